@@ -1,0 +1,316 @@
+"""CPU oracle of the routed sparse-attention step of Memory Sparse Attention (MSA).
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module. It shares no code,
+table or helper with the CUDA library, and the library never calls it.
+
+Everything is plain numpy in fp64, one document / one chunk / one query row at
+a time, in the order the method states its steps:
+
+1. chunk-mean pooling of each document's per-token routing keys into the
+   compressed routing keys K_r (256-token chunks)
+   -- "MSA架构：突破大模型记忆瓶颈的稀疏注意力技术", §2.1 item 2 and §3.1
+      (the ``chunk_mean_pooling`` example: a mean over each 256-token chunk);
+   -- "MSA (Memory Sparse Attention)" (robocikowo.com), Komponenty: the
+      Router's K_r is a compressed document representation; Pułapki
+      implementacyjne: build the bank offline with chunked mean pooling.
+2. Parallel (document-wise) RoPE on the bank keys: positions restart at 0 at
+   every document's first token
+   -- "MSA架构…", §2.2; robocikowo.com, Komponenty (Document-wise RoPE,
+      Parallel RoPE) and Pułapki implementacyjne (RoPE consistency).
+3. the routing query q_r of a query block = mean of its tokens' routing queries.
+4. router: cosine similarity between q_r and every chunk of K_r; a document's
+   score is the max over its chunks
+   -- "MSA架构…", §2.1 item 1 (cosine top-k router); robocikowo.com,
+      Komponenty (Router / Routing Projector).
+5. top-k documents per (query block, KV head), larger score first, equal
+   scores to the lower document index
+   -- robocikowo.com, Hiperparametry (Top-k documents), Paradygmat wykonania.
+6. one softmax attention over the selected documents' K/V (all visible) plus
+   the causal local context, whose queries and keys carry Global RoPE at
+   positions k_off + u with k_off = top_k * max document length
+   -- robocikowo.com, Komponenty (Memory Sparse Attention Layer: append the
+      selected documents' K/V to the local context; Global RoPE), Pułapki
+      implementacyjne (Global RoPE with a k-offset for the active context),
+      Paradygmat wykonania (only the k selected documents take part).
+
+Readings where the pages are silent (each is listed in the design doc):
+the document score is the max over its chunks; a ragged last chunk is the mean
+over its actual tokens; q_r is the unnormalised block mean; a zero-norm cosine
+is 0; RoPE is rotate-half with theta_i = base^(-2i/d); the softmax scale is
+1/sqrt(d); query head hq reads KV head hq // (Hq/Hkv); the Tq queries are the
+last Tq local tokens and local key u is visible to local query i iff u <= i.
+
+Parity pins: every function here is pinned in tests/test_oracle_pins.py
+against closed forms, invariants, library special cases or brute force.
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, List, Sequence, Tuple
+
+import numpy as np
+
+CHUNK = 256
+
+
+# --------------------------------------------------------------------------
+# 1. document layout and chunk-mean pooling
+# --------------------------------------------------------------------------
+
+def doc_offsets(doc_lens: Sequence[int]) -> np.ndarray:
+    """Token offset of every document in the concatenated bank, length n+1."""
+    off = np.zeros(len(doc_lens) + 1, dtype=np.int64)
+    for j, L in enumerate(doc_lens):
+        if L < 1:
+            raise ValueError("every document holds at least one token")
+        off[j + 1] = off[j] + int(L)
+    return off
+
+
+def chunk_spans(doc_len: int, chunk: int = CHUNK) -> List[Tuple[int, int]]:
+    """[start, end) token spans of one document's chunks, relative to the document."""
+    return [(s, min(s + chunk, doc_len)) for s in range(0, doc_len, chunk)]
+
+
+def chunk_mean_pool(R_doc: np.ndarray, chunk: int = CHUNK) -> np.ndarray:
+    """K_r rows of one document: the arithmetic mean of each chunk's actual tokens.
+
+    R_doc: [L, d_r] per-token routing keys of one document and one KV head.
+    Returns [ceil(L/chunk), d_r] in fp64.
+    """
+    R_doc = np.asarray(R_doc, dtype=np.float64)
+    rows = []
+    for s, e in chunk_spans(R_doc.shape[0], chunk):
+        total = np.zeros(R_doc.shape[1], dtype=np.float64)
+        for t in range(s, e):
+            total += R_doc[t]
+        rows.append(total / (e - s))
+    return np.stack(rows)
+
+
+def build_routing_keys(R_head: np.ndarray, doc_lens: Sequence[int],
+                       chunk: int = CHUNK) -> Tuple[np.ndarray, np.ndarray]:
+    """K_r of one KV head over the whole bank.
+
+    R_head: [Ntok, d_r] routing keys of one KV head, documents concatenated.
+    Returns (K_r [Nch, d_r], chunk_doc [Nch]) where chunk_doc[c] is the
+    document that owns chunk c.
+    """
+    off = doc_offsets(doc_lens)
+    kr, owner = [], []
+    for j, L in enumerate(doc_lens):
+        rows = chunk_mean_pool(R_head[off[j]:off[j + 1]], chunk)
+        kr.append(rows)
+        owner.extend([j] * rows.shape[0])
+    return np.concatenate(kr, axis=0), np.asarray(owner, dtype=np.int64)
+
+
+# --------------------------------------------------------------------------
+# 2. RoPE (rotate-half), Parallel and Global placement
+# --------------------------------------------------------------------------
+
+def rope_inv_freq(d: int, base: float) -> np.ndarray:
+    """theta_i = base^(-2i/d), i < d/2, in fp64."""
+    i = np.arange(d // 2, dtype=np.float64)
+    return base ** (-2.0 * i / d)
+
+
+def rope(x: np.ndarray, pos, base: float) -> np.ndarray:
+    """Rotate-half RoPE: pair (x_i, x_{i+d/2}) is turned by pos * theta_i.
+
+    x: [..., d]; pos: scalar or array broadcastable to x.shape[:-1].
+    x'_i = x_i cos - x_{i+d/2} sin;  x'_{i+d/2} = x_{i+d/2} cos + x_i sin.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    h = d // 2
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * rope_inv_freq(d, base)
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = x[..., :h], x[..., h:]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
+def parallel_rope_positions(doc_lens: Sequence[int]) -> np.ndarray:
+    """Position of every bank token: its index inside its own document."""
+    return np.concatenate([np.arange(int(L), dtype=np.int64) for L in doc_lens])
+
+
+def parallel_rope_bank(K_head: np.ndarray, doc_lens: Sequence[int], base: float) -> np.ndarray:
+    """Bank keys of one KV head with document-wise (Parallel) RoPE applied."""
+    return rope(K_head, parallel_rope_positions(doc_lens), base)
+
+
+def k_offset(top_k: int, doc_lens: Sequence[int]) -> int:
+    """Global-RoPE offset of the active context: top_k * (longest document)."""
+    return int(top_k) * int(max(int(L) for L in doc_lens))
+
+
+# --------------------------------------------------------------------------
+# 3-5. routing
+# --------------------------------------------------------------------------
+
+def block_mean_query(Qr_tokens: np.ndarray, route_block: int) -> np.ndarray:
+    """q_r of each routing block: mean of its tokens' routing queries.
+
+    Qr_tokens: [Tq, d_r] for one (sequence, KV head). Returns [Tq/route_block, d_r].
+    """
+    Qr_tokens = np.asarray(Qr_tokens, dtype=np.float64)
+    Tq = Qr_tokens.shape[0]
+    if Tq % route_block:
+        raise ValueError("query tokens must split into whole routing blocks")
+    out = []
+    for s in range(0, Tq, route_block):
+        total = np.zeros(Qr_tokens.shape[1], dtype=np.float64)
+        for t in range(s, s + route_block):
+            total += Qr_tokens[t]
+        out.append(total / route_block)
+    return np.stack(out)
+
+
+def cosine(q: np.ndarray, k: np.ndarray) -> float:
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    den = math.sqrt(float(q @ q)) * math.sqrt(float(k @ k))
+    return float(q @ k) / max(den, 1e-30)
+
+
+def route_doc_scores(q_r: np.ndarray, K_r: np.ndarray, chunk_doc: np.ndarray,
+                     n_docs: int) -> np.ndarray:
+    """Document scores of one routing query: max over each document's chunk cosines."""
+    scores = np.full(n_docs, -np.inf, dtype=np.float64)
+    for c in range(K_r.shape[0]):
+        s = cosine(q_r, K_r[c])
+        j = int(chunk_doc[c])
+        if s > scores[j]:
+            scores[j] = s
+    return scores
+
+
+def chunk_cosines(q_r: np.ndarray, K_r: np.ndarray) -> np.ndarray:
+    """All chunk cosines of one routing query at once (same definition, vectorised)."""
+    q = np.asarray(q_r, dtype=np.float64)
+    K = np.asarray(K_r, dtype=np.float64)
+    den = np.sqrt(q @ q) * np.sqrt(np.einsum("cd,cd->c", K, K))
+    return (K @ q) / np.maximum(den, 1e-30)
+
+
+def doc_max(chunk_scores: np.ndarray, chunk_doc: np.ndarray, n_docs: int) -> np.ndarray:
+    out = np.full(n_docs, -np.inf, dtype=np.float64)
+    np.maximum.at(out, chunk_doc, chunk_scores)
+    return out
+
+
+def select_top_k(doc_scores: np.ndarray, top_k: int) -> np.ndarray:
+    """Indices of the top_k documents, ordered by (score desc, index asc)."""
+    n = len(doc_scores)
+    if not 1 <= top_k <= n:
+        raise ValueError("1 <= top_k <= n_docs")
+    order = sorted(range(n), key=lambda j: (-float(doc_scores[j]), j))
+    return np.asarray(order[:top_k], dtype=np.int64)
+
+
+# --------------------------------------------------------------------------
+# 6. routed attention
+# --------------------------------------------------------------------------
+
+def softmax_attention(q: np.ndarray, keys: np.ndarray, values: np.ndarray) -> np.ndarray:
+    """softmax(q . keys^T / sqrt(d)) . values for one query row, fp64, max-subtracted."""
+    q = np.asarray(q, dtype=np.float64)
+    d = q.shape[-1]
+    logits = (np.asarray(keys, dtype=np.float64) @ q) / math.sqrt(d)
+    m = logits.max()
+    w = np.exp(logits - m)
+    return (w @ np.asarray(values, dtype=np.float64)) / w.sum()
+
+
+def routed_attention_row(q: np.ndarray, q_index: int, k_off: int, base: float,
+                         mem_k_rot: np.ndarray, mem_v: np.ndarray,
+                         local_k: np.ndarray, local_v: np.ndarray) -> np.ndarray:
+    """Output of one query row.
+
+    q:        [d] un-rotated query of the local token at index q_index.
+    mem_k_rot:[M, d] keys of the selected documents with Parallel RoPE applied.
+    mem_v:    [M, d] their values.
+    local_k/v:[Lc, d] un-rotated local keys / values; keys 0..q_index are visible.
+    """
+    q_rot = rope(q, k_off + q_index, base)
+    vis = q_index + 1
+    loc_k_rot = rope(local_k[:vis], k_off + np.arange(vis), base)
+    keys = np.concatenate([np.asarray(mem_k_rot, dtype=np.float64), loc_k_rot], axis=0)
+    values = np.concatenate([np.asarray(mem_v, dtype=np.float64),
+                             np.asarray(local_v[:vis], dtype=np.float64)], axis=0)
+    return softmax_attention(q_rot, keys, values)
+
+
+# --------------------------------------------------------------------------
+# the whole step on explicit (small) tensors
+# --------------------------------------------------------------------------
+
+def forward(inputs: Dict[str, np.ndarray], doc_lens: Sequence[int], top_k: int,
+            route_block: int, base: float = 10000.0, chunk: int = CHUNK,
+            selection=None) -> Dict[str, np.ndarray]:
+    """The routed sparse-attention step on fully materialised inputs.
+
+    inputs (all real-valued arrays, converted to fp64):
+      K, V   [Hkv, Ntok, d]  bank keys (un-rotated) and values
+      R      [Hkv, Ntok, d_r] per-token routing keys
+      Q      [B, Hq, Tq, d]  un-rotated queries (the last Tq local tokens)
+      Qr     [B, Hkv, Tq, d_r] per-token routing queries
+      LK, LV [B, Hkv, Lc, d] un-rotated local keys / values
+    selection: optional [B, nblk, Hkv, k] document indices to attend over
+      instead of the oracle's own top-k (used when several sets are correct).
+
+    Returns K_r [Hkv, Nch, d_r], K_rot [Hkv, Ntok, d], q_r [B, nblk, Hkv, d_r],
+    doc_scores [B, nblk, Hkv, n], topk [B, nblk, Hkv, k], out [B, Hq, Tq, d].
+    """
+    K = np.asarray(inputs["K"], dtype=np.float64)
+    V = np.asarray(inputs["V"], dtype=np.float64)
+    R = np.asarray(inputs["R"], dtype=np.float64)
+    Q = np.asarray(inputs["Q"], dtype=np.float64)
+    Qr = np.asarray(inputs["Qr"], dtype=np.float64)
+    LK = np.asarray(inputs["LK"], dtype=np.float64)
+    LV = np.asarray(inputs["LV"], dtype=np.float64)
+    Hkv, Ntok, d = K.shape
+    B, Hq, Tq, _ = Q.shape
+    Lc = LK.shape[2]
+    n = len(doc_lens)
+    G = Hq // Hkv
+    nblk = Tq // route_block
+    off = doc_offsets(doc_lens)
+    k_off = k_offset(top_k, doc_lens)
+
+    K_r, chunk_doc = [], None
+    K_rot = np.empty_like(K)
+    for h in range(Hkv):
+        kr, chunk_doc = build_routing_keys(R[h], doc_lens, chunk)
+        K_r.append(kr)
+        K_rot[h] = parallel_rope_bank(K[h], doc_lens, base)
+    K_r = np.stack(K_r)
+
+    q_r = np.empty((B, nblk, Hkv, R.shape[2]))
+    scores = np.empty((B, nblk, Hkv, n))
+    topk = np.empty((B, nblk, Hkv, top_k), dtype=np.int64)
+    for b in range(B):
+        for h in range(Hkv):
+            qb = block_mean_query(Qr[b, h], route_block)
+            for blk in range(nblk):
+                q_r[b, blk, h] = qb[blk]
+                scores[b, blk, h] = route_doc_scores(qb[blk], K_r[h], chunk_doc, n)
+                topk[b, blk, h] = select_top_k(scores[b, blk, h], top_k)
+    sel = topk if selection is None else np.asarray(selection, dtype=np.int64)
+
+    out = np.empty((B, Hq, Tq, d))
+    for b in range(B):
+        for hq in range(Hq):
+            h = hq // G
+            for t in range(Tq):
+                blk = t // route_block
+                docs = sel[b, blk, h]
+                mk = np.concatenate([K_rot[h, off[j]:off[j + 1]] for j in docs], axis=0)
+                mv = np.concatenate([V[h, off[j]:off[j + 1]] for j in docs], axis=0)
+                i = Lc - Tq + t
+                out[b, hq, t] = routed_attention_row(Q[b, hq, t], i, k_off, base, mk, mv,
+                                                     LK[b, h], LV[b, h])
+    return {"K_r": K_r, "K_rot": K_rot, "q_r": q_r, "doc_scores": scores, "topk": topk,
+            "out": out, "k_off": k_off}
