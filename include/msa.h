@@ -1,0 +1,178 @@
+/*
+ * msa.h — C ABI of the routed sparse-attention step of Memory Sparse Attention
+ * (MSA) on NVIDIA B200 (sm_100a).
+ *
+ * The step, as the pages state it:
+ *   - a memory bank of documents; each document's per-token routing keys are
+ *     compressed by chunk-mean pooling over 256-token chunks into K_r
+ *     ("MSA架构：突破大模型记忆瓶颈的稀疏注意力技术", §2.1 item 2, §3.1);
+ *   - the bank keys carry document-wise (Parallel) RoPE, positions restarting at
+ *     0 in every document ("MSA (Memory Sparse Attention)", robocikowo.com,
+ *     Komponenty: Document-wise RoPE; "MSA架构…", §2.2);
+ *   - a router scores the query's routing vector against K_r by cosine
+ *     similarity and keeps the top-k documents ("MSA架构…", §2.1 item 1;
+ *     robocikowo.com, Komponenty: Router (Routing Projector); Hiperparametry:
+ *     Top-k documents);
+ *   - attention runs over the selected documents' K/V appended to the local
+ *     context, whose queries and keys carry Global RoPE with a k-offset
+ *     (robocikowo.com, Komponenty: Memory Sparse Attention Layer; Pułapki
+ *     implementacyjne: RoPE consistency; Paradygmat wykonania).
+ *
+ * Readings this library takes where the pages are silent: a document's score
+ * is the max of its chunks' cosines; a ragged last chunk is the mean of its
+ * actual tokens; q_r of a routing block is the mean of its tokens' routing
+ * queries; equal scores go to the lower document index; the Global-RoPE offset
+ * is k_off = top_k * (longest document in the bank); local token u sits at
+ * position k_off + u; the Tq queries are the last Tq local tokens; local key u
+ * is visible to local query i iff u <= i; every selected document token is
+ * visible to every query; softmax scale 1/sqrt(d); RoPE is rotate-half with
+ * theta_i = base^(-2i/d); query head hq reads KV head hq / (Hq/Hkv).
+ *
+ * Conventions for every entry point:
+ *   - All tensors are caller-owned, row-major, densely packed, bf16 unless
+ *     stated, and live in device memory unless the argument says "host".
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
+ *     asynchronous on it; host arrays are read before the call returns.
+ *   - Every call returns an msa_status and never throws. Argument errors are
+ *     detected on the host before any launch. CUDA errors map to MSA_ERR_CUDA.
+ *     Device-side bounded waits that expire set a flag read by
+ *     msa_get_device_error() (MSA_ERR_TIMEOUT).
+ *   - There is no CPU fallback: without a usable sm_100 device the calls that
+ *     launch work return MSA_ERR_CUDA or MSA_ERR_UNSUPPORTED.
+ *   - Supported shapes: head_dim = route_dim in {64, 128}; n_q_heads a
+ *     multiple of n_kv_heads; G = n_q_heads / n_kv_heads and route_block with
+ *     G * route_block <= 16; 1 <= top_k <= min(n_docs, 64).
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1, /* a null pointer, an out-of-range size or index */
+  MSA_ERR_UNSUPPORTED = 2, /* a valid shape this build does not implement */
+  MSA_ERR_OOM = 3,         /* device or pinned allocation failed */
+  MSA_ERR_CUDA = 4,        /* a CUDA runtime or driver call failed */
+  MSA_ERR_TIMEOUT = 5,     /* a bounded device-side wait expired */
+  MSA_ERR_HOST_TIER = 6    /* the pinned-host K/V tier could not serve a fetch */
+} msa_status;
+
+typedef enum {
+  MSA_KV_DEVICE = 0,      /* bank K/V in device memory */
+  MSA_KV_PINNED_HOST = 1  /* bank K/V in pinned (page-locked) host memory */
+} msa_kv_location;
+
+/* Opaque bank handle. Owns: K_r (fp32) and its inverse norms, document and
+ * chunk offsets, RoPE tables, workspace, and (host tier) the device staging
+ * pool, side stream and events. */
+typedef struct msa_bank msa_bank;
+
+typedef struct {
+  int32_t n_docs;          /* number of documents, >= 1 */
+  int32_t n_kv_heads;      /* Hkv, >= 1 */
+  int32_t head_dim;        /* d: 64 or 128 */
+  int32_t route_dim;       /* d_r: equal to head_dim */
+  const int64_t* doc_lens; /* host [n_docs], each >= 1 token */
+  float rope_base;         /* RoPE base, > 1 (10000 in the workloads) */
+  int32_t kv_location;     /* msa_kv_location */
+  const void* k;           /* bank keys   [Hkv, kv_rows, d]; Parallel RoPE already applied
+                              (msa_build_bank applies it in place) */
+  const void* v;           /* bank values [Hkv, kv_rows, d] */
+  int64_t kv_rows;         /* rows per head in k/v; 0 means Ntok = sum(doc_lens) */
+  const int64_t* doc_rows; /* host [n_docs] or NULL: first row of document j inside
+                              each head's k/v; NULL means the prefix sums of doc_lens.
+                              Several documents may share rows (an aliased pool). */
+} msa_bank_config;
+
+/* Creates a bank: validates the layout, computes document/chunk offsets and
+ * the Parallel-RoPE table (angles in fp64), allocates K_r. Launches nothing
+ * that reads k/v; the handle keeps the k/v pointers (caller-owned; they must
+ * outlive the handle). On error *out is set to NULL. */
+msa_status msa_bank_create(const msa_bank_config* cfg, msa_bank** out);
+
+/* Frees everything the handle owns (synchronises the device first). NULL is a no-op. */
+msa_status msa_bank_destroy(msa_bank* bank);
+
+/* Offline bank build for documents [doc_begin, doc_end):
+ *  - pools K_r[h, c] = mean of the per-token routing keys of chunk c over its
+ *    actual tokens (fp32 accumulate, fp32 store) and 1/||K_r[h, c]||;
+ *  - if k_slice != NULL, applies Parallel RoPE in place to k_slice (position of
+ *    a token = its index inside its document), rounding to bf16.
+ * r_slice: [Hkv][T][d_r] routing keys of those documents, where T = their total
+ *   length and row 0 is the first token of doc_begin; head h starts at
+ *   r_slice + h * r_head_stride elements (r_head_stride >= T).
+ * k_slice: same layout for the keys, head stride k_head_stride (>= T); for a
+ *   device bank, pass the bank's own k + doc_rows[doc_begin] * d with stride
+ *   kv_rows. For a pinned-host bank, pass a device copy and copy it back.
+ * Building in slices lets routing keys that do not fit in HBM stream through.
+ * (robocikowo.com, Pułapki implementacyjne: encode offline, chunked mean pooling.) */
+msa_status msa_build_bank(msa_bank* bank, int32_t doc_begin, int32_t doc_end,
+                          const void* r_slice, int64_t r_head_stride,
+                          void* k_slice, int64_t k_head_stride, void* stream);
+
+/* Sizes and device pointers owned by the bank: K_r fp32 [Hkv, n_chunks, d_r],
+ * inverse norms fp32 [Hkv, n_chunks]. Any output pointer may be NULL. */
+msa_status msa_bank_info(const msa_bank* bank, int64_t* n_tokens, int64_t* n_chunks,
+                         int64_t* max_doc_len, const float** k_r, const float** k_r_inv_norm);
+
+/* One step's queries. */
+typedef struct {
+  int32_t batch;        /* B */
+  int32_t n_q_heads;    /* Hq, a multiple of Hkv */
+  int32_t q_tokens;     /* Tq: the last Tq local tokens are the queries */
+  int32_t local_len;    /* Lc >= Tq */
+  int32_t route_block;  /* Bq: query tokens per routing block; Tq % Bq == 0 */
+  const void* q;        /* [B, Hq, Tq, d]   queries, no RoPE applied */
+  const void* qr;       /* [B, Hkv, Tq, d_r] per-token routing queries */
+  const void* local_k;  /* [B, Hkv, Lc, d]  local keys, no RoPE applied */
+  const void* local_v;  /* [B, Hkv, Lc, d]  local values */
+} msa_query;
+
+/* Pre-allocates the workspace and Global-RoPE table for steps up to the given
+ * sizes, so that later calls allocate nothing (required before capturing
+ * calls into a CUDA graph). */
+msa_status msa_reserve(msa_bank* bank, const msa_query* shape, int32_t top_k);
+
+/* Router: q_r per (sequence, routing block, KV head) = mean of the block's
+ * routing queries; score of chunk c = cos(q_r, K_r[h, c]); document score =
+ * max over its chunks; selection = top_k documents, ordered by (score desc,
+ * index asc).
+ * doc_scores:  [B, nblk, Hkv, n_docs] fp32, or NULL.
+ * topk_idx:    [B, nblk, Hkv, top_k] int32 (required).
+ * topk_scores: [B, nblk, Hkv, top_k] fp32, or NULL.  (nblk = Tq / Bq) */
+msa_status msa_route(msa_bank* bank, const msa_query* q, int32_t top_k, float* doc_scores,
+                     int32_t* topk_idx, float* topk_scores, void* stream);
+
+/* Routed attention: for query head hq at local index i = Lc - Tq + t,
+ * out[b, hq, t] = softmax over { all tokens of the documents in
+ * topk_idx[b, t / Bq, hq / G] (bank keys, Parallel RoPE) } and { local keys
+ * u <= i with Global RoPE at k_off + u }, query with Global RoPE at k_off + i,
+ * scale 1/sqrt(d), applied to the matching values. k_off = top_k * max_doc_len.
+ * topk_idx: [B, nblk, Hkv, top_k] int32 in [0, n_docs) (checked on the device;
+ *   an out-of-range index sets MSA_ERR_INVALID_ARG in the device error flag and
+ *   that document is skipped).
+ * out: [B, Hq, Tq, d] fp32. */
+msa_status msa_attend(msa_bank* bank, const msa_query* q, int32_t top_k,
+                      const int32_t* topk_idx, float* out, void* stream);
+
+/* msa_route followed by msa_attend on one stream; topk_idx receives the selection. */
+msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_t* topk_idx,
+                       float* out, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device-side error flag
+ * (MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_INVALID_ARG). */
+msa_status msa_get_device_error(msa_bank* bank, void* stream);
+
+/* Static description of a status code. */
+const char* msa_status_string(msa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */

@@ -1,0 +1,184 @@
+"""Python binding of libmsa (routed sparse attention of Memory Sparse Attention on B200).
+
+Argument marshalling only: every step runs in the CUDA library. The functions
+carry the names of the C entry points in include/msa.h and take raw integers
+(device pointers, host arrays via numpy, stream handles). `ptr()` turns a
+torch tensor into its device pointer after checking dtype and contiguity.
+
+Importing this module loads libmsa.so and fails loudly when it is missing;
+there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmsa.so")
+
+MSA_OK = 0
+MSA_ERR_INVALID_ARG = 1
+MSA_ERR_UNSUPPORTED = 2
+MSA_ERR_OOM = 3
+MSA_ERR_CUDA = 4
+MSA_ERR_TIMEOUT = 5
+MSA_ERR_HOST_TIER = 6
+
+MSA_KV_DEVICE = 0
+MSA_KV_PINNED_HOST = 1
+
+
+class MsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {msa_status_string(status)} (status {status})")
+        self.status = status
+
+
+class msa_bank_config(ctypes.Structure):
+    _fields_ = [
+        ("n_docs", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("route_dim", ctypes.c_int32), ("doc_lens", ctypes.POINTER(ctypes.c_int64)),
+        ("rope_base", ctypes.c_float), ("kv_location", ctypes.c_int32), ("k", ctypes.c_void_p),
+        ("v", ctypes.c_void_p), ("kv_rows", ctypes.c_int64), ("doc_rows", ctypes.POINTER(ctypes.c_int64)),
+    ]
+
+
+class msa_query(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("q_tokens", ctypes.c_int32),
+        ("local_len", ctypes.c_int32), ("route_block", ctypes.c_int32), ("q", ctypes.c_void_p),
+        ("qr", ctypes.c_void_p), ("local_k", ctypes.c_void_p), ("local_v", ctypes.c_void_p),
+    ]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libmsa.so is not built ({LIB_PATH}); run python -m sparse_attention_routed_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    sig = {
+        "msa_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "msa_bank_create": ([ctypes.POINTER(msa_bank_config), ctypes.POINTER(vp)], ctypes.c_int),
+        "msa_bank_destroy": ([vp], ctypes.c_int),
+        "msa_build_bank": ([vp, i32, i32, vp, i64, vp, i64, vp], ctypes.c_int),
+        "msa_bank_info": ([vp, ctypes.POINTER(i64), ctypes.POINTER(i64), ctypes.POINTER(i64),
+                           ctypes.POINTER(vp), ctypes.POINTER(vp)], ctypes.c_int),
+        "msa_reserve": ([vp, ctypes.POINTER(msa_query), i32], ctypes.c_int),
+        "msa_route": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp, vp], ctypes.c_int),
+        "msa_attend": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp], ctypes.c_int),
+        "msa_forward": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp], ctypes.c_int),
+        "msa_get_device_error": ([vp, vp], ctypes.c_int),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+LIB = _load()
+
+# Every symbol include/msa.h declares, in declaration order.
+EXPORTED = ["msa_bank_create", "msa_bank_destroy", "msa_build_bank", "msa_bank_info", "msa_reserve",
+            "msa_route", "msa_attend", "msa_forward", "msa_get_device_error", "msa_status_string"]
+
+
+def msa_status_string(status: int) -> str:
+    return LIB.msa_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != MSA_OK:
+        raise MsaError(status, where)
+
+
+def ptr(t, dtype=None) -> int:
+    """Device (or pinned host) pointer of a contiguous torch tensor; 0 for None."""
+    if t is None:
+        return 0
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def make_query(batch, n_q_heads, q_tokens, local_len, route_block, q=0, qr=0, local_k=0, local_v=0) -> msa_query:
+    return msa_query(batch, n_q_heads, q_tokens, local_len, route_block, q or None, qr or None,
+                     local_k or None, local_v or None)
+
+
+def msa_bank_create(n_docs: int, n_kv_heads: int, head_dim: int, doc_lens, k: int, v: int,
+                    rope_base: float = 10000.0, kv_location: int = MSA_KV_DEVICE, kv_rows: int = 0,
+                    doc_rows=None, route_dim: Optional[int] = None, check: bool = True):
+    """Returns (status, handle). doc_lens / doc_rows are host int64 sequences."""
+    lens = np.ascontiguousarray(np.asarray(doc_lens, dtype=np.int64))
+    rows = None if doc_rows is None else np.ascontiguousarray(np.asarray(doc_rows, dtype=np.int64))
+    cfg = msa_bank_config(
+        n_docs, n_kv_heads, head_dim, head_dim if route_dim is None else route_dim,
+        lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), rope_base, kv_location, k or None, v or None,
+        kv_rows, None if rows is None else rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)))
+    handle = ctypes.c_void_p()
+    st = LIB.msa_bank_create(ctypes.byref(cfg), ctypes.byref(handle))
+    if check:
+        _check(st, "msa_bank_create")
+    return st, handle.value
+
+
+def msa_bank_destroy(bank) -> int:
+    return LIB.msa_bank_destroy(bank)
+
+
+def msa_build_bank(bank, doc_begin, doc_end, r_slice, r_head_stride, k_slice, k_head_stride, stream=0,
+                   check=True) -> int:
+    st = LIB.msa_build_bank(bank, doc_begin, doc_end, r_slice or None, r_head_stride, k_slice or None,
+                            k_head_stride, stream or None)
+    if check:
+        _check(st, "msa_build_bank")
+    return st
+
+
+def msa_bank_info(bank):
+    n_tok, n_ch, max_len = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    kr, kinv = ctypes.c_void_p(), ctypes.c_void_p()
+    _check(LIB.msa_bank_info(bank, ctypes.byref(n_tok), ctypes.byref(n_ch), ctypes.byref(max_len),
+                             ctypes.byref(kr), ctypes.byref(kinv)), "msa_bank_info")
+    return {"n_tokens": n_tok.value, "n_chunks": n_ch.value, "max_doc_len": max_len.value,
+            "k_r": kr.value, "k_r_inv_norm": kinv.value}
+
+
+def msa_reserve(bank, query: msa_query, top_k: int, check=True) -> int:
+    st = LIB.msa_reserve(bank, ctypes.byref(query), top_k)
+    if check:
+        _check(st, "msa_reserve")
+    return st
+
+
+def msa_route(bank, query: msa_query, top_k: int, doc_scores: int, topk_idx: int, topk_scores: int,
+              stream=0, check=True) -> int:
+    st = LIB.msa_route(bank, ctypes.byref(query), top_k, doc_scores or None, topk_idx or None,
+                       topk_scores or None, stream or None)
+    if check:
+        _check(st, "msa_route")
+    return st
+
+
+def msa_attend(bank, query: msa_query, top_k: int, topk_idx: int, out: int, stream=0, check=True) -> int:
+    st = LIB.msa_attend(bank, ctypes.byref(query), top_k, topk_idx or None, out or None, stream or None)
+    if check:
+        _check(st, "msa_attend")
+    return st
+
+
+def msa_forward(bank, query: msa_query, top_k: int, topk_idx: int, out: int, stream=0, check=True) -> int:
+    st = LIB.msa_forward(bank, ctypes.byref(query), top_k, topk_idx or None, out or None, stream or None)
+    if check:
+        _check(st, "msa_forward")
+    return st
+
+
+def msa_get_device_error(bank, stream=0) -> int:
+    return LIB.msa_get_device_error(bank, stream or None)

@@ -1,0 +1,516 @@
+// sparse_attend (decode): one fused softmax attention over the selected
+// documents' K/V (Parallel RoPE already in the bank keys, every token visible)
+// plus the causal local context (Global RoPE at k_off + u applied here).
+//   "MSA (Memory Sparse Attention)" (robocikowo.com), Komponenty (Memory Sparse
+//   Attention Layer: append the top-k documents' K/V to the local context),
+//   Pułapki implementacyjne (Global RoPE with a k-offset for the active query
+//   context), Paradygmat wykonania (only the k selected documents take part).
+//
+// Design (B200, HBM-bound):
+//  * Problem p = (sequence, routing block, KV head). Its key list is the tiles
+//    of 64 keys of each selected document followed by the local tiles up to
+//    the last query's position. The list is cut into n_splits equal ranges,
+//    one CTA each (split-KV), so ragged documents balance by construction.
+//  * One producer lane streams K and V tiles with 2-D TMA loads (128-byte
+//    swizzle, evict-first L2 policy) into an NS-stage ring guarded by
+//    full/empty mbarriers; 4 consumer warps take tiles round-robin.
+//  * The problem's query rows (G heads x Bq tokens <= 16) are few, so the MMA
+//    runs "keys as M": S^T = K Q^T with mma.sync m16n8k16 (keys fill M=16, the
+//    rows sit in N=8), then O^T += V^T P^T with V^T fed by ldmatrix.trans and
+//    P^T produced in registers by movmatrix.trans. Padding is at most N-side.
+//  * Online softmax in the exp2 domain; each CTA leaves (m, l, O) per row and
+//    attend_merge combines the splits.
+#include "common.cuh"
+#include "internal.h"
+
+namespace msa {
+namespace {
+
+constexpr int kTile = 64;          // keys per tile
+constexpr int kWarps = 4;          // consumer warps
+constexpr int kBufs = 1;           // ring slots owned by each consumer warp
+constexpr int kStages = kWarps * kBufs;
+constexpr int kMaxTopK = 64;
+constexpr int kRowsMax = 16;
+constexpr int kMT = kTile / 16;    // 16-key m-tiles per tile
+
+// Ring ownership: relative tile n goes to consumer warp n % kWarps; that warp's
+// q-th tile (q = n / kWarps) uses slot w + kWarps * (q % kBufs). Every slot is
+// filled and drained by one producer and one consumer warp in order, so each
+// mbarrier wait targets the phase right after one the waiter saw complete
+// (a parity wait is only unambiguous under that condition).
+__device__ __forceinline__ void slot_of(int n, int& stage, int& use) {
+  const int w = n % kWarps, q = n / kWarps;
+  stage = w + kWarps * (q % kBufs);
+  use = q / kBufs;
+}
+
+template <int D>
+struct Cfg {
+  static constexpr int kBoxes = D / 64;                 // 128-byte-wide TMA boxes per row
+  static constexpr int kBoxBytes = kTile * 128;
+  static constexpr int kTileBytes = kTile * D * 2;      // one of K or V
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kRingBytes = kStages * kStageBytes;
+};
+
+struct TileRef {
+  int di;  // document slot (0..k-1) or k for the local context
+  int tt;  // tile index inside it
+};
+
+__device__ __forceinline__ TileRef locate(const int* tile_start, int k, int j, int hint) {
+  int di = hint;
+  while (di < k && j >= tile_start[di + 1]) ++di;
+  return {di, j - tile_start[di]};
+}
+
+template <int D, int NT>
+__global__ void __launch_bounds__((kWarps + 1) * 32, 1)
+    attend_decode_kernel(const __grid_constant__ CUtensorMap tm_bk, const __grid_constant__ CUtensorMap tm_bv,
+                         const __grid_constant__ CUtensorMap tm_lk, const __grid_constant__ CUtensorMap tm_lv,
+                         const AttendArgs a) {
+  using C = Cfg<D>;
+  static_assert(kWarps * NT * 8 * (D + 2) * 4 <= C::kRingBytes, "merge scratch must fit in the ring");
+  extern __shared__ uint8_t smem_raw[];
+  // 128-byte swizzle is defined on shared-memory address bits: align the ring to 1 KiB there.
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  uint8_t* ring = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kRingBytes);
+  uint64_t* empty = full + kStages;
+  int* tile_start = reinterpret_cast<int*>(empty + kStages);         // [kMaxTopK + 2]
+  int* doc_len_s = tile_start + kMaxTopK + 2;                          // [kMaxTopK]
+  long long* doc_base_s = reinterpret_cast<long long*>(doc_len_s + kMaxTopK);  // [kMaxTopK]
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int p = blockIdx.y, split = blockIdx.x;
+  const int G = a.n_q_heads / a.n_kv_heads;
+  const int nblk = a.q_tokens / a.route_block;
+  const int h = p % a.n_kv_heads;
+  const int blk = (p / a.n_kv_heads) % nblk;
+  const int b = p / (a.n_kv_heads * nblk);
+  const int rows = G * a.route_block;
+  const int i_first = a.local_len - a.q_tokens + blk * a.route_block;  // local index of row 0's token
+  const int i_max = i_first + a.route_block - 1;
+  const int k = a.top_k;
+
+  if (tid < k) {
+    const int j = a.sel[(int64_t)p * k + tid];
+    int len = 0;
+    long long base = 0;
+    if (j >= 0 && j < a.n_docs) {
+      len = a.doc_len[j];
+      base = (long long)h * a.kv_rows + a.doc_row[j];
+    } else {
+      atomicCAS(a.err, 0, kErrInvalidArg);
+    }
+    doc_len_s[tid] = len;
+    doc_base_s[tid] = base;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int d = 0; d < k; ++d) {
+      tile_start[d] = acc;
+      acc += (doc_len_s[d] + kTile - 1) / kTile;
+    }
+    tile_start[k] = acc;
+    tile_start[k + 1] = acc + (i_max + 1 + kTile - 1) / kTile;
+  }
+  __syncthreads();
+  const int T = tile_start[k + 1];
+  const int t0 = (int)(((long long)T * split) / a.n_splits);
+  const int t1 = (int)(((long long)T * (split + 1)) / a.n_splits);
+  const int ntiles = t1 - t0;
+
+  if (warp == kWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && ntiles > 0) {
+      prefetch_tensormap(&tm_bk);
+      prefetch_tensormap(&tm_bv);
+      prefetch_tensormap(&tm_lk);
+      prefetch_tensormap(&tm_lv);
+      const uint64_t pol = l2_policy_evict_first();
+      int hint = 0;
+      int issued = 0;
+      for (int n = 0; n < ntiles; ++n) {
+        int stage, use;
+        slot_of(n, stage, use);
+        if (use > 0 && !mbar_wait_bounded(&empty[stage], (use - 1) & 1, a.err)) break;
+        const TileRef tr = locate(tile_start, k, t0 + n, hint);
+        hint = tr.di;
+        const CUtensorMap* mk;
+        const CUtensorMap* mv;
+        int y;
+        if (tr.di < k) {
+          mk = &tm_bk; mv = &tm_bv;
+          y = (int)(doc_base_s[tr.di] + (long long)tr.tt * kTile);
+        } else {
+          mk = &tm_lk; mv = &tm_lv;
+          y = (b * a.n_kv_heads + h) * a.local_len + tr.tt * kTile;
+        }
+        uint8_t* kdst = ring + stage * C::kStageBytes;
+        uint8_t* vdst = kdst + C::kTileBytes;
+        mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+#pragma unroll
+        for (int bx = 0; bx < C::kBoxes; ++bx) {
+          tma_load_2d(kdst + bx * C::kBoxBytes, mk, bx * 64, y, &full[stage], pol);
+          tma_load_2d(vdst + bx * C::kBoxBytes, mv, bx * 64, y, &full[stage], pol);
+        }
+        ++issued;
+      }
+      // No copy may still be landing when the CTA ends: wait for the last fill
+      // of every slot (consumers normally have already).
+      for (int n = max(0, issued - kStages); n < issued; ++n) {
+        int stage, use;
+        slot_of(n, stage, use);
+        mbar_wait_bounded(&full[stage], use & 1, nullptr);
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers
+  const int g = lane >> 2, c = lane & 3;
+  // Query fragments (B operand of S^T = K Q^T): row 8*nt + g, dims
+  // 16*ks + 2c + {0,1} and 16*ks + 8 + 2c + {0,1}; Global RoPE at k_off + i.
+  uint32_t qf[D / 16][NT][2];
+  int lim[NT][2];  // causal limit (local index) of this thread's two columns per n-tile
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int r = nt * 8 + 2 * c + e;
+      lim[nt][e] = (r < rows) ? i_first + r / G : i_max;
+    }
+    const int r = nt * 8 + g;
+    if (r < rows) {
+      const int t = blk * a.route_block + r / G;
+      const int hq = h * G + r % G;
+      const int i = a.local_len - a.q_tokens + t;
+      const uint16_t* qrow = a.q + (((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t) * D;
+      const float2* cs = a.gtab + (int64_t)i * (D / 2);
+#pragma unroll
+      for (int ks = 0; ks < D / 32; ++ks) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float xo[2], yo[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int d0 = 16 * ks + 8 * hf + 2 * c + e;
+            const float x = __uint_as_float((uint32_t)qrow[d0] << 16);
+            const float y = __uint_as_float((uint32_t)qrow[d0 + D / 2] << 16);
+            const float2 t2 = __ldg(cs + d0);
+            xo[e] = x * t2.x - y * t2.y;
+            yo[e] = y * t2.x + x * t2.y;
+          }
+          qf[ks][nt][hf] = pack_bf16(xo[0], xo[1]);
+          qf[ks + D / 32][nt][hf] = pack_bf16(yo[0], yo[1]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) qf[ks][nt][0] = qf[ks][nt][1] = 0u;
+    }
+  }
+
+  float m_run[NT][2], l_run[NT][2];
+  float acc[D / 16][NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    m_run[nt][0] = m_run[nt][1] = -INFINITY;
+    l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+    for (int md = 0; md < D / 16; ++md)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[md][nt][e] = 0.f;
+  }
+
+  int hint = 0;
+  bool ok = true;
+  for (int n = warp; n < ntiles && ok; n += kWarps) {
+    int stage, use;
+    slot_of(n, stage, use);
+    if (!mbar_wait_bounded(&full[stage], use & 1, a.err)) { ok = false; break; }
+    const TileRef tr = locate(tile_start, k, t0 + n, hint);
+    hint = tr.di;
+    uint8_t* kt = ring + stage * C::kStageBytes;
+    uint8_t* vt = kt + C::kTileBytes;
+    const bool local = tr.di >= k;
+    const int key0 = tr.tt * kTile;
+    const int nvalid = local ? 0 : min(kTile, doc_len_s[tr.di] - key0);
+
+    if (local) {
+      // Global RoPE of the local keys, in shared memory: pair (i, i + D/2)
+      // lives in the same swizzled slot of chunk i/8 and chunk (i + D/2)/8.
+      constexpr int kPairChunks = D / 16;  // 16-byte chunks per half row
+      for (int unit = lane; unit < kTile * kPairChunks; unit += 32) {
+        const int r = unit / kPairChunks, ch = unit % kPairChunks;
+        const int u = key0 + r;
+        if (u >= a.local_len) continue;
+        uint8_t* px;
+        uint8_t* py;
+        if constexpr (D == 128) {
+          px = kt + swz128(r, ch);
+          py = kt + C::kBoxBytes + swz128(r, ch);
+        } else {
+          px = kt + swz128(r, ch);
+          py = kt + swz128(r, ch + 4);
+        }
+        uint4 xv = *reinterpret_cast<uint4*>(px), yv = *reinterpret_cast<uint4*>(py);
+        uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w}, ys[4] = {yv.x, yv.y, yv.z, yv.w};
+        const float4* cs = reinterpret_cast<const float4*>(a.gtab + (int64_t)u * (D / 2) + ch * 8);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float4 t4 = __ldg(cs + j);
+          const float x0 = bf16_lo(xs[j]), x1 = bf16_hi(xs[j]);
+          const float y0 = bf16_lo(ys[j]), y1 = bf16_hi(ys[j]);
+          xs[j] = pack_bf16(x0 * t4.x - y0 * t4.y, x1 * t4.z - y1 * t4.w);
+          ys[j] = pack_bf16(y0 * t4.x + x0 * t4.y, y1 * t4.z + x1 * t4.w);
+        }
+        *reinterpret_cast<uint4*>(px) = make_uint4(xs[0], xs[1], xs[2], xs[3]);
+        *reinterpret_cast<uint4*>(py) = make_uint4(ys[0], ys[1], ys[2], ys[3]);
+      }
+      __syncwarp();
+    }
+
+    // ---- S^T = K Q^T : 4 m-tiles of 16 keys x NT n-tiles of 8 rows
+    float s[kMT][NT][4];
+    const uint32_t kbase = smem_addr(kt);
+#pragma unroll
+    for (int mt = 0; mt < kMT; ++mt) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[mt][nt][e] = 0.f;
+      const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const int col = ks * 16 + (lane >> 4) * 8;
+        const uint32_t addr = kbase + (col >> 6) * C::kBoxBytes + swz128(row, (col & 63) >> 3);
+        uint32_t af[4];
+        ldmatrix_x4(af, addr);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[mt][nt], af, qf[ks][nt][0], qf[ks][nt][1]);
+      }
+    }
+
+    // ---- mask, scale, online softmax (per column = query row)
+    float alpha[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int kk = mt * 16 + g + hf * 8;
+            const bool vis = local ? (key0 + kk <= lim[nt][e]) : (kk < nvalid);
+            float v = s[mt][nt][hf * 2 + e] * a.scale_log2;
+            v = vis ? v : -INFINITY;
+            s[mt][nt][hf * 2 + e] = v;
+            mx[e] = fmaxf(mx[e], v);
+          }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 4));
+        mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 8));
+        mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 16));
+        const float m_new = fmaxf(m_run[nt][e], mx[e]);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        alpha[nt][e] = exp2f(m_run[nt][e] - m_use);
+        m_run[nt][e] = m_new;
+        float sum = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const float pv = exp2f(s[mt][nt][hf * 2 + e] - m_use);
+            s[mt][nt][hf * 2 + e] = pv;
+            sum += pv;
+          }
+        l_run[nt][e] = l_run[nt][e] * alpha[nt][e] + sum;
+      }
+#pragma unroll
+      for (int md = 0; md < D / 16; ++md) {
+        acc[md][nt][0] *= alpha[nt][0];
+        acc[md][nt][1] *= alpha[nt][1];
+        acc[md][nt][2] *= alpha[nt][0];
+        acc[md][nt][3] *= alpha[nt][1];
+      }
+    }
+
+    // ---- P^T fragments: transpose each 8x8 (keys x rows) block with movmatrix
+    uint32_t pb[kMT][NT][2];
+#pragma unroll
+    for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        pb[mt][nt][0] = movmatrix_trans(pack_bf16(s[mt][nt][0], s[mt][nt][1]));
+        pb[mt][nt][1] = movmatrix_trans(pack_bf16(s[mt][nt][2], s[mt][nt][3]));
+      }
+
+    // ---- O^T += V^T P^T
+    const uint32_t vbase = smem_addr(vt);
+#pragma unroll
+    for (int mt = 0; mt < kMT; ++mt) {
+      const int key = mt * 16 + (lane & 7) + (lane >> 4) * 8;
+#pragma unroll
+      for (int md = 0; md < D / 16; ++md) {
+        const int dim = md * 16 + ((lane >> 3) & 1) * 8;
+        const uint32_t addr = vbase + (dim >> 6) * C::kBoxBytes + swz128(key, (dim & 63) >> 3);
+        uint32_t af[4];
+        ldmatrix_x4_trans(af, addr);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(acc[md][nt], af, pb[mt][nt][0], pb[mt][nt][1]);
+      }
+    }
+
+    if (local) fence_proxy_async();  // generic writes above precede the next TMA into this stage
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+  }
+
+  // ------------------------------------------------------------ CTA merge
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float v = l_run[nt][e];
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 16);
+      l_run[nt][e] = v;
+    }
+  named_barrier_sync(1, kWarps * 32);  // every consumer is done reading the ring
+  constexpr int R = NT * 8;
+  float* sc_o = reinterpret_cast<float*>(ring);            // [kWarps][R][D]
+  float* sc_m = sc_o + kWarps * R * D;                       // [kWarps][R]
+  float* sc_l = sc_m + kWarps * R;                           // [kWarps][R]
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int r = nt * 8 + 2 * c + e;
+#pragma unroll
+      for (int md = 0; md < D / 16; ++md) {
+        sc_o[(warp * R + r) * D + md * 16 + g] = acc[md][nt][e];
+        sc_o[(warp * R + r) * D + md * 16 + g + 8] = acc[md][nt][e + 2];
+      }
+      if (g == 0) {
+        sc_m[warp * R + r] = m_run[nt][e];
+        sc_l[warp * R + r] = l_run[nt][e];
+      }
+    }
+  named_barrier_sync(1, kWarps * 32);
+  const int64_t slot = (int64_t)p * a.n_splits + split;
+  for (int idx = tid; idx < rows * D; idx += kWarps * 32) {
+    const int r = idx / D, dim = idx % D;
+    float mstar = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) mstar = fmaxf(mstar, sc_m[w * R + r]);
+    float o = 0.f, l = 0.f;
+    if (mstar != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float f = exp2f(sc_m[w * R + r] - mstar);
+        o += f * sc_o[(w * R + r) * D + dim];
+        l += f * sc_l[w * R + r];
+      }
+    }
+    a.part_o[(slot * rows + r) * D + dim] = o;
+    if (dim == 0) {
+      a.part_ml[(slot * rows + r) * 2 + 0] = mstar;
+      a.part_ml[(slot * rows + r) * 2 + 1] = l;
+    }
+  }
+}
+
+// One warp per (problem, row): log-sum-exp merge of the splits.
+__global__ void attend_merge_kernel(MergeArgs a) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = a.n_q_heads / a.n_kv_heads;
+  const int rows = G * a.route_block;
+  const int nblk = a.q_tokens / a.route_block;
+  const int P = a.batch * nblk * a.n_kv_heads;
+  if (warp >= P * rows) return;
+  const int p = warp / rows, r = warp % rows;
+  const int h = p % a.n_kv_heads;
+  const int blk = (p / a.n_kv_heads) % nblk;
+  const int b = p / (a.n_kv_heads * nblk);
+  const int t = blk * a.route_block + r / G;
+  const int hq = h * G + r % G;
+  const int D = a.head_dim;
+  float M = -INFINITY;
+  for (int s = 0; s < a.n_splits; ++s)
+    M = fmaxf(M, a.part_ml[(((int64_t)p * a.n_splits + s) * rows + r) * 2]);
+  float L = 0.f;
+  float o[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < a.n_splits; ++s) {
+    const int64_t sl = ((int64_t)p * a.n_splits + s) * rows + r;
+    const float m = a.part_ml[sl * 2];
+    if (m == -INFINITY) continue;
+    const float f = exp2f(m - M);
+    L += f * a.part_ml[sl * 2 + 1];
+    for (int j = 0; j < D / 32; ++j) o[j] += f * a.part_o[sl * D + lane + 32 * j];
+  }
+  const float inv = (L > 0.f) ? 1.0f / L : 0.f;
+  float* dst = a.out + (((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t) * D;
+  for (int j = 0; j < D / 32; ++j) dst[lane + 32 * j] = o[j] * inv;
+}
+
+template <int D, int NT>
+cudaError_t launch_decode_t(const AttendArgs& a, const AttendMaps& m, cudaStream_t s) {
+  auto kern = attend_decode_kernel<D, NT>;
+  const size_t smem = attend_smem_bytes(D);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int nblk = a.q_tokens / a.route_block;
+  dim3 grid(a.n_splits, a.batch * nblk * a.n_kv_heads);
+  kern<<<grid, (kWarps + 1) * 32, smem, s>>>(m.bank_k, m.bank_v, m.loc_k, m.loc_v, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int attend_rows_per_problem(int group, int route_block) { return group * route_block; }
+int attend_tile_rows() { return kTile; }
+
+size_t attend_smem_bytes(int head_dim) {
+  const size_t ring = (size_t)kStages * 2 * kTile * head_dim * 2;
+  const size_t scratch = (size_t)kWarps * kRowsMax * (head_dim + 2) * 4;
+  const size_t body = ring > scratch ? ring : scratch;
+  return 1024 + body + 2 * kStages * 8 + (kMaxTopK + 2) * 4 + kMaxTopK * 4 + kMaxTopK * 8;
+}
+
+cudaError_t launch_attend_decode(const AttendArgs& a, const AttendMaps& m, int head_dim, cudaStream_t s) {
+  const int rows = (a.n_q_heads / a.n_kv_heads) * a.route_block;
+  if (head_dim == 128) {
+    if (rows <= 8) return launch_decode_t<128, 1>(a, m, s);
+    return launch_decode_t<128, 2>(a, m, s);
+  }
+  if (rows <= 8) return launch_decode_t<64, 1>(a, m, s);
+  return launch_decode_t<64, 2>(a, m, s);
+}
+
+cudaError_t launch_attend_merge(const MergeArgs& a, cudaStream_t s) {
+  const int nblk = a.q_tokens / a.route_block;
+  const int rows = (a.n_q_heads / a.n_kv_heads) * a.route_block;
+  const int64_t warps = (int64_t)a.batch * nblk * a.n_kv_heads * rows;
+  const int blocks = (int)((warps + 3) / 4);
+  attend_merge_kernel<<<blocks, 128, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

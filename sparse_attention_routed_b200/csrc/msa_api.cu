@@ -1,0 +1,529 @@
+// Host side of libmsa: argument validation, the bank handle, RoPE tables,
+// TMA descriptors, workspace, and the C entry points declared in msa.h.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "../../include/msa.h"
+#include "common.cuh"
+#include "internal.h"
+
+using namespace msa;
+
+namespace {
+
+constexpr int kChunk = 256;  // routing chunk ("MSA架构…" §2.1 item 2: 256-token chunks)
+constexpr int kMaxTopK = 64;
+constexpr int kMaxRows = 16;
+
+msa_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return MSA_OK;
+  if (e == cudaErrorMemoryAllocation) return MSA_ERR_OOM;
+  return MSA_ERR_CUDA;
+}
+
+#define MSA_CUDA(call)                                \
+  do {                                                \
+    cudaError_t e_ = (call);                          \
+    if (e_ != cudaSuccess) return from_cuda(e_);      \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [rows][d], boxes of box_rows rows x 64 elements (128 bytes), 128-byte swizzle.
+msa_status make_map(CUtensorMap* map, const void* base, int64_t rows, int d, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return MSA_ERR_CUDA;
+  if (!aligned16(base) || rows <= 0 || rows >= (int64_t(1) << 31)) return MSA_ERR_INVALID_ARG;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
+}
+
+// (cos, sin) of pos * base^(-2i/d) for positions p0 .. p0+n-1, angles in fp64
+// reduced mod 2*pi before the fp32 rounding.
+std::vector<float2> rope_table(int64_t p0, int64_t n, int d, double base) {
+  std::vector<float2> t((size_t)n * (d / 2));
+  const double two_pi = 6.283185307179586476925286766559;
+  std::vector<double> inv(d / 2);
+  for (int i = 0; i < d / 2; ++i) inv[i] = std::pow(base, -2.0 * i / d);
+  for (int64_t p = 0; p < n; ++p)
+    for (int i = 0; i < d / 2; ++i) {
+      const double ang = std::fmod((double)(p0 + p) * inv[i], two_pi);
+      t[(size_t)p * (d / 2) + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+    }
+  return t;
+}
+
+template <typename T>
+msa_status upload(T** dst, const std::vector<T>& src) {
+  *dst = nullptr;
+  if (src.empty()) return MSA_OK;
+  MSA_CUDA(cudaMalloc(dst, src.size() * sizeof(T)));
+  MSA_CUDA(cudaMemcpy(*dst, src.data(), src.size() * sizeof(T), cudaMemcpyHostToDevice));
+  return MSA_OK;
+}
+
+}  // namespace
+
+struct msa_bank {
+  // configuration
+  int n_docs = 0, hkv = 0, d = 0, dr = 0, kv_loc = 0;
+  double base = 10000.0;
+  const void* k = nullptr;
+  const void* v = nullptr;
+  int64_t kv_rows = 0, ntok = 0, nch = 0, max_len = 0;
+  std::vector<int64_t> doc_lens, doc_off, doc_rows;
+  std::vector<int32_t> chunk_off;
+  int sms = 148;
+  // device, owned
+  int64_t* d_doc_row = nullptr;
+  int32_t* d_doc_len = nullptr;
+  int32_t* d_chunk_off = nullptr;
+  int64_t* d_chunk_tok = nullptr;  // relative to the bank's first token
+  int32_t* d_chunk_len = nullptr;
+  int32_t* d_chunk_pos = nullptr;
+  float2* d_ptab = nullptr;
+  float* d_kr = nullptr;
+  float* d_kr_inv = nullptr;
+  int* d_err = nullptr;
+  // Global RoPE table cache
+  float2* d_gtab = nullptr;
+  int64_t gtab_koff = -1;
+  int gtab_lc = 0;
+  size_t gtab_cap = 0;
+  // workspace
+  uint8_t* ws = nullptr;
+  size_t ws_cap = 0;
+  // TMA descriptors of the bank K/V (device tier)
+  CUtensorMap map_k{}, map_v{};
+  std::vector<void*> owned;
+};
+
+namespace {
+
+void free_bank(msa_bank* b) {
+  if (!b) return;
+  cudaDeviceSynchronize();
+  void* ptrs[] = {b->d_doc_row, b->d_doc_len, b->d_chunk_off, b->d_chunk_tok, b->d_chunk_len,
+                  b->d_chunk_pos, b->d_ptab, b->d_kr, b->d_kr_inv, b->d_err, b->d_gtab, b->ws};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  delete b;
+}
+
+struct StepShape {
+  int B, Hq, Tq, Lc, Bq, G, nblk, rows, P, k;
+};
+
+msa_status check_query(const msa_bank* bank, const msa_query* q, int top_k, StepShape* s, bool need_attn) {
+  if (!bank || !q) return MSA_ERR_INVALID_ARG;
+  if (q->batch < 1 || q->n_q_heads < 1 || q->q_tokens < 1 || q->local_len < 1 || q->route_block < 1)
+    return MSA_ERR_INVALID_ARG;
+  if (q->n_q_heads % bank->hkv) return MSA_ERR_INVALID_ARG;
+  if (q->q_tokens > q->local_len || q->q_tokens % q->route_block) return MSA_ERR_INVALID_ARG;
+  if (top_k < 1 || top_k > bank->n_docs) return MSA_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK) return MSA_ERR_UNSUPPORTED;
+  if (!q->qr || !aligned16(q->qr)) return MSA_ERR_INVALID_ARG;
+  s->B = q->batch;
+  s->Hq = q->n_q_heads;
+  s->Tq = q->q_tokens;
+  s->Lc = q->local_len;
+  s->Bq = q->route_block;
+  s->G = q->n_q_heads / bank->hkv;
+  s->nblk = q->q_tokens / q->route_block;
+  s->rows = s->G * s->Bq;
+  s->P = s->B * s->nblk * bank->hkv;
+  s->k = top_k;
+  if (need_attn) {
+    if (!q->q || !q->local_k || !q->local_v) return MSA_ERR_INVALID_ARG;
+    if (!aligned16(q->q) || !aligned16(q->local_k) || !aligned16(q->local_v)) return MSA_ERR_INVALID_ARG;
+    if (s->rows > kMaxRows) return MSA_ERR_UNSUPPORTED;
+    if ((int64_t)s->B * bank->hkv * s->Lc >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+    if (bank->kv_loc != MSA_KV_DEVICE) return MSA_ERR_UNSUPPORTED;
+  }
+  if ((int64_t)s->B * s->nblk > 65535 || s->P > 65535) return MSA_ERR_UNSUPPORTED;
+  return MSA_OK;
+}
+
+int choose_splits(const msa_bank* bank, const StepShape& s) {
+  const double avg_len = (double)bank->ntok / bank->n_docs;
+  const int64_t tiles = (int64_t)s.k * (int64_t)std::ceil(avg_len / 64.0) + (s.Lc + 63) / 64;
+  const int64_t target = (int64_t)bank->sms * 2 * 8;  // ~8 waves of 2 resident CTAs per SM
+  int64_t S = (target + s.P - 1) / s.P;
+  S = std::min<int64_t>(S, std::max<int64_t>(1, tiles / 8));
+  return (int)std::max<int64_t>(1, S);
+}
+
+struct Workspace {
+  float* q_r;
+  float* q_r_inv;
+  float* scores;
+  int32_t* idx;
+  float* part_o;
+  float* part_ml;
+  size_t bytes;
+};
+
+size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
+
+Workspace layout(const msa_bank* bank, const StepShape& s, int splits, uint8_t* base) {
+  Workspace w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* p = base ? base + off : nullptr;
+    off += align_up(bytes);
+    return p;
+  };
+  const size_t rows_route = (size_t)s.B * s.nblk;
+  w.q_r = (float*)take(rows_route * bank->hkv * bank->dr * 4);
+  w.q_r_inv = (float*)take(rows_route * bank->hkv * 4);
+  w.scores = (float*)take(rows_route * bank->hkv * bank->n_docs * 4);
+  w.idx = (int32_t*)take((size_t)s.P * s.k * 4);
+  w.part_o = (float*)take((size_t)s.P * splits * s.rows * bank->d * 4);
+  w.part_ml = (float*)take((size_t)s.P * splits * s.rows * 2 * 4);
+  w.bytes = off;
+  return w;
+}
+
+bool capturing(cudaStream_t s) {
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  return cudaStreamIsCapturing(s, &st) == cudaSuccess && st != cudaStreamCaptureStatusNone;
+}
+
+// Grows the workspace; refuses while `s` is being captured (call msa_reserve first).
+msa_status ensure_workspace(msa_bank* bank, size_t bytes, cudaStream_t s) {
+  if (bytes <= bank->ws_cap) return MSA_OK;
+  if (capturing(s)) return MSA_ERR_INVALID_ARG;
+  if (bank->ws) {
+    MSA_CUDA(cudaDeviceSynchronize());
+    cudaFree(bank->ws);
+    bank->ws = nullptr;
+    bank->ws_cap = 0;
+  }
+  MSA_CUDA(cudaMalloc(&bank->ws, bytes));
+  bank->ws_cap = bytes;
+  return MSA_OK;
+}
+
+msa_status ensure_gtab(msa_bank* bank, int64_t koff, int lc, cudaStream_t s) {
+  if (bank->gtab_koff == koff && bank->gtab_lc >= lc) return MSA_OK;
+  if (capturing(s)) return MSA_ERR_INVALID_ARG;
+  std::vector<float2> t = rope_table(koff, lc, bank->d, bank->base);
+  const size_t bytes = t.size() * sizeof(float2);
+  if (bytes > bank->gtab_cap) {
+    MSA_CUDA(cudaDeviceSynchronize());
+    if (bank->d_gtab) cudaFree(bank->d_gtab);
+    bank->d_gtab = nullptr;
+    bank->gtab_cap = 0;
+    MSA_CUDA(cudaMalloc(&bank->d_gtab, bytes));
+    bank->gtab_cap = bytes;
+  } else {
+    MSA_CUDA(cudaDeviceSynchronize());  // an in-flight step may still read the old table
+  }
+  MSA_CUDA(cudaMemcpy(bank->d_gtab, t.data(), bytes, cudaMemcpyHostToDevice));
+  bank->gtab_koff = koff;
+  bank->gtab_lc = lc;
+  return MSA_OK;
+}
+
+msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, const Workspace& w,
+                      float* doc_scores, int32_t* idx, float* top_scores, cudaStream_t st) {
+  QrArgs qa{(const uint16_t*)q->qr, w.q_r, w.q_r_inv, s.B, bank->hkv, s.Tq, s.Bq, bank->dr};
+  MSA_CUDA(launch_qr_prep(qa, st));
+  RouteArgs ra{};
+  ra.k_r = bank->d_kr;
+  ra.k_r_inv = bank->d_kr_inv;
+  ra.chunk_off = bank->d_chunk_off;
+  ra.q_r = w.q_r;
+  ra.q_r_inv = w.q_r_inv;
+  ra.doc_scores = doc_scores ? doc_scores : w.scores;
+  ra.nch = bank->nch;
+  ra.rows = s.B * s.nblk;
+  ra.n_kv_heads = bank->hkv;
+  ra.n_docs = bank->n_docs;
+  ra.route_dim = bank->dr;
+  MSA_CUDA(launch_route(ra, st));
+  TopkArgs ta{ra.doc_scores, idx, top_scores, s.P, bank->n_docs, s.k};
+  MSA_CUDA(launch_topk(ta, st));
+  return MSA_OK;
+}
+
+msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, int splits, const Workspace& w,
+                       const int32_t* idx, float* out, cudaStream_t st) {
+  AttendMaps maps;
+  maps.bank_k = bank->map_k;
+  maps.bank_v = bank->map_v;
+  msa_status rc = make_map(&maps.loc_k, q->local_k, (int64_t)s.B * bank->hkv * s.Lc, bank->d, attend_tile_rows());
+  if (rc != MSA_OK) return rc;
+  rc = make_map(&maps.loc_v, q->local_v, (int64_t)s.B * bank->hkv * s.Lc, bank->d, attend_tile_rows());
+  if (rc != MSA_OK) return rc;
+  AttendArgs a{};
+  a.q = (const uint16_t*)q->q;
+  a.sel = idx;
+  a.doc_row = bank->d_doc_row;
+  a.doc_len = bank->d_doc_len;
+  a.gtab = bank->d_gtab;
+  a.part_o = w.part_o;
+  a.part_ml = w.part_ml;
+  a.err = bank->d_err;
+  a.kv_rows = bank->kv_rows;
+  a.batch = s.B;
+  a.n_q_heads = s.Hq;
+  a.n_kv_heads = bank->hkv;
+  a.q_tokens = s.Tq;
+  a.local_len = s.Lc;
+  a.route_block = s.Bq;
+  a.top_k = s.k;
+  a.n_docs = bank->n_docs;
+  a.n_splits = splits;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)bank->d));
+  MSA_CUDA(launch_attend_decode(a, maps, bank->d, st));
+  MergeArgs m{w.part_o, w.part_ml, out, s.B, s.Hq, bank->hkv, s.Tq, s.Bq, splits, bank->d};
+  MSA_CUDA(launch_attend_merge(m, st));
+  return MSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* msa_status_string(msa_status s) {
+  switch (s) {
+    case MSA_OK: return "ok";
+    case MSA_ERR_INVALID_ARG: return "invalid argument";
+    case MSA_ERR_UNSUPPORTED: return "unsupported shape or configuration";
+    case MSA_ERR_OOM: return "out of memory";
+    case MSA_ERR_CUDA: return "CUDA error";
+    case MSA_ERR_TIMEOUT: return "device-side wait timed out";
+    case MSA_ERR_HOST_TIER: return "host K/V tier error";
+  }
+  return "unknown status";
+}
+
+msa_status msa_bank_create(const msa_bank_config* cfg, msa_bank** out) {
+  if (!out) return MSA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg || cfg->n_docs < 1 || cfg->n_kv_heads < 1 || !cfg->doc_lens) return MSA_ERR_INVALID_ARG;
+  if ((cfg->head_dim != 64 && cfg->head_dim != 128) || cfg->route_dim != cfg->head_dim)
+    return MSA_ERR_INVALID_ARG;
+  if (!(cfg->rope_base > 1.0f)) return MSA_ERR_INVALID_ARG;
+  if (cfg->kv_location != MSA_KV_DEVICE && cfg->kv_location != MSA_KV_PINNED_HOST) return MSA_ERR_INVALID_ARG;
+  if (!cfg->k || !cfg->v || !aligned16(cfg->k) || !aligned16(cfg->v)) return MSA_ERR_INVALID_ARG;
+
+  msa_bank* b = new (std::nothrow) msa_bank();
+  if (!b) return MSA_ERR_OOM;
+  b->n_docs = cfg->n_docs;
+  b->hkv = cfg->n_kv_heads;
+  b->d = cfg->head_dim;
+  b->dr = cfg->route_dim;
+  b->base = cfg->rope_base;
+  b->kv_loc = cfg->kv_location;
+  b->k = cfg->k;
+  b->v = cfg->v;
+  b->doc_lens.assign(cfg->doc_lens, cfg->doc_lens + cfg->n_docs);
+  b->doc_off.assign(b->n_docs + 1, 0);
+  b->chunk_off.assign(b->n_docs + 1, 0);
+  for (int j = 0; j < b->n_docs; ++j) {
+    const int64_t L = b->doc_lens[j];
+    if (L < 1 || L >= (int64_t(1) << 30)) {
+      delete b;
+      return MSA_ERR_INVALID_ARG;
+    }
+    b->doc_off[j + 1] = b->doc_off[j] + L;
+    const int64_t nc = b->chunk_off[j] + (L + kChunk - 1) / kChunk;
+    if (nc >= (int64_t(1) << 31)) {
+      delete b;
+      return MSA_ERR_UNSUPPORTED;
+    }
+    b->chunk_off[j + 1] = (int32_t)nc;
+    b->max_len = std::max(b->max_len, L);
+  }
+  b->ntok = b->doc_off[b->n_docs];
+  b->nch = b->chunk_off[b->n_docs];
+  b->kv_rows = cfg->kv_rows > 0 ? cfg->kv_rows : b->ntok;
+  b->doc_rows.resize(b->n_docs);
+  for (int j = 0; j < b->n_docs; ++j) {
+    b->doc_rows[j] = cfg->doc_rows ? cfg->doc_rows[j] : b->doc_off[j];
+    if (b->doc_rows[j] < 0 || b->doc_rows[j] + b->doc_lens[j] > b->kv_rows) {
+      delete b;
+      return MSA_ERR_INVALID_ARG;
+    }
+  }
+  if ((int64_t)b->hkv * b->kv_rows >= (int64_t(1) << 31)) {
+    delete b;
+    return MSA_ERR_UNSUPPORTED;
+  }
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&b->sms, cudaDevAttrMultiProcessorCount, dev);
+
+  // chunk table
+  std::vector<int64_t> ctok(b->nch);
+  std::vector<int32_t> clen(b->nch), cpos(b->nch), dlen(b->n_docs);
+  for (int j = 0; j < b->n_docs; ++j) {
+    dlen[j] = (int32_t)b->doc_lens[j];
+    for (int c = b->chunk_off[j]; c < b->chunk_off[j + 1]; ++c) {
+      const int64_t s = (int64_t)(c - b->chunk_off[j]) * kChunk;
+      ctok[c] = b->doc_off[j] + s;
+      clen[c] = (int32_t)std::min<int64_t>(kChunk, b->doc_lens[j] - s);
+      cpos[c] = (int32_t)s;
+    }
+  }
+  msa_status rc = MSA_OK;
+  auto fail = [&](msa_status r) {
+    free_bank(b);
+    return r;
+  };
+  if ((rc = upload(&b->d_doc_row, b->doc_rows)) != MSA_OK) return fail(rc);
+  if ((rc = upload(&b->d_doc_len, dlen)) != MSA_OK) return fail(rc);
+  if ((rc = upload(&b->d_chunk_off, b->chunk_off)) != MSA_OK) return fail(rc);
+  if ((rc = upload(&b->d_chunk_tok, ctok)) != MSA_OK) return fail(rc);
+  if ((rc = upload(&b->d_chunk_len, clen)) != MSA_OK) return fail(rc);
+  if ((rc = upload(&b->d_chunk_pos, cpos)) != MSA_OK) return fail(rc);
+  if ((rc = upload(&b->d_ptab, rope_table(0, b->max_len, b->d, b->base))) != MSA_OK) return fail(rc);
+  if (cudaMalloc(&b->d_kr, (size_t)b->hkv * b->nch * b->dr * 4) != cudaSuccess) return fail(MSA_ERR_OOM);
+  if (cudaMalloc(&b->d_kr_inv, (size_t)b->hkv * b->nch * 4) != cudaSuccess) return fail(MSA_ERR_OOM);
+  if (cudaMalloc(&b->d_err, sizeof(int)) != cudaSuccess) return fail(MSA_ERR_OOM);
+  if (cudaMemset(b->d_err, 0, sizeof(int)) != cudaSuccess) return fail(MSA_ERR_CUDA);
+  if (b->kv_loc == MSA_KV_DEVICE) {
+    if ((rc = make_map(&b->map_k, b->k, (int64_t)b->hkv * b->kv_rows, b->d, attend_tile_rows())) != MSA_OK) return fail(rc);
+    if ((rc = make_map(&b->map_v, b->v, (int64_t)b->hkv * b->kv_rows, b->d, attend_tile_rows())) != MSA_OK) return fail(rc);
+  }
+  *out = b;
+  return MSA_OK;
+}
+
+msa_status msa_bank_destroy(msa_bank* bank) {
+  free_bank(bank);
+  return MSA_OK;
+}
+
+// Strides are in rows; a row is d * 2 >= 128 bytes, so every head of an aligned slice stays aligned.
+msa_status msa_build_bank(msa_bank* bank, int32_t doc_begin, int32_t doc_end, const void* r_slice,
+                          int64_t r_head_stride, void* k_slice, int64_t k_head_stride, void* stream) {
+  if (!bank || !r_slice) return MSA_ERR_INVALID_ARG;
+  if (doc_begin < 0 || doc_end > bank->n_docs || doc_begin >= doc_end) return MSA_ERR_INVALID_ARG;
+  const int64_t T = bank->doc_off[doc_end] - bank->doc_off[doc_begin];
+  if (r_head_stride < T || !aligned16(r_slice)) return MSA_ERR_INVALID_ARG;
+  if (k_slice && (k_head_stride < T || !aligned16(k_slice))) return MSA_ERR_INVALID_ARG;
+  const int64_t c0 = bank->chunk_off[doc_begin], c1 = bank->chunk_off[doc_end];
+  if (c1 - c0 >= (int64_t(1) << 31) / bank->hkv) return MSA_ERR_UNSUPPORTED;
+  BankBuildArgs a{};
+  a.r = (const uint16_t*)r_slice;
+  a.r_head_stride = r_head_stride * bank->dr;
+  a.k = (uint16_t*)k_slice;
+  a.tok_base = bank->doc_off[doc_begin];
+  a.k_head_stride = k_head_stride * bank->d;
+  a.chunk_tok = bank->d_chunk_tok + c0;
+  a.chunk_len = bank->d_chunk_len + c0;
+  a.chunk_pos = bank->d_chunk_pos + c0;
+  a.rope_tab = bank->d_ptab;
+  a.k_r = bank->d_kr;
+  a.k_r_inv = bank->d_kr_inv;
+  a.nch_total = bank->nch;
+  a.chunk0 = c0;
+  a.n_chunks = (int32_t)(c1 - c0);
+  a.n_kv_heads = bank->hkv;
+  a.head_dim = bank->d;
+  return from_cuda(launch_bank_build(a, (cudaStream_t)stream));
+}
+
+msa_status msa_bank_info(const msa_bank* bank, int64_t* n_tokens, int64_t* n_chunks, int64_t* max_doc_len,
+                         const float** k_r, const float** k_r_inv_norm) {
+  if (!bank) return MSA_ERR_INVALID_ARG;
+  if (n_tokens) *n_tokens = bank->ntok;
+  if (n_chunks) *n_chunks = bank->nch;
+  if (max_doc_len) *max_doc_len = bank->max_len;
+  if (k_r) *k_r = bank->d_kr;
+  if (k_r_inv_norm) *k_r_inv_norm = bank->d_kr_inv;
+  return MSA_OK;
+}
+
+msa_status msa_reserve(msa_bank* bank, const msa_query* shape, int32_t top_k) {
+  StepShape s;
+  const bool attn = shape && shape->q && shape->local_k && shape->local_v;
+  msa_status rc = check_query(bank, shape, top_k, &s, attn);
+  if (rc != MSA_OK) return rc;
+  const int splits = choose_splits(bank, s);
+  if ((rc = ensure_workspace(bank, layout(bank, s, splits, nullptr).bytes, nullptr)) != MSA_OK) return rc;
+  return ensure_gtab(bank, (int64_t)top_k * bank->max_len, s.Lc, nullptr);
+}
+
+msa_status msa_route(msa_bank* bank, const msa_query* q, int32_t top_k, float* doc_scores, int32_t* topk_idx,
+                     float* topk_scores, void* stream) {
+  StepShape s;
+  msa_status rc = check_query(bank, q, top_k, &s, false);
+  if (rc != MSA_OK) return rc;
+  if (!topk_idx) return MSA_ERR_INVALID_ARG;
+  const int splits = 1;
+  Workspace w = layout(bank, s, splits, nullptr);
+  if ((rc = ensure_workspace(bank, w.bytes, (cudaStream_t)stream)) != MSA_OK) return rc;
+  w = layout(bank, s, splits, bank->ws);
+  return route_impl(bank, q, s, w, doc_scores, topk_idx, topk_scores, (cudaStream_t)stream);
+}
+
+msa_status msa_attend(msa_bank* bank, const msa_query* q, int32_t top_k, const int32_t* topk_idx, float* out,
+                      void* stream) {
+  StepShape s;
+  msa_status rc = check_query(bank, q, top_k, &s, true);
+  if (rc != MSA_OK) return rc;
+  if (!topk_idx || !out) return MSA_ERR_INVALID_ARG;
+  const int splits = choose_splits(bank, s);
+  Workspace w = layout(bank, s, splits, nullptr);
+  if ((rc = ensure_workspace(bank, w.bytes, (cudaStream_t)stream)) != MSA_OK) return rc;
+  if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->max_len, s.Lc, (cudaStream_t)stream)) != MSA_OK) return rc;
+  w = layout(bank, s, splits, bank->ws);
+  return attend_impl(bank, q, s, splits, w, topk_idx, out, (cudaStream_t)stream);
+}
+
+msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_t* topk_idx, float* out,
+                       void* stream) {
+  StepShape s;
+  msa_status rc = check_query(bank, q, top_k, &s, true);
+  if (rc != MSA_OK) return rc;
+  if (!topk_idx || !out) return MSA_ERR_INVALID_ARG;
+  const int splits = choose_splits(bank, s);
+  Workspace w = layout(bank, s, splits, nullptr);
+  if ((rc = ensure_workspace(bank, w.bytes, (cudaStream_t)stream)) != MSA_OK) return rc;
+  if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->max_len, s.Lc, (cudaStream_t)stream)) != MSA_OK) return rc;
+  w = layout(bank, s, splits, bank->ws);
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((rc = route_impl(bank, q, s, w, nullptr, topk_idx, nullptr, st)) != MSA_OK) return rc;
+  return attend_impl(bank, q, s, splits, w, topk_idx, out, st);
+}
+
+msa_status msa_get_device_error(msa_bank* bank, void* stream) {
+  if (!bank) return MSA_ERR_INVALID_ARG;
+  MSA_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+  int v = 0;
+  MSA_CUDA(cudaMemcpy(&v, bank->d_err, sizeof(int), cudaMemcpyDeviceToHost));
+  MSA_CUDA(cudaMemset(bank->d_err, 0, sizeof(int)));
+  return (msa_status)v;
+}
+
+}  // extern "C"

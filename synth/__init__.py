@@ -52,9 +52,10 @@ def _mix64_int(z: int) -> int:
 
 def mix64(z: np.ndarray) -> np.ndarray:
     """SplitMix64 finaliser on a uint64 array (wrapping arithmetic)."""
-    z = np.asarray(z, dtype=np.uint64)
-    z = (z ^ (z >> np.uint64(30))) * np.uint64(0xBF58476D1CE4E5B9)
-    z = (z ^ (z >> np.uint64(27))) * np.uint64(0x94D049BB133111EB)
+    z = np.atleast_1d(np.asarray(z, dtype=np.uint64))
+    with np.errstate(over="ignore"):
+        z = (z ^ (z >> np.uint64(30))) * np.uint64(0xBF58476D1CE4E5B9)
+        z = (z ^ (z >> np.uint64(27))) * np.uint64(0x94D049BB133111EB)
     return z ^ (z >> np.uint64(31))
 
 
@@ -64,8 +65,11 @@ def stream_key(seed: int, tensor_id: int) -> int:
 
 def u64_at(key: int, idx) -> np.ndarray:
     """The idx-th (0-based) SplitMix64 output of the stream started at key."""
-    idx = np.asarray(idx, dtype=np.uint64)
-    return mix64(np.uint64(key) + (idx + np.uint64(1)) * np.uint64(GAMMA))
+    scalar = np.ndim(idx) == 0
+    idx = np.atleast_1d(np.asarray(idx, dtype=np.uint64))
+    with np.errstate(over="ignore"):
+        out = mix64(np.uint64(key) + (idx + np.uint64(1)) * np.uint64(GAMMA))
+    return out[0] if scalar else out
 
 
 def _round_f64_to_bf16(x: np.ndarray) -> np.ndarray:

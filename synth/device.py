@@ -1,0 +1,54 @@
+"""Device-resident synthetic inputs (torch allocates, libmsasynth.so fills).
+
+Same values as the numpy generator in synth/__init__.py, bit for bit.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import (NORMAL_TABLE_BITS, T_K, T_LK, T_LV, T_Q, T_QR, T_R, T_V, Workload, device_normal_bf16,
+               planted_qr_bits)
+
+_TABLES = {}
+
+
+def _table(device) -> torch.Tensor:
+    key = str(device)
+    if key not in _TABLES:
+        _TABLES[key] = torch.from_numpy(NORMAL_TABLE_BITS.view(np.int16).copy()).to(device)
+    return _TABLES[key]
+
+
+def fill_normal(t: torch.Tensor, seed: int, tensor_id: int, start: int = 0) -> torch.Tensor:
+    """Fill a contiguous bf16 CUDA tensor with elements [start, start + numel) of a stream."""
+    assert t.dtype == torch.bfloat16 and t.is_cuda and t.is_contiguous()
+    device_normal_bf16(t.data_ptr(), seed, tensor_id, start, t.numel(), _table(t.device).data_ptr(),
+                       torch.cuda.current_stream(t.device).cuda_stream)
+    return t
+
+
+def normal(shape, seed: int, tensor_id: int, device="cuda", start: int = 0) -> torch.Tensor:
+    return fill_normal(torch.empty(shape, dtype=torch.bfloat16, device=device), seed, tensor_id, start)
+
+
+def bank_tensors(w: Workload, device="cuda", with_r: bool = True):
+    """K, V, R of the bank as [Hkv, Ntok, d] bf16 (K without RoPE)."""
+    shape = (w.n_kv_heads, w.n_tokens, w.head_dim)
+    K = normal(shape, w.seed, T_K, device)
+    V = normal(shape, w.seed, T_V, device)
+    R = normal((w.n_kv_heads, w.n_tokens, w.route_dim), w.seed, T_R, device) if with_r else None
+    return K, V, R
+
+
+def query_tensors(w: Workload, device="cuda"):
+    """Q [B,Hq,Tq,d], Qr [B,Hkv,Tq,d_r], local K/V [B,Hkv,Lc,d], all bf16."""
+    Q = normal((w.batch, w.n_q_heads, w.q_tokens, w.head_dim), w.seed, T_Q, device)
+    if w.planted:
+        bits = planted_qr_bits(w)
+        Qr = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device).contiguous()
+    else:
+        Qr = normal((w.batch, w.n_kv_heads, w.q_tokens, w.route_dim), w.seed, T_QR, device)
+    LK = normal((w.batch, w.n_kv_heads, w.local_len, w.head_dim), w.seed, T_LK, device)
+    LV = normal((w.batch, w.n_kv_heads, w.local_len, w.head_dim), w.seed, T_LV, device)
+    return Q, Qr, LK, LV

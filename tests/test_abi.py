@@ -1,0 +1,75 @@
+"""The C-ABI library loads and exports every entry point include/msa.h declares.
+Host-side argument checks return before any CUDA call, so they run without a GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import sparse_attention_routed_b200 as msa
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "msa.h")
+
+
+def declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(msa_\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_declarations_are_exported():
+    names = declared()
+    assert len(names) >= 10
+    assert sorted(names) == sorted(msa.EXPORTED)
+    lib = ctypes.CDLL(msa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    for s in range(7):
+        assert msa.msa_status_string(s) and msa.msa_status_string(s) != "unknown status"
+    assert msa.msa_status_string(99) == "unknown status"
+
+
+def test_bank_create_rejects_bad_arguments():
+    lens = np.array([10, 20], dtype=np.int64)
+    fake = 0x10000  # never dereferenced: validation fails first
+    cases = [
+        dict(n_docs=0, n_kv_heads=1, head_dim=64),
+        dict(n_docs=2, n_kv_heads=0, head_dim=64),
+        dict(n_docs=2, n_kv_heads=1, head_dim=96),
+        dict(n_docs=2, n_kv_heads=1, head_dim=64, route_dim=128),
+        dict(n_docs=2, n_kv_heads=1, head_dim=64, rope_base=0.5),
+        dict(n_docs=2, n_kv_heads=1, head_dim=64, kv_location=7),
+        dict(n_docs=2, n_kv_heads=1, head_dim=64, k=0),
+        dict(n_docs=2, n_kv_heads=1, head_dim=64, k=fake + 2),   # misaligned
+    ]
+    for c in cases:
+        kw = dict(doc_lens=lens, k=fake, v=fake)
+        kw.update(c)
+        st, h = msa.msa_bank_create(kw.pop("n_docs"), kw.pop("n_kv_heads"), kw.pop("head_dim"), check=False, **kw)
+        assert st == msa.MSA_ERR_INVALID_ARG and not h, c
+    st, h = msa.msa_bank_create(2, 1, 64, np.array([10, 0]), fake, fake, check=False)
+    assert st == msa.MSA_ERR_INVALID_ARG and not h
+    st, h = msa.msa_bank_create(2, 1, 64, lens, fake, fake, kv_rows=25, check=False)   # rows too short
+    assert st == msa.MSA_ERR_INVALID_ARG and not h
+
+
+def test_null_handles_are_rejected():
+    q = msa.make_query(1, 4, 1, 8, 1, 0x10000, 0x10000, 0x10000, 0x10000)
+    assert msa.msa_route(None, q, 1, 0, 0x10000, 0, check=False) == msa.MSA_ERR_INVALID_ARG
+    assert msa.msa_attend(None, q, 1, 0x10000, 0x10000, check=False) == msa.MSA_ERR_INVALID_ARG
+    assert msa.msa_forward(None, q, 1, 0x10000, 0x10000, check=False) == msa.MSA_ERR_INVALID_ARG
+    assert msa.msa_build_bank(None, 0, 1, 0x10000, 8, 0, 0, check=False) == msa.MSA_ERR_INVALID_ARG
+    assert msa.msa_bank_destroy(None) == msa.MSA_OK
+
+
+def test_product_path_does_not_import_oracle():
+    pkg = os.path.dirname(msa.__file__)
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(root, f), errors="ignore").read()
+                assert "oracle" not in re.sub(r"#.*|//.*", "", text).lower().replace("oracle/", ""), f
