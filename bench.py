@@ -1,0 +1,369 @@
+#!/usr/bin/env python3
+"""Benchmark of the routed sparse-attention decode step (MSA) on B200.
+
+Workload: batched decode on a shared 4.19M-token memory bank -- batch 8, 32
+query heads / 8 KV heads, head_dim 128, 1024 documents x 4096 tokens, 4096-token
+local context, 1 query token, top_k = 16 documents per (sequence, KV head),
+bf16 storage, fp32 accumulation, seeded synthetic N(0,1) inputs.
+
+One step = msa_route + msa_attend through the C ABI (identical to msa_forward):
+q_r, cosine router over every chunk of K_r, top-k, split-KV attention, merge.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU: each rank runs an independent replica (the step does not shard);
+value = all ranks' queries / max-over-ranks device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "decode_4m"
+METRIC = "decode queries/s on 4M-tok bank; router+attn HBM GB/s as % of B200 peak"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "decode_512k"],
+                    help="decode_512k: the same step on a 128-document bank (profiling captures)")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------- CPU oracle
+def oracle_sample(seconds: float):
+    """Times the oracle as it stands on a bounded sample of the decode workload.
+
+    Sample: whole decode queries (one sequence each): the oracle's router over
+    every chunk of the 4.19M-token bank for all 8 KV heads (per-chunk cosine
+    loop, per-document max, top-k by full sort), then the oracle's attention for
+    all 32 query heads over the 16 selected documents plus the 4096 local tokens.
+    K_r is offline state (built once per bank), so a stand-in K_r of the right
+    shape is drawn from the generator (the oracle's cost does not depend on
+    its values); the selected documents' K/V and the local K/V are regenerated
+    exactly. Queries run until `seconds` of oracle time are spent (>= 1 query).
+    """
+    import synth
+    from oracle import msa_oracle as O
+
+    w = synth.WORKLOADS[WORKLOAD]
+    n, L, d, Hkv, G = w.n_docs, w.doc_len, w.head_dim, w.n_kv_heads, w.n_q_heads // w.n_kv_heads
+    nch_doc = L // 256
+    chunk_doc = np.repeat(np.arange(n), nch_doc)
+    kr = synth.normal_f32(99, 1, 0, Hkv * n * nch_doc * d).reshape(Hkv, n * nch_doc, d).astype(np.float64)
+    f64 = lambda bits: synth.bf16_bits_to_f32(bits).astype(np.float64)
+    Qr = f64(synth.query_bits(w, synth.T_QR, (w.batch, Hkv, 1, d)))
+    Q = f64(synth.query_bits(w, synth.T_Q, (w.batch, w.n_q_heads, 1, d)))
+    k_off = O.k_offset(w.top_k, w.doc_lens())
+    b = 0  # the same query is repeated: the oracle's work per query does not depend on its values
+    cache = {}
+    spent, queries = 0.0, 0
+    while queries == 0 or spent < seconds:
+        t0 = time.perf_counter()
+        sel = []
+        for h in range(Hkv):
+            s = O.route_doc_scores(Qr[b, h, 0], kr[h], chunk_doc, n)
+            sel.append(O.select_top_k(s, w.top_k))
+        spent += time.perf_counter() - t0
+        for h in range(Hkv):
+            docs = sel[h]
+            if h not in cache:  # input regeneration, not timed
+                mk = np.concatenate([f64(synth.bank_rows_bits(w, synth.T_K, h, int(j) * L, L)) for j in docs])
+                mv = np.concatenate([f64(synth.bank_rows_bits(w, synth.T_V, h, int(j) * L, L)) for j in docs])
+                base = (b * Hkv + h) * w.local_len * d
+                lk = f64(synth.normal_bf16_bits(w.seed, synth.T_LK, base, w.local_len * d)).reshape(-1, d)
+                lv = f64(synth.normal_bf16_bits(w.seed, synth.T_LV, base, w.local_len * d)).reshape(-1, d)
+                cache[h] = (mk, mv, lk, lv)
+            mk, mv, lk, lv = cache[h]
+            t0 = time.perf_counter()
+            mk_rot = O.parallel_rope_bank(mk, [L] * len(docs), w.rope_base)
+            for g in range(G):
+                O.routed_attention_row(Q[b, h * G + g, 0], w.local_len - 1, k_off, w.rope_base,
+                                       mk_rot, mv, lk, lv)
+            spent += time.perf_counter() - t0
+        queries += 1
+    threads = int(os.environ.get("OMP_NUM_THREADS", "0")) or os.cpu_count()
+    return queries / spent, queries, spent, threads
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    qps, nq, spent, cores = oracle_sample(max(2.0, min(args.cpu_seconds, 5.0 * max(1, args.steps) / 100)))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": qps, "unit": "queries/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * 8 / qps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "batch": 8, "bank_tokens": 4194304},
+        "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{nq} decode queries (router over all 16384 chunks x 8 KV heads, "
+                                   f"top-16, attention for 32 heads), {spent:.1f} s of oracle time"},
+        "e2e": {"value": qps, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        self.t_start = self.t_end = None
+
+    def mark(self, start: bool):
+        if start:
+            self.t_start = time.time()
+        else:
+            self.t_end = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxes.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        load = [s for s in sms if s > 0.5 * (max(sms) if sms else 1)]
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(maxes) if maxes else None, "reasons": sorted(reasons), "samples": len(sms)}
+
+
+# ----------------------------------------------------------------- ours
+def profile_traffic(kernel_file: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current source."""
+    prof = os.path.join(ROOT, "profiles", "attend_decode.decode_4m.txt")
+    src = os.path.join(ROOT, "sparse_attention_routed_b200", "csrc", kernel_file)
+    if not os.path.exists(prof):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    vals = {}
+    for line in open(prof):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("source_sha256") != sha:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    from sparse_attention_routed_b200 import msa_attend, msa_route, ptr
+    from sparse_attention_routed_b200.runner import Bank
+    from synth.device import bank_tensors, query_tensors
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    w = synth.WORKLOADS[args.workload]
+    K, V, R = bank_tensors(w)
+    bank = Bank(K, V, w.doc_lens(), w.rope_base)
+    bank.build(R)
+    torch.cuda.synchronize()
+    del R
+    torch.cuda.empty_cache()
+    Q, Qr, LK, LV = query_tensors(w)
+    qry = bank.query(Q, Qr, LK, LV, w.route_block)
+    bank.reserve(qry, w.top_k)
+    B, k, Hkv, d = w.batch, w.top_k, w.n_kv_heads, w.head_dim
+    idx = torch.empty((B, 1, Hkv, k), dtype=torch.int32, device="cuda")
+    out = torch.empty((B, w.n_q_heads, 1, d), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    def step():
+        msa_route(bank.handle, qry, k, 0, idx.data_ptr(), 0, sh)
+        msa_attend(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert bank.device_error() == 0
+
+    # algorithmic bytes of one step (selection is fixed by the fixed inputs)
+    sel = idx.cpu().numpy()
+    uniq = {(int(j), h) for b in range(B) for h in range(Hkv) for j in sel[b, 0, h]}
+    kv_sel = len(uniq) * w.doc_len * d * 2 * 2
+    kv_local = B * Hkv * w.local_len * d * 2 * 2
+    q_out = B * w.n_q_heads * d * (2 + 4)
+    nch = bank.info["n_chunks"]
+    router = Hkv * nch * (d * 4 + 4) + B * Hkv * w.n_docs * 4 * 2 + B * Hkv * d * 2
+    attn_bytes = kv_sel + kv_local + q_out
+    step_bytes = attn_bytes + router
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    time.sleep(0.4)
+    n = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark(True)
+    t_begin.record(stream)
+    for i in range(n):
+        ev[i][0].record(stream)
+        msa_route(bank.handle, qry, k, 0, idx.data_ptr(), 0, sh)
+        ev[i][1].record(stream)
+        msa_attend(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
+        ev[i][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(False)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = t_begin.elapsed_time(t_end)
+    route_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / n
+    attend_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / n
+    assert bank.device_error() == 0
+
+    # e2e: pinned host inputs of each decode step (queries, routing queries and the
+    # newest local token's K/V) copied in, the step run, output + selection copied out.
+    q_h = Q.cpu().pin_memory()
+    qr_h = Qr.cpu().pin_memory()
+    kv_h = torch.stack([LK[:, :, -1], LV[:, :, -1]]).cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    idx_h = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
+    h2d = q_h.numel() * 2 + qr_h.numel() * 2 + kv_h.numel() * 2
+    d2h = out_h.numel() * 4 + idx_h.numel() * 4
+    n_e2e = max(10, n // 2)
+
+    def e2e_step():
+        Q.copy_(q_h, non_blocking=True)
+        Qr.copy_(qr_h, non_blocking=True)
+        LK[:, :, -1].copy_(kv_h[0], non_blocking=True)
+        LV[:, :, -1].copy_(kv_h[1], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        idx_h.copy_(idx, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    t = torch.tensor([total_ms, e2e_ms, route_ms, attend_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    total_ms, e2e_ms, route_ms, attend_ms = t.tolist()
+    ms_step = total_ms / n
+    value = world * B * n / (total_ms / 1000.0)
+    e2e_value = world * B * n_e2e / (e2e_ms / 1000.0)
+
+    if rank == 0:
+        peak, peak_kind = peaks()
+        achieved = attn_bytes / (attend_ms / 1000.0) / 1e9
+        traffic = profile_traffic("attend_decode.cu")
+        line = {
+            "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": n,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "batch": B, "q_heads": w.n_q_heads, "kv_heads": Hkv,
+                       "head_dim": d, "bank_docs": w.n_docs, "doc_len": w.doc_len, "local_len": w.local_len,
+                       "top_k": k, "parallelism": f"replicas x{world}",
+                       "l2": f"inputs larger than L2: {step_bytes / 1e9:.2f} GB of HBM per step vs 126 MB L2"},
+            "router_attn_hbm": {"bytes_per_step": step_bytes, "GBps": step_bytes / (ms_step / 1000.0) / 1e9,
+                                "frac_of_peak": step_bytes / (ms_step / 1000.0) / 1e9 / peak,
+                                "route_ms": route_ms, "attend_ms": attend_ms},
+            "roofline": {"kernel": "sparse_attend (attend_decode + attend_merge launches)", "bound": "hbm",
+                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": attn_bytes},
+            "clocks": clk,
+            "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 5 * n,
+        }
+        if world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
+            qps, nq, spent, cores = oracle_sample(args.cpu_seconds)
+            line["cpu_baseline"] = {
+                "value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                "sample": f"{nq} decode queries (router over all 16384 chunks x 8 KV heads, top-16, "
+                          f"attention for 32 heads), {spent:.1f} s of oracle time"}
+        print(json.dumps(line), flush=True)
+    bank.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -197,6 +197,9 @@ def planted_targets(seed: int, batch: int, n_docs: int, count: int) -> np.ndarra
 WORKLOADS = {
     "tiny": Workload("tiny", 0, 1, 4, 4, 64, 16, 512, 256, 16, 16, 2),
     "decode_4m": Workload("decode_4m", 1, 8, 32, 8, 128, 1024, 4096, 4096, 1, 1, 16),
+    # same step as decode_4m on a 128-document bank: identical attention bytes per
+    # step, 2 GB of K/V on the device (for hardware-counter captures)
+    "decode_512k": Workload("decode_512k", 1, 8, 32, 8, 128, 128, 4096, 4096, 1, 1, 16),
     "prefill": Workload("prefill", 2, 1, 32, 8, 128, 256, 8192, 4096, 4096, 64, 8),
     "ragged_planted": Workload("ragged_planted", 3, 4, 64, 8, 128, 8192, 0, 2048, 1, 1, 32,
                                ragged=(512, 16384), planted=4, host_tier=True),
