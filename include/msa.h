@@ -164,6 +164,25 @@ msa_status msa_attend(msa_bank* bank, const msa_query* q, int32_t top_k,
 msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_t* topk_idx,
                        float* out, void* stream);
 
+/* msa_route without any allocation, for callers that must not allocate device
+ * memory while they run (inside a CUDA-graph capture, under a fixed memory
+ * budget or pool, or where a cudaMalloc's implicit synchronisation is not
+ * acceptable). The pages describe no such entry point; it exists for those
+ * callers only. Same arguments, outputs and results as msa_route.
+ * Scratch: q_r, 1/|q_r| and (when doc_scores is NULL) the document scores live
+ * in one 4 MiB device array that libmsa defines at file scope; every GPU that
+ * loads the library holds it until the process exits. A step needing more than
+ * 4 MiB (rows * Hkv * (4*d_r + 4 + 4*n_docs) bytes, each part rounded up to 256)
+ * returns MSA_ERR_UNSUPPORTED before any launch; pass doc_scores to keep the
+ * scores out of the scratch. Nothing in the scratch needs to start at zero:
+ * every word the kernels read was written earlier in the same call.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any stream
+ * capture. All calls share the one array, so calls whose work overlaps on the
+ * GPU (e.g. on two streams without ordering) race and corrupt each other. */
+msa_status msa_route_noalloc(msa_bank* bank, const msa_query* q, int32_t top_k, float* doc_scores,
+                             int32_t* topk_idx, float* topk_scores, void* stream);
+
 /* Synchronises `stream`, then returns and clears the device-side error flag
  * (MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_INVALID_ARG). */
 msa_status msa_get_device_error(msa_bank* bank, void* stream);

@@ -5,8 +5,8 @@ carry the names of the C entry points in include/msa.h and take raw integers
 (device pointers, host arrays via numpy, stream handles). `ptr()` turns a
 torch tensor into its device pointer after checking dtype and contiguity.
 
-Importing this module loads libmsa.so and fails loudly when it is missing;
-there is no fallback path.
+The first call loads libmsa.so (lib()) and fails loudly when it is missing or
+lacks an entry point; there is no fallback path.
 """
 from __future__ import annotations
 
@@ -71,6 +71,7 @@ def _load():
         "msa_attend": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp], ctypes.c_int),
         "msa_forward": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp], ctypes.c_int),
         "msa_get_device_error": ([vp, vp], ctypes.c_int),
+        "msa_route_noalloc": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -79,15 +80,30 @@ def _load():
     return lib
 
 
-LIB = _load()
+_LIB = None
+
+
+def lib():
+    """The loaded libmsa.so (loaded on first use)."""
+    global _LIB
+    if _LIB is None:
+        _LIB = _load()
+    return _LIB
+
+
+def __getattr__(name):
+    if name == "LIB":
+        return lib()
+    raise AttributeError(name)
 
 # Every symbol include/msa.h declares, in declaration order.
 EXPORTED = ["msa_bank_create", "msa_bank_destroy", "msa_build_bank", "msa_bank_info", "msa_reserve",
-            "msa_route", "msa_attend", "msa_forward", "msa_get_device_error", "msa_status_string"]
+            "msa_route", "msa_attend", "msa_forward", "msa_route_noalloc", "msa_get_device_error",
+            "msa_status_string"]
 
 
 def msa_status_string(status: int) -> str:
-    return LIB.msa_status_string(int(status)).decode()
+    return lib().msa_status_string(int(status)).decode()
 
 
 def _check(status: int, where: str) -> None:
@@ -122,19 +138,19 @@ def msa_bank_create(n_docs: int, n_kv_heads: int, head_dim: int, doc_lens, k: in
         lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), rope_base, kv_location, k or None, v or None,
         kv_rows, None if rows is None else rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)))
     handle = ctypes.c_void_p()
-    st = LIB.msa_bank_create(ctypes.byref(cfg), ctypes.byref(handle))
+    st = lib().msa_bank_create(ctypes.byref(cfg), ctypes.byref(handle))
     if check:
         _check(st, "msa_bank_create")
     return st, handle.value
 
 
 def msa_bank_destroy(bank) -> int:
-    return LIB.msa_bank_destroy(bank)
+    return lib().msa_bank_destroy(bank)
 
 
 def msa_build_bank(bank, doc_begin, doc_end, r_slice, r_head_stride, k_slice, k_head_stride, stream=0,
                    check=True) -> int:
-    st = LIB.msa_build_bank(bank, doc_begin, doc_end, r_slice or None, r_head_stride, k_slice or None,
+    st = lib().msa_build_bank(bank, doc_begin, doc_end, r_slice or None, r_head_stride, k_slice or None,
                             k_head_stride, stream or None)
     if check:
         _check(st, "msa_build_bank")
@@ -144,14 +160,14 @@ def msa_build_bank(bank, doc_begin, doc_end, r_slice, r_head_stride, k_slice, k_
 def msa_bank_info(bank):
     n_tok, n_ch, max_len = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
     kr, kinv = ctypes.c_void_p(), ctypes.c_void_p()
-    _check(LIB.msa_bank_info(bank, ctypes.byref(n_tok), ctypes.byref(n_ch), ctypes.byref(max_len),
+    _check(lib().msa_bank_info(bank, ctypes.byref(n_tok), ctypes.byref(n_ch), ctypes.byref(max_len),
                              ctypes.byref(kr), ctypes.byref(kinv)), "msa_bank_info")
     return {"n_tokens": n_tok.value, "n_chunks": n_ch.value, "max_doc_len": max_len.value,
             "k_r": kr.value, "k_r_inv_norm": kinv.value}
 
 
 def msa_reserve(bank, query: msa_query, top_k: int, check=True) -> int:
-    st = LIB.msa_reserve(bank, ctypes.byref(query), top_k)
+    st = lib().msa_reserve(bank, ctypes.byref(query), top_k)
     if check:
         _check(st, "msa_reserve")
     return st
@@ -159,7 +175,7 @@ def msa_reserve(bank, query: msa_query, top_k: int, check=True) -> int:
 
 def msa_route(bank, query: msa_query, top_k: int, doc_scores: int, topk_idx: int, topk_scores: int,
               stream=0, check=True) -> int:
-    st = LIB.msa_route(bank, ctypes.byref(query), top_k, doc_scores or None, topk_idx or None,
+    st = lib().msa_route(bank, ctypes.byref(query), top_k, doc_scores or None, topk_idx or None,
                        topk_scores or None, stream or None)
     if check:
         _check(st, "msa_route")
@@ -167,18 +183,28 @@ def msa_route(bank, query: msa_query, top_k: int, doc_scores: int, topk_idx: int
 
 
 def msa_attend(bank, query: msa_query, top_k: int, topk_idx: int, out: int, stream=0, check=True) -> int:
-    st = LIB.msa_attend(bank, ctypes.byref(query), top_k, topk_idx or None, out or None, stream or None)
+    st = lib().msa_attend(bank, ctypes.byref(query), top_k, topk_idx or None, out or None, stream or None)
     if check:
         _check(st, "msa_attend")
     return st
 
 
 def msa_forward(bank, query: msa_query, top_k: int, topk_idx: int, out: int, stream=0, check=True) -> int:
-    st = LIB.msa_forward(bank, ctypes.byref(query), top_k, topk_idx or None, out or None, stream or None)
+    st = lib().msa_forward(bank, ctypes.byref(query), top_k, topk_idx or None, out or None, stream or None)
     if check:
         _check(st, "msa_forward")
     return st
 
 
+def msa_route_noalloc(bank, query: msa_query, top_k: int, doc_scores: int, topk_idx: int, topk_scores: int,
+                      stream=0, check=True) -> int:
+    """msa_route with its scratch in the library's fixed 4 MiB device array (no allocation)."""
+    st = lib().msa_route_noalloc(bank, ctypes.byref(query), top_k, doc_scores or None, topk_idx or None,
+                               topk_scores or None, stream or None)
+    if check:
+        _check(st, "msa_route_noalloc")
+    return st
+
+
 def msa_get_device_error(bank, stream=0) -> int:
-    return LIB.msa_get_device_error(bank, stream or None)
+    return lib().msa_get_device_error(bank, stream or None)

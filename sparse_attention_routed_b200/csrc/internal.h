@@ -89,9 +89,22 @@ struct MergeArgs {
 };
 cudaError_t launch_attend_merge(const MergeArgs& a, cudaStream_t s);
 
+// Device pointers and sizes of a bank that the routing kernels read.
+struct BankRouteView {
+  const float* k_r;
+  const float* k_r_inv;
+  const int32_t* chunk_off;
+  int64_t nch;
+  int32_t n_docs, n_kv_heads, route_dim;
+};
+
 // Host-side helpers.
 int attend_rows_per_problem(int group, int route_block);
 int attend_tile_rows();  // keys per TMA tile of the decode attention kernel
 size_t attend_smem_bytes(int head_dim);
 
 }  // namespace msa
+
+struct msa_bank;
+// Fills `v` from a bank handle (no allocation, no CUDA call).
+void msa_bank_route_view(const msa_bank* bank, msa::BankRouteView* v);

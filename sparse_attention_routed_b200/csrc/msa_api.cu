@@ -310,6 +310,16 @@ msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, i
 
 }  // namespace
 
+void msa_bank_route_view(const msa_bank* bank, msa::BankRouteView* v) {
+  v->k_r = bank->d_kr;
+  v->k_r_inv = bank->d_kr_inv;
+  v->chunk_off = bank->d_chunk_off;
+  v->nch = bank->nch;
+  v->n_docs = bank->n_docs;
+  v->n_kv_heads = bank->hkv;
+  v->route_dim = bank->dr;
+}
+
 extern "C" {
 
 const char* msa_status_string(msa_status s) {

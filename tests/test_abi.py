@@ -22,6 +22,7 @@ def test_header_declarations_are_exported():
     names = declared()
     assert len(names) >= 10
     assert sorted(names) == sorted(msa.EXPORTED)
+    msa.lib()
     lib = ctypes.CDLL(msa.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
