@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "decode_512k"],
                     help="decode_512k: the same step on a 128-document bank (profiling captures)")
+    ap.add_argument("--route-only", action="store_true",
+                    help="time msa_route alone on the full bank's K_r with a stand-in 1-document K/V "
+                         "(routing keys streamed in slices; a few GB on the device, for profiling captures)")
     return ap.parse_args()
 
 
@@ -357,10 +360,60 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_route_only(args):
+    """msa_route alone over the full K_r of the workload (profiling aid, not the headline)."""
+    import torch
+
+    import synth
+    from sparse_attention_routed_b200 import msa_route
+    from sparse_attention_routed_b200.runner import Bank
+    from synth.device import fill_normal, query_tensors
+
+    w = synth.WORKLOADS[args.workload]
+    Hkv, d, L = w.n_kv_heads, w.head_dim, int(w.doc_lens().max())
+    K = torch.zeros((Hkv, L, d), dtype=torch.bfloat16, device="cuda")   # every document aliases these rows
+    V = torch.zeros_like(K)
+    bank = Bank(K, V, w.doc_lens(), w.rope_base, doc_rows=np.zeros(w.n_docs, dtype=np.int64))
+    off = np.concatenate([[0], np.cumsum(w.doc_lens())])
+    step = 64
+    for j0 in range(0, w.n_docs, step):
+        j1 = min(w.n_docs, j0 + step)
+        T = int(off[j1] - off[j0])
+        R = torch.empty((Hkv, T, d), dtype=torch.bfloat16, device="cuda")
+        for h in range(Hkv):
+            fill_normal(R[h], w.seed, synth.T_R, (h * w.n_tokens + int(off[j0])) * d)
+        bank.build(R, j0, j1, rope=False)
+        torch.cuda.synchronize()
+        del R
+    Q, Qr, LK, LV = query_tensors(w)
+    qry = bank.query(Q, Qr, LK, LV, w.route_block)
+    idx = torch.empty((w.batch, 1, Hkv, w.top_k), dtype=torch.int32, device="cuda")
+    sh = torch.cuda.current_stream().cuda_stream
+    for _ in range(max(3, args.warmup)):
+        msa_route(bank.handle, qry, w.top_k, 0, idx.data_ptr(), 0, sh)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        msa_route(bank.handle, qry, w.top_k, 0, idx.data_ptr(), 0, sh)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    kr_bytes = Hkv * bank.info["n_chunks"] * (d * 4 + 4)
+    peak, kind = peaks()
+    print(json.dumps({"mode": "route-only", "workload": args.workload, "route_ms": ms,
+                      "k_r_bytes": kr_bytes, "GBps": kr_bytes / (ms / 1e3) / 1e9,
+                      "frac_of_peak": kr_bytes / (ms / 1e3) / 1e9 / peak, "peak_kind": kind,
+                      "device_error": bank.device_error()}), flush=True)
+    bank.close()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.route_only:
+        run_route_only(args)
     else:
         run_ours(args)
 

@@ -8,51 +8,66 @@
 //
 // Design (B200, HBM-bound):
 //  * Problem p = (sequence, routing block, KV head). Its key list is the tiles
-//    of 64 keys of each selected document followed by the local tiles up to
+//    of TILE keys of each selected document followed by the local tiles up to
 //    the last query's position. The list is cut into n_splits equal ranges,
 //    one CTA each (split-KV), so ragged documents balance by construction.
 //  * One producer lane streams K and V tiles with 2-D TMA loads (128-byte
-//    swizzle, evict-first L2 policy) into an NS-stage ring guarded by
-//    full/empty mbarriers; 4 consumer warps take tiles round-robin.
+//    swizzle, evict-first L2 policy) into a ring of WARPS x BUFS slots; consumer
+//    warp w owns slots w, w + WARPS, ... and takes relative tiles w, w + WARPS, ...
 //  * The problem's query rows (G heads x Bq tokens <= 16) are few, so the MMA
 //    runs "keys as M": S^T = K Q^T with mma.sync m16n8k16 (keys fill M=16, the
 //    rows sit in N=8), then O^T += V^T P^T with V^T fed by ldmatrix.trans and
 //    P^T produced in registers by movmatrix.trans. Padding is at most N-side.
-//  * Online softmax in the exp2 domain; each CTA leaves (m, l, O) per row and
-//    attend_merge combines the splits.
+//  * Online softmax in the exp2 domain; the consumer warps merge in shared
+//    memory, each CTA leaves (m, l, O) per row, and the last CTA of a problem
+//    to finish (a wrapping atomic counter) merges all splits into the output.
 #include "common.cuh"
 #include "internal.h"
 
 namespace msa {
 namespace {
 
-constexpr int kTile = 64;          // keys per tile
-constexpr int kWarps = 4;          // consumer warps
-constexpr int kBufs = 1;           // ring slots owned by each consumer warp
-constexpr int kStages = kWarps * kBufs;
 constexpr int kMaxTopK = 64;
+constexpr int kMaxSplits = 64;
 constexpr int kRowsMax = 16;
-constexpr int kMT = kTile / 16;    // 16-key m-tiles per tile
 
-// Ring ownership: relative tile n goes to consumer warp n % kWarps; that warp's
-// q-th tile (q = n / kWarps) uses slot w + kWarps * (q % kBufs). Every slot is
-// filled and drained by one producer and one consumer warp in order, so each
-// mbarrier wait targets the phase right after one the waiter saw complete
-// (a parity wait is only unambiguous under that condition).
-__device__ __forceinline__ void slot_of(int n, int& stage, int& use) {
-  const int w = n % kWarps, q = n / kWarps;
-  stage = w + kWarps * (q % kBufs);
-  use = q / kBufs;
-}
-
-template <int D>
-struct Cfg {
-  static constexpr int kBoxes = D / 64;                 // 128-byte-wide TMA boxes per row
-  static constexpr int kBoxBytes = kTile * 128;
-  static constexpr int kTileBytes = kTile * D * 2;      // one of K or V
-  static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kRingBytes = kStages * kStageBytes;
+template <int D_, int TILE_, int WARPS_, int BUFS_>
+struct Shape {
+  static constexpr int D = D_;
+  static constexpr int TILE = TILE_;                  // keys per tile
+  static constexpr int WARPS = WARPS_;                // consumer warps
+  static constexpr int BUFS = BUFS_;                  // ring slots per consumer warp
+  static constexpr int STAGES = WARPS * BUFS;
+  static constexpr int MT = TILE / 16;                // 16-key m-tiles per tile
+  static constexpr int BOXES = D / 64;                // 128-byte-wide TMA boxes per row
+  static constexpr int BOX_BYTES = TILE * 128;
+  static constexpr int TILE_BYTES = TILE * D * 2;     // one of K or V
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+  static constexpr int THREADS = (WARPS + 1) * 32;
+  // resident CTAs per SM the ring allows (227 KiB of shared memory per SM)
+  static constexpr int MINB = RING_BYTES <= 70 * 1024 ? 3 : (RING_BYTES <= 108 * 1024 ? 2 : 1);
+  static_assert(TILE % 16 == 0 && TILE <= 256, "tile");
 };
+
+// The shape the library launches (one place to change it; the macros exist so
+// that other shapes can be compiled for measurement).
+#ifndef MSA_DECODE_TILE
+#define MSA_DECODE_TILE 32
+#endif
+#ifndef MSA_DECODE_WARPS
+#define MSA_DECODE_WARPS 4
+#endif
+#ifndef MSA_DECODE_BUFS
+#define MSA_DECODE_BUFS 1
+#endif
+// Cost of a local tile (Global RoPE in shared memory) relative to a bank tile,
+// used to cut each problem's tile list into splits of equal cost.
+#ifndef MSA_DECODE_LOCAL_W
+#define MSA_DECODE_LOCAL_W 2
+#endif
+template <int D>
+using Decode = Shape<D, MSA_DECODE_TILE, MSA_DECODE_WARPS, MSA_DECODE_BUFS>;
 
 struct TileRef {
   int di;  // document slot (0..k-1) or k for the local context
@@ -65,22 +80,45 @@ __device__ __forceinline__ TileRef locate(const int* tile_start, int k, int j, i
   return {di, j - tile_start[di]};
 }
 
-template <int D, int NT>
-__global__ void __launch_bounds__((kWarps + 1) * 32, 1)
+// Relative tile n goes to consumer warp n % WARPS; that warp's q-th tile uses
+// slot w + WARPS * (q % BUFS). Every slot is filled and drained by one producer
+// and one consumer in order, so each mbarrier parity wait targets the phase
+// right after one the waiter saw complete (the only case where it is unambiguous).
+template <class S>
+__device__ __forceinline__ void slot_of(int n, int& stage, int& use) {
+  const int w = n % S::WARPS, q = n / S::WARPS;
+  stage = w + S::WARPS * (q % S::BUFS);
+  use = q / S::BUFS;
+}
+
+template <class S>
+constexpr size_t smem_bytes(int nt) {
+  // ring, or the merge scratch that reuses it
+  size_t scratch = (size_t)S::WARPS * nt * 8 * (S::D + 2) * 4;
+  size_t body = (size_t)S::RING_BYTES > scratch ? (size_t)S::RING_BYTES : scratch;
+  return 1024 + body + 2 * S::STAGES * 8 + (kMaxTopK + 2) * 4 + kMaxTopK * 4 + kMaxTopK * 8 +
+         kMaxSplits * kRowsMax * 4 + 64;
+}
+
+template <class S, int NT>
+__global__ void __launch_bounds__(S::THREADS, S::MINB)
     attend_decode_kernel(const __grid_constant__ CUtensorMap tm_bk, const __grid_constant__ CUtensorMap tm_bv,
                          const __grid_constant__ CUtensorMap tm_lk, const __grid_constant__ CUtensorMap tm_lv,
                          const AttendArgs a) {
-  using C = Cfg<D>;
-  static_assert(kWarps * NT * 8 * (D + 2) * 4 <= C::kRingBytes, "merge scratch must fit in the ring");
+  constexpr int D = S::D, TILE = S::TILE, WARPS = S::WARPS, MT = S::MT;
+  constexpr int R = NT * 8;
+  static_assert((size_t)WARPS * R * (D + 2) * 4 <= (size_t)S::RING_BYTES, "merge scratch must fit in the ring");
   extern __shared__ uint8_t smem_raw[];
   // 128-byte swizzle is defined on shared-memory address bits: align the ring to 1 KiB there.
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint8_t* ring = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kRingBytes);
-  uint64_t* empty = full + kStages;
-  int* tile_start = reinterpret_cast<int*>(empty + kStages);         // [kMaxTopK + 2]
-  int* doc_len_s = tile_start + kMaxTopK + 2;                          // [kMaxTopK]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::RING_BYTES);
+  uint64_t* empty = full + S::STAGES;
+  int* tile_start = reinterpret_cast<int*>(empty + S::STAGES);                 // [kMaxTopK + 2]
+  int* doc_len_s = tile_start + kMaxTopK + 2;                                  // [kMaxTopK]
   long long* doc_base_s = reinterpret_cast<long long*>(doc_len_s + kMaxTopK);  // [kMaxTopK]
+  float* wgt_s = reinterpret_cast<float*>(doc_base_s + kMaxTopK);              // [kMaxSplits][kRowsMax]
+  int* flag_s = reinterpret_cast<int*>(wgt_s + kMaxSplits * kRowsMax);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -109,7 +147,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
     doc_base_s[tid] = base;
   }
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < S::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -120,18 +158,24 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
     int acc = 0;
     for (int d = 0; d < k; ++d) {
       tile_start[d] = acc;
-      acc += (doc_len_s[d] + kTile - 1) / kTile;
+      acc += (doc_len_s[d] + TILE - 1) / TILE;
     }
     tile_start[k] = acc;
-    tile_start[k + 1] = acc + (i_max + 1 + kTile - 1) / kTile;
+    tile_start[k + 1] = acc + (i_max + 1 + TILE - 1) / TILE;
   }
   __syncthreads();
-  const int T = tile_start[k + 1];
-  const int t0 = (int)(((long long)T * split) / a.n_splits);
-  const int t1 = (int)(((long long)T * (split + 1)) / a.n_splits);
+  // split boundaries in cost units: bank tiles cost 1, local tiles LOCAL_W
+  const int Tb = tile_start[k], T = tile_start[k + 1];
+  constexpr int LW = MSA_DECODE_LOCAL_W;
+  const long long cost = (long long)Tb + (long long)LW * (T - Tb);
+  auto tile_at = [&](long long cpos) -> int {
+    return cpos <= Tb ? (int)cpos : Tb + (int)((cpos - Tb + LW - 1) / LW);
+  };
+  const int t0 = tile_at((cost * split) / a.n_splits);
+  const int t1 = tile_at((cost * (split + 1)) / a.n_splits);
   const int ntiles = t1 - t0;
 
-  if (warp == kWarps) {
+  if (warp == WARPS) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && ntiles > 0) {
       prefetch_tensormap(&tm_bk);
@@ -141,37 +185,39 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
       const uint64_t pol = l2_policy_evict_first();
       int hint = 0;
       int issued = 0;
+      auto tile_coord = [&](const TileRef& tr, const CUtensorMap*& mk, const CUtensorMap*& mv, int& y) {
+        if (tr.di < k) {
+          mk = &tm_bk; mv = &tm_bv;
+          y = (int)(doc_base_s[tr.di] + (long long)tr.tt * TILE);
+        } else {
+          mk = &tm_lk; mv = &tm_lv;
+          y = (b * a.n_kv_heads + h) * a.local_len + tr.tt * TILE;
+        }
+      };
       for (int n = 0; n < ntiles; ++n) {
         int stage, use;
-        slot_of(n, stage, use);
+        slot_of<S>(n, stage, use);
         if (use > 0 && !mbar_wait_bounded(&empty[stage], (use - 1) & 1, a.err)) break;
         const TileRef tr = locate(tile_start, k, t0 + n, hint);
         hint = tr.di;
-        const CUtensorMap* mk;
-        const CUtensorMap* mv;
+        const CUtensorMap *mk, *mv;
         int y;
-        if (tr.di < k) {
-          mk = &tm_bk; mv = &tm_bv;
-          y = (int)(doc_base_s[tr.di] + (long long)tr.tt * kTile);
-        } else {
-          mk = &tm_lk; mv = &tm_lv;
-          y = (b * a.n_kv_heads + h) * a.local_len + tr.tt * kTile;
-        }
-        uint8_t* kdst = ring + stage * C::kStageBytes;
-        uint8_t* vdst = kdst + C::kTileBytes;
-        mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+        tile_coord(tr, mk, mv, y);
+        uint8_t* kdst = ring + stage * S::STAGE_BYTES;
+        uint8_t* vdst = kdst + S::TILE_BYTES;
+        mbar_arrive_expect_tx(&full[stage], S::STAGE_BYTES);
 #pragma unroll
-        for (int bx = 0; bx < C::kBoxes; ++bx) {
-          tma_load_2d(kdst + bx * C::kBoxBytes, mk, bx * 64, y, &full[stage], pol);
-          tma_load_2d(vdst + bx * C::kBoxBytes, mv, bx * 64, y, &full[stage], pol);
+        for (int bx = 0; bx < S::BOXES; ++bx) {
+          tma_load_2d(kdst + bx * S::BOX_BYTES, mk, bx * 64, y, &full[stage], pol);
+          tma_load_2d(vdst + bx * S::BOX_BYTES, mv, bx * 64, y, &full[stage], pol);
         }
         ++issued;
       }
       // No copy may still be landing when the CTA ends: wait for the last fill
       // of every slot (consumers normally have already).
-      for (int n = max(0, issued - kStages); n < issued; ++n) {
+      for (int n = max(0, issued - S::STAGES); n < issued; ++n) {
         int stage, use;
-        slot_of(n, stage, use);
+        slot_of<S>(n, stage, use);
         mbar_wait_bounded(&full[stage], use & 1, nullptr);
       }
     }
@@ -235,24 +281,23 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
   }
 
   int hint = 0;
-  bool ok = true;
-  for (int n = warp; n < ntiles && ok; n += kWarps) {
+  for (int n = warp; n < ntiles; n += WARPS) {
     int stage, use;
-    slot_of(n, stage, use);
-    if (!mbar_wait_bounded(&full[stage], use & 1, a.err)) { ok = false; break; }
+    slot_of<S>(n, stage, use);
+    if (!mbar_wait_bounded(&full[stage], use & 1, a.err)) break;
     const TileRef tr = locate(tile_start, k, t0 + n, hint);
     hint = tr.di;
-    uint8_t* kt = ring + stage * C::kStageBytes;
-    uint8_t* vt = kt + C::kTileBytes;
+    uint8_t* kt = ring + stage * S::STAGE_BYTES;
+    uint8_t* vt = kt + S::TILE_BYTES;
     const bool local = tr.di >= k;
-    const int key0 = tr.tt * kTile;
-    const int nvalid = local ? 0 : min(kTile, doc_len_s[tr.di] - key0);
+    const int key0 = tr.tt * TILE;
+    const int nvalid = local ? 0 : min(TILE, doc_len_s[tr.di] - key0);
 
     if (local) {
       // Global RoPE of the local keys, in shared memory: pair (i, i + D/2)
       // lives in the same swizzled slot of chunk i/8 and chunk (i + D/2)/8.
       constexpr int kPairChunks = D / 16;  // 16-byte chunks per half row
-      for (int unit = lane; unit < kTile * kPairChunks; unit += 32) {
+      for (int unit = lane; unit < TILE * kPairChunks; unit += 32) {
         const int r = unit / kPairChunks, ch = unit % kPairChunks;
         const int u = key0 + r;
         if (u >= a.local_len) continue;
@@ -260,7 +305,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
         uint8_t* py;
         if constexpr (D == 128) {
           px = kt + swz128(r, ch);
-          py = kt + C::kBoxBytes + swz128(r, ch);
+          py = kt + S::BOX_BYTES + swz128(r, ch);
         } else {
           px = kt + swz128(r, ch);
           py = kt + swz128(r, ch + 4);
@@ -282,25 +327,34 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
       __syncwarp();
     }
 
-    // ---- S^T = K Q^T : 4 m-tiles of 16 keys x NT n-tiles of 8 rows
-    float s[kMT][NT][4];
+    // ---- S^T = K Q^T : MT m-tiles of 16 keys x NT n-tiles of 8 rows; even and
+    // odd k-steps accumulate separately (two short mma dependency chains).
+    float s[MT][NT][4];
     const uint32_t kbase = smem_addr(kt);
 #pragma unroll
-    for (int mt = 0; mt < kMT; ++mt) {
+    for (int mt = 0; mt < MT; ++mt) {
+      float s2[NT][4];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) s[mt][nt][e] = 0.f;
+        for (int e = 0; e < 4; ++e) s[mt][nt][e] = s2[nt][e] = 0.f;
       const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
         const int col = ks * 16 + (lane >> 4) * 8;
-        const uint32_t addr = kbase + (col >> 6) * C::kBoxBytes + swz128(row, (col & 63) >> 3);
+        const uint32_t addr = kbase + (col >> 6) * S::BOX_BYTES + swz128(row, (col & 63) >> 3);
         uint32_t af[4];
         ldmatrix_x4(af, addr);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[mt][nt], af, qf[ks][nt][0], qf[ks][nt][1]);
+        for (int nt = 0; nt < NT; ++nt) {
+          if (ks & 1) mma_bf16_16816(s2[nt], af, qf[ks][nt][0], qf[ks][nt][1]);
+          else mma_bf16_16816(s[mt][nt], af, qf[ks][nt][0], qf[ks][nt][1]);
+        }
       }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[mt][nt][e] += s2[nt][e];
     }
 
     // ---- mask, scale, online softmax (per column = query row)
@@ -309,7 +363,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
     for (int nt = 0; nt < NT; ++nt) {
       float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-      for (int mt = 0; mt < kMT; ++mt)
+      for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
@@ -332,7 +386,7 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
         m_run[nt][e] = m_new;
         float sum = 0.f;
 #pragma unroll
-        for (int mt = 0; mt < kMT; ++mt)
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
             const float pv = exp2f(s[mt][nt][hf * 2 + e] - m_use);
@@ -351,9 +405,9 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
     }
 
     // ---- P^T fragments: transpose each 8x8 (keys x rows) block with movmatrix
-    uint32_t pb[kMT][NT][2];
+    uint32_t pb[MT][NT][2];
 #pragma unroll
-    for (int mt = 0; mt < kMT; ++mt)
+    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         pb[mt][nt][0] = movmatrix_trans(pack_bf16(s[mt][nt][0], s[mt][nt][1]));
@@ -363,12 +417,12 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
     // ---- O^T += V^T P^T
     const uint32_t vbase = smem_addr(vt);
 #pragma unroll
-    for (int mt = 0; mt < kMT; ++mt) {
+    for (int mt = 0; mt < MT; ++mt) {
       const int key = mt * 16 + (lane & 7) + (lane >> 4) * 8;
 #pragma unroll
       for (int md = 0; md < D / 16; ++md) {
         const int dim = md * 16 + ((lane >> 3) & 1) * 8;
-        const uint32_t addr = vbase + (dim >> 6) * C::kBoxBytes + swz128(key, (dim & 63) >> 3);
+        const uint32_t addr = vbase + (dim >> 6) * S::BOX_BYTES + swz128(key, (dim & 63) >> 3);
         uint32_t af[4];
         ldmatrix_x4_trans(af, addr);
 #pragma unroll
@@ -392,11 +446,11 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
       v += __shfl_xor_sync(0xffffffffu, v, 16);
       l_run[nt][e] = v;
     }
-  named_barrier_sync(1, kWarps * 32);  // every consumer is done reading the ring
-  constexpr int R = NT * 8;
-  float* sc_o = reinterpret_cast<float*>(ring);            // [kWarps][R][D]
-  float* sc_m = sc_o + kWarps * R * D;                       // [kWarps][R]
-  float* sc_l = sc_m + kWarps * R;                           // [kWarps][R]
+  constexpr int CT = WARPS * 32;  // consumer threads
+  named_barrier_sync(1, CT);      // every consumer is done reading the ring
+  float* sc_o = reinterpret_cast<float*>(ring);            // [WARPS][R][D]
+  float* sc_m = sc_o + WARPS * R * D;                      // [WARPS][R]
+  float* sc_l = sc_m + WARPS * R;                          // [WARPS][R]
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -412,17 +466,17 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
         sc_l[warp * R + r] = l_run[nt][e];
       }
     }
-  named_barrier_sync(1, kWarps * 32);
+  named_barrier_sync(1, CT);
   const int64_t slot = (int64_t)p * a.n_splits + split;
-  for (int idx = tid; idx < rows * D; idx += kWarps * 32) {
+  for (int idx = tid; idx < rows * D; idx += CT) {
     const int r = idx / D, dim = idx % D;
     float mstar = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) mstar = fmaxf(mstar, sc_m[w * R + r]);
+    for (int w = 0; w < WARPS; ++w) mstar = fmaxf(mstar, sc_m[w * R + r]);
     float o = 0.f, l = 0.f;
     if (mstar != -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
+      for (int w = 0; w < WARPS; ++w) {
         const float f = exp2f(sc_m[w * R + r] - mstar);
         o += f * sc_o[(w * R + r) * D + dim];
         l += f * sc_l[w * R + r];
@@ -434,83 +488,80 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
       a.part_ml[(slot * rows + r) * 2 + 1] = l;
     }
   }
-}
 
-// One warp per (problem, row): log-sum-exp merge of the splits.
-__global__ void attend_merge_kernel(MergeArgs a) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const int G = a.n_q_heads / a.n_kv_heads;
-  const int rows = G * a.route_block;
-  const int nblk = a.q_tokens / a.route_block;
-  const int P = a.batch * nblk * a.n_kv_heads;
-  if (warp >= P * rows) return;
-  const int p = warp / rows, r = warp % rows;
-  const int h = p % a.n_kv_heads;
-  const int blk = (p / a.n_kv_heads) % nblk;
-  const int b = p / (a.n_kv_heads * nblk);
-  const int t = blk * a.route_block + r / G;
-  const int hq = h * G + r % G;
-  const int D = a.head_dim;
-  float M = -INFINITY;
-  for (int s = 0; s < a.n_splits; ++s)
-    M = fmaxf(M, a.part_ml[(((int64_t)p * a.n_splits + s) * rows + r) * 2]);
-  float L = 0.f;
-  float o[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int s = 0; s < a.n_splits; ++s) {
-    const int64_t sl = ((int64_t)p * a.n_splits + s) * rows + r;
-    const float m = a.part_ml[sl * 2];
-    if (m == -INFINITY) continue;
-    const float f = exp2f(m - M);
-    L += f * a.part_ml[sl * 2 + 1];
-    for (int j = 0; j < D / 32; ++j) o[j] += f * a.part_o[sl * D + lane + 32 * j];
+  // ------------------------------------------------------------ split merge
+  // The last CTA of this problem to get here combines every split. Writers
+  // fence before the counter bump; the last one fences before reading.
+  __threadfence();
+  named_barrier_sync(1, CT);
+  if (tid == 0) {
+    const unsigned old = atomicInc(reinterpret_cast<unsigned*>(a.counters + p), (unsigned)(a.n_splits - 1));
+    *flag_s = (old == (unsigned)(a.n_splits - 1));
   }
-  const float inv = (L > 0.f) ? 1.0f / L : 0.f;
-  float* dst = a.out + (((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t) * D;
-  for (int j = 0; j < D / 32; ++j) dst[lane + 32 * j] = o[j] * inv;
+  named_barrier_sync(1, CT);
+  if (!*flag_s) return;
+  __threadfence();
+  const int nS = a.n_splits;
+  const float* pm = a.part_ml + (int64_t)p * nS * rows * 2;
+  for (int i = tid; i < rows; i += CT) {
+    float M = -INFINITY;
+    for (int sp = 0; sp < nS; ++sp) M = fmaxf(M, __ldcg(pm + (sp * rows + i) * 2));
+    float L = 0.f;
+    for (int sp = 0; sp < nS; ++sp) {
+      const float m = __ldcg(pm + (sp * rows + i) * 2);
+      const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
+      wgt_s[sp * kRowsMax + i] = f;
+      L += f * __ldcg(pm + (sp * rows + i) * 2 + 1);
+    }
+    const float inv = (L > 0.f) ? 1.0f / L : 0.f;
+    for (int sp = 0; sp < nS; ++sp) wgt_s[sp * kRowsMax + i] *= inv;
+  }
+  named_barrier_sync(1, CT);
+  const float* po = a.part_o + (int64_t)p * nS * rows * D;
+  for (int idx = tid; idx < rows * D; idx += CT) {
+    const int r = idx / D, dim = idx % D;
+    float o = 0.f;
+#pragma unroll 8
+    for (int sp = 0; sp < nS; ++sp) o += wgt_s[sp * kRowsMax + r] * __ldcg(po + ((int64_t)sp * rows + r) * D + dim);
+    const int t = blk * a.route_block + r / G;
+    const int hq = h * G + r % G;
+    a.out[(((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t) * D + dim] = o;
+  }
 }
 
-template <int D, int NT>
+template <class S, int NT>
 cudaError_t launch_decode_t(const AttendArgs& a, const AttendMaps& m, cudaStream_t s) {
-  auto kern = attend_decode_kernel<D, NT>;
-  const size_t smem = attend_smem_bytes(D);
+  auto kern = attend_decode_kernel<S, NT>;
+  const size_t smem = smem_bytes<S>(NT);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int nblk = a.q_tokens / a.route_block;
   dim3 grid(a.n_splits, a.batch * nblk * a.n_kv_heads);
-  kern<<<grid, (kWarps + 1) * 32, smem, s>>>(m.bank_k, m.bank_v, m.loc_k, m.loc_v, a);
+  kern<<<grid, S::THREADS, smem, s>>>(m.bank_k, m.bank_v, m.loc_k, m.loc_v, a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-int attend_rows_per_problem(int group, int route_block) { return group * route_block; }
-int attend_tile_rows() { return kTile; }
+int attend_tile_rows() { return Decode<128>::TILE; }
+int attend_max_splits() { return kMaxSplits; }
 
-size_t attend_smem_bytes(int head_dim) {
-  const size_t ring = (size_t)kStages * 2 * kTile * head_dim * 2;
-  const size_t scratch = (size_t)kWarps * kRowsMax * (head_dim + 2) * 4;
-  const size_t body = ring > scratch ? ring : scratch;
-  return 1024 + body + 2 * kStages * 8 + (kMaxTopK + 2) * 4 + kMaxTopK * 4 + kMaxTopK * 8;
+int attend_ctas_per_sm(int head_dim) {
+  const size_t per = head_dim == 128 ? smem_bytes<Decode<128>>(2) : smem_bytes<Decode<64>>(2);
+  const size_t total = 227 * 1024;
+  int n = (int)(total / (per + 1024));
+  return n < 1 ? 1 : n;
 }
 
 cudaError_t launch_attend_decode(const AttendArgs& a, const AttendMaps& m, int head_dim, cudaStream_t s) {
   const int rows = (a.n_q_heads / a.n_kv_heads) * a.route_block;
+  if (a.n_splits < 1 || a.n_splits > kMaxSplits || rows > kRowsMax) return cudaErrorInvalidValue;
   if (head_dim == 128) {
-    if (rows <= 8) return launch_decode_t<128, 1>(a, m, s);
-    return launch_decode_t<128, 2>(a, m, s);
+    if (rows <= 8) return launch_decode_t<Decode<128>, 1>(a, m, s);
+    return launch_decode_t<Decode<128>, 2>(a, m, s);
   }
-  if (rows <= 8) return launch_decode_t<64, 1>(a, m, s);
-  return launch_decode_t<64, 2>(a, m, s);
-}
-
-cudaError_t launch_attend_merge(const MergeArgs& a, cudaStream_t s) {
-  const int nblk = a.q_tokens / a.route_block;
-  const int rows = (a.n_q_heads / a.n_kv_heads) * a.route_block;
-  const int64_t warps = (int64_t)a.batch * nblk * a.n_kv_heads * rows;
-  const int blocks = (int)((warps + 3) / 4);
-  attend_merge_kernel<<<blocks, 128, 0, s>>>(a);
-  return cudaGetLastError();
+  if (rows <= 8) return launch_decode_t<Decode<64>, 1>(a, m, s);
+  return launch_decode_t<Decode<64>, 2>(a, m, s);
 }
 
 }  // namespace msa

@@ -77,7 +77,21 @@ __global__ void __launch_bounds__(256) bank_build_kernel(BankBuildArgs a) {
       dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
       dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
-    if (lane == 0) a.k_r_inv[h * a.nch_total + gc] = 1.0f / fmaxf(sqrtf(ss), 1e-30f);
+    const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-30f);
+    if (lane == 0) a.k_r_inv[h * a.nch_total + gc] = inv;
+    if (lane < LANES_PER_ROW) {
+      // normalised key split into bf16 hi + lo for the tensor-core router
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float x0 = acc[2 * j] * inv, x1 = acc[2 * j + 1] * inv;
+        hi[j] = pack_bf16(x0, x1);
+        lo[j] = pack_bf16(x0 - bf16_lo(hi[j]), x1 - bf16_hi(hi[j]));
+      }
+      const int64_t o = (h * a.nch_total + gc) * D + vec * 8;
+      *reinterpret_cast<uint4*>(a.k_hat_hi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(a.k_hat_lo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
   }
 
   // ---- Parallel RoPE in place: pair (i, i + D/2) turned by pos * theta_i

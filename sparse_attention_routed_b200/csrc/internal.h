@@ -21,6 +21,8 @@ struct BankBuildArgs {
   const float2* rope_tab;   // [max_doc_len][d/2] (cos, sin) of Parallel RoPE
   float* k_r;               // [Hkv][nch_total][d_r] (pointer at chunk 0 of the bank)
   float* k_r_inv;           // [Hkv][nch_total]
+  uint16_t* k_hat_hi;       // [Hkv][nch_total][d_r] bf16 of K_r / |K_r|
+  uint16_t* k_hat_lo;       // [Hkv][nch_total][d_r] bf16 of the remainder (hi + lo = K_r / |K_r|)
   int64_t nch_total;
   int64_t chunk0;           // global index of the slice's first chunk
   int32_t n_chunks;         // chunks in the slice
@@ -38,18 +40,30 @@ struct QrArgs {
 };
 cudaError_t launch_qr_prep(const QrArgs& a, cudaStream_t s);
 
-// Cosine of every (query row, chunk) and per-document max.
+// Cosine of every (query row, chunk) and per-document max, on tensor cores:
+// K_r / |K_r| is stored as bf16 hi + lo (tensor maps over [Hkv * nch, d_r]),
+// q_r / |q_r| is split the same way, and the three products hi*hi + hi*lo +
+// lo*hi carry the dot product to ~1e-5 relative.
 struct RouteArgs {
-  const float* k_r;        // [Hkv][nch][d_r]
-  const float* k_r_inv;    // [Hkv][nch]
   const int32_t* chunk_off;// [n_docs+1]
-  const float* q_r;        // [rows][Hkv][d_r]
+  const float* q_r;        // [rows][Hkv][d_r]   (used when qr == nullptr)
   const float* q_r_inv;    // [rows][Hkv]
   float* doc_scores;       // [rows][Hkv][n_docs]
   int64_t nch;
   int32_t rows, n_kv_heads, n_docs, route_dim;
+  // Optional: compute q_r in the router from the bf16 routing queries
+  // [B, Hkv, Tq, d_r] (rows = B * Tq / route_block); then q_r/q_r_inv are unused.
+  const uint16_t* qr;
+  int32_t q_tokens, route_block;
+  int* err;                // device error flag for expired waits, or nullptr
 };
-cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+// Largest routing block for which the router computes q_r itself.
+constexpr int kRouteFuseMaxBlock = 4;
+struct RouteMaps {
+  CUtensorMap k_hat_hi, k_hat_lo;  // boxes of route_tile_rows() chunks x 64 dims
+};
+cudaError_t launch_route(const RouteArgs& a, const RouteMaps& m, cudaStream_t s);
+int route_tile_rows();
 
 // Top-k per row of doc_scores, ordered (score desc, index asc).
 struct TopkArgs {
@@ -69,6 +83,8 @@ struct AttendArgs {
   const float2* gtab;       // [Lc][d/2] Global RoPE (cos, sin) at k_off + u
   float* part_o;            // [P][S][rows][d]   rows = G * route_block
   float* part_ml;           // [P][S][rows][2]   (running max in log2 units, sum)
+  float* out;               // [B, Hq, Tq, d] fp32
+  int* counters;            // [P] split-completion counters, zero between calls
   int* err;
   int64_t kv_rows;          // rows per head in the bank tensor map
   int32_t batch, n_q_heads, n_kv_heads, q_tokens, local_len, route_block, top_k, n_docs;
@@ -81,26 +97,18 @@ struct AttendMaps {
 cudaError_t launch_attend_decode(const AttendArgs& a, const AttendMaps& m, int head_dim,
                                  cudaStream_t s);
 
-struct MergeArgs {
-  const float* part_o;
-  const float* part_ml;
-  float* out;               // [B, Hq, Tq, d]
-  int32_t batch, n_q_heads, n_kv_heads, q_tokens, route_block, n_splits, head_dim;
-};
-cudaError_t launch_attend_merge(const MergeArgs& a, cudaStream_t s);
-
 // Device pointers and sizes of a bank that the routing kernels read.
 struct BankRouteView {
-  const float* k_r;
-  const float* k_r_inv;
+  RouteMaps maps;
   const int32_t* chunk_off;
   int64_t nch;
   int32_t n_docs, n_kv_heads, route_dim;
 };
 
 // Host-side helpers.
-int attend_rows_per_problem(int group, int route_block);
-int attend_tile_rows();  // keys per TMA tile of the decode attention kernel
+int attend_tile_rows();               // keys per TMA tile of the decode attention kernel
+int attend_max_splits();              // upper bound on n_splits
+int attend_ctas_per_sm(int head_dim); // resident CTAs per SM (shared-memory bound)
 size_t attend_smem_bytes(int head_dim);
 
 }  // namespace msa

@@ -21,6 +21,7 @@ namespace {
 constexpr int kChunk = 256;  // routing chunk ("MSA架构…" §2.1 item 2: 256-token chunks)
 constexpr int kMaxTopK = 64;
 constexpr int kMaxRows = 16;
+constexpr size_t kCounterBytes = 65536 * sizeof(int);  // one split counter per problem (P <= 65535)
 
 msa_status from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return MSA_OK;
@@ -110,6 +111,8 @@ struct msa_bank {
   float2* d_ptab = nullptr;
   float* d_kr = nullptr;
   float* d_kr_inv = nullptr;
+  uint16_t* d_khi = nullptr;  // bf16 K_r/|K_r| (hi), router operand
+  uint16_t* d_klo = nullptr;  // bf16 remainder (lo)
   int* d_err = nullptr;
   // Global RoPE table cache
   float2* d_gtab = nullptr;
@@ -119,8 +122,9 @@ struct msa_bank {
   // workspace
   uint8_t* ws = nullptr;
   size_t ws_cap = 0;
-  // TMA descriptors of the bank K/V (device tier)
+  // TMA descriptors of the bank K/V (device tier) and of the router operands
   CUtensorMap map_k{}, map_v{};
+  RouteMaps route_maps{};
   std::vector<void*> owned;
 };
 
@@ -130,7 +134,7 @@ void free_bank(msa_bank* b) {
   if (!b) return;
   cudaDeviceSynchronize();
   void* ptrs[] = {b->d_doc_row, b->d_doc_len, b->d_chunk_off, b->d_chunk_tok, b->d_chunk_len,
-                  b->d_chunk_pos, b->d_ptab, b->d_kr, b->d_kr_inv, b->d_err, b->d_gtab, b->ws};
+                  b->d_chunk_pos, b->d_ptab, b->d_kr, b->d_kr_inv, b->d_khi, b->d_klo, b->d_err, b->d_gtab, b->ws};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   delete b;
@@ -170,16 +174,32 @@ msa_status check_query(const msa_bank* bank, const msa_query* q, int top_k, Step
   return MSA_OK;
 }
 
+// Splits per problem. Every split of a problem carries the same work, so the
+// grid should fill whole waves of resident CTAs: among split counts that leave
+// every warp at least ~4 tiles, take the one whose last wave is fullest
+// (ties to fewer CTAs, which means fewer partials to merge).
 int choose_splits(const msa_bank* bank, const StepShape& s) {
   const double avg_len = (double)bank->ntok / bank->n_docs;
-  const int64_t tiles = (int64_t)s.k * (int64_t)std::ceil(avg_len / 64.0) + (s.Lc + 63) / 64;
-  const int64_t target = (int64_t)bank->sms * 2 * 8;  // ~8 waves of 2 resident CTAs per SM
-  int64_t S = (target + s.P - 1) / s.P;
-  S = std::min<int64_t>(S, std::max<int64_t>(1, tiles / 8));
-  return (int)std::max<int64_t>(1, S);
+  const int tile = attend_tile_rows();
+  const int64_t tiles = (int64_t)s.k * (int64_t)std::ceil(avg_len / tile) + (s.Lc + tile - 1) / tile;
+  const int64_t resident = (int64_t)bank->sms * attend_ctas_per_sm(bank->d);
+  const int64_t s_max = std::max<int64_t>(1, std::min<int64_t>(attend_max_splits(), tiles / 16));
+  int best = 1;
+  double best_eff = -1.0;
+  for (int64_t S = 1; S <= s_max; ++S) {
+    const double waves = (double)(s.P * S) / resident;
+    if (waves < 1.0 && S < s_max) continue;  // fill the machine at least once when possible
+    const double eff = waves / std::ceil(waves);
+    if (eff > best_eff + 0.01) {
+      best_eff = eff;
+      best = (int)S;
+    }
+  }
+  return best;
 }
 
 struct Workspace {
+  int* counters;
   float* q_r;
   float* q_r_inv;
   float* scores;
@@ -200,6 +220,7 @@ Workspace layout(const msa_bank* bank, const StepShape& s, int splits, uint8_t* 
     return p;
   };
   const size_t rows_route = (size_t)s.B * s.nblk;
+  w.counters = (int*)take(kCounterBytes);  // always first: a fixed place that stays zero between calls
   w.q_r = (float*)take(rows_route * bank->hkv * bank->dr * 4);
   w.q_r_inv = (float*)take(rows_route * bank->hkv * 4);
   w.scores = (float*)take(rows_route * bank->hkv * bank->n_docs * 4);
@@ -226,6 +247,7 @@ msa_status ensure_workspace(msa_bank* bank, size_t bytes, cudaStream_t s) {
     bank->ws_cap = 0;
   }
   MSA_CUDA(cudaMalloc(&bank->ws, bytes));
+  MSA_CUDA(cudaMemset(bank->ws, 0, bytes));
   bank->ws_cap = bytes;
   return MSA_OK;
 }
@@ -253,11 +275,16 @@ msa_status ensure_gtab(msa_bank* bank, int64_t koff, int lc, cudaStream_t s) {
 
 msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, const Workspace& w,
                       float* doc_scores, int32_t* idx, float* top_scores, cudaStream_t st) {
-  QrArgs qa{(const uint16_t*)q->qr, w.q_r, w.q_r_inv, s.B, bank->hkv, s.Tq, s.Bq, bank->dr};
-  MSA_CUDA(launch_qr_prep(qa, st));
   RouteArgs ra{};
-  ra.k_r = bank->d_kr;
-  ra.k_r_inv = bank->d_kr_inv;
+  const bool fuse = s.Bq <= kRouteFuseMaxBlock;  // the router forms q_r itself
+  if (!fuse) {
+    QrArgs qa{(const uint16_t*)q->qr, w.q_r, w.q_r_inv, s.B, bank->hkv, s.Tq, s.Bq, bank->dr};
+    MSA_CUDA(launch_qr_prep(qa, st));
+  } else {
+    ra.qr = (const uint16_t*)q->qr;
+    ra.q_tokens = s.Tq;
+    ra.route_block = s.Bq;
+  }
   ra.chunk_off = bank->d_chunk_off;
   ra.q_r = w.q_r;
   ra.q_r_inv = w.q_r_inv;
@@ -267,7 +294,8 @@ msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, co
   ra.n_kv_heads = bank->hkv;
   ra.n_docs = bank->n_docs;
   ra.route_dim = bank->dr;
-  MSA_CUDA(launch_route(ra, st));
+  ra.err = bank->d_err;
+  MSA_CUDA(launch_route(ra, bank->route_maps, st));
   TopkArgs ta{ra.doc_scores, idx, top_scores, s.P, bank->n_docs, s.k};
   MSA_CUDA(launch_topk(ta, st));
   return MSA_OK;
@@ -290,6 +318,8 @@ msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, i
   a.gtab = bank->d_gtab;
   a.part_o = w.part_o;
   a.part_ml = w.part_ml;
+  a.out = out;
+  a.counters = w.counters;
   a.err = bank->d_err;
   a.kv_rows = bank->kv_rows;
   a.batch = s.B;
@@ -303,16 +333,13 @@ msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, i
   a.n_splits = splits;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)bank->d));
   MSA_CUDA(launch_attend_decode(a, maps, bank->d, st));
-  MergeArgs m{w.part_o, w.part_ml, out, s.B, s.Hq, bank->hkv, s.Tq, s.Bq, splits, bank->d};
-  MSA_CUDA(launch_attend_merge(m, st));
   return MSA_OK;
 }
 
 }  // namespace
 
 void msa_bank_route_view(const msa_bank* bank, msa::BankRouteView* v) {
-  v->k_r = bank->d_kr;
-  v->k_r_inv = bank->d_kr_inv;
+  v->maps = bank->route_maps;
   v->chunk_off = bank->d_chunk_off;
   v->nch = bank->nch;
   v->n_docs = bank->n_docs;
@@ -418,6 +445,12 @@ msa_status msa_bank_create(const msa_bank_config* cfg, msa_bank** out) {
   if ((rc = upload(&b->d_ptab, rope_table(0, b->max_len, b->d, b->base))) != MSA_OK) return fail(rc);
   if (cudaMalloc(&b->d_kr, (size_t)b->hkv * b->nch * b->dr * 4) != cudaSuccess) return fail(MSA_ERR_OOM);
   if (cudaMalloc(&b->d_kr_inv, (size_t)b->hkv * b->nch * 4) != cudaSuccess) return fail(MSA_ERR_OOM);
+  if (cudaMalloc(&b->d_khi, (size_t)b->hkv * b->nch * b->dr * 2) != cudaSuccess) return fail(MSA_ERR_OOM);
+  if (cudaMalloc(&b->d_klo, (size_t)b->hkv * b->nch * b->dr * 2) != cudaSuccess) return fail(MSA_ERR_OOM);
+  if ((rc = make_map(&b->route_maps.k_hat_hi, b->d_khi, (int64_t)b->hkv * b->nch, b->dr, route_tile_rows())) != MSA_OK)
+    return fail(rc);
+  if ((rc = make_map(&b->route_maps.k_hat_lo, b->d_klo, (int64_t)b->hkv * b->nch, b->dr, route_tile_rows())) != MSA_OK)
+    return fail(rc);
   if (cudaMalloc(&b->d_err, sizeof(int)) != cudaSuccess) return fail(MSA_ERR_OOM);
   if (cudaMemset(b->d_err, 0, sizeof(int)) != cudaSuccess) return fail(MSA_ERR_CUDA);
   if (b->kv_loc == MSA_KV_DEVICE) {
@@ -455,6 +488,8 @@ msa_status msa_build_bank(msa_bank* bank, int32_t doc_begin, int32_t doc_end, co
   a.rope_tab = bank->d_ptab;
   a.k_r = bank->d_kr;
   a.k_r_inv = bank->d_kr_inv;
+  a.k_hat_hi = bank->d_khi;
+  a.k_hat_lo = bank->d_klo;
   a.nch_total = bank->nch;
   a.chunk0 = c0;
   a.n_chunks = (int32_t)(c1 - c0);
@@ -533,6 +568,8 @@ msa_status msa_get_device_error(msa_bank* bank, void* stream) {
   int v = 0;
   MSA_CUDA(cudaMemcpy(&v, bank->d_err, sizeof(int), cudaMemcpyDeviceToHost));
   MSA_CUDA(cudaMemset(bank->d_err, 0, sizeof(int)));
+  // A step cut short may leave split counters mid-count: reset them.
+  if (v != 0 && bank->ws) MSA_CUDA(cudaMemset(bank->ws, 0, kCounterBytes));
   return (msa_status)v;
 }
 

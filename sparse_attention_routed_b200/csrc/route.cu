@@ -41,109 +41,258 @@ __global__ void qr_prep_kernel(QrArgs a) {
 }
 
 // ---------------------------------------------------------------- router
-// Warp per document: the warp streams the document's K_r rows (one 16-byte
-// vector per lane per chunk for d_r = 128) and keeps a running max per query
-// row. NR rows are scored per pass; the per-row dot products are finished by
-// a reduce-scatter butterfly so that after log2(32) steps lane l holds the
-// total of row l >> (5 - log2 NR).
-template <int DR, int NR>
-__global__ void __launch_bounds__(256) route_kernel(RouteArgs a, int row0) {
-  constexpr int VEC = DR / 32;  // floats per lane per chunk (4 or 2)
-  constexpr int LOG_NR = (NR == 1) ? 0 : (NR == 2) ? 1 : (NR == 4) ? 2 : (NR == 8) ? 3 : (NR == 16) ? 4 : 5;
-  __shared__ __align__(16) float qs[NR * DR];
-  __shared__ float qinv[NR];
-  const int h = blockIdx.y;
-  const int nrows = min(NR, a.rows - row0);
-  for (int i = threadIdx.x; i < NR * DR; i += blockDim.x) {
-    const int r = i / DR;
-    qs[i] = (r < nrows) ? a.q_r[((int64_t)(row0 + r) * a.n_kv_heads + h) * DR + (i % DR)] : 0.f;
+// Scoring the whole bank is the step's bottleneck (robocikowo.com, Złożoność
+// obliczeniowa): K_r is the one large stream, at 2 multiply-adds per byte for
+// 8 query rows -- more than the fp32 FMA pipes sustain at HBM speed -- so the
+// contraction runs on tensor cores:
+//   S^T[chunk, row] = sum_d Khat[chunk, d] * Qhat[row, d],
+// with Khat = K_r/|K_r| and Qhat = q_r/|q_r| each split into bf16 hi + lo and
+// the products lo*hi + hi*lo + hi*hi accumulated in fp32 by mma.sync m16n8k16
+// (chunks as M, query rows as N). The score is then the cosine itself.
+// Khat tiles of RITEM chunks arrive by 2-D TMA (128-byte swizzle) into a ring
+// whose slots each consumer warp owns; CTA (x, h) owns documents
+// x, x + gridDim.x, ... of KV head h, its j-th document going to warp
+// j % RWARPS, which keeps a running max per row over the document's chunks.
+constexpr int RWARPS = 4;
+constexpr int RBUFS = 2;
+constexpr int RSLOTS = RWARPS * RBUFS;
+constexpr int RITEM = 16;            // chunks per tile (one m16 tile)
+constexpr int RNT_MAX = 2;           // n-tiles of 8 query rows per pass
+constexpr int RDOCS = 512;           // documents per CTA whose chunk ranges are staged in shared memory
+
+template <int DR, int NT>
+struct RouteShape {
+  static constexpr int BOXES = DR / 64;
+  static constexpr int BOX_BYTES = RITEM * 128;
+  static constexpr int MAT_BYTES = BOXES * BOX_BYTES;  // hi or lo tile
+  static constexpr int SLOT_BYTES = 2 * MAT_BYTES;
+  static constexpr int NR = NT * 8;
+  static constexpr size_t bytes() {
+    return 1024 + (size_t)RSLOTS * SLOT_BYTES + 2 * RSLOTS * 8 + 2 * (size_t)NR * DR * 2 + 2 * RDOCS * 4;
   }
-  for (int r = threadIdx.x; r < NR; r += blockDim.x)
-    qinv[r] = (r < nrows) ? a.q_r_inv[(int64_t)(row0 + r) * a.n_kv_heads + h] : 0.f;
+};
+
+template <int DR, int NT>
+__global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
+    route_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo,
+                 const RouteArgs a, int row0) {
+  using SH = RouteShape<DR, NT>;
+  constexpr int NR = SH::NR;
+  constexpr int THREADS = (RWARPS + 1) * 32;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* ring = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + RSLOTS * SH::SLOT_BYTES);
+  uint64_t* empty = full + RSLOTS;
+  // fp32 q_r rows live in the ring until the split below (before any TMA is issued)
+  float* qs = reinterpret_cast<float*>(ring);                   // [NR][DR] fp32
+  static_assert(SH::NR * DR * 4 <= RSLOTS * SH::SLOT_BYTES, "q_r scratch must fit in the ring");
+  uint16_t* qhi = reinterpret_cast<uint16_t*>(empty + RSLOTS);  // [NR][DR] bf16
+  uint16_t* qlo = qhi + NR * DR;                                // [NR][DR] bf16
+  int* c_beg = reinterpret_cast<int*>(qlo + NR * DR);           // [RDOCS] chunk range of the
+  int* c_end = c_beg + RDOCS;                                   // CTA's j-th document
+  const int h = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nrows = min(NR, a.rows - row0);
+
+  if (tid == 0) {
+    for (int s = 0; s < RSLOTS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    fence_barrier_init();
+  }
+  const int n_mine = (a.n_docs - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;  // <= RDOCS (host check)
+  for (int j = tid; j < n_mine; j += THREADS) {
+    const int doc = blockIdx.x + j * gridDim.x;
+    c_beg[j] = a.chunk_off[doc];
+    c_end[j] = a.chunk_off[doc + 1];
+  }
+  // ---- query rows of this pass: q_r (block mean) in fp32
+  if (a.qr != nullptr) {
+    const int nblk = a.q_tokens / a.route_block;
+    const float inv_b = 1.0f / (float)a.route_block;
+    for (int i = tid; i < NR * DR; i += THREADS) {
+      const int r = i / DR, dd = i % DR;
+      float v = 0.f;
+      if (r < nrows) {
+        const int row = row0 + r, bb = row / nblk, blk = row % nblk;
+        const uint16_t* src =
+            a.qr + (((int64_t)bb * a.n_kv_heads + h) * a.q_tokens + (int64_t)blk * a.route_block) * DR + dd;
+        for (int t = 0; t < a.route_block; ++t) v += __uint_as_float((uint32_t)src[(int64_t)t * DR] << 16);
+        v *= inv_b;
+      }
+      qs[i] = v;
+    }
+  } else {
+    for (int i = tid; i < NR * DR; i += THREADS) {
+      const int r = i / DR;
+      qs[i] = (r < nrows) ? a.q_r[((int64_t)(row0 + r) * a.n_kv_heads + h) * DR + (i % DR)] : 0.f;
+    }
+  }
+  __syncthreads();
+  // ---- normalise and split into bf16 hi + lo
+  for (int r = warp; r < NR; r += THREADS / 32) {
+    float ss = 0.f;
+    for (int i = lane; i < DR; i += 32) ss += qs[r * DR + i] * qs[r * DR + i];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-30f);
+    for (int i = lane; i < DR; i += 32) {
+      const float x = qs[r * DR + i] * inv;
+      const __nv_bfloat16 hb = __float2bfloat16_rn(x);
+      const __nv_bfloat16 lb = __float2bfloat16_rn(x - __bfloat162float(hb));
+      qhi[r * DR + i] = *reinterpret_cast<const uint16_t*>(&hb);
+      qlo[r * DR + i] = *reinterpret_cast<const uint16_t*>(&lb);
+    }
+  }
   __syncthreads();
 
-  const int lane = threadIdx.x & 31;
-  // This lane's slice of every query row.
-  float q[NR][VEC];
+  if (warp == RWARPS) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tm_hi);
+      prefetch_tensormap(&tm_lo);
+      const uint64_t pol = l2_policy_evict_first();
+      int qw[RWARPS] = {};  // items issued per consumer warp (constant-indexed: registers)
+      bool ok = true;
+      for (int j0 = 0; ok && j0 < n_mine; j0 += RWARPS) {
 #pragma unroll
-  for (int r = 0; r < NR; ++r)
+        for (int w = 0; w < RWARPS; ++w) {
+          const int j = j0 + w;
+          if (!ok || j >= n_mine) break;
+          const int c1 = c_end[j];
+          for (int cs = c_beg[j]; cs < c1; cs += RITEM) {
+            const int slot = w + RWARPS * (qw[w] % RBUFS), use = qw[w] / RBUFS;
+            if (use > 0 && !mbar_wait_bounded(&empty[slot], (use - 1) & 1, a.err)) {
+              ok = false;
+              break;
+            }
+            ++qw[w];
+            uint8_t* dst = ring + slot * SH::SLOT_BYTES;
+            const int y = (int)((int64_t)h * a.nch + cs);
+            mbar_arrive_expect_tx(&full[slot], SH::SLOT_BYTES);
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) q[r][v] = qs[r * DR + lane * VEC + v];
-  const int my_row = lane >> (5 - LOG_NR);
-  const float my_qinv = qinv[my_row];
-
-  const float* kr = a.k_r + (int64_t)h * a.nch * DR;
-  const float* kinv = a.k_r_inv + (int64_t)h * a.nch;
-  const int warps_total = gridDim.x * (blockDim.x >> 5);
-  for (int doc = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); doc < a.n_docs; doc += warps_total) {
-    const int c0 = a.chunk_off[doc], c1 = a.chunk_off[doc + 1];
-    float best = -INFINITY;
-    for (int c = c0; c < c1; c += 4) {
-      float kv[4][VEC];
-      float ki[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int cc = min(c + u, c1 - 1);
-        if constexpr (VEC == 4) {
-          float4 t = __ldcs(reinterpret_cast<const float4*>(kr + (int64_t)cc * DR) + lane);
-          kv[u][0] = t.x; kv[u][1] = t.y; kv[u][2] = t.z; kv[u][3] = t.w;
-        } else {
-          float2 t = __ldcs(reinterpret_cast<const float2*>(kr + (int64_t)cc * DR) + lane);
-          kv[u][0] = t.x; kv[u][1] = t.y;
-        }
-        ki[u] = __ldg(kinv + cc);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        float p[NR];
-#pragma unroll
-        for (int r = 0; r < NR; ++r) {
-          float s = 0.f;
-#pragma unroll
-          for (int v = 0; v < VEC; ++v) s = fmaf(q[r][v], kv[u][v], s);
-          p[r] = s;
-        }
-        // reduce-scatter: halve the live rows per step on lane bits 4..(5-LOG_NR)
-#pragma unroll
-        for (int step = 0; step < LOG_NR; ++step) {
-          const int off = 16 >> step;
-          const int half = NR >> (step + 1);
-          const bool upper = (lane & off) != 0;
-#pragma unroll
-          for (int i = 0; i < half; ++i) {
-            const float send = upper ? p[i] : p[i + half];
-            const float keep = upper ? p[i + half] : p[i];
-            p[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+            for (int bx = 0; bx < SH::BOXES; ++bx) {
+              tma_load_2d(dst + bx * SH::BOX_BYTES, &tm_hi, bx * 64, y, &full[slot], pol);
+              tma_load_2d(dst + SH::MAT_BYTES + bx * SH::BOX_BYTES, &tm_lo, bx * 64, y, &full[slot], pol);
+            }
           }
         }
-        float tot = p[0];
-#pragma unroll
-        for (int off = (16 >> LOG_NR); off > 0; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
-        const float sc = tot * ki[u] * my_qinv;
-        if (c + u < c1) best = fmaxf(best, sc);
       }
+      // no copy may still be landing when the CTA ends
+#pragma unroll
+      for (int w = 0; w < RWARPS; ++w)
+        for (int q = max(0, qw[w] - RBUFS); q < qw[w]; ++q)
+          mbar_wait_bounded(&full[w + RWARPS * (q % RBUFS)], (q / RBUFS) & 1, nullptr);
     }
-    // lanes holding the same row agree; the first of each group writes
-    if ((lane & ((32 >> LOG_NR) - 1)) == 0 && my_row < nrows)
-      a.doc_scores[((int64_t)(row0 + my_row) * a.n_kv_heads + h) * a.n_docs + doc] = best;
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers
+  const int g = lane >> 2, c = lane & 3;
+  // B fragments (k = dims, n = rows): row 8*nt + g, dims 16ks + 2c (+1), +8.
+  uint32_t bh[DR / 16][NT][2], bl[DR / 16][NT][2];
+#pragma unroll
+  for (int ks = 0; ks < DR / 16; ++ks)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int o = (nt * 8 + g) * DR + ks * 16 + hf * 8 + 2 * c;
+        bh[ks][nt][hf] = *reinterpret_cast<const uint32_t*>(qhi + o);
+        bl[ks][nt][hf] = *reinterpret_cast<const uint32_t*>(qlo + o);
+      }
+  const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;  // ldmatrix row of this lane
+  int qc = 0;
+  for (int j = warp; j < n_mine; j += RWARPS) {
+    const int doc = blockIdx.x + j * gridDim.x;
+    const int c1 = c_end[j];
+    float best[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) best[nt][0] = best[nt][1] = -INFINITY;
+    bool ok = true;
+    for (int cs = c_beg[j]; cs < c1; cs += RITEM) {
+      const int n = min(RITEM, c1 - cs);
+      const int slot = warp + RWARPS * (qc % RBUFS), use = qc / RBUFS;
+      ++qc;
+      if (!mbar_wait_bounded(&full[slot], use & 1, a.err)) {
+        ok = false;
+        break;
+      }
+      const uint32_t hbase = smem_addr(ring + slot * SH::SLOT_BYTES);
+      const uint32_t lbase = hbase + SH::MAT_BYTES;
+      float acc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < DR / 16; ++ks) {
+        const int col = ks * 16 + (lane >> 4) * 8;
+        const uint32_t off = (col >> 6) * SH::BOX_BYTES + swz128(arow, (col & 63) >> 3);
+        uint32_t ah[4], al[4];
+        ldmatrix_x4(ah, hbase + off);
+        ldmatrix_x4(al, lbase + off);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_bf16_16816(acc[nt], al, bh[ks][nt][0], bh[ks][nt][1]);
+          mma_bf16_16816(acc[nt], ah, bl[ks][nt][0], bl[ks][nt][1]);
+          mma_bf16_16816(acc[nt], ah, bh[ks][nt][0], bh[ks][nt][1]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+      // rows of the C tile are chunks g and g + 8; mask those past the document
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float v = fmaxf(g < n ? acc[nt][e] : -INFINITY, g + 8 < n ? acc[nt][e + 2] : -INFINITY);
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+          best[nt][e] = fmaxf(best[nt][e], v);
+        }
+    }
+    if (!ok) break;
+    if (g == 0) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int r = nt * 8 + 2 * c + e;
+          if (r < nrows) a.doc_scores[((int64_t)(row0 + r) * a.n_kv_heads + h) * a.n_docs + doc] = best[nt][e];
+        }
+    }
   }
 }
 
-template <int DR>
-cudaError_t launch_route_dr(const RouteArgs& a, cudaStream_t s) {
-  const int warps_per_block = 8;
-  int blocks_x = (a.n_docs + warps_per_block - 1) / warps_per_block;
-  for (int row0 = 0; row0 < a.rows; row0 += 32) {
-    const int nr = a.rows - row0;
-    dim3 grid(blocks_x, a.n_kv_heads);
-    if (nr <= 1) route_kernel<DR, 1><<<grid, 256, 0, s>>>(a, row0);
-    else if (nr <= 2) route_kernel<DR, 2><<<grid, 256, 0, s>>>(a, row0);
-    else if (nr <= 4) route_kernel<DR, 4><<<grid, 256, 0, s>>>(a, row0);
-    else if (nr <= 8) route_kernel<DR, 8><<<grid, 256, 0, s>>>(a, row0);
-    else if (nr <= 16) route_kernel<DR, 16><<<grid, 256, 0, s>>>(a, row0);
-    else route_kernel<DR, 32><<<grid, 256, 0, s>>>(a, row0);
-  }
+template <int DR, int NT>
+cudaError_t launch_route_t(const RouteArgs& a, const RouteMaps& m, int row0, int sms, cudaStream_t s) {
+  auto kern = route_kernel<DR, NT>;
+  const size_t smem = RouteShape<DR, NT>::bytes();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = (int)((227 * 1024) / (smem + 1024));
+  per_sm = per_sm < 1 ? 1 : (per_sm > 3 ? 3 : per_sm);
+  // one wave of resident CTAs, unless a CTA would own more than RDOCS documents
+  int gx = (sms * per_sm) / a.n_kv_heads;
+  gx = gx < 1 ? 1 : (gx > a.n_docs ? a.n_docs : gx);
+  if ((a.n_docs + gx - 1) / gx > RDOCS) gx = (a.n_docs + RDOCS - 1) / RDOCS;
+  if (gx > 65535) return cudaErrorInvalidValue;
+  kern<<<dim3(gx, a.n_kv_heads), (RWARPS + 1) * 32, smem, s>>>(m.k_hat_hi, m.k_hat_lo, a, row0);
   return cudaGetLastError();
+}
+
+template <int DR>
+cudaError_t launch_route_dr(const RouteArgs& a, const RouteMaps& m, cudaStream_t s) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  for (int row0 = 0; row0 < a.rows; row0 += 8 * RNT_MAX) {
+    const int nr = a.rows - row0;
+    const cudaError_t e = nr <= 8 ? launch_route_t<DR, 1>(a, m, row0, sms, s) : launch_route_t<DR, 2>(a, m, row0, sms, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 // ---------------------------------------------------------------- top-k
@@ -173,15 +322,33 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(TopkArgs a) {
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
     __syncthreads();
-    if (tid == 0) {
-      uint32_t cum = 0;
-      int dg = 0;
-      for (int d = 255; d >= 0; --d) {
-        if (cum + hist[d] >= remaining) { dg = d; break; }
-        cum += hist[d];
+    if (tid < 32) {
+      // Suffix scan over the 256 bins (largest digit first): lane l owns bins
+      // 255-8l .. 248-8l; the lane whose range crosses `remaining` picks the digit.
+      uint32_t cnt[8], tot = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[j] = hist[255 - (tid * 8 + j)];
+        tot += cnt[j];
       }
-      s_prefix = prefix | ((uint32_t)dg << shift);
-      s_remaining = remaining - cum;
+      uint32_t incl = tot;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (tid >= off) incl += v;
+      }
+      const uint32_t excl = incl - tot;
+      if (excl < remaining && remaining <= incl) {
+        uint32_t cum = excl;
+        int dg = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (cum + cnt[j] >= remaining) { dg = 255 - (tid * 8 + j); break; }
+          cum += cnt[j];
+        }
+        s_prefix = prefix | ((uint32_t)dg << shift);
+        s_remaining = remaining - cum;
+      }
     }
     __syncthreads();
     prefix = s_prefix;
@@ -246,10 +413,12 @@ cudaError_t launch_qr_prep(const QrArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
-  if (a.route_dim == 128) return launch_route_dr<128>(a, s);
-  return launch_route_dr<64>(a, s);
+cudaError_t launch_route(const RouteArgs& a, const RouteMaps& m, cudaStream_t s) {
+  if (a.route_dim == 128) return launch_route_dr<128>(a, m, s);
+  return launch_route_dr<64>(a, m, s);
 }
+
+int route_tile_rows() { return RITEM; }
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   topk_kernel<<<a.rows, TOPK_THREADS, 0, s>>>(a);

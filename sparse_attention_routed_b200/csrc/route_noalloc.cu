@@ -79,8 +79,6 @@ extern "C" msa_status msa_route_noalloc(msa_bank* bank, const msa_query* q, int3
                  q->route_block, v.route_dim};
   if (msa::launch_qr_prep(qa, s) != cudaSuccess) return MSA_ERR_CUDA;
   msa::RouteArgs ra{};
-  ra.k_r = v.k_r;
-  ra.k_r_inv = v.k_r_inv;
   ra.chunk_off = v.chunk_off;
   ra.q_r = q_r;
   ra.q_r_inv = q_inv;
@@ -90,7 +88,7 @@ extern "C" msa_status msa_route_noalloc(msa_bank* bank, const msa_query* q, int3
   ra.n_kv_heads = v.n_kv_heads;
   ra.n_docs = v.n_docs;
   ra.route_dim = v.route_dim;
-  if (msa::launch_route(ra, s) != cudaSuccess) return MSA_ERR_CUDA;
+  if (msa::launch_route(ra, v.maps, s) != cudaSuccess) return MSA_ERR_CUDA;
   msa::TopkArgs ta{scores, topk_idx, topk_scores, (int32_t)(rows * v.n_kv_heads), v.n_docs, top_k};
   if (msa::launch_topk(ta, s) != cudaSuccess) return MSA_ERR_CUDA;
   return MSA_OK;

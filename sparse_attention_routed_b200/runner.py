@@ -39,13 +39,16 @@ class Bank:
                                          ptr(K), ptr(V), rope_base, kv_location, self.kv_rows, doc_rows)
         self.info = msa_bank_info(self.handle)
 
-    def build(self, R: torch.Tensor, doc_begin: int = 0, doc_end=None, K_slice=None, stream=None):
+    def build(self, R: torch.Tensor, doc_begin: int = 0, doc_end=None, K_slice=None, stream=None,
+              rope: bool = True):
         """Pools K_r from R [Hkv, T, d_r] of docs [doc_begin, doc_end); RoPEs K_slice
-        (default: the bank's own K rows of those documents) in place."""
+        (default: the bank's own K rows of those documents) in place unless rope=False."""
         doc_end = len(self.doc_lens) if doc_end is None else doc_end
         off = np.concatenate([[0], np.cumsum(self.doc_lens)])
         tok0 = int(off[doc_begin])
-        if K_slice is None:
+        if not rope:
+            k_ptr, k_stride = 0, 0
+        elif K_slice is None:
             K_slice = self.K
             k_ptr = self.K.data_ptr() + tok0 * self.head_dim * 2
             k_stride = self.kv_rows
