@@ -43,8 +43,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "decode_512k"],
-                    help="decode_512k: the same step on a 128-document bank (profiling captures)")
+    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "decode_512k", "prefill"],
+                    help="decode_512k: the same step on a 128-document bank (profiling captures); "
+                         "prefill: 4096 query tokens in 64-token routing blocks (tensor-bound)")
     ap.add_argument("--route-only", action="store_true",
                     help="time msa_route alone on the full bank's K_r with a stand-in 1-document K/V "
                          "(routing keys streamed in slices; a few GB on the device, for profiling captures)")
@@ -58,6 +59,23 @@ def peaks():
             m = json.load(f)
         return float(m["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def tensor_peak():
+    """Dense bf16 TFLOP/s: the burst figure (a kernel timed alone)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+def launches_per_step(w) -> int:
+    """Kernels libmsa launches for one route + attend step of workload w."""
+    rows_route = w.batch * (w.q_tokens // w.route_block)
+    n = (0 if w.route_block <= 4 else 1) + (rows_route + 15) // 16 + 1     # qr_prep, router passes, top-k
+    n += 1 if (w.n_q_heads // w.n_kv_heads) * w.route_block <= 16 else 2   # decode kernel | rope_local + prefill
+    return n
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -220,6 +238,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
     w = synth.WORKLOADS[args.workload]
+    prefill = args.workload == "prefill"
     K, V, R = bank_tensors(w)
     bank = Bank(K, V, w.doc_lens(), w.rope_base)
     bank.build(R)
@@ -230,8 +249,9 @@ def run_ours(args):
     qry = bank.query(Q, Qr, LK, LV, w.route_block)
     bank.reserve(qry, w.top_k)
     B, k, Hkv, d = w.batch, w.top_k, w.n_kv_heads, w.head_dim
-    idx = torch.empty((B, 1, Hkv, k), dtype=torch.int32, device="cuda")
-    out = torch.empty((B, w.n_q_heads, 1, d), dtype=torch.float32, device="cuda")
+    nblk = w.q_tokens // w.route_block
+    idx = torch.empty((B, nblk, Hkv, k), dtype=torch.int32, device="cuda")
+    out = torch.empty((B, w.n_q_heads, w.q_tokens, d), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
 
@@ -244,16 +264,23 @@ def run_ours(args):
     torch.cuda.synchronize()
     assert bank.device_error() == 0
 
-    # algorithmic bytes of one step (selection is fixed by the fixed inputs)
+    # algorithmic bytes and FLOPs of one step (the selection is fixed by the fixed inputs)
     sel = idx.cpu().numpy()
-    uniq = {(int(j), h) for b in range(B) for h in range(Hkv) for j in sel[b, 0, h]}
-    kv_sel = len(uniq) * w.doc_len * d * 2 * 2
+    lens = w.doc_lens()
+    uniq = {(int(j), h) for b in range(B) for blk in range(nblk) for h in range(Hkv) for j in sel[b, blk, h]}
+    kv_sel = sum(int(lens[j]) for j, _ in uniq) * d * 2 * 2
     kv_local = B * Hkv * w.local_len * d * 2 * 2
-    q_out = B * w.n_q_heads * d * (2 + 4)
+    q_out = B * w.n_q_heads * w.q_tokens * d * (2 + 4)
     nch = bank.info["n_chunks"]
-    router = Hkv * nch * (d * 4 + 4) + B * Hkv * w.n_docs * 4 * 2 + B * Hkv * d * 2
+    router = Hkv * nch * (d * 4) + B * nblk * Hkv * w.n_docs * 4 * 2 + B * Hkv * w.q_tokens * d * 2
     attn_bytes = kv_sel + kv_local + q_out
     step_bytes = attn_bytes + router
+    G = w.n_q_heads // w.n_kv_heads
+    mem_keys = sum(int(lens[j]) for b in range(B) for blk in range(nblk) for h in range(Hkv)
+                   for j in sel[b, blk, h]) * G * w.route_block
+    first = w.local_len - w.q_tokens
+    loc_keys = B * w.n_q_heads * sum(first + t + 1 for t in range(w.q_tokens))
+    attn_flops = 4 * d * (mem_keys + loc_keys)
 
     if world > 1:
         dist.barrier()
@@ -282,11 +309,12 @@ def run_ours(args):
     attend_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / n
     assert bank.device_error() == 0
 
-    # e2e: pinned host inputs of each decode step (queries, routing queries and the
-    # newest local token's K/V) copied in, the step run, output + selection copied out.
+    # e2e: pinned host inputs of each step copied in -- decode: queries, routing
+    # queries and the newest local token's K/V; prefill: queries, routing queries
+    # and the whole local K/V (the prompt) -- the step run, output + selection copied out.
     q_h = Q.cpu().pin_memory()
     qr_h = Qr.cpu().pin_memory()
-    kv_h = torch.stack([LK[:, :, -1], LV[:, :, -1]]).cpu().pin_memory()
+    kv_h = (torch.stack([LK, LV]) if prefill else torch.stack([LK[:, :, -1], LV[:, :, -1]])).cpu().pin_memory()
     out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     idx_h = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
     h2d = q_h.numel() * 2 + qr_h.numel() * 2 + kv_h.numel() * 2
@@ -296,8 +324,12 @@ def run_ours(args):
     def e2e_step():
         Q.copy_(q_h, non_blocking=True)
         Qr.copy_(qr_h, non_blocking=True)
-        LK[:, :, -1].copy_(kv_h[0], non_blocking=True)
-        LV[:, :, -1].copy_(kv_h[1], non_blocking=True)
+        if prefill:
+            LK.copy_(kv_h[0], non_blocking=True)
+            LV.copy_(kv_h[1], non_blocking=True)
+        else:
+            LK[:, :, -1].copy_(kv_h[0], non_blocking=True)
+            LV[:, :, -1].copy_(kv_h[1], non_blocking=True)
         step()
         out_h.copy_(out, non_blocking=True)
         idx_h.copy_(idx, non_blocking=True)
@@ -321,32 +353,44 @@ def run_ours(args):
         dist.barrier()
     total_ms, e2e_ms, route_ms, attend_ms = t.tolist()
     ms_step = total_ms / n
-    value = world * B * n / (total_ms / 1000.0)
-    e2e_value = world * B * n_e2e / (e2e_ms / 1000.0)
+    units = B * (w.q_tokens if prefill else 1)   # queries (decode) or query tokens (prefill) per step
+    value = world * units * n / (total_ms / 1000.0)
+    e2e_value = world * units * n_e2e / (e2e_ms / 1000.0)
 
     if rank == 0:
         peak, peak_kind = peaks()
-        achieved = attn_bytes / (attend_ms / 1000.0) / 1e9
-        traffic = profile_traffic("attend_decode.cu")
+        if prefill:
+            tpeak, tkind = tensor_peak()
+            achieved = attn_flops / (attend_ms / 1000.0) / 1e12
+            roofline = {"kernel": "sparse_attend (rope_local + attend_prefill launches)", "bound": "tensor",
+                        "achieved": achieved, "peak": tpeak, "peak_kind": tkind, "unit": "TFLOP/s",
+                        "frac": achieved / tpeak, "traffic": None, "algorithmic_flops_per_launch": attn_flops,
+                        "hbm_bytes_algorithmic": attn_bytes}
+            metric, unit = "prefill query tokens/s (4096-token prompt, 64-token routing blocks)", "tokens/s"
+        else:
+            achieved = attn_bytes / (attend_ms / 1000.0) / 1e9
+            roofline = {"kernel": "sparse_attend (attend_decode launch)", "bound": "hbm",
+                        "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                        "frac": achieved / peak, "traffic": profile_traffic("attend_decode.cu"),
+                        "algorithmic_bytes_per_launch": attn_bytes}
+            metric, unit = METRIC, "queries/s"
         line = {
-            "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": n,
+            "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": n,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": args.workload, "batch": B, "q_heads": w.n_q_heads, "kv_heads": Hkv,
                        "head_dim": d, "bank_docs": w.n_docs, "doc_len": w.doc_len, "local_len": w.local_len,
-                       "top_k": k, "parallelism": f"replicas x{world}",
+                       "q_tokens": w.q_tokens, "route_block": w.route_block, "top_k": k,
+                       "parallelism": f"replicas x{world}",
                        "l2": f"inputs larger than L2: {step_bytes / 1e9:.2f} GB of HBM per step vs 126 MB L2"},
             "router_attn_hbm": {"bytes_per_step": step_bytes, "GBps": step_bytes / (ms_step / 1000.0) / 1e9,
                                 "frac_of_peak": step_bytes / (ms_step / 1000.0) / 1e9 / peak,
                                 "route_ms": route_ms, "attend_ms": attend_ms},
-            "roofline": {"kernel": "sparse_attend (attend_decode + attend_merge launches)", "bound": "hbm",
-                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic,
-                         "algorithmic_bytes_per_launch": attn_bytes},
+            "roofline": roofline,
             "clocks": clk,
-            "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": 5 * n,
+            "gpu_launches": launches_per_step(w) * n,
         }
         if world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
             qps, nq, spent, cores = oracle_sample(args.cpu_seconds)

@@ -96,6 +96,12 @@ struct AttendMaps {
 };
 cudaError_t launch_attend_decode(const AttendArgs& a, const AttendMaps& m, int head_dim,
                                  cudaStream_t s);
+// Many-row problems (G * route_block > 16); loc_k must map the RoPE'd local keys.
+cudaError_t launch_attend_prefill(const AttendArgs& a, const AttendMaps& m, int head_dim, cudaStream_t s);
+int attend_prefill_tile_rows();
+// out[row] = Global RoPE of lk[row] at k_off + (row % local_len) (rows = B * Hkv * Lc).
+cudaError_t launch_rope_local(const uint16_t* lk, uint16_t* out, const float2* gtab, int64_t rows, int local_len,
+                              int head_dim, cudaStream_t s);
 
 // Device pointers and sizes of a bank that the routing kernels read.
 struct BankRouteView {

@@ -123,7 +123,8 @@ struct msa_bank {
   uint8_t* ws = nullptr;
   size_t ws_cap = 0;
   // TMA descriptors of the bank K/V (device tier) and of the router operands
-  CUtensorMap map_k{}, map_v{};
+  CUtensorMap map_k{}, map_v{};      // boxes of the decode kernel's tile
+  CUtensorMap map_k64{}, map_v64{};  // boxes of the prefill kernel's tile
   RouteMaps route_maps{};
   std::vector<void*> owned;
 };
@@ -166,7 +167,6 @@ msa_status check_query(const msa_bank* bank, const msa_query* q, int top_k, Step
   if (need_attn) {
     if (!q->q || !q->local_k || !q->local_v) return MSA_ERR_INVALID_ARG;
     if (!aligned16(q->q) || !aligned16(q->local_k) || !aligned16(q->local_v)) return MSA_ERR_INVALID_ARG;
-    if (s->rows > kMaxRows) return MSA_ERR_UNSUPPORTED;
     if ((int64_t)s->B * bank->hkv * s->Lc >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
     if (bank->kv_loc != MSA_KV_DEVICE) return MSA_ERR_UNSUPPORTED;
   }
@@ -206,6 +206,7 @@ struct Workspace {
   int32_t* idx;
   float* part_o;
   float* part_ml;
+  uint16_t* local_rot;  // prefill: local keys with Global RoPE applied
   size_t bytes;
 };
 
@@ -225,8 +226,10 @@ Workspace layout(const msa_bank* bank, const StepShape& s, int splits, uint8_t* 
   w.q_r_inv = (float*)take(rows_route * bank->hkv * 4);
   w.scores = (float*)take(rows_route * bank->hkv * bank->n_docs * 4);
   w.idx = (int32_t*)take((size_t)s.P * s.k * 4);
-  w.part_o = (float*)take((size_t)s.P * splits * s.rows * bank->d * 4);
-  w.part_ml = (float*)take((size_t)s.P * splits * s.rows * 2 * 4);
+  const bool prefill = s.rows > kMaxRows;
+  w.part_o = (float*)take(prefill ? 0 : (size_t)s.P * splits * s.rows * bank->d * 4);
+  w.part_ml = (float*)take(prefill ? 0 : (size_t)s.P * splits * s.rows * 2 * 4);
+  w.local_rot = (uint16_t*)take(prefill ? (size_t)s.B * bank->hkv * s.Lc * bank->d * 2 : 0);
   w.bytes = off;
   return w;
 }
@@ -303,12 +306,16 @@ msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, co
 
 msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, int splits, const Workspace& w,
                        const int32_t* idx, float* out, cudaStream_t st) {
+  const bool prefill = s.rows > kMaxRows;
+  const int box = prefill ? attend_prefill_tile_rows() : attend_tile_rows();
+  const int64_t lrows = (int64_t)s.B * bank->hkv * s.Lc;
   AttendMaps maps;
-  maps.bank_k = bank->map_k;
-  maps.bank_v = bank->map_v;
-  msa_status rc = make_map(&maps.loc_k, q->local_k, (int64_t)s.B * bank->hkv * s.Lc, bank->d, attend_tile_rows());
+  maps.bank_k = prefill ? bank->map_k64 : bank->map_k;
+  maps.bank_v = prefill ? bank->map_v64 : bank->map_v;
+  if (prefill) MSA_CUDA(launch_rope_local((const uint16_t*)q->local_k, w.local_rot, bank->d_gtab, lrows, s.Lc, bank->d, st));
+  msa_status rc = make_map(&maps.loc_k, prefill ? (const void*)w.local_rot : q->local_k, lrows, bank->d, box);
   if (rc != MSA_OK) return rc;
-  rc = make_map(&maps.loc_v, q->local_v, (int64_t)s.B * bank->hkv * s.Lc, bank->d, attend_tile_rows());
+  rc = make_map(&maps.loc_v, q->local_v, lrows, bank->d, box);
   if (rc != MSA_OK) return rc;
   AttendArgs a{};
   a.q = (const uint16_t*)q->q;
@@ -332,7 +339,11 @@ msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, i
   a.n_docs = bank->n_docs;
   a.n_splits = splits;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)bank->d));
-  MSA_CUDA(launch_attend_decode(a, maps, bank->d, st));
+  if (prefill) {
+    MSA_CUDA(launch_attend_prefill(a, maps, bank->d, st));
+  } else {
+    MSA_CUDA(launch_attend_decode(a, maps, bank->d, st));
+  }
   return MSA_OK;
 }
 
@@ -456,6 +467,10 @@ msa_status msa_bank_create(const msa_bank_config* cfg, msa_bank** out) {
   if (b->kv_loc == MSA_KV_DEVICE) {
     if ((rc = make_map(&b->map_k, b->k, (int64_t)b->hkv * b->kv_rows, b->d, attend_tile_rows())) != MSA_OK) return fail(rc);
     if ((rc = make_map(&b->map_v, b->v, (int64_t)b->hkv * b->kv_rows, b->d, attend_tile_rows())) != MSA_OK) return fail(rc);
+    if ((rc = make_map(&b->map_k64, b->k, (int64_t)b->hkv * b->kv_rows, b->d, attend_prefill_tile_rows())) != MSA_OK)
+      return fail(rc);
+    if ((rc = make_map(&b->map_v64, b->v, (int64_t)b->hkv * b->kv_rows, b->d, attend_prefill_tile_rows())) != MSA_OK)
+      return fail(rc);
   }
   *out = b;
   return MSA_OK;

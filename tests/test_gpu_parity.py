@@ -24,6 +24,11 @@ SMALL = {
     "one_token": Workload("one_token", 15, 1, 2, 2, 128, 3, 0, 1, 1, 1, 1, ragged=(1, 3)),
     "planted_small": Workload("planted_small", 16, 2, 8, 8, 128, 30, 0, 64, 1, 1, 4, ragged=(300, 1500),
                               planted=4),
+    # many-row problems (prefill kernel): 4 heads x 64 tokens = 256 rows over 2 CTAs
+    "prefill_small": Workload("prefill_small", 17, 1, 8, 2, 128, 24, 600, 256, 256, 64, 3),
+    # 3 heads x 48 tokens = 144 rows (a 16-row tail CTA), ragged docs, queries not at the local start
+    "prefill_ragged": Workload("prefill_ragged", 18, 2, 6, 2, 128, 20, 0, 300, 96, 48, 4, ragged=(1, 900)),
+    "prefill_d64": Workload("prefill_d64", 19, 1, 4, 1, 64, 12, 0, 200, 64, 32, 12, ragged=(50, 400)),
 }
 
 
