@@ -12,7 +12,7 @@
 // barrier counts the 8 warps). Per 64-key tile each warp computes
 // S = Q K^T and O += P V with mma.sync m16n8k16 in the FlashAttention-2
 // register layout (the S accumulator fragments are the P operand fragments).
-// The local keys arrive already turned by Global RoPE (rope_local_kernel);
+// The local keys arrive already turned by Global RoPE (rope_rows_kernel);
 // queries are turned while their fragments are built.
 #include "common.cuh"
 #include "internal.h"
@@ -37,15 +37,17 @@ struct PShape {
                                  PMAX_TOPK * 8;
 };
 
-// Global RoPE of the local keys at k_off + u, written to a workspace copy.
-__global__ void rope_local_kernel(const uint16_t* __restrict__ lk, uint16_t* __restrict__ out,
-                                  const float2* __restrict__ gtab, int64_t rows, int local_len, int d) {
+// Global RoPE of a [rows, d] tensor into a workspace copy: row r sits at local
+// index offset + r % period (local keys: period Lc, offset 0; queries: period
+// Tq, offset Lc - Tq), i.e. at position k_off + that index.
+__global__ void rope_rows_kernel(const uint16_t* __restrict__ lk, uint16_t* __restrict__ out,
+                                 const float2* __restrict__ gtab, int64_t rows, int period, int offset, int d) {
   const int half_vecs = d / 16;  // 16-byte vectors per half row
   const int64_t unit = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (unit >= rows * half_vecs) return;
   const int64_t row = unit / half_vecs;
   const int vec = (int)(unit % half_vecs);
-  const int u = (int)(row % local_len);
+  const int u = offset + (int)(row % period);
   const uint4 x = *reinterpret_cast<const uint4*>(lk + row * d + vec * 8);
   const uint4 y = *reinterpret_cast<const uint4*>(lk + row * d + d / 2 + vec * 8);
   const float4* cs = reinterpret_cast<const float4*>(gtab + (int64_t)u * (d / 2) + vec * 8);
@@ -345,11 +347,11 @@ cudaError_t launch_prefill_t(const AttendArgs& a, const AttendMaps& m, cudaStrea
 
 int attend_prefill_tile_rows() { return PT; }
 
-cudaError_t launch_rope_local(const uint16_t* lk, uint16_t* out, const float2* gtab, int64_t rows, int local_len,
-                              int head_dim, cudaStream_t s) {
+cudaError_t launch_rope_rows(const uint16_t* in, uint16_t* out, const float2* gtab, int64_t rows, int period,
+                             int offset, int head_dim, cudaStream_t s) {
   const int64_t units = rows * (head_dim / 16);
   const int blocks = (int)((units + 255) / 256);
-  rope_local_kernel<<<blocks, 256, 0, s>>>(lk, out, gtab, rows, local_len, head_dim);
+  rope_rows_kernel<<<blocks, 256, 0, s>>>(in, out, gtab, rows, period, offset, head_dim);
   return cudaGetLastError();
 }
 

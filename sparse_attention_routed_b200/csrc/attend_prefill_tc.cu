@@ -1,0 +1,335 @@
+// sparse_attend (prefill) on the 5th-generation tensor cores: tcgen05.mma with
+// accumulators in tensor memory (TMEM), operands staged by TMA.
+//   "MSA (Memory Sparse Attention)" (robocikowo.com), Komponenty (Memory Sparse
+//   Attention Layer), Pułapki implementacyjne (Global RoPE with a k-offset),
+//   Paradygmat wykonania (only the k selected documents take part).
+//
+// One CTA owns 128 query rows of one problem (sequence, 64- or 128-token
+// routing block, KV head; rows ordered head-major) and walks the problem's key
+// list in tiles of 128 keys: the selected documents' tiles, then the local
+// tiles up to its last row's position.
+//   warp 0     TMA producer: the query tile once (queries pre-turned by Global
+//              RoPE), then K and V tiles into a 2-stage ring.
+//   warp 1     allocates 512 TMEM columns; one lane issues, per tile j,
+//              S_j = Q K_j^T (M = N = K = 128, into one of two S buffers) and
+//              then O += P_{j-1} V_{j-1} (P from shared memory, V read as an
+//              MN-major operand), and commits each group to an mbarrier.
+//   warps 4-7  softmax, one thread per row (TMEM lane = row): read S_j with
+//              tcgen05.ld, mask (document tails, causal local keys), write
+//              P_j = exp2(S_j * scale - m) as bf16 into a 128-byte-swizzled
+//              K-major tile. The reference max m of a row moves only when the
+//              row max rises by more than 2^8; then the row of O is rescaled in
+//              TMEM (warp-collective tcgen05.ld/st after the previous P V).
+// Every mbarrier parity wait targets the phase right after one the same waiter
+// saw complete, so no wait can be satisfied by an older phase.
+#include "common.cuh"
+#include "internal.h"
+
+namespace msa {
+namespace {
+
+constexpr int TN = 128;               // keys per tile
+constexpr int TM = 128;               // query rows per CTA
+constexpr int TD = 128;               // head dim
+constexpr int TMEM_COLS = 512;        // S0 [0,128) S1 [128,256) O [256,384)
+constexpr int O_COL = 256;
+constexpr int THREADS = 256;
+constexpr int BOX = TN * 128;         // one 64-element-wide box of a 128-row tile (16 KB)
+constexpr int TILE = 2 * BOX;         // 128 x 128 bf16 (32 KB)
+constexpr int TOPK_MAX = 64;
+constexpr float kLazy = 8.0f;         // rescale O only when a row max grows by more than 2^8
+
+// shared memory layout (offsets from a 1 KiB-aligned base)
+constexpr int OFF_Q = 0;
+constexpr int OFF_K0 = OFF_Q + TILE;           // K[s] = OFF_K0 + s * 2 * TILE, V[s] = K[s] + TILE
+constexpr int OFF_P0 = OFF_K0 + 4 * TILE;      // P[b] = OFF_P0 + b * TILE
+constexpr int OFF_BAR = OFF_P0 + 2 * TILE;
+constexpr int N_BAR = 13;
+constexpr int OFF_TMEM = OFF_BAR + N_BAR * 8;
+constexpr int OFF_TAB = OFF_TMEM + 8;
+constexpr size_t SMEM_BYTES = 1024 + OFF_TAB + (TOPK_MAX + 2) * 4 + TOPK_MAX * 4 + TOPK_MAX * 8;
+static_assert(SMEM_BYTES <= 232448, "shared memory");
+
+__global__ void __launch_bounds__(THREADS, 1)
+    attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_bk,
+                             const __grid_constant__ CUtensorMap tm_bv, const __grid_constant__ CUtensorMap tm_lk,
+                             const __grid_constant__ CUtensorMap tm_lv, const AttendArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;    // [2]
+  uint64_t* kv_empty = bars + 3;   // [2]
+  uint64_t* s_full = bars + 5;     // [2]
+  uint64_t* s_free = bars + 7;     // [2]
+  uint64_t* p_full = bars + 9;     // [2]
+  uint64_t* p_free = bars + 11;    // [2]
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
+  int* tile_start = reinterpret_cast<int*>(sm + OFF_TAB);
+  int* doc_len_s = tile_start + TOPK_MAX + 2;
+  long long* doc_base_s = reinterpret_cast<long long*>(doc_len_s + TOPK_MAX);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int p = blockIdx.y;
+  const int G = a.n_q_heads / a.n_kv_heads;
+  const int Bq = a.route_block;
+  const int nblk = a.q_tokens / Bq;
+  const int h = p % a.n_kv_heads;
+  const int blk = (p / a.n_kv_heads) % nblk;
+  const int b = p / (a.n_kv_heads * nblk);
+  const int row0 = blockIdx.x * TM;  // rows ordered (head, token); 128 | G * Bq
+  const int i_first = a.local_len - a.q_tokens + blk * Bq;
+  const int r_end = row0 + TM - 1;
+  const int i_max = i_first + (r_end / Bq != row0 / Bq ? Bq - 1 : r_end % Bq);
+  const int k = a.top_k;
+
+  if (tid < k) {
+    const int j = a.sel[(int64_t)p * k + tid];
+    int len = 0;
+    long long base = 0;
+    if (j >= 0 && j < a.n_docs) {
+      len = a.doc_len[j];
+      base = (long long)h * a.kv_rows + a.doc_row[j];
+    } else {
+      atomicCAS(a.err, 0, kErrInvalidArg);
+    }
+    doc_len_s[tid] = len;
+    doc_base_s[tid] = base;
+  }
+  if (tid == 0) {
+    // s_free and p_full collect one arrival per softmax warp; the rest one arrival each
+    for (int i = 0; i < N_BAR; ++i) mbar_init(&bars[i], (i >= 7 && i <= 10) ? 4 : 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_base_s, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid == 0) {
+    int acc = 0;
+    for (int d = 0; d < k; ++d) {
+      tile_start[d] = acc;
+      acc += (doc_len_s[d] + TN - 1) / TN;
+    }
+    tile_start[k] = acc;
+    tile_start[k + 1] = acc + (i_max + 1 + TN - 1) / TN;
+  }
+  __syncthreads();
+  const int T = tile_start[k + 1];
+  const uint32_t tmem = *tmem_base_s;
+  const uint32_t sbase = smem_addr(sm);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_bk);
+      prefetch_tensormap(&tm_bv);
+      prefetch_tensormap(&tm_lk);
+      prefetch_tensormap(&tm_lv);
+      const uint64_t pol = l2_policy_evict_last();  // the problem's other CTAs read the same tiles
+      // query tile: two 64-row segments x two 64-dim boxes
+      mbar_arrive_expect_tx(q_full, TILE);
+#pragma unroll
+      for (int sg = 0; sg < 2; ++sg) {
+        const int r = row0 + 64 * sg;
+        const int hq = h * G + r / Bq;
+        const int y = (int)(((int64_t)b * a.n_q_heads + hq) * a.q_tokens + (int64_t)blk * Bq + r % Bq);
+#pragma unroll
+        for (int dh = 0; dh < 2; ++dh)
+          tma_load_2d(sm + OFF_Q + dh * BOX + sg * (64 * 128), &tm_q, dh * 64, y, q_full, pol);
+      }
+      int di = 0;
+      for (int n = 0; n < T; ++n) {
+        const int st = n & 1, use = n >> 1;
+        if (use > 0 && !mbar_wait_bounded(&kv_empty[st], (use - 1) & 1, a.err)) break;
+        while (di < k && n >= tile_start[di + 1]) ++di;
+        const int tt = n - tile_start[di];
+        const CUtensorMap *mk, *mv;
+        int y;
+        if (di < k) {
+          mk = &tm_bk; mv = &tm_bv;
+          y = (int)(doc_base_s[di] + (long long)tt * TN);
+        } else {
+          mk = &tm_lk; mv = &tm_lv;
+          y = (b * a.n_kv_heads + h) * a.local_len + tt * TN;
+        }
+        uint8_t* kd = sm + OFF_K0 + st * 2 * TILE;
+        mbar_arrive_expect_tx(&kv_full[st], 2 * TILE);
+#pragma unroll
+        for (int dh = 0; dh < 2; ++dh) {
+          tma_load_2d(kd + dh * BOX, mk, dh * 64, y, &kv_full[st], pol);
+          tma_load_2d(kd + TILE + dh * BOX, mv, dh * 64, y, &kv_full[st], pol);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = umma_idesc_bf16(TM, TN, false);
+      const uint32_t idesc_pv = umma_idesc_bf16(TM, TD, true);
+      bool ok = mbar_wait_bounded(q_full, 0, a.err);
+      auto issue_pv = [&](int i) -> bool {
+        if (!mbar_wait_bounded(&p_full[i & 1], (i >> 1) & 1, a.err)) return false;
+        tc_fence_after();
+        const uint32_t pa = sbase + OFF_P0 + (i & 1) * TILE;
+        const uint32_t vb = sbase + OFF_K0 + (i & 1) * 2 * TILE + TILE;
+#pragma unroll
+        for (int kk = 0; kk < TN / 16; ++kk) {
+          const uint64_t ad = umma_desc_sw128(pa + (kk >> 2) * BOX + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = umma_desc_sw128(vb + kk * 2048, BOX, 1024);
+          umma_bf16_ss(tmem + O_COL, ad, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&kv_empty[i & 1]);
+        umma_commit(&p_free[i & 1]);
+        return true;
+      };
+      for (int j = 0; ok && j < T; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait_bounded(&kv_full[st], (j >> 1) & 1, a.err)) break;
+        if (j >= 2 && !mbar_wait_bounded(&s_free[j & 1], ((j - 2) >> 1) & 1, a.err)) break;
+        tc_fence_after();
+        const uint32_t qa = sbase + OFF_Q;
+        const uint32_t kb = sbase + OFF_K0 + st * 2 * TILE;
+#pragma unroll
+        for (int ks = 0; ks < TD / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * BOX + (ks & 3) * 32;
+          umma_bf16_ss(tmem + (j & 1) * TN, umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024),
+                       idesc_qk, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[j & 1]);
+        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok && T > 0) issue_pv(T - 1);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int r = (warp - 4) * 32 + lane;         // row inside the CTA tile = TMEM lane
+    const int R = row0 + r;                        // row of the problem
+    const int g = R / Bq, t_in = R % Bq;
+    const int lim = i_first + t_in;                // causal limit among local keys
+    const uint32_t tl = tmem + ((uint32_t)((warp - 4) * 32) << 16);
+    float m_ref = -INFINITY, l = 0.f;
+    int di = 0;
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      if (!mbar_wait_bounded(&s_full[j & 1], (j >> 1) & 1, a.err)) { ok = false; break; }
+      tc_fence_after();
+      while (di < k && j >= tile_start[di + 1]) ++di;
+      const bool local = di >= k;
+      const int key0 = (j - tile_start[di]) * TN;
+      const int nvalid = local ? TN : min(TN, doc_len_s[di] - key0);
+      const int vis_end = local ? max(0, min(TN, lim - key0 + 1)) : nvalid;  // keys [0, vis_end) are visible
+      const uint32_t scol = tl + (j & 1) * TN;
+      // pass 1: tile max
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < TN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(scol + c * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (c * 32 + e < vis_end) mt = fmaxf(mt, __uint_as_float(v[e]) * a.scale_log2);
+      }
+      const float m_new = fmaxf(m_ref, mt);
+      const bool need = m_new > m_ref + kLazy;  // also true when m_ref = -inf and the tile has a key
+      float alpha = 1.f;
+      if (need) {
+        alpha = exp2f(m_ref - m_new);  // 0 when m_ref = -inf
+        l *= alpha;
+        m_ref = m_new;
+      }
+      if (__any_sync(0xffffffffu, need && j > 0)) {
+        // O holds the sum up to tile j-1: wait for that P V, then rescale this warp's rows
+        if (!mbar_wait_bounded(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < TD / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tl + O_COL + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tl + O_COL + c * 32, o);
+        }
+        tmem_wait_st();
+      }
+      if (j >= 2 && !mbar_wait_bounded(&p_free[j & 1], ((j - 2) >> 1) & 1, a.err)) { ok = false; break; }
+      // pass 2: P = exp2(S * scale - m_ref) as bf16, K-major 128-byte-swizzled rows
+      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      uint8_t* prow = sm + OFF_P0 + (j & 1) * TILE;
+#pragma unroll
+      for (int c = 0; c < TN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(scol + c * 32, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float p0 = (c * 32 + e < vis_end) ? exp2f(__uint_as_float(v[e]) * a.scale_log2 - m_use) : 0.f;
+          const float p1 = (c * 32 + e + 1 < vis_end) ? exp2f(__uint_as_float(v[e + 1]) * a.scale_log2 - m_use) : 0.f;
+          l += p0 + p1;
+          pk[e >> 1] = pack_bf16(p0, p1);
+        }
+        uint8_t* box = prow + (c >> 1) * BOX;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(box + swz128(r, (c & 1) * 4 + q)) =
+              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      }
+      fence_proxy_async();  // P is read by the tensor cores (async proxy)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&p_full[j & 1]);
+        mbar_arrive(&s_free[j & 1]);
+      }
+    }
+    // ---- epilogue: O / l once the last P V has completed
+    if (ok && T > 0 && mbar_wait_bounded(&p_free[(T - 1) & 1], ((T - 1) >> 1) & 1, a.err)) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.0f / l : 0.f;
+      const int hq = h * G + g;
+      const int t = blk * Bq + t_in;
+      float* dst = a.out + (((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t) * TD;
+#pragma unroll
+      for (int c = 0; c < TD / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tl + O_COL + c * 32, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dst + c * 32 + e) =
+              make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                          __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+      }
+    }
+  }
+  // ---- teardown: every role is done with TMEM and shared memory
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+}  // namespace
+
+bool attend_prefill_tc_supported(int head_dim, int group, int route_block) {
+  return head_dim == TD && (route_block == 64 || route_block == 128) && (group * route_block) % TM == 0;
+}
+int attend_prefill_tc_tile_rows() { return TN; }
+
+cudaError_t launch_attend_prefill_tc(const AttendArgs& a, const AttendMaps& m, const CUtensorMap& q_map,
+                                     cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(attend_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int nblk = a.q_tokens / a.route_block;
+  const int rows = (a.n_q_heads / a.n_kv_heads) * a.route_block;
+  dim3 grid(rows / TM, a.batch * nblk * a.n_kv_heads);
+  attend_prefill_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(q_map, m.bank_k, m.bank_v, m.loc_k, m.loc_v, a);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

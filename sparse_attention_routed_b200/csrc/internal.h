@@ -99,9 +99,16 @@ cudaError_t launch_attend_decode(const AttendArgs& a, const AttendMaps& m, int h
 // Many-row problems (G * route_block > 16); loc_k must map the RoPE'd local keys.
 cudaError_t launch_attend_prefill(const AttendArgs& a, const AttendMaps& m, int head_dim, cudaStream_t s);
 int attend_prefill_tile_rows();
-// out[row] = Global RoPE of lk[row] at k_off + (row % local_len) (rows = B * Hkv * Lc).
-cudaError_t launch_rope_local(const uint16_t* lk, uint16_t* out, const float2* gtab, int64_t rows, int local_len,
-                              int head_dim, cudaStream_t s);
+// out[row] = Global RoPE of in[row] at local index offset + row % period (gtab row).
+cudaError_t launch_rope_rows(const uint16_t* in, uint16_t* out, const float2* gtab, int64_t rows, int period,
+                             int offset, int head_dim, cudaStream_t s);
+// tcgen05/TMEM prefill for head_dim 128, routing blocks of 64 or 128 tokens and
+// G * route_block a multiple of 128; loc_k must map the RoPE'd local keys and
+// q_map the RoPE'd queries [B * Hq * Tq, 128] in boxes of 64 x 64.
+bool attend_prefill_tc_supported(int head_dim, int group, int route_block);
+int attend_prefill_tc_tile_rows();
+cudaError_t launch_attend_prefill_tc(const AttendArgs& a, const AttendMaps& m, const CUtensorMap& q_map,
+                                     cudaStream_t s);
 
 // Device pointers and sizes of a bank that the routing kernels read.
 struct BankRouteView {

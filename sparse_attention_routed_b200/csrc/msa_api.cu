@@ -124,7 +124,8 @@ struct msa_bank {
   size_t ws_cap = 0;
   // TMA descriptors of the bank K/V (device tier) and of the router operands
   CUtensorMap map_k{}, map_v{};      // boxes of the decode kernel's tile
-  CUtensorMap map_k64{}, map_v64{};  // boxes of the prefill kernel's tile
+  CUtensorMap map_k64{}, map_v64{};  // boxes of the mma.sync prefill kernel's tile
+  CUtensorMap map_k128{}, map_v128{};  // boxes of the tcgen05 prefill kernel's tile
   RouteMaps route_maps{};
   std::vector<void*> owned;
 };
@@ -207,6 +208,7 @@ struct Workspace {
   float* part_o;
   float* part_ml;
   uint16_t* local_rot;  // prefill: local keys with Global RoPE applied
+  uint16_t* q_rot;      // tcgen05 prefill: queries with Global RoPE applied
   size_t bytes;
 };
 
@@ -230,6 +232,8 @@ Workspace layout(const msa_bank* bank, const StepShape& s, int splits, uint8_t* 
   w.part_o = (float*)take(prefill ? 0 : (size_t)s.P * splits * s.rows * bank->d * 4);
   w.part_ml = (float*)take(prefill ? 0 : (size_t)s.P * splits * s.rows * 2 * 4);
   w.local_rot = (uint16_t*)take(prefill ? (size_t)s.B * bank->hkv * s.Lc * bank->d * 2 : 0);
+  const bool tc = prefill && attend_prefill_tc_supported(bank->d, s.G, s.Bq);
+  w.q_rot = (uint16_t*)take(tc ? (size_t)s.B * s.Hq * s.Tq * bank->d * 2 : 0);
   w.bytes = off;
   return w;
 }
@@ -307,12 +311,21 @@ msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, co
 msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, int splits, const Workspace& w,
                        const int32_t* idx, float* out, cudaStream_t st) {
   const bool prefill = s.rows > kMaxRows;
-  const int box = prefill ? attend_prefill_tile_rows() : attend_tile_rows();
+  const bool tc = prefill && attend_prefill_tc_supported(bank->d, s.G, s.Bq);
+  const int box = tc ? attend_prefill_tc_tile_rows() : prefill ? attend_prefill_tile_rows() : attend_tile_rows();
   const int64_t lrows = (int64_t)s.B * bank->hkv * s.Lc;
   AttendMaps maps;
-  maps.bank_k = prefill ? bank->map_k64 : bank->map_k;
-  maps.bank_v = prefill ? bank->map_v64 : bank->map_v;
-  if (prefill) MSA_CUDA(launch_rope_local((const uint16_t*)q->local_k, w.local_rot, bank->d_gtab, lrows, s.Lc, bank->d, st));
+  maps.bank_k = tc ? bank->map_k128 : prefill ? bank->map_k64 : bank->map_k;
+  maps.bank_v = tc ? bank->map_v128 : prefill ? bank->map_v64 : bank->map_v;
+  if (prefill)
+    MSA_CUDA(launch_rope_rows((const uint16_t*)q->local_k, w.local_rot, bank->d_gtab, lrows, s.Lc, 0, bank->d, st));
+  CUtensorMap q_map{};
+  if (tc) {
+    const int64_t qrows = (int64_t)s.B * s.Hq * s.Tq;
+    MSA_CUDA(launch_rope_rows((const uint16_t*)q->q, w.q_rot, bank->d_gtab, qrows, s.Tq, s.Lc - s.Tq, bank->d, st));
+    msa_status r0 = make_map(&q_map, w.q_rot, qrows, bank->d, 64);
+    if (r0 != MSA_OK) return r0;
+  }
   msa_status rc = make_map(&maps.loc_k, prefill ? (const void*)w.local_rot : q->local_k, lrows, bank->d, box);
   if (rc != MSA_OK) return rc;
   rc = make_map(&maps.loc_v, q->local_v, lrows, bank->d, box);
@@ -339,7 +352,9 @@ msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, i
   a.n_docs = bank->n_docs;
   a.n_splits = splits;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)bank->d));
-  if (prefill) {
+  if (tc) {
+    MSA_CUDA(launch_attend_prefill_tc(a, maps, q_map, st));
+  } else if (prefill) {
     MSA_CUDA(launch_attend_prefill(a, maps, bank->d, st));
   } else {
     MSA_CUDA(launch_attend_decode(a, maps, bank->d, st));
@@ -470,6 +485,12 @@ msa_status msa_bank_create(const msa_bank_config* cfg, msa_bank** out) {
     if ((rc = make_map(&b->map_k64, b->k, (int64_t)b->hkv * b->kv_rows, b->d, attend_prefill_tile_rows())) != MSA_OK)
       return fail(rc);
     if ((rc = make_map(&b->map_v64, b->v, (int64_t)b->hkv * b->kv_rows, b->d, attend_prefill_tile_rows())) != MSA_OK)
+      return fail(rc);
+    if ((rc = make_map(&b->map_k128, b->k, (int64_t)b->hkv * b->kv_rows, b->d, attend_prefill_tc_tile_rows())) !=
+        MSA_OK)
+      return fail(rc);
+    if ((rc = make_map(&b->map_v128, b->v, (int64_t)b->hkv * b->kv_rows, b->d, attend_prefill_tc_tile_rows())) !=
+        MSA_OK)
       return fail(rc);
   }
   *out = b;
