@@ -43,7 +43,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "decode_512k", "prefill"],
+    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "decode_512k", "prefill", "prefill_64docs"],
                     help="decode_512k: the same step on a 128-document bank (profiling captures); "
                          "prefill: 4096 query tokens in 64-token routing blocks (tensor-bound)")
     ap.add_argument("--route-only", action="store_true",
@@ -238,7 +238,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
     w = synth.WORKLOADS[args.workload]
-    prefill = args.workload == "prefill"
+    prefill = args.workload.startswith("prefill")
     K, V, R = bank_tensors(w)
     bank = Bank(K, V, w.doc_lens(), w.rope_base)
     bank.build(R)

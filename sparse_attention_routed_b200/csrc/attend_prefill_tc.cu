@@ -14,8 +14,10 @@
 //              S_j = Q K_j^T (M = N = K = 128, into one of two S buffers) and
 //              then O += P_{j-1} V_{j-1} (P from shared memory, V read as an
 //              MN-major operand), and commits each group to an mbarrier.
-//   warps 4-7  softmax, one thread per row (TMEM lane = row): read S_j with
-//              tcgen05.ld, mask (document tails, causal local keys), write
+//   warps 2-9  softmax, two warpgroups: each row is split over two threads,
+//              one per 64-key half (TMEM lane = row); they read S_j with
+//              tcgen05.ld, mask (document tails, causal local keys), exchange
+//              half-row maxima through shared memory, and write
 //              P_j = exp2(S_j * scale - m) as bf16 into a 128-byte-swizzled
 //              K-major tile. The reference max m of a row moves only when the
 //              row max rises by more than 2^8; then the row of O is rescaled in
@@ -33,7 +35,7 @@ constexpr int TM = 128;               // query rows per CTA
 constexpr int TD = 128;               // head dim
 constexpr int TMEM_COLS = 512;        // S0 [0,128) S1 [128,256) O [256,384)
 constexpr int O_COL = 256;
-constexpr int THREADS = 256;
+constexpr int THREADS = 320;           // producer, MMA, 8 softmax warps
 constexpr int BOX = TN * 128;         // one 64-element-wide box of a 128-row tile (16 KB)
 constexpr int TILE = 2 * BOX;         // 128 x 128 bf16 (32 KB)
 constexpr int TOPK_MAX = 64;
@@ -46,7 +48,10 @@ constexpr int OFF_P0 = OFF_K0 + 4 * TILE;      // P[b] = OFF_P0 + b * TILE
 constexpr int OFF_BAR = OFF_P0 + 2 * TILE;
 constexpr int N_BAR = 13;
 constexpr int OFF_TMEM = OFF_BAR + N_BAR * 8;
-constexpr int OFF_TAB = OFF_TMEM + 8;
+constexpr int OFF_TAB = OFF_TMEM + 16;
+// TMEM columns used to exchange per-row values between the two softmax warpgroups
+constexpr int MX_COL = 384;   // + 2 * parity + warpgroup: half-row maxima
+constexpr int L_COL = 388;    // + warpgroup: half-row sums
 constexpr size_t SMEM_BYTES = 1024 + OFF_TAB + (TOPK_MAX + 2) * 4 + TOPK_MAX * 4 + TOPK_MAX * 8;
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 
@@ -65,6 +70,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* p_full = bars + 9;     // [2]
   uint64_t* p_free = bars + 11;    // [2]
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
+  int* abort_s = reinterpret_cast<int*>(sm + OFF_TMEM + 4);   // set when a wait expired: softmax warps stop together
+
   int* tile_start = reinterpret_cast<int*>(sm + OFF_TAB);
   int* doc_len_s = tile_start + TOPK_MAX + 2;
   long long* doc_base_s = reinterpret_cast<long long*>(doc_len_s + TOPK_MAX);
@@ -98,8 +105,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   if (tid == 0) {
     // s_free and p_full collect one arrival per softmax warp; the rest one arrival each
-    for (int i = 0; i < N_BAR; ++i) mbar_init(&bars[i], (i >= 7 && i <= 10) ? 4 : 1);
+    for (int i = 0; i < N_BAR; ++i) mbar_init(&bars[i], (i >= 7 && i <= 10) ? 8 : 1);
     fence_barrier_init();
+    *abort_s = 0;
   }
   if (warp == 1) tmem_alloc(tmem_base_s, TMEM_COLS);
   tc_fence_before();
@@ -202,36 +210,61 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (ok && T > 0) issue_pv(T - 1);
     }
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------------------ softmax
-    const int r = (warp - 4) * 32 + lane;         // row inside the CTA tile = TMEM lane
+    // warps 2..9 = two warpgroups; warpgroup wg takes keys [64 wg, 64 wg + 64)
+    // of every row, warp w reads TMEM lanes 32 (w % 4) .. +31 (its rows).
+    const int wg = (warp - 2) >> 2;
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;                  // row inside the CTA tile = TMEM lane
     const int R = row0 + r;                        // row of the problem
     const int g = R / Bq, t_in = R % Bq;
     const int lim = i_first + t_in;                // causal limit among local keys
-    const uint32_t tl = tmem + ((uint32_t)((warp - 4) * 32) << 16);
+    const int c0 = wg * (TN / 2);                  // this warpgroup's first key / S column
+    const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     float m_ref = -INFINITY, l = 0.f;
     int di = 0;
-    bool ok = true;
     for (int j = 0; j < T; ++j) {
-      if (!mbar_wait_bounded(&s_full[j & 1], (j >> 1) & 1, a.err)) { ok = false; break; }
+      bool okw = mbar_wait_bounded(&s_full[j & 1], (j >> 1) & 1, a.err);
+      if (j >= 2) okw = okw && mbar_wait_bounded(&p_free[j & 1], ((j - 2) >> 1) & 1, a.err);  // P buffer reusable
       tc_fence_after();
       while (di < k && j >= tile_start[di + 1]) ++di;
       const bool local = di >= k;
       const int key0 = (j - tile_start[di]) * TN;
       const int nvalid = local ? TN : min(TN, doc_len_s[di] - key0);
       const int vis_end = local ? max(0, min(TN, lim - key0 + 1)) : nvalid;  // keys [0, vis_end) are visible
-      const uint32_t scol = tl + (j & 1) * TN;
-      // pass 1: tile max
-      float mt = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < TN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(scol + c * 32, v);
+      uint32_t v0[32], v1[32];  // S of keys c0 .. c0+31 and c0+32 .. c0+63
+      {
+        const uint32_t scol = tl + (j & 1) * TN + c0;
+        tmem_ld32(scol, v0);
+        tmem_ld32(scol + 32, v1);
         tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (c * 32 + e < vis_end) mt = fmaxf(mt, __uint_as_float(v[e]) * a.scale_log2);
       }
+#define SV(e) __uint_as_float((e) < 32 ? v0[(e) & 31] : v1[(e) & 31])
+      // every key of this half visible for every row of the warp: no per-key masks
+      const bool full = __all_sync(0xffffffffu, vis_end >= c0 + TN / 2);
+      float mt;
+      if (full) {
+        float m4[4] = {SV(0), SV(1), SV(2), SV(3)};
+#pragma unroll
+        for (int e = 4; e < TN / 2; ++e) m4[e & 3] = fmaxf(m4[e & 3], SV(e));
+        mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale_log2;
+      } else {
+        mt = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < TN / 2; ++e)
+          if (c0 + e < vis_end) mt = fmaxf(mt, SV(e));
+        mt = (mt == -INFINITY) ? mt : mt * a.scale_log2;
+      }
+      tmem_st1(tl + MX_COL + (j & 1) * 2 + wg, __float_as_uint(mt));
+      tmem_wait_st();
+      if (!okw) *abort_s = 1;
+      tc_fence_before();
+      named_barrier_sync(1, 2 * 4 * 32);
+      tc_fence_after();
+      if (*abort_s) break;
+      mt = fmaxf(mt, __uint_as_float(tmem_ld1(tl + MX_COL + (j & 1) * 2 + (wg ^ 1))));
+      tmem_wait_ld();
       const float m_new = fmaxf(m_ref, mt);
       const bool need = m_new > m_ref + kLazy;  // also true when m_ref = -inf and the tile has a key
       float alpha = 1.f;
@@ -240,43 +273,46 @@ __global__ void __launch_bounds__(THREADS, 1)
         l *= alpha;
         m_ref = m_new;
       }
+      // P = exp2(S * scale - m_ref) as bf16 into this warpgroup's 64-key box of the K-major tile
+      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      uint8_t* box = sm + OFF_P0 + (j & 1) * TILE + wg * BOX;
+      const float sc = a.scale_log2;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = q * 8 + 2 * u;
+          float p0 = ex2_approx(fmaf(SV(e), sc, -m_use));
+          float p1 = ex2_approx(fmaf(SV(e + 1), sc, -m_use));
+          if (!full) {
+            p0 = (c0 + e < vis_end) ? p0 : 0.f;
+            p1 = (c0 + e + 1 < vis_end) ? p1 : 0.f;
+          }
+          ls[u] += p0 + p1;
+          pk[u] = pack_bf16(p0, p1);
+        }
+        *reinterpret_cast<uint4*>(box + swz128(r, q)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+#undef SV
+      // (after P, so that S is no longer live) the rescale must land before P V of this tile
       if (__any_sync(0xffffffffu, need && j > 0)) {
-        // O holds the sum up to tile j-1: wait for that P V, then rescale this warp's rows
-        if (!mbar_wait_bounded(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err)) { ok = false; break; }
+        // O holds the sum up to tile j-1: wait for that P V, then rescale this
+        // warp's rows in this warpgroup's half of the O columns
+        if (!mbar_wait_bounded(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err)) *abort_s = 1;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < TD / 32; ++c) {
+        for (int c = 0; c < TD / 64; ++c) {
           uint32_t o[32];
-          tmem_ld32(tl + O_COL + c * 32, o);
+          tmem_ld32(tl + O_COL + c0 + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tl + O_COL + c * 32, o);
+          tmem_st32(tl + O_COL + c0 + c * 32, o);
         }
         tmem_wait_st();
-      }
-      if (j >= 2 && !mbar_wait_bounded(&p_free[j & 1], ((j - 2) >> 1) & 1, a.err)) { ok = false; break; }
-      // pass 2: P = exp2(S * scale - m_ref) as bf16, K-major 128-byte-swizzled rows
-      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      uint8_t* prow = sm + OFF_P0 + (j & 1) * TILE;
-#pragma unroll
-      for (int c = 0; c < TN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(scol + c * 32, v);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float p0 = (c * 32 + e < vis_end) ? exp2f(__uint_as_float(v[e]) * a.scale_log2 - m_use) : 0.f;
-          const float p1 = (c * 32 + e + 1 < vis_end) ? exp2f(__uint_as_float(v[e + 1]) * a.scale_log2 - m_use) : 0.f;
-          l += p0 + p1;
-          pk[e >> 1] = pack_bf16(p0, p1);
-        }
-        uint8_t* box = prow + (c >> 1) * BOX;
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          *reinterpret_cast<uint4*>(box + swz128(r, (c & 1) * 4 + q)) =
-              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       }
       fence_proxy_async();  // P is read by the tensor cores (async proxy)
       tc_fence_before();
@@ -286,17 +322,24 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_arrive(&s_free[j & 1]);
       }
     }
-    // ---- epilogue: O / l once the last P V has completed
-    if (ok && T > 0 && mbar_wait_bounded(&p_free[(T - 1) & 1], ((T - 1) >> 1) & 1, a.err)) {
+    // ---- epilogue: O / l once the last P V has completed; l sums both halves of the keys
+    tmem_st1(tl + L_COL + wg, __float_as_uint(l));
+    tmem_wait_st();
+    tc_fence_before();
+    named_barrier_sync(1, 2 * 4 * 32);
+    tc_fence_after();
+    const float lt = l + __uint_as_float(tmem_ld1(tl + L_COL + (wg ^ 1)));
+    tmem_wait_ld();
+    if (!*abort_s && T > 0 && mbar_wait_bounded(&p_free[(T - 1) & 1], ((T - 1) >> 1) & 1, a.err)) {
       tc_fence_after();
-      const float inv = l > 0.f ? 1.0f / l : 0.f;
+      const float inv = lt > 0.f ? 1.0f / lt : 0.f;
       const int hq = h * G + g;
       const int t = blk * Bq + t_in;
-      float* dst = a.out + (((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t) * TD;
+      float* dst = a.out + (((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t) * TD + c0;
 #pragma unroll
-      for (int c = 0; c < TD / 32; ++c) {
+      for (int c = 0; c < TD / 64; ++c) {
         uint32_t o[32];
-        tmem_ld32(tl + O_COL + c * 32, o);
+        tmem_ld32(tl + O_COL + c0 + c * 32, o);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; e += 4)

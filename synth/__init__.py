@@ -201,6 +201,8 @@ WORKLOADS = {
     # step, 2 GB of K/V on the device (for hardware-counter captures)
     "decode_512k": Workload("decode_512k", 1, 8, 32, 8, 128, 128, 4096, 4096, 1, 1, 16),
     "prefill": Workload("prefill", 2, 1, 32, 8, 128, 256, 8192, 4096, 4096, 64, 8),
+    # the prefill step on a 64-document bank: same work per CTA, 2 GB of K/V (hardware-counter captures)
+    "prefill_64docs": Workload("prefill_64docs", 2, 1, 32, 8, 128, 64, 8192, 4096, 4096, 64, 8),
     "ragged_planted": Workload("ragged_planted", 3, 4, 64, 8, 128, 8192, 0, 2048, 1, 1, 32,
                                ragged=(512, 16384), planted=4, host_tier=True),
     "bank_100m": Workload("bank_100m", 4, 16, 32, 8, 128, 24414, 4096, 4096, 1, 1, 16,
