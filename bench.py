@@ -43,7 +43,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "decode_512k", "prefill", "prefill_64docs"],
+    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "decode_512k", "prefill", "prefill_64docs", "ragged_planted", "bank_100m"],
                     help="decode_512k: the same step on a 128-document bank (profiling captures); "
                          "prefill: 4096 query tokens in 64-token routing blocks (tensor-bound)")
     ap.add_argument("--route-only", action="store_true",
@@ -452,12 +452,111 @@ def run_route_only(args):
     bank.close()
 
 
+def run_host_tier(args):
+    """Decode steps on a bank whose K/V live in pinned host memory (69M / 100M tokens):
+    route on the device, copy the selected documents' K/V slabs over PCIe, attend."""
+    import torch
+
+    import synth
+    from sparse_attention_routed_b200 import MSA_KV_PINNED_HOST, msa_attend, msa_route
+    from sparse_attention_routed_b200.runner import Bank
+    from synth.device import fill_normal, host_kv_pool, query_tensors
+
+    w = synth.WORKLOADS[args.workload]
+    Hkv, d, B, k = w.n_kv_heads, w.head_dim, w.batch, w.top_k
+    t0 = time.time()
+    Kh, Vh = host_kv_pool(w)
+    bank = Bank(Kh, Vh, w.doc_lens(), w.rope_base, kv_location=MSA_KV_PINNED_HOST, doc_rows=w.doc_kv_rows())
+    lens = w.doc_lens()
+    off = np.concatenate([[0], np.cumsum(lens)])
+    for j0 in range(0, w.n_docs, 64):          # routing keys streamed through the build
+        j1 = min(w.n_docs, j0 + 64)
+        T = int(off[j1] - off[j0])
+        R = torch.empty((Hkv, T, d), dtype=torch.bfloat16, device="cuda")
+        for h in range(Hkv):
+            fill_normal(R[h], w.seed, synth.T_R, (h * w.n_tokens + int(off[j0])) * d)
+        bank.build(R, j0, j1, rope=False)
+        del R
+    torch.cuda.synchronize()
+    setup_s = time.time() - t0
+    Q, Qr, LK, LV = query_tensors(w)
+    qry = bank.query(Q, Qr, LK, LV, w.route_block)
+    idx = torch.empty((B, 1, Hkv, k), dtype=torch.int32, device="cuda")
+    out = torch.empty((B, w.n_q_heads, 1, d), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    for _ in range(max(3, args.warmup)):
+        msa_route(bank.handle, qry, k, 0, idx.data_ptr(), 0, sh)
+        msa_attend(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
+    torch.cuda.synchronize()
+    assert bank.device_error() == 0
+    sel = idx.cpu().numpy()
+    uniq = {(int(j), h) for b in range(B) for h in range(Hkv) for j in sel[b, 0, h]}
+    pcie_bytes = sum(int(lens[j]) for j, _ in uniq) * d * 2 * 2
+    recall = None
+    if w.planted:
+        tg = synth.planted_targets(w.seed, B, w.n_docs, w.planted)
+        recall = float(np.mean([tg[b, h % w.planted] in sel[b, 0, h] for b in range(B) for h in range(Hkv)]))
+    # pinned H2D reference bandwidth (1 GiB, best of 3)
+    hbuf = torch.empty(1 << 30, dtype=torch.uint8, pin_memory=True)
+    dbuf = torch.empty(1 << 30, dtype=torch.uint8, device="cuda")
+    best = 1e9
+    for _ in range(3):
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        dbuf.copy_(hbuf, non_blocking=True)
+        a1.record(stream)
+        a1.synchronize()
+        best = min(best, a0.elapsed_time(a1))
+    h2d_peak = (1 << 30) / (best / 1e3) / 1e9
+    del hbuf, dbuf
+    n = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    time.sleep(0.4)
+    torch.cuda.synchronize()
+    for i in range(n):
+        ev[i][0].record(stream)
+        msa_route(bank.handle, qry, k, 0, idx.data_ptr(), 0, sh)
+        ev[i][1].record(stream)
+        msa_attend(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    route_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / n
+    attend_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / n
+    step_ms = route_ms + attend_ms
+    router_bytes = Hkv * bank.info["n_chunks"] * d * 4
+    peak, kind = peaks()
+    line = {
+        "metric": f"decode queries/s, pinned-host K/V tier ({w.n_tokens / 1e6:.1f}M-token bank)",
+        "value": B / (step_ms / 1e3), "unit": "queries/s", "n_gpus": 1, "steps": n, "warmup": args.warmup,
+        "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": B, "q_heads": w.n_q_heads, "kv_heads": Hkv,
+                   "head_dim": d, "bank_docs": w.n_docs, "bank_tokens": w.n_tokens, "local_len": w.local_len,
+                   "top_k": k, "kv_slabs_pinned": w.kv_slabs, "pinned_kv_bytes": 2 * Kh.numel() * 2},
+        "roofline": {"kernel": "selected K/V slabs over PCIe (cudaMemcpyAsync per slab)", "bound": "pcie",
+                     "achieved": pcie_bytes / (attend_ms / 1e3) / 1e9, "peak": h2d_peak,
+                     "peak_kind": "measured pinned H2D copy, 1 GiB", "unit": "GB/s",
+                     "frac": pcie_bytes / (attend_ms / 1e3) / 1e9 / h2d_peak, "bytes_per_step": pcie_bytes},
+        "router": {"ms": route_ms, "bytes": router_bytes, "GBps": router_bytes / (route_ms / 1e3) / 1e9,
+                   "frac_of_hbm_peak": router_bytes / (route_ms / 1e3) / 1e9 / peak},
+        "planted_recall": recall, "setup_s": setup_s, "clocks": clk,
+        "gpu_launches": launches_per_step(w) * n,
+    }
+    print(json.dumps(line), flush=True)
+    bank.close()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
     elif args.route_only:
         run_route_only(args)
+    elif args.workload in ("ragged_planted", "bank_100m"):
+        run_host_tier(args)
     else:
         run_ours(args)
 

@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(S::THREADS, S::MINB)
     long long base = 0;
     if (j >= 0 && j < a.n_docs) {
       len = a.doc_len[j];
-      base = (long long)h * a.kv_rows + a.doc_row[j];
+      base = a.sel_base ? (long long)a.sel_base[(int64_t)p * k + tid] : (long long)h * a.kv_rows + a.doc_row[j];
     } else {
       atomicCAS(a.err, 0, kErrInvalidArg);
     }

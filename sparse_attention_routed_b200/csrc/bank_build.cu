@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(256) bank_build_kernel(BankBuildArgs a) {
   const int pos0 = a.chunk_pos[c];
 
   // ---- pooling: sum the chunk's rows in fp32, divide by its actual length
-  {
+  if (a.r != nullptr) {
     const int sub = lane / LANES_PER_ROW;   // which row of the pair/quad
     const int vec = lane % LANES_PER_ROW;   // which 8 dims
     const uint16_t* base = a.r + h * a.r_head_stride + tok0 * D + vec * 8;

@@ -79,6 +79,8 @@ struct AttendArgs {
   const uint16_t* q;        // [B, Hq, Tq, d]
   const int32_t* sel;       // [B*nblk*Hkv][top_k]
   const int64_t* doc_row;   // [n_docs] first row of the document inside each head's K/V
+  const int64_t* sel_base;  // [P][top_k] or nullptr: row of each selected (document, head) slab in the
+                            // K/V tensor maps (host tier: the device staging pool)
   const int32_t* doc_len;   // [n_docs]
   const float2* gtab;       // [Lc][d/2] Global RoPE (cos, sin) at k_off + u
   float* part_o;            // [P][S][rows][d]   rows = G * route_block

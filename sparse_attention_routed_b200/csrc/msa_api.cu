@@ -8,6 +8,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <unordered_map>
 #include <vector>
 
 #include "../../include/msa.h"
@@ -127,7 +128,18 @@ struct msa_bank {
   CUtensorMap map_k64{}, map_v64{};  // boxes of the mma.sync prefill kernel's tile
   CUtensorMap map_k128{}, map_v128{};  // boxes of the tcgen05 prefill kernel's tile
   RouteMaps route_maps{};
-  std::vector<void*> owned;
+  // pinned-host K/V tier: selected slabs are copied into a device staging pool
+  static constexpr int kSide = 4;    // copies round-robin over several streams (copy engines)
+  cudaStream_t side[kSide] = {};
+  cudaEvent_t ev_fetch[kSide] = {};
+  int32_t* h_idx = nullptr;   // pinned copy of the selection
+  int64_t* h_base = nullptr;  // pinned staging row of every selection entry
+  int64_t* d_base = nullptr;  // device copy of h_base
+  size_t sel_cap = 0;         // entries of h_idx / h_base / d_base
+  uint16_t* stage_k = nullptr;
+  uint16_t* stage_v = nullptr;
+  int64_t stage_cap = 0;      // rows of stage_k / stage_v
+  int64_t last_fetch_bytes = 0;
 };
 
 namespace {
@@ -135,6 +147,15 @@ namespace {
 void free_bank(msa_bank* b) {
   if (!b) return;
   cudaDeviceSynchronize();
+  for (int i = 0; i < msa_bank::kSide; ++i) {
+    if (b->side[i]) cudaStreamDestroy(b->side[i]);
+    if (b->ev_fetch[i]) cudaEventDestroy(b->ev_fetch[i]);
+  }
+  if (b->h_idx) cudaFreeHost(b->h_idx);
+  if (b->h_base) cudaFreeHost(b->h_base);
+  if (b->d_base) cudaFree(b->d_base);
+  if (b->stage_k) cudaFree(b->stage_k);
+  if (b->stage_v) cudaFree(b->stage_v);
   void* ptrs[] = {b->d_doc_row, b->d_doc_len, b->d_chunk_off, b->d_chunk_tok, b->d_chunk_len,
                   b->d_chunk_pos, b->d_ptab, b->d_kr, b->d_kr_inv, b->d_khi, b->d_klo, b->d_err, b->d_gtab, b->ws};
   for (void* p : ptrs)
@@ -169,7 +190,6 @@ msa_status check_query(const msa_bank* bank, const msa_query* q, int top_k, Step
     if (!q->q || !q->local_k || !q->local_v) return MSA_ERR_INVALID_ARG;
     if (!aligned16(q->q) || !aligned16(q->local_k) || !aligned16(q->local_v)) return MSA_ERR_INVALID_ARG;
     if ((int64_t)s->B * bank->hkv * s->Lc >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
-    if (bank->kv_loc != MSA_KV_DEVICE) return MSA_ERR_UNSUPPORTED;
   }
   if ((int64_t)s->B * s->nblk > 65535 || s->P > 65535) return MSA_ERR_UNSUPPORTED;
   return MSA_OK;
@@ -308,6 +328,93 @@ msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, co
   return MSA_OK;
 }
 
+// Pinned-host tier ("MSA (Memory Sparse Attention)", robocikowo.com, Komponenty:
+// K_r in GPU memory, full K/V in CPU RAM; Pułapki implementacyjne: pinned memory
+// and asynchronous prefetch). The selection is read back, every distinct
+// (document, KV head) slab it names is copied from pinned host memory into the
+// device staging pool on the bank's side streams (one cudaMemcpyAsync per slab
+// and per K/V, round-robin over the streams so that copy engines overlap their
+// per-copy costs), and `st` waits for the copies. Returns the staging row of every
+// selection entry in bank->d_base. Host-synchronising: not capturable.
+msa_status host_fetch(msa_bank* bank, const StepShape& s, const int32_t* idx_dev, cudaStream_t st) {
+  const size_t n = (size_t)s.P * s.k;
+  if (!bank->side[0]) {
+    for (int i = 0; i < msa_bank::kSide; ++i) {
+      MSA_CUDA(cudaStreamCreateWithFlags(&bank->side[i], cudaStreamNonBlocking));
+      MSA_CUDA(cudaEventCreateWithFlags(&bank->ev_fetch[i], cudaEventDisableTiming));
+    }
+  }
+  if (n > bank->sel_cap) {
+    MSA_CUDA(cudaDeviceSynchronize());
+    if (bank->h_idx) cudaFreeHost(bank->h_idx);
+    if (bank->h_base) cudaFreeHost(bank->h_base);
+    if (bank->d_base) cudaFree(bank->d_base);
+    bank->h_idx = nullptr;
+    bank->h_base = nullptr;
+    bank->d_base = nullptr;
+    bank->sel_cap = 0;
+    if (cudaHostAlloc(&bank->h_idx, n * 4, cudaHostAllocDefault) != cudaSuccess) return MSA_ERR_HOST_TIER;
+    if (cudaHostAlloc(&bank->h_base, n * 8, cudaHostAllocDefault) != cudaSuccess) return MSA_ERR_HOST_TIER;
+    MSA_CUDA(cudaMalloc(&bank->d_base, n * 8));
+    bank->sel_cap = n;
+  }
+  MSA_CUDA(cudaMemcpyAsync(bank->h_idx, idx_dev, n * 4, cudaMemcpyDeviceToHost, st));
+  MSA_CUDA(cudaStreamSynchronize(st));  // also retires every earlier step that read the staging pool
+  std::unordered_map<int64_t, int64_t> slot;
+  slot.reserve(n * 2);
+  std::vector<std::pair<int64_t, int64_t>> uniq;  // (doc * Hkv + head, staging row)
+  int64_t rows = 0;
+  for (size_t e = 0; e < n; ++e) {
+    const int p = (int)(e / s.k);
+    const int h = p % bank->hkv;
+    const int j = bank->h_idx[e];
+    if (j < 0 || j >= bank->n_docs) return MSA_ERR_INVALID_ARG;
+    const int64_t key = (int64_t)j * bank->hkv + h;
+    auto it = slot.find(key);
+    if (it == slot.end()) {
+      it = slot.emplace(key, rows).first;
+      uniq.emplace_back(key, rows);
+      rows += bank->doc_lens[j];
+    }
+    bank->h_base[e] = it->second;
+  }
+  if (rows >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  if (rows > bank->stage_cap) {
+    if (capturing(st)) return MSA_ERR_INVALID_ARG;
+    if (bank->stage_k) cudaFree(bank->stage_k);
+    if (bank->stage_v) cudaFree(bank->stage_v);
+    bank->stage_k = bank->stage_v = nullptr;
+    bank->stage_cap = 0;
+    const size_t bytes = (size_t)rows * bank->d * 2;
+    if (cudaMalloc(&bank->stage_k, bytes) != cudaSuccess || cudaMalloc(&bank->stage_v, bytes) != cudaSuccess)
+      return MSA_ERR_OOM;
+    bank->stage_cap = rows;
+  }
+  const size_t row_bytes = (size_t)bank->d * 2;
+  const uint16_t* hk = static_cast<const uint16_t*>(bank->k);
+  const uint16_t* hv = static_cast<const uint16_t*>(bank->v);
+  int64_t bytes = 0;
+  int c = 0;
+  for (const auto& u : uniq) {
+    const int j = (int)(u.first / bank->hkv), h = (int)(u.first % bank->hkv);
+    const int64_t src = ((int64_t)h * bank->kv_rows + bank->doc_rows[j]) * bank->d;
+    const size_t len = (size_t)bank->doc_lens[j] * row_bytes;
+    if (cudaMemcpyAsync(bank->stage_k + u.second * bank->d, hk + src, len, cudaMemcpyHostToDevice,
+                        bank->side[c++ % msa_bank::kSide]) != cudaSuccess ||
+        cudaMemcpyAsync(bank->stage_v + u.second * bank->d, hv + src, len, cudaMemcpyHostToDevice,
+                        bank->side[c++ % msa_bank::kSide]) != cudaSuccess)
+      return MSA_ERR_HOST_TIER;
+    bytes += 2 * (int64_t)len;
+  }
+  MSA_CUDA(cudaMemcpyAsync(bank->d_base, bank->h_base, n * 8, cudaMemcpyHostToDevice, bank->side[0]));
+  for (int i = 0; i < msa_bank::kSide; ++i) {
+    MSA_CUDA(cudaEventRecord(bank->ev_fetch[i], bank->side[i]));
+    MSA_CUDA(cudaStreamWaitEvent(st, bank->ev_fetch[i], 0));
+  }
+  bank->last_fetch_bytes = bytes;
+  return MSA_OK;
+}
+
 msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, int splits, const Workspace& w,
                        const int32_t* idx, float* out, cudaStream_t st) {
   const bool prefill = s.rows > kMaxRows;
@@ -315,8 +422,17 @@ msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, i
   const int box = tc ? attend_prefill_tc_tile_rows() : prefill ? attend_prefill_tile_rows() : attend_tile_rows();
   const int64_t lrows = (int64_t)s.B * bank->hkv * s.Lc;
   AttendMaps maps;
-  maps.bank_k = tc ? bank->map_k128 : prefill ? bank->map_k64 : bank->map_k;
-  maps.bank_v = tc ? bank->map_v128 : prefill ? bank->map_v64 : bank->map_v;
+  const int64_t* sel_base = nullptr;
+  if (bank->kv_loc == MSA_KV_PINNED_HOST) {
+    msa_status rf = host_fetch(bank, s, idx, st);
+    if (rf != MSA_OK) return rf;
+    if ((rf = make_map(&maps.bank_k, bank->stage_k, bank->stage_cap, bank->d, box)) != MSA_OK) return rf;
+    if ((rf = make_map(&maps.bank_v, bank->stage_v, bank->stage_cap, bank->d, box)) != MSA_OK) return rf;
+    sel_base = bank->d_base;
+  } else {
+    maps.bank_k = tc ? bank->map_k128 : prefill ? bank->map_k64 : bank->map_k;
+    maps.bank_v = tc ? bank->map_v128 : prefill ? bank->map_v64 : bank->map_v;
+  }
   if (prefill)
     MSA_CUDA(launch_rope_rows((const uint16_t*)q->local_k, w.local_rot, bank->d_gtab, lrows, s.Lc, 0, bank->d, st));
   CUtensorMap q_map{};
@@ -334,6 +450,7 @@ msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, i
   a.q = (const uint16_t*)q->q;
   a.sel = idx;
   a.doc_row = bank->d_doc_row;
+  a.sel_base = sel_base;
   a.doc_len = bank->d_doc_len;
   a.gtab = bank->d_gtab;
   a.part_o = w.part_o;
@@ -505,10 +622,10 @@ msa_status msa_bank_destroy(msa_bank* bank) {
 // Strides are in rows; a row is d * 2 >= 128 bytes, so every head of an aligned slice stays aligned.
 msa_status msa_build_bank(msa_bank* bank, int32_t doc_begin, int32_t doc_end, const void* r_slice,
                           int64_t r_head_stride, void* k_slice, int64_t k_head_stride, void* stream) {
-  if (!bank || !r_slice) return MSA_ERR_INVALID_ARG;
+  if (!bank || (!r_slice && !k_slice)) return MSA_ERR_INVALID_ARG;
   if (doc_begin < 0 || doc_end > bank->n_docs || doc_begin >= doc_end) return MSA_ERR_INVALID_ARG;
   const int64_t T = bank->doc_off[doc_end] - bank->doc_off[doc_begin];
-  if (r_head_stride < T || !aligned16(r_slice)) return MSA_ERR_INVALID_ARG;
+  if (r_slice && (r_head_stride < T || !aligned16(r_slice))) return MSA_ERR_INVALID_ARG;
   if (k_slice && (k_head_stride < T || !aligned16(k_slice))) return MSA_ERR_INVALID_ARG;
   const int64_t c0 = bank->chunk_off[doc_begin], c1 = bank->chunk_off[doc_end];
   if (c1 - c0 >= (int64_t(1) << 31) / bank->hkv) return MSA_ERR_UNSUPPORTED;

@@ -55,9 +55,10 @@ class Bank:
         else:
             k_ptr = ptr(K_slice, torch.bfloat16)
             k_stride = K_slice.shape[1]
-        assert R.is_contiguous() and R.dtype == torch.bfloat16
-        msa_build_bank(self.handle, doc_begin, doc_end, R.data_ptr(), R.shape[1], k_ptr, k_stride,
-                       _stream(stream))
+        if R is not None:
+            assert R.is_contiguous() and R.dtype == torch.bfloat16
+        msa_build_bank(self.handle, doc_begin, doc_end, 0 if R is None else R.data_ptr(),
+                       0 if R is None else R.shape[1], k_ptr, k_stride, _stream(stream))
 
     def k_r(self) -> torch.Tensor:
         """A copy of K_r [Hkv, n_chunks, d_r] fp32 (device)."""

@@ -135,6 +135,7 @@ class Workload:
     ragged: Optional[tuple] = None   # (lo, hi) inclusive, lengths not multiples of 256
     planted: int = 0                 # planted target docs per sequence
     host_tier: bool = False
+    kv_slabs: int = 0                # > 0: K/V of document j are the rows of slab (j mod kv_slabs)
     rope_base: float = 10000.0
     doc_lens_cache: Optional[np.ndarray] = field(default=None, repr=False)
 
@@ -153,6 +154,21 @@ class Workload:
     @property
     def n_tokens(self) -> int:
         return int(self.doc_lens().sum())
+
+    @property
+    def max_len(self) -> int:
+        return int(self.doc_lens().max())
+
+    @property
+    def kv_rows(self) -> int:
+        """Rows per head of the K/V tensors (the slab pool when aliased)."""
+        return self.kv_slabs * self.max_len if self.kv_slabs else self.n_tokens
+
+    def doc_kv_rows(self) -> np.ndarray:
+        """First K/V row of every document inside each head's K/V tensor."""
+        if self.kv_slabs:
+            return (np.arange(self.n_docs, dtype=np.int64) % self.kv_slabs) * self.max_len
+        return np.concatenate([[0], np.cumsum(self.doc_lens())[:-1]]).astype(np.int64)
 
     def scaled(self, **kw) -> "Workload":
         d = dict(self.__dict__)
@@ -203,10 +219,13 @@ WORKLOADS = {
     "prefill": Workload("prefill", 2, 1, 32, 8, 128, 256, 8192, 4096, 4096, 64, 8),
     # the prefill step on a 64-document bank: same work per CTA, 2 GB of K/V (hardware-counter captures)
     "prefill_64docs": Workload("prefill_64docs", 2, 1, 32, 8, 128, 64, 8192, 4096, 4096, 64, 8),
+    # K/V of these two banks (283 GB, 410 GB) exceed host RAM: the pinned pool holds
+    # kv_slabs distinct slabs and document j reads slab j mod kv_slabs (routing keys
+    # stay distinct per document; the bytes each step moves over PCIe are unchanged)
     "ragged_planted": Workload("ragged_planted", 3, 4, 64, 8, 128, 8192, 0, 2048, 1, 1, 32,
-                               ragged=(512, 16384), planted=4, host_tier=True),
+                               ragged=(512, 16384), planted=4, host_tier=True, kv_slabs=256),
     "bank_100m": Workload("bank_100m", 4, 16, 32, 8, 128, 24414, 4096, 4096, 1, 1, 16,
-                          host_tier=True),
+                          host_tier=True, kv_slabs=1024),
 }
 
 
@@ -215,10 +234,20 @@ WORKLOADS = {
 # ----------------------------------------------------------------------------
 
 def bank_rows_bits(w: Workload, tensor_id: int, head: int, tok0: int, ntok: int) -> np.ndarray:
-    """bf16 bits of rows [tok0, tok0+ntok) of head `head` of a [Hkv, Ntok, d] bank tensor."""
+    """bf16 bits of rows [tok0, tok0+ntok) of head `head` of a [Hkv, Ntok, d] bank tensor
+    (the routing keys; K and V too when the bank is not aliased)."""
     d = w.head_dim
     start = (head * w.n_tokens + tok0) * d
     return normal_bf16_bits(w.seed, tensor_id, start, ntok * d).reshape(ntok, d)
+
+
+def doc_kv_bits(w: Workload, tensor_id: int, head: int, doc: int, t0: int = 0, n=None) -> np.ndarray:
+    """bf16 bits of tokens [t0, t0+n) of document `doc` in K (T_K) or V (T_V)."""
+    d = w.head_dim
+    n = int(w.doc_lens()[doc]) - t0 if n is None else n
+    row = int(w.doc_kv_rows()[doc]) + t0
+    start = (head * w.kv_rows + row) * d
+    return normal_bf16_bits(w.seed, tensor_id, start, n * d).reshape(n, d)
 
 
 def query_bits(w: Workload, tensor_id: int, shape) -> np.ndarray:

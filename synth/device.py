@@ -33,8 +33,8 @@ def normal(shape, seed: int, tensor_id: int, device="cuda", start: int = 0) -> t
 
 
 def bank_tensors(w: Workload, device="cuda", with_r: bool = True):
-    """K, V, R of the bank as [Hkv, Ntok, d] bf16 (K without RoPE)."""
-    shape = (w.n_kv_heads, w.n_tokens, w.head_dim)
+    """K, V as [Hkv, kv_rows, d] and R as [Hkv, Ntok, d_r], bf16 (K without RoPE)."""
+    shape = (w.n_kv_heads, w.kv_rows, w.head_dim)
     K = normal(shape, w.seed, T_K, device)
     V = normal(shape, w.seed, T_V, device)
     R = normal((w.n_kv_heads, w.n_tokens, w.route_dim), w.seed, T_R, device) if with_r else None
@@ -52,3 +52,24 @@ def query_tensors(w: Workload, device="cuda"):
     LK = normal((w.batch, w.n_kv_heads, w.local_len, w.head_dim), w.seed, T_LK, device)
     LV = normal((w.batch, w.n_kv_heads, w.local_len, w.head_dim), w.seed, T_LV, device)
     return Q, Qr, LK, LV
+
+
+def host_kv_pool(w: Workload, device="cuda"):
+    """The pinned-host K/V tier of an aliased bank: [Hkv, kv_slabs * max_len, d] bf16
+    in pinned host memory, K with Parallel RoPE (slab rows at positions 0..max_len-1,
+    so every document reading the first L_j rows of a slab sees positions 0..L_j-1).
+    The RoPE runs on the device through a bank whose documents are the slabs."""
+    from sparse_attention_routed_b200.runner import Bank
+    assert w.kv_slabs > 0
+    K, V, _ = bank_tensors(w, device, with_r=False)
+    slabs = Bank(K, V, [w.max_len] * w.kv_slabs, w.rope_base)
+    slabs.build(None)
+    torch.cuda.synchronize()
+    slabs.close()
+    Kh = torch.empty(K.shape, dtype=K.dtype, pin_memory=True)
+    Vh = torch.empty(V.shape, dtype=V.dtype, pin_memory=True)
+    Kh.copy_(K)
+    Vh.copy_(V)
+    del K, V
+    torch.cuda.empty_cache()
+    return Kh, Vh

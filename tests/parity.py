@@ -26,8 +26,15 @@ def oracle_inputs(w: synth.Workload) -> dict:
     N, Hkv, d = w.n_tokens, w.n_kv_heads, w.head_dim
     def gen(tid, shape):
         return synth.normal_f32(w.seed, tid, 0, int(np.prod(shape))).reshape(shape).astype(np.float64)
+    if w.kv_slabs:
+        def kv(tid):
+            return np.stack([np.concatenate([f64(synth.doc_kv_bits(w, tid, h, j)) for j in range(w.n_docs)])
+                             for h in range(Hkv)])
+        K, V = kv(synth.T_K), kv(synth.T_V)
+    else:
+        K, V = gen(synth.T_K, (Hkv, N, d)), gen(synth.T_V, (Hkv, N, d))
     inp = {
-        "K": gen(synth.T_K, (Hkv, N, d)), "V": gen(synth.T_V, (Hkv, N, d)),
+        "K": K, "V": V,
         "R": gen(synth.T_R, (Hkv, N, w.route_dim)),
         "Q": gen(synth.T_Q, (w.batch, w.n_q_heads, w.q_tokens, d)),
         "LK": gen(synth.T_LK, (w.batch, Hkv, w.local_len, d)),

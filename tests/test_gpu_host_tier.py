@@ -1,0 +1,88 @@
+"""Pinned-host K/V tier: K/V in pinned host memory, the selected documents'
+slabs copied into a device staging pool each step. Checked against the CPU
+oracle, and bit for bit against a device-resident bank over the same K/V."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import msa_oracle as O
+from synth import Workload
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+HOST = {
+    # decode, G = 4, ragged documents, 5 slabs for 40 documents (aliased pool)
+    "host_decode": Workload("host_decode", 31, 2, 8, 2, 128, 40, 0, 300, 1, 1, 6, ragged=(1, 700),
+                            host_tier=True, kv_slabs=5),
+    # planted targets, G = 8
+    "host_planted": Workload("host_planted", 32, 2, 16, 2, 128, 30, 0, 100, 1, 1, 4, ragged=(300, 1500),
+                             planted=4, host_tier=True, kv_slabs=7),
+    # 256-row problems (tcgen05 prefill) reading the staging pool
+    "host_prefill": Workload("host_prefill", 33, 1, 8, 2, 128, 16, 0, 256, 128, 64, 3, ragged=(100, 900),
+                             host_tier=True, kv_slabs=4),
+}
+
+
+def _run(w, host: bool):
+    import sparse_attention_routed_b200 as msa
+    from sparse_attention_routed_b200.runner import Bank
+    from synth.device import bank_tensors, host_kv_pool, query_tensors
+    if host:
+        K, V = host_kv_pool(w)
+        _, _, R = bank_tensors(w)
+        kv_loc = msa.MSA_KV_PINNED_HOST
+    else:
+        K, V, R = bank_tensors(w)
+        slabs = Bank(K, V, [w.max_len] * w.kv_slabs, w.rope_base)   # same RoPE'd slabs, on the device
+        slabs.build(None)
+        torch.cuda.synchronize()
+        slabs.close()
+        kv_loc = msa.MSA_KV_DEVICE
+    Q, Qr, LK, LV = query_tensors(w)
+    bank = Bank(K, V, w.doc_lens(), w.rope_base, kv_location=kv_loc, doc_rows=w.doc_kv_rows())
+    bank.build(R, rope=False)
+    qry = bank.query(Q, Qr, LK, LV, w.route_block)
+    idx, tsc, scores = bank.route(qry, w.top_k)
+    out = bank.attend(qry, w.top_k, idx)
+    idx2, out2 = bank.forward(qry, w.top_k)
+    torch.cuda.synchronize()
+    assert bank.device_error() == 0
+    res = dict(idx=idx.cpu().numpy(), tsc=tsc.cpu().numpy(), scores=scores.cpu().numpy(), out=out.cpu().numpy(),
+               idx2=idx2.cpu().numpy(), out2=out2.cpu().numpy())
+    # an out-of-range selection index is caught on the host before any copy
+    bad = idx.clone()
+    bad[0, 0, 0, 0] = w.n_docs
+    if host:
+        st = msa.msa_attend(bank.handle, qry, w.top_k, bad.data_ptr(), out.data_ptr(),
+                            torch.cuda.current_stream().cuda_stream, check=False)
+        res["bad_status"] = st
+    bank.close()
+    return res
+
+
+@pytest.mark.parametrize("name", list(HOST))
+def test_host_tier_parity(name):
+    w = HOST[name]
+    g = _run(w, host=True)
+    inp = P.oracle_inputs(w)
+    ref = O.forward(inp, w.doc_lens(), w.top_k, w.route_block, w.rope_base)
+    rows = g["scores"].reshape(-1, w.n_docs)
+    P.check_scores(rows, ref["doc_scores"].reshape(-1, w.n_docs))
+    P.check_topk(g["idx"].reshape(-1, w.top_k), g["tsc"].reshape(-1, w.top_k), rows,
+                 ref["doc_scores"].reshape(-1, w.n_docs), w.top_k)
+    ref2 = O.forward(inp, w.doc_lens(), w.top_k, w.route_block, w.rope_base, selection=g["idx"])
+    P.check_out(g["out"], ref2["out"])
+    np.testing.assert_array_equal(g["idx2"], g["idx"])
+    np.testing.assert_array_equal(g["out2"], g["out"])
+    import sparse_attention_routed_b200 as msa
+    assert g["bad_status"] == msa.MSA_ERR_INVALID_ARG
+
+
+def test_host_tier_equals_device_bank():
+    w = HOST["host_decode"]
+    gh = _run(w, host=True)
+    gd = _run(w, host=False)
+    np.testing.assert_array_equal(gh["idx"], gd["idx"])
+    np.testing.assert_array_equal(gh["out"], gd["out"])
