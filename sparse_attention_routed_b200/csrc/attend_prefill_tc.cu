@@ -9,7 +9,10 @@
 // list in tiles of 128 keys: the selected documents' tiles, then the local
 // tiles up to its last row's position.
 //   warp 0     TMA producer: the query tile once (queries pre-turned by Global
-//              RoPE), then K and V tiles into a 2-stage ring.
+//              RoPE), then K and V tiles into two separate 2-slot rings, in
+//              the order K_0, K_1, V_0, K_2, V_1, ...: a K slot frees as soon
+//              as its S MMA completes, a V slot only after its P V, so the
+//              loads of the next keys never wait behind the softmax.
 //   warp 1     allocates 512 TMEM columns; one lane issues, per tile j,
 //              S_j = Q K_j^T (M = N = K = 128, into one of two S buffers) and
 //              then O += P_{j-1} V_{j-1} (P from shared memory, V read as an
@@ -43,10 +46,11 @@ constexpr float kLazy = 8.0f;         // rescale O only when a row max grows by 
 
 // shared memory layout (offsets from a 1 KiB-aligned base)
 constexpr int OFF_Q = 0;
-constexpr int OFF_K0 = OFF_Q + TILE;           // K[s] = OFF_K0 + s * 2 * TILE, V[s] = K[s] + TILE
-constexpr int OFF_P0 = OFF_K0 + 4 * TILE;      // P[b] = OFF_P0 + b * TILE
+constexpr int OFF_K0 = OFF_Q + TILE;           // K[s] = OFF_K0 + s * TILE
+constexpr int OFF_V0 = OFF_K0 + 2 * TILE;      // V[s] = OFF_V0 + s * TILE
+constexpr int OFF_P0 = OFF_V0 + 2 * TILE;      // P[b] = OFF_P0 + b * TILE
 constexpr int OFF_BAR = OFF_P0 + 2 * TILE;
-constexpr int N_BAR = 13;
+constexpr int N_BAR = 17;
 constexpr int OFF_TMEM = OFF_BAR + N_BAR * 8;
 constexpr int OFF_TAB = OFF_TMEM + 16;
 // TMEM columns used to exchange per-row values between the two softmax warpgroups
@@ -63,12 +67,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sm = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;    // [2]
-  uint64_t* kv_empty = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;     // [2]
-  uint64_t* s_free = bars + 7;     // [2]
-  uint64_t* p_full = bars + 9;     // [2]
-  uint64_t* p_free = bars + 11;    // [2]
+  uint64_t* s_full = bars + 1;     // [2]
+  uint64_t* s_free = bars + 3;     // [2]  one arrival per softmax warp
+  uint64_t* p_full = bars + 5;     // [2]  one arrival per softmax warp
+  uint64_t* p_free = bars + 7;     // [2]
+  uint64_t* k_full = bars + 9;     // [2]
+  uint64_t* k_empty = bars + 11;   // [2]
+  uint64_t* v_full = bars + 13;    // [2]
+  uint64_t* v_empty = bars + 15;   // [2]
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
   int* abort_s = reinterpret_cast<int*>(sm + OFF_TMEM + 4);   // set when a wait expired: softmax warps stop together
 
@@ -105,7 +111,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   if (tid == 0) {
     // s_free and p_full collect one arrival per softmax warp; the rest one arrival each
-    for (int i = 0; i < N_BAR; ++i) mbar_init(&bars[i], (i >= 7 && i <= 10) ? 8 : 1);
+    for (int i = 0; i < N_BAR; ++i) mbar_init(&bars[i], (i >= 3 && i <= 6) ? 8 : 1);
     fence_barrier_init();
     *abort_s = 0;
   }
@@ -147,28 +153,34 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int dh = 0; dh < 2; ++dh)
           tma_load_2d(sm + OFF_Q + dh * BOX + sg * (64 * 128), &tm_q, dh * 64, y, q_full, pol);
       }
-      int di = 0;
-      for (int n = 0; n < T; ++n) {
-        const int st = n & 1, use = n >> 1;
-        if (use > 0 && !mbar_wait_bounded(&kv_empty[st], (use - 1) & 1, a.err)) break;
+      // key tile n -> (tensor map pair, first row); tiles are visited in order, so
+      // one cursor per ring suffices
+      auto coord = [&](int n, int& di, bool& local) -> int {
         while (di < k && n >= tile_start[di + 1]) ++di;
+        local = di >= k;
         const int tt = n - tile_start[di];
-        const CUtensorMap *mk, *mv;
-        int y;
-        if (di < k) {
-          mk = &tm_bk; mv = &tm_bv;
-          y = (int)(doc_base_s[di] + (long long)tt * TN);
-        } else {
-          mk = &tm_lk; mv = &tm_lv;
-          y = (b * a.n_kv_heads + h) * a.local_len + tt * TN;
-        }
-        uint8_t* kd = sm + OFF_K0 + st * 2 * TILE;
-        mbar_arrive_expect_tx(&kv_full[st], 2 * TILE);
-#pragma unroll
-        for (int dh = 0; dh < 2; ++dh) {
-          tma_load_2d(kd + dh * BOX, mk, dh * 64, y, &kv_full[st], pol);
-          tma_load_2d(kd + TILE + dh * BOX, mv, dh * 64, y, &kv_full[st], pol);
-        }
+        return local ? (b * a.n_kv_heads + h) * a.local_len + tt * TN : (int)(doc_base_s[di] + (long long)tt * TN);
+      };
+      int dk = 0, dv = 0;
+      auto load = [&](int n, bool is_v, int& di) -> bool {
+        const int st = n & 1, use = n >> 1;
+        uint64_t* empty = is_v ? v_empty : k_empty;
+        uint64_t* full = is_v ? v_full : k_full;
+        if (use > 0 && !mbar_wait_bounded(&empty[st], (use - 1) & 1, a.err)) return false;
+        bool local;
+        const int y = coord(n, di, local);
+        const CUtensorMap* m = is_v ? (local ? &tm_lv : &tm_bv) : (local ? &tm_lk : &tm_bk);
+        uint8_t* dst = sm + (is_v ? OFF_V0 : OFF_K0) + st * TILE;
+        mbar_arrive_expect_tx(&full[st], TILE);
+        tma_load_2d(dst, m, 0, y, &full[st], pol);
+        tma_load_2d(dst + BOX, m, 64, y, &full[st], pol);
+        return true;
+      };
+      // K runs one tile ahead of V: K_n is needed for S_n, V_n only after the softmax of tile n
+      bool ok = true;
+      for (int n = 0; ok && n <= T; ++n) {
+        if (n < T) ok = load(n, false, dk);
+        if (ok && n >= 1) ok = load(n - 1, true, dv);
       }
     }
   } else if (warp == 1) {
@@ -179,26 +191,27 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = mbar_wait_bounded(q_full, 0, a.err);
       auto issue_pv = [&](int i) -> bool {
         if (!mbar_wait_bounded(&p_full[i & 1], (i >> 1) & 1, a.err)) return false;
+        if (!mbar_wait_bounded(&v_full[i & 1], (i >> 1) & 1, a.err)) return false;
         tc_fence_after();
         const uint32_t pa = sbase + OFF_P0 + (i & 1) * TILE;
-        const uint32_t vb = sbase + OFF_K0 + (i & 1) * 2 * TILE + TILE;
+        const uint32_t vb = sbase + OFF_V0 + (i & 1) * TILE;
 #pragma unroll
         for (int kk = 0; kk < TN / 16; ++kk) {
           const uint64_t ad = umma_desc_sw128(pa + (kk >> 2) * BOX + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = umma_desc_sw128(vb + kk * 2048, BOX, 1024);
           umma_bf16_ss(tmem + O_COL, ad, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&kv_empty[i & 1]);
+        umma_commit(&v_empty[i & 1]);
         umma_commit(&p_free[i & 1]);
         return true;
       };
       for (int j = 0; ok && j < T; ++j) {
         const int st = j & 1;
-        if (!mbar_wait_bounded(&kv_full[st], (j >> 1) & 1, a.err)) break;
+        if (!mbar_wait_bounded(&k_full[st], (j >> 1) & 1, a.err)) break;
         if (j >= 2 && !mbar_wait_bounded(&s_free[j & 1], ((j - 2) >> 1) & 1, a.err)) break;
         tc_fence_after();
         const uint32_t qa = sbase + OFF_Q;
-        const uint32_t kb = sbase + OFF_K0 + st * 2 * TILE;
+        const uint32_t kb = sbase + OFF_K0 + st * TILE;
 #pragma unroll
         for (int ks = 0; ks < TD / 16; ++ks) {
           const uint32_t off = (ks >> 2) * BOX + (ks & 3) * 32;
@@ -206,6 +219,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                        idesc_qk, ks > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[j & 1]);
+        umma_commit(&k_empty[st]);
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok && T > 0) issue_pv(T - 1);
