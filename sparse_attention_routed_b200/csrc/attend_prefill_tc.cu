@@ -9,20 +9,21 @@
 // list in tiles of 128 keys: the selected documents' tiles, then the local
 // tiles up to its last row's position.
 //   warp 0     TMA producer: the query tile once (queries pre-turned by Global
-//              RoPE), then K and V tiles into two separate 2-slot rings, in
+//              RoPE), then K and V tiles into two separate 3-slot rings, in
 //              the order K_0, K_1, V_0, K_2, V_1, ...: a K slot frees as soon
 //              as its S MMA completes, a V slot only after its P V, so the
 //              loads of the next keys never wait behind the softmax.
 //   warp 1     allocates 512 TMEM columns; one lane issues, per tile j,
 //              S_j = Q K_j^T (M = N = K = 128, into one of two S buffers) and
-//              then O += P_{j-1} V_{j-1} (P from shared memory, V read as an
-//              MN-major operand), and commits each group to an mbarrier.
+//              then O += P_{j-1} V_{j-1} (P read from TMEM as the A operand, V
+//              from shared memory as an MN-major operand), and commits each
+//              group to an mbarrier.
 //   warps 2-9  softmax, two warpgroups: each row is split over two threads,
 //              one per 64-key half (TMEM lane = row); they read S_j with
 //              tcgen05.ld, mask (document tails, causal local keys), exchange
-//              half-row maxima through shared memory, and write
-//              P_j = exp2(S_j * scale - m) as bf16 into a 128-byte-swizzled
-//              K-major tile. The reference max m of a row moves only when the
+//              half-row maxima through already-read S columns, and write
+//              P_j = exp2(S_j * scale - m) as packed bf16 pairs into one of two
+//              P buffers in TMEM. The reference max m of a row moves only when the
 //              row max rises by more than 2^8; then the row of O is rescaled in
 //              TMEM (warp-collective tcgen05.ld/st after the previous P V).
 // Every mbarrier parity wait targets the phase right after one the same waiter
@@ -36,8 +37,10 @@ namespace {
 constexpr int TN = 128;               // keys per tile
 constexpr int TM = 128;               // query rows per CTA
 constexpr int TD = 128;               // head dim
-constexpr int TMEM_COLS = 512;        // S0 [0,128) S1 [128,256) O [256,384)
+constexpr int TMEM_COLS = 512;        // S0 [0,128) S1 [128,256) O [256,384) P0 [384,448) P1 [448,512)
 constexpr int O_COL = 256;
+constexpr int P_COL = 384;            // P_b = P_COL + 64 b: 128 keys as 64 packed bf16 pairs
+constexpr int NSLOT = 3;              // depth of the K ring and of the V ring
 constexpr int THREADS = 320;           // producer, MMA, 8 softmax warps
 constexpr int BOX = TN * 128;         // one 64-element-wide box of a 128-row tile (16 KB)
 constexpr int TILE = 2 * BOX;         // 128 x 128 bf16 (32 KB)
@@ -46,16 +49,12 @@ constexpr float kLazy = 8.0f;         // rescale O only when a row max grows by 
 
 // shared memory layout (offsets from a 1 KiB-aligned base)
 constexpr int OFF_Q = 0;
-constexpr int OFF_K0 = OFF_Q + TILE;           // K[s] = OFF_K0 + s * TILE
-constexpr int OFF_V0 = OFF_K0 + 2 * TILE;      // V[s] = OFF_V0 + s * TILE
-constexpr int OFF_P0 = OFF_V0 + 2 * TILE;      // P[b] = OFF_P0 + b * TILE
-constexpr int OFF_BAR = OFF_P0 + 2 * TILE;
-constexpr int N_BAR = 17;
+constexpr int OFF_K0 = OFF_Q + TILE;              // K[s] = OFF_K0 + s * TILE
+constexpr int OFF_V0 = OFF_K0 + NSLOT * TILE;     // V[s] = OFF_V0 + s * TILE
+constexpr int OFF_BAR = OFF_V0 + NSLOT * TILE;
+constexpr int N_BAR = 9 + 4 * NSLOT;
 constexpr int OFF_TMEM = OFF_BAR + N_BAR * 8;
 constexpr int OFF_TAB = OFF_TMEM + 16;
-// TMEM columns used to exchange per-row values between the two softmax warpgroups
-constexpr int MX_COL = 384;   // + 2 * parity + warpgroup: half-row maxima
-constexpr int L_COL = 388;    // + warpgroup: half-row sums
 constexpr size_t SMEM_BYTES = 1024 + OFF_TAB + (TOPK_MAX + 2) * 4 + TOPK_MAX * 4 + TOPK_MAX * 8;
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 
@@ -71,10 +70,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* s_free = bars + 3;     // [2]  one arrival per softmax warp
   uint64_t* p_full = bars + 5;     // [2]  one arrival per softmax warp
   uint64_t* p_free = bars + 7;     // [2]
-  uint64_t* k_full = bars + 9;     // [2]
-  uint64_t* k_empty = bars + 11;   // [2]
-  uint64_t* v_full = bars + 13;    // [2]
-  uint64_t* v_empty = bars + 15;   // [2]
+  uint64_t* k_full = bars + 9;     // [NSLOT] each
+  uint64_t* k_empty = k_full + NSLOT;
+  uint64_t* v_full = k_empty + NSLOT;
+  uint64_t* v_empty = v_full + NSLOT;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
   int* abort_s = reinterpret_cast<int*>(sm + OFF_TMEM + 4);   // set when a wait expired: softmax warps stop together
 
@@ -163,7 +162,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       };
       int dk = 0, dv = 0;
       auto load = [&](int n, bool is_v, int& di) -> bool {
-        const int st = n & 1, use = n >> 1;
+        const int st = n % NSLOT, use = n / NSLOT;
         uint64_t* empty = is_v ? v_empty : k_empty;
         uint64_t* full = is_v ? v_full : k_full;
         if (use > 0 && !mbar_wait_bounded(&empty[st], (use - 1) & 1, a.err)) return false;
@@ -191,23 +190,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = mbar_wait_bounded(q_full, 0, a.err);
       auto issue_pv = [&](int i) -> bool {
         if (!mbar_wait_bounded(&p_full[i & 1], (i >> 1) & 1, a.err)) return false;
-        if (!mbar_wait_bounded(&v_full[i & 1], (i >> 1) & 1, a.err)) return false;
+        if (!mbar_wait_bounded(&v_full[i % NSLOT], (i / NSLOT) & 1, a.err)) return false;
         tc_fence_after();
-        const uint32_t pa = sbase + OFF_P0 + (i & 1) * TILE;
-        const uint32_t vb = sbase + OFF_V0 + (i & 1) * TILE;
+        const uint32_t pt = tmem + P_COL + (i & 1) * (TN / 2);
+        const uint32_t vb = sbase + OFF_V0 + (i % NSLOT) * TILE;
 #pragma unroll
         for (int kk = 0; kk < TN / 16; ++kk) {
-          const uint64_t ad = umma_desc_sw128(pa + (kk >> 2) * BOX + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = umma_desc_sw128(vb + kk * 2048, BOX, 1024);
-          umma_bf16_ss(tmem + O_COL, ad, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem + O_COL, pt + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&v_empty[i & 1]);
+        umma_commit(&v_empty[i % NSLOT]);
         umma_commit(&p_free[i & 1]);
         return true;
       };
       for (int j = 0; ok && j < T; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait_bounded(&k_full[st], (j >> 1) & 1, a.err)) break;
+        const int st = j % NSLOT;
+        if (!mbar_wait_bounded(&k_full[st], (j / NSLOT) & 1, a.err)) break;
         if (j >= 2 && !mbar_wait_bounded(&s_free[j & 1], ((j - 2) >> 1) & 1, a.err)) break;
         tc_fence_after();
         const uint32_t qa = sbase + OFF_Q;
@@ -270,14 +268,17 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (c0 + e < vis_end) mt = fmaxf(mt, SV(e));
         mt = (mt == -INFINITY) ? mt : mt * a.scale_log2;
       }
-      tmem_st1(tl + MX_COL + (j & 1) * 2 + wg, __float_as_uint(mt));
+      // each warpgroup posts its half-row max in the first S column of its own
+      // half (already read) and takes the partner's from the partner's half
+      const uint32_t sbuf = tl + (j & 1) * TN;
+      tmem_st1(sbuf + c0, __float_as_uint(mt));
       tmem_wait_st();
       if (!okw) *abort_s = 1;
       tc_fence_before();
       named_barrier_sync(1, 2 * 4 * 32);
       tc_fence_after();
       if (*abort_s) break;
-      mt = fmaxf(mt, __uint_as_float(tmem_ld1(tl + MX_COL + (j & 1) * 2 + (wg ^ 1))));
+      mt = fmaxf(mt, __uint_as_float(tmem_ld1(sbuf + (c0 ^ (TN / 2)))));
       tmem_wait_ld();
       const float m_new = fmaxf(m_ref, mt);
       const bool need = m_new > m_ref + kLazy;  // also true when m_ref = -inf and the tile has a key
@@ -287,27 +288,27 @@ __global__ void __launch_bounds__(THREADS, 1)
         l *= alpha;
         m_ref = m_new;
       }
-      // P = exp2(S * scale - m_ref) as bf16 into this warpgroup's 64-key box of the K-major tile
+      // P = exp2(S * scale - m_ref) as bf16 pairs into this warpgroup's 32 columns of P_(j&1)
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      uint8_t* box = sm + OFF_P0 + (j & 1) * TILE + wg * BOX;
+      const uint32_t pcol = tl + P_COL + (j & 1) * (TN / 2) + c0 / 2;
       const float sc = a.scale_log2;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        uint32_t pk[4];
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int e = q * 8 + 2 * u;
+        for (int u = 0; u < 16; ++u) {
+          const int e = hh * 32 + 2 * u;
           float p0 = ex2_approx(fmaf(SV(e), sc, -m_use));
           float p1 = ex2_approx(fmaf(SV(e + 1), sc, -m_use));
           if (!full) {
             p0 = (c0 + e < vis_end) ? p0 : 0.f;
             p1 = (c0 + e + 1 < vis_end) ? p1 : 0.f;
           }
-          ls[u] += p0 + p1;
+          ls[u & 3] += p0 + p1;
           pk[u] = pack_bf16(p0, p1);
         }
-        *reinterpret_cast<uint4*>(box + swz128(r, q)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        tmem_st16(pcol + hh * 16, pk);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
 #undef SV
@@ -328,7 +329,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tmem_wait_st();
       }
-      fence_proxy_async();  // P is read by the tensor cores (async proxy)
+      tmem_wait_st();  // P (and any rescaled O) is in TMEM before the MMA may read it
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -337,12 +338,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
     // ---- epilogue: O / l once the last P V has completed; l sums both halves of the keys
-    tmem_st1(tl + L_COL + wg, __float_as_uint(l));
+    // row sums through the second S column of each half of buffer 0 (no S MMA is left)
+    tmem_st1(tl + c0 + 1, __float_as_uint(l));
     tmem_wait_st();
     tc_fence_before();
     named_barrier_sync(1, 2 * 4 * 32);
     tc_fence_after();
-    const float lt = l + __uint_as_float(tmem_ld1(tl + L_COL + (wg ^ 1)));
+    const float lt = l + __uint_as_float(tmem_ld1(tl + ((c0 + 1) ^ (TN / 2))));
     tmem_wait_ld();
     if (!*abort_s && T > 0 && mbar_wait_bounded(&p_free[(T - 1) & 1], ((T - 1) >> 1) & 1, a.err)) {
       tc_fence_after();
