@@ -46,6 +46,27 @@ constexpr int BOX = TN * 128;         // one 64-element-wide box of a 128-row ti
 constexpr int TILE = 2 * BOX;         // 128 x 128 bf16 (32 KB)
 constexpr int TOPK_MAX = 64;
 constexpr float kLazy = 8.0f;         // rescale O only when a row max grows by more than 2^8
+#ifndef MSA_PF_POLY
+#define MSA_PF_POLY 1                 // of every 4 key pairs, how many take exp2 on the FMA pipe
+#endif
+constexpr int kPolyPairs = MSA_PF_POLY;
+
+// 2^x on the FMA and integer pipes, to share the exponentials of a tile between
+// them and the special-function unit. Range reduction x = n + f with n the
+// nearest integer (adding 1.5 * 2^23 leaves n in the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f from a cubic whose coefficients are a Remez
+// (equioscillating relative error) fit on that interval, max relative error
+// 7.5e-5 -- far below the 2^-9 of the bf16 rounding P gets next; 2^n is
+// added to the exponent field. x is clamped at -125 so the result stays normal
+// (its weight next to the row max is then below 2^-125 anyway).
+__device__ __forceinline__ float exp2_poly3(float x) {
+  x = fmaxf(x, -125.f);
+  const float big = 12582912.f;
+  const float j = x + big;
+  const float f = x - (j - big);
+  const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.242611125f), f, 0.693260968f), f, 0.999928057f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(j) << 23));
+}
 
 // shared memory layout (offsets from a 1 KiB-aligned base)
 constexpr int OFF_Q = 0;
@@ -299,8 +320,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const int e = hh * 32 + 2 * u;
-          float p0 = ex2_approx(fmaf(SV(e), sc, -m_use));
-          float p1 = ex2_approx(fmaf(SV(e + 1), sc, -m_use));
+          const bool poly = u >= 4 - kPolyPairs;
+          const float x0 = fmaf(SV(e), sc, -m_use), x1 = fmaf(SV(e + 1), sc, -m_use);
+          float p0 = poly ? exp2_poly3(x0) : ex2_approx(x0);
+          float p1 = poly ? exp2_poly3(x1) : ex2_approx(x1);
           if (!full) {
             p0 = (c0 + e < vis_end) ? p0 : 0.f;
             p1 = (c0 + e + 1 < vis_end) ? p1 : 0.f;
