@@ -134,7 +134,15 @@ def oracle_sample(seconds: float):
     return queries / spent, queries, spent, threads
 
 
+def base_config(w) -> dict:
+    """The workload description both arms print."""
+    return {"workload": w.name, "batch": w.batch, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
+            "head_dim": w.head_dim, "bank_docs": w.n_docs, "doc_len": w.doc_len, "local_len": w.local_len,
+            "q_tokens": w.q_tokens, "route_block": w.route_block, "top_k": w.top_k}
+
+
 def run_reference(args):
+    import synth
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -143,7 +151,9 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": qps, "unit": "queries/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * 8 / qps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": WORKLOAD, "batch": 8, "bank_tokens": 4194304},
+        "data": "synthetic",
+        "config": dict(base_config(synth.WORKLOADS[WORKLOAD]), parallelism="oracle on host cores",
+                       l2="n/a (host cores)"),
         "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
                          "sample": f"{nq} decode queries (router over all 16384 chunks x 8 KV heads, "
                                    f"top-16, attention for 32 heads), {spent:.1f} s of oracle time"},
@@ -218,6 +228,23 @@ def profile_traffic(kernel_file: str):
         return float(vals["dram_bytes_per_launch"])
     except (KeyError, ValueError):
         return None
+
+
+def max_over_ranks(values, device="cpu"):
+    """Each timing's maximum over all ranks (the slowest replica sets the job's
+    time); the values unchanged on a single process."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world: int, units_per_step: float, steps: int, total_ms: float) -> float:
+    """Whole-job throughput of `world` replicas that each processed `units_per_step`
+    units in each of `steps` steps, over the max-over-ranks time `total_ms`."""
+    return world * units_per_step * steps / (total_ms / 1000.0)
 
 
 def run_ours(args):
@@ -347,15 +374,13 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
 
-    t = torch.tensor([total_ms, e2e_ms, route_ms, attend_ms], dtype=torch.float64, device="cuda")
+    total_ms, e2e_ms, route_ms, attend_ms = max_over_ranks([total_ms, e2e_ms, route_ms, attend_ms], "cuda")
     if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
         dist.barrier()
-    total_ms, e2e_ms, route_ms, attend_ms = t.tolist()
     ms_step = total_ms / n
     units = B * (w.q_tokens if prefill else 1)   # queries (decode) or query tokens (prefill) per step
-    value = world * units * n / (total_ms / 1000.0)
-    e2e_value = world * units * n_e2e / (e2e_ms / 1000.0)
+    value = job_throughput(world, units, n, total_ms)
+    e2e_value = job_throughput(world, units, n_e2e, e2e_ms)
 
     if rank == 0:
         peak, peak_kind = peaks()
@@ -378,11 +403,8 @@ def run_ours(args):
             "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": n,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": args.workload, "batch": B, "q_heads": w.n_q_heads, "kv_heads": Hkv,
-                       "head_dim": d, "bank_docs": w.n_docs, "doc_len": w.doc_len, "local_len": w.local_len,
-                       "q_tokens": w.q_tokens, "route_block": w.route_block, "top_k": k,
-                       "parallelism": f"replicas x{world}",
-                       "l2": f"inputs larger than L2: {step_bytes / 1e9:.2f} GB of HBM per step vs 126 MB L2"},
+            "config": dict(base_config(w), parallelism=f"replicas x{world}",
+                           l2=f"inputs larger than L2: {step_bytes / 1e9:.2f} GB of HBM per step vs 126 MB L2"),
             "router_attn_hbm": {"bytes_per_step": step_bytes, "GBps": step_bytes / (ms_step / 1000.0) / 1e9,
                                 "frac_of_peak": step_bytes / (ms_step / 1000.0) / 1e9 / peak,
                                 "route_ms": route_ms, "attend_ms": attend_ms},

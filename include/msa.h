@@ -40,8 +40,19 @@
  *   - There is no CPU fallback: without a usable sm_100 device the calls that
  *     launch work return MSA_ERR_CUDA or MSA_ERR_UNSUPPORTED.
  *   - Supported shapes: head_dim = route_dim in {64, 128}; n_q_heads a
- *     multiple of n_kv_heads; G = n_q_heads / n_kv_heads and route_block with
- *     G * route_block <= 16; 1 <= top_k <= min(n_docs, 64).
+ *     multiple of n_kv_heads; 1 <= top_k <= min(n_docs, 64); q_tokens a
+ *     multiple of route_block; batch * (q_tokens / route_block) * n_kv_heads
+ *     <= 65535. With G = n_q_heads / n_kv_heads, a routing block holds
+ *     G * route_block query rows per KV head: up to 16 rows run the split-KV
+ *     decode kernel, more rows the prefill kernels (tensor-memory tcgen05
+ *     kernel when head_dim = 128, route_block is 64 or 128 and G * route_block
+ *     is a multiple of 128; an mma.sync kernel otherwise).
+ *   - Bank K/V may live in pinned host memory (MSA_KV_PINNED_HOST): msa_attend
+ *     and msa_forward then read the step's selection back to the host, copy
+ *     every distinct selected (document, KV head) slab into a device staging
+ *     pool with cudaMemcpyAsync on side streams, and attend from there. Those
+ *     two calls synchronise the stream once per call and cannot be captured
+ *     into a CUDA graph; msa_route never touches host K/V.
  */
 #ifndef MSA_H_
 #define MSA_H_
@@ -182,6 +193,16 @@ msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_
  * GPU (e.g. on two streams without ordering) race and corrupt each other. */
 msa_status msa_route_noalloc(msa_bank* bank, const msa_query* q, int32_t top_k, float* doc_scores,
                              int32_t* topk_idx, float* topk_scores, void* stream);
+
+/* Failure-detection check of the device-side bounded waits (the pages describe
+ * no such call): launches one small kernel on `stream` whose thread waits on an
+ * mbarrier phase that nothing ever completes, with the same poll limit every
+ * kernel of this library uses (2^22 polls of mbarrier.try_wait). The wait gives
+ * up, raises the bank's device error flag and the kernel returns normally: no
+ * fault, and the context stays usable. A following msa_get_device_error()
+ * returns MSA_ERR_TIMEOUT (and clears the flag). Returns MSA_ERR_INVALID_ARG for
+ * a NULL bank, MSA_ERR_CUDA if the launch fails. */
+msa_status msa_check_wait_timeout(msa_bank* bank, void* stream);
 
 /* Synchronises `stream`, then returns and clears the device-side error flag
  * (MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_INVALID_ARG). */

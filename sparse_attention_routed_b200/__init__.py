@@ -72,6 +72,7 @@ def _load():
         "msa_forward": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp], ctypes.c_int),
         "msa_get_device_error": ([vp, vp], ctypes.c_int),
         "msa_route_noalloc": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp, vp], ctypes.c_int),
+        "msa_check_wait_timeout": ([vp, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -98,8 +99,8 @@ def __getattr__(name):
 
 # Every symbol include/msa.h declares, in declaration order.
 EXPORTED = ["msa_bank_create", "msa_bank_destroy", "msa_build_bank", "msa_bank_info", "msa_reserve",
-            "msa_route", "msa_attend", "msa_forward", "msa_route_noalloc", "msa_get_device_error",
-            "msa_status_string"]
+            "msa_route", "msa_attend", "msa_forward", "msa_route_noalloc", "msa_check_wait_timeout",
+            "msa_get_device_error", "msa_status_string"]
 
 
 def msa_status_string(status: int) -> str:
@@ -204,6 +205,10 @@ def msa_route_noalloc(bank, query: msa_query, top_k: int, doc_scores: int, topk_
     if check:
         _check(st, "msa_route_noalloc")
     return st
+
+
+def msa_check_wait_timeout(bank, stream=0) -> None:
+    _check(lib().msa_check_wait_timeout(bank, stream or None), "msa_check_wait_timeout")
 
 
 def msa_get_device_error(bank, stream=0) -> int:

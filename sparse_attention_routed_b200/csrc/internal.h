@@ -126,6 +126,10 @@ int attend_max_splits();              // upper bound on n_splits
 int attend_ctas_per_sm(int head_dim); // resident CTAs per SM (shared-memory bound)
 size_t attend_smem_bytes(int head_dim);
 
+// One CTA whose bounded wait on a never-completed mbarrier phase expires and
+// raises kErrTimeout in *err.
+cudaError_t launch_wait_timeout(int* err, cudaStream_t s);
+
 }  // namespace msa
 
 struct msa_bank;

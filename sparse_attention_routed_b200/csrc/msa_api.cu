@@ -715,6 +715,12 @@ msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_
   return attend_impl(bank, q, s, splits, w, topk_idx, out, st);
 }
 
+msa_status msa_check_wait_timeout(msa_bank* bank, void* stream) {
+  if (!bank) return MSA_ERR_INVALID_ARG;
+  MSA_CUDA(launch_wait_timeout(bank->d_err, (cudaStream_t)stream));
+  return MSA_OK;
+}
+
 msa_status msa_get_device_error(msa_bank* bank, void* stream) {
   if (!bank) return MSA_ERR_INVALID_ARG;
   MSA_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
