@@ -14,9 +14,15 @@ namespace msa {
 constexpr int kErrInvalidArg = 1;
 constexpr int kErrTimeout = 5;
 
-// A bounded wait gives up after this many polls (each try_wait already blocks
-// for a hardware-chosen interval), i.e. on the order of a second.
-constexpr uint32_t kMaxPolls = 1u << 22;
+// Each poll of a bounded wait is an mbarrier.try_wait that suspends the thread
+// for up to kWaitHintNs (it resumes as soon as the phase completes), so that
+// waiting warps do not spin through issue slots their SM sub-partition's other
+// warps need; a wait gives up after kMaxPolls polls, on the order of a second.
+#ifndef MSA_WAIT_HINT_NS
+#define MSA_WAIT_HINT_NS 1000
+#endif
+constexpr uint32_t kWaitHintNs = MSA_WAIT_HINT_NS;
+constexpr uint32_t kMaxPolls = kWaitHintNs ? (1u << 30) / kWaitHintNs : (1u << 22);
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -56,13 +62,23 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
+  if (kWaitHintNs) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(kWaitHintNs)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+  }
   return ok != 0;
 }
 
