@@ -74,7 +74,10 @@ def launches_per_step(w) -> int:
     """Kernels libmsa launches for one route + attend step of workload w."""
     rows_route = w.batch * (w.q_tokens // w.route_block)
     n = (0 if w.route_block <= 4 else 1) + (rows_route + 15) // 16 + 1     # qr_prep, router passes, top-k
-    n += 1 if (w.n_q_heads // w.n_kv_heads) * w.route_block <= 16 else 2   # decode kernel | rope_local + prefill
+    rows = (w.n_q_heads // w.n_kv_heads) * w.route_block
+    tc = w.head_dim == 128 and w.route_block in (64, 128) and rows % 128 == 0
+    # decode kernel | rope_local (+ rope of the queries for the tcgen05 kernel) + prefill kernel
+    n += 1 if rows <= 16 else (3 if tc else 2)
     return n
 
 
@@ -210,19 +213,32 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- ours
-def profile_traffic(kernel_file: str):
-    """DRAM bytes per launch from the committed ncu summary, if it matches the current source."""
-    prof = os.path.join(ROOT, "profiles", "attend_decode.decode_4m.txt")
-    src = os.path.join(ROOT, "sparse_attention_routed_b200", "csrc", kernel_file)
+KERNEL_SOURCES = {
+    "attend_decode": ["attend_decode.cu", "common.cuh"],
+    "attend_prefill_tc": ["attend_prefill_tc.cu", "common.cuh"],
+}
+
+
+def source_sha(kernel: str) -> str:
+    """sha256 over the source files a kernel is compiled from (its .cu and the shared header)."""
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(ROOT, "sparse_attention_routed_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
+def profile_traffic(profile: str, kernel: str):
+    """DRAM bytes per launch from a committed ncu summary under profiles/, or None
+    when the kernel's sources changed since the counters were taken."""
+    prof = os.path.join(ROOT, "profiles", profile)
     if not os.path.exists(prof):
         return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
     vals = {}
     for line in open(prof):
         if ":" in line:
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
-    if vals.get("source_sha256") != sha:
+    if vals.get("source_sha256") != source_sha(kernel):
         return None
     try:
         return float(vals["dram_bytes_per_launch"])
@@ -389,14 +405,16 @@ def run_ours(args):
             achieved = attn_flops / (attend_ms / 1000.0) / 1e12
             roofline = {"kernel": "sparse_attend (rope_local + attend_prefill launches)", "bound": "tensor",
                         "achieved": achieved, "peak": tpeak, "peak_kind": tkind, "unit": "TFLOP/s",
-                        "frac": achieved / tpeak, "traffic": None, "algorithmic_flops_per_launch": attn_flops,
+                        "frac": achieved / tpeak,
+                        "traffic": profile_traffic("attend_prefill_tc.prefill.txt", "attend_prefill_tc"),
+                        "algorithmic_flops_per_launch": attn_flops,
                         "hbm_bytes_algorithmic": attn_bytes}
             metric, unit = "prefill query tokens/s (4096-token prompt, 64-token routing blocks)", "tokens/s"
         else:
             achieved = attn_bytes / (attend_ms / 1000.0) / 1e9
             roofline = {"kernel": "sparse_attend (attend_decode launch)", "bound": "hbm",
                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                        "frac": achieved / peak, "traffic": profile_traffic("attend_decode.cu"),
+                        "frac": achieved / peak, "traffic": profile_traffic("attend_decode.decode_4m.txt", "attend_decode"),
                         "algorithmic_bytes_per_launch": attn_bytes}
             metric, unit = METRIC, "queries/s"
         line = {
