@@ -59,13 +59,25 @@ constexpr int kPolyPairs = MSA_PF_POLY;
 // 7.5e-5 -- far below the 2^-9 of the bf16 rounding P gets next; 2^n is
 // added to the exponent field. x is clamped at -125 so the result stays normal
 // (its weight next to the row max is then below 2^-125 anyway).
-__device__ __forceinline__ float exp2_poly3(float x) {
-  x = fmaxf(x, -125.f);
-  const float big = 12582912.f;
-  const float j = x + big;
-  const float f = x - (j - big);
-  const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.242611125f), f, 0.693260968f), f, 0.999928057f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(j) << 23));
+// Two lanes at once with the packed fp32x2 FMA/add of sm_100.
+__device__ __forceinline__ float2 exp2_poly3x2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 big = make_float2(12582912.f, 12582912.f), nbig = make_float2(-12582912.f, -12582912.f);
+  const float2 j = __fadd2_rn(x, big);
+  const float2 f = __ffma2_rn(__fadd2_rn(j, nbig), make_float2(-1.f, -1.f), x);  // x - (j - big)
+  float2 p = __ffma2_rn(make_float2(0.0551716685f, 0.0551716685f), f, make_float2(0.242611125f, 0.242611125f));
+  p = __ffma2_rn(p, f, make_float2(0.693260968f, 0.693260968f));
+  p = __ffma2_rn(p, f, make_float2(0.999928057f, 0.999928057f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(j.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(j.y) << 23)));
+}
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 // shared memory layout (offsets from a 1 KiB-aligned base)
@@ -280,7 +292,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (full) {
         float m4[4] = {SV(0), SV(1), SV(2), SV(3)};
 #pragma unroll
-        for (int e = 4; e < TN / 2; ++e) m4[e & 3] = fmaxf(m4[e & 3], SV(e));
+        for (int pr = 2; pr < TN / 4; ++pr) m4[pr & 3] = max3f(m4[pr & 3], SV(2 * pr), SV(2 * pr + 1));
         mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale_log2;
       } else {
         mt = -INFINITY;
@@ -312,28 +324,27 @@ __global__ void __launch_bounds__(THREADS, 1)
       // P = exp2(S * scale - m_ref) as bf16 pairs into this warpgroup's 32 columns of P_(j&1)
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
       const uint32_t pcol = tl + P_COL + (j & 1) * (TN / 2) + c0 / 2;
-      const float sc = a.scale_log2;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_use, -m_use);
+      float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t pk[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const int e = hh * 32 + 2 * u;
-          const bool poly = u >= 4 - kPolyPairs;
-          const float x0 = fmaf(SV(e), sc, -m_use), x1 = fmaf(SV(e + 1), sc, -m_use);
-          float p0 = poly ? exp2_poly3(x0) : ex2_approx(x0);
-          float p1 = poly ? exp2_poly3(x1) : ex2_approx(x1);
+          const bool poly = (u & 3) >= 4 - kPolyPairs;
+          const float2 x = __ffma2_rn(make_float2(SV(e), SV(e + 1)), sc2, nm2);
+          float2 pp = poly ? exp2_poly3x2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
           if (!full) {
-            p0 = (c0 + e < vis_end) ? p0 : 0.f;
-            p1 = (c0 + e + 1 < vis_end) ? p1 : 0.f;
+            pp.x = (c0 + e < vis_end) ? pp.x : 0.f;
+            pp.y = (c0 + e + 1 < vis_end) ? pp.y : 0.f;
           }
-          ls[u & 3] += p0 + p1;
-          pk[u] = pack_bf16(p0, p1);
+          ls[u & 1] = __fadd2_rn(ls[u & 1], pp);
+          pk[u] = pack_bf16(pp.x, pp.y);
         }
         tmem_st16(pcol + hh * 16, pk);
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
 #undef SV
       // (after P, so that S is no longer live) the rescale must land before P V of this tile
       if (__any_sync(0xffffffffu, need && j > 0)) {
