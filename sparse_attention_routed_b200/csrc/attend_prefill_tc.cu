@@ -221,15 +221,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t idesc_qk = umma_idesc_bf16(TM, TN, false);
       const uint32_t idesc_pv = umma_idesc_bf16(TM, TD, true);
       bool ok = mbar_wait_bounded(q_full, 0, a.err);
+      const uint64_t qdesc = umma_desc_sw128(sbase + OFF_Q, 16, 1024);
+      const uint64_t kdesc0 = umma_desc_sw128(sbase + OFF_K0, 16, 1024);
       auto issue_pv = [&](int i) -> bool {
         if (!mbar_wait_bounded(&p_full[i & 1], (i >> 1) & 1, a.err)) return false;
         if (!mbar_wait_bounded(&v_full[i % NSLOT], (i / NSLOT) & 1, a.err)) return false;
         tc_fence_after();
         const uint32_t pt = tmem + P_COL + (i & 1) * (TN / 2);
         const uint32_t vb = sbase + OFF_V0 + (i % NSLOT) * TILE;
+        const uint64_t vdesc = umma_desc_sw128(vb, BOX, 1024);
 #pragma unroll
         for (int kk = 0; kk < TN / 16; ++kk) {
-          const uint64_t bd = umma_desc_sw128(vb + kk * 2048, BOX, 1024);
+          const uint64_t bd = vdesc + (uint64_t)((kk * 2048) >> 4);
           umma_bf16_ts(tmem + O_COL, pt + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&v_empty[i % NSLOT]);
@@ -241,12 +244,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!mbar_wait_bounded(&k_full[st], (j / NSLOT) & 1, a.err)) break;
         if (j >= 2 && !mbar_wait_bounded(&s_free[j & 1], ((j - 2) >> 1) & 1, a.err)) break;
         tc_fence_after();
-        const uint32_t qa = sbase + OFF_Q;
-        const uint32_t kb = sbase + OFF_K0 + st * TILE;
+        // shared memory addresses stay below 2^18, so the 14-bit start field
+        // of a descriptor never carries: offsets add to it directly
+        const uint64_t kdesc = kdesc0 + (uint64_t)((st * TILE) >> 4);
 #pragma unroll
         for (int ks = 0; ks < TD / 16; ++ks) {
           const uint32_t off = (ks >> 2) * BOX + (ks & 3) * 32;
-          umma_bf16_ss(tmem + (j & 1) * TN, umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024),
+          umma_bf16_ss(tmem + (j & 1) * TN, qdesc + (uint64_t)(off >> 4), kdesc + (uint64_t)(off >> 4),
                        idesc_qk, ks > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[j & 1]);
