@@ -14,18 +14,24 @@
 //              as its S MMA completes, a V slot only after its P V, so the
 //              loads of the next keys never wait behind the softmax.
 //   warp 1     allocates 512 TMEM columns; one lane issues, per tile j,
-//              S_j = Q K_j^T (M = N = K = 128, into one of two S buffers) and
-//              then O += P_{j-1} V_{j-1} (P read from TMEM as the A operand, V
-//              from shared memory as an MN-major operand), and commits each
-//              group to an mbarrier.
-//   warps 2-9  softmax, two warpgroups: each row is split over two threads,
-//              one per 64-key half (TMEM lane = row); they read S_j with
-//              tcgen05.ld, mask (document tails, causal local keys), exchange
-//              half-row maxima through already-read S columns, and write
-//              P_j = exp2(S_j * scale - m) as packed bf16 pairs into one of two
-//              P buffers in TMEM. The reference max m of a row moves only when the
-//              row max rises by more than 2^8; then the row of O is rescaled in
-//              TMEM (warp-collective tcgen05.ld/st after the previous P V).
+//              S_j = Q K_j^T (M = N = K = 128, into one of two S buffers, once
+//              both P V of tile j-2, which read P over that buffer, completed)
+//              and then, for tile j-1, O_0 += P_0 V[0:64) and O_1 += P_1
+//              V[64:128) (P read from TMEM as the A operand, V from shared
+//              memory as an MN-major operand), each as soon as its warpgroup
+//              has written P; every group is committed to an mbarrier.
+//   warps 2-9  softmax, two warpgroups; warpgroup h owns keys [64 h, 64 h + 64)
+//              of every tile and keeps, per row (TMEM lane = row), its own
+//              reference max, running sum and output accumulator O_h over
+//              those keys, so the two never wait for each other inside the
+//              key loop. Each thread reads its 64 S values with tcgen05.ld,
+//              masks (document tails, causal local keys), and writes
+//              P = exp2(S * scale - m) as packed bf16 pairs over the S columns
+//              it has just read. m moves only when the half-row max rises by
+//              more than 2^8; then the row of O_h is rescaled in TMEM (after
+//              the previous P V into it). At the end the two halves' (m, l, O)
+//              are merged per row -- exact, as a softmax over the union of
+//              two key sets -- and each warpgroup writes 64 of the 128 dims.
 // Every mbarrier parity wait targets the phase right after one the same waiter
 // saw complete, so no wait can be satisfied by an older phase.
 #include "common.cuh"
@@ -37,9 +43,8 @@ namespace {
 constexpr int TN = 128;               // keys per tile
 constexpr int TM = 128;               // query rows per CTA
 constexpr int TD = 128;               // head dim
-constexpr int TMEM_COLS = 512;        // S0 [0,128) S1 [128,256) O [256,384) P0 [384,448) P1 [448,512)
-constexpr int O_COL = 256;
-constexpr int P_COL = 384;            // P_b = P_COL + 64 b: 128 keys as 64 packed bf16 pairs
+constexpr int TMEM_COLS = 512;        // S0 [0,128) S1 [128,256) O_0 [256,384) O_1 [384,512)
+constexpr int O_COL = 256;            // O_h = O_COL + 128 h
 constexpr int NSLOT = 3;              // depth of the K ring and of the V ring
 constexpr int THREADS = 320;           // producer, MMA, 8 softmax warps
 constexpr int BOX = TN * 128;         // one 64-element-wide box of a 128-row tile (16 KB)
@@ -85,7 +90,7 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_K0 = OFF_Q + TILE;              // K[s] = OFF_K0 + s * TILE
 constexpr int OFF_V0 = OFF_K0 + NSLOT * TILE;     // V[s] = OFF_V0 + s * TILE
 constexpr int OFF_BAR = OFF_V0 + NSLOT * TILE;
-constexpr int N_BAR = 9 + 4 * NSLOT;
+constexpr int N_BAR = 12 + 4 * NSLOT;
 constexpr int OFF_TMEM = OFF_BAR + N_BAR * 8;
 constexpr int OFF_TAB = OFF_TMEM + 16;
 constexpr size_t SMEM_BYTES = 1024 + OFF_TAB + (TOPK_MAX + 2) * 4 + TOPK_MAX * 4 + TOPK_MAX * 8;
@@ -99,11 +104,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sm = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* s_full = bars + 1;     // [2]
-  uint64_t* s_free = bars + 3;     // [2]  one arrival per softmax warp
-  uint64_t* p_full = bars + 5;     // [2]  one arrival per softmax warp
-  uint64_t* p_free = bars + 7;     // [2]
-  uint64_t* k_full = bars + 9;     // [NSLOT] each
+  uint64_t* s_full = bars + 1;     // [buffer]
+  uint64_t* s_free = bars + 3;     // [buffer]  both P V that read P over the buffer completed
+  uint64_t* p_full = bars + 5;     // [warpgroup * 2 + buffer]  one arrival per warp of the warpgroup
+  uint64_t* pv_done = bars + 9;    // [warpgroup]  one phase per tile
+  uint64_t* o_done = bars + 11;    // one phase: every MMA of the CTA has completed
+  uint64_t* k_full = bars + 12;    // [NSLOT] each
   uint64_t* k_empty = k_full + NSLOT;
   uint64_t* v_full = k_empty + NSLOT;
   uint64_t* v_empty = v_full + NSLOT;
@@ -142,8 +148,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     doc_base_s[tid] = base;
   }
   if (tid == 0) {
-    // s_free and p_full collect one arrival per softmax warp; the rest one arrival each
-    for (int i = 0; i < N_BAR; ++i) mbar_init(&bars[i], (i >= 3 && i <= 6) ? 8 : 1);
+    // p_full collects one arrival per warp of a warpgroup; the rest one arrival each
+    for (int i = 0; i < N_BAR; ++i) mbar_init(&bars[i], (i >= 5 && i <= 8) ? 4 : 1);
     fence_barrier_init();
     *abort_s = 0;
   }
@@ -223,20 +229,25 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = mbar_wait_bounded(q_full, 0, a.err);
       const uint64_t qdesc = umma_desc_sw128(sbase + OFF_Q, 16, 1024);
       const uint64_t kdesc0 = umma_desc_sw128(sbase + OFF_K0, 16, 1024);
+      // O_h += P_h V_i[64 h, 64 h + 64) for both warpgroups h of tile i
       auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait_bounded(&p_full[i & 1], (i >> 1) & 1, a.err)) return false;
         if (!mbar_wait_bounded(&v_full[i % NSLOT], (i / NSLOT) & 1, a.err)) return false;
-        tc_fence_after();
-        const uint32_t pt = tmem + P_COL + (i & 1) * (TN / 2);
         const uint32_t vb = sbase + OFF_V0 + (i % NSLOT) * TILE;
         const uint64_t vdesc = umma_desc_sw128(vb, BOX, 1024);
 #pragma unroll
-        for (int kk = 0; kk < TN / 16; ++kk) {
-          const uint64_t bd = vdesc + (uint64_t)((kk * 2048) >> 4);
-          umma_bf16_ts(tmem + O_COL, pt + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait_bounded(&p_full[h * 2 + (i & 1)], (i >> 1) & 1, a.err)) return false;
+          tc_fence_after();
+          const uint32_t pt = tmem + (i & 1) * TN + h * (TN / 2);  // P_h over S_h's first 32 columns
+#pragma unroll
+          for (int kk = 0; kk < TN / 32; ++kk) {
+            const uint64_t bd = vdesc + (uint64_t)(((h * 4 + kk) * 2048) >> 4);
+            umma_bf16_ts(tmem + O_COL + h * TD, pt + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&pv_done[h]);
         }
         umma_commit(&v_empty[i % NSLOT]);
-        umma_commit(&p_free[i & 1]);
+        umma_commit(&s_free[i & 1]);
         return true;
       };
       for (int j = 0; ok && j < T; ++j) {
@@ -257,12 +268,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         umma_commit(&k_empty[st]);
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
-      if (ok && T > 0) issue_pv(T - 1);
+      if (ok && T > 0 && issue_pv(T - 1)) umma_commit(o_done);
     }
   } else {
     // ------------------------------------------------------------ softmax
-    // warps 2..9 = two warpgroups; warpgroup wg takes keys [64 wg, 64 wg + 64)
-    // of every row, warp w reads TMEM lanes 32 (w % 4) .. +31 (its rows).
+    // warps 2..9 = two warpgroups; warpgroup wg owns keys [64 wg, 64 wg + 64)
+    // of every tile; warp w reads TMEM lanes 32 (w % 4) .. +31 (its rows).
     const int wg = (warp - 2) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;                  // row inside the CTA tile = TMEM lane
@@ -271,24 +282,25 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int lim = i_first + t_in;                // causal limit among local keys
     const int c0 = wg * (TN / 2);                  // this warpgroup's first key / S column
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+    const uint32_t ocol = tl + O_COL + wg * TD;    // this warpgroup's O
     float m_ref = -INFINITY, l = 0.f;
     int di = 0;
+    bool ok = true;
     for (int j = 0; j < T; ++j) {
-      bool okw = mbar_wait_bounded(&s_full[j & 1], (j >> 1) & 1, a.err);
-      if (j >= 2) okw = okw && mbar_wait_bounded(&p_free[j & 1], ((j - 2) >> 1) & 1, a.err);  // P buffer reusable
+      // S_j was issued only after both P V of tile j-2 completed: its columns are free for P_j
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[j & 1], (j >> 1) & 1, a.err));
+      if (!ok) break;
       tc_fence_after();
       while (di < k && j >= tile_start[di + 1]) ++di;
       const bool local = di >= k;
       const int key0 = (j - tile_start[di]) * TN;
       const int nvalid = local ? TN : min(TN, doc_len_s[di] - key0);
       const int vis_end = local ? max(0, min(TN, lim - key0 + 1)) : nvalid;  // keys [0, vis_end) are visible
+      const uint32_t scol = tl + (j & 1) * TN + c0;
       uint32_t v0[32], v1[32];  // S of keys c0 .. c0+31 and c0+32 .. c0+63
-      {
-        const uint32_t scol = tl + (j & 1) * TN + c0;
-        tmem_ld32(scol, v0);
-        tmem_ld32(scol + 32, v1);
-        tmem_wait_ld();
-      }
+      tmem_ld32(scol, v0);
+      tmem_ld32(scol + 32, v1);
+      tmem_wait_ld();
 #define SV(e) __uint_as_float((e) < 32 ? v0[(e) & 31] : v1[(e) & 31])
       // every key of this half visible for every row of the warp: no per-key masks
       const bool full = __all_sync(0xffffffffu, vis_end >= c0 + TN / 2);
@@ -305,29 +317,16 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (c0 + e < vis_end) mt = fmaxf(mt, SV(e));
         mt = (mt == -INFINITY) ? mt : mt * a.scale_log2;
       }
-      // each warpgroup posts its half-row max in the first S column of its own
-      // half (already read) and takes the partner's from the partner's half
-      const uint32_t sbuf = tl + (j & 1) * TN;
-      tmem_st1(sbuf + c0, __float_as_uint(mt));
-      tmem_wait_st();
-      if (!okw) *abort_s = 1;
-      tc_fence_before();
-      named_barrier_sync(1, 2 * 4 * 32);
-      tc_fence_after();
-      if (*abort_s) break;
-      mt = fmaxf(mt, __uint_as_float(tmem_ld1(sbuf + (c0 ^ (TN / 2)))));
-      tmem_wait_ld();
       const float m_new = fmaxf(m_ref, mt);
-      const bool need = m_new > m_ref + kLazy;  // also true when m_ref = -inf and the tile has a key
+      const bool need = m_new > m_ref + kLazy;  // also true when m_ref = -inf and the half-tile has a key
       float alpha = 1.f;
       if (need) {
         alpha = exp2f(m_ref - m_new);  // 0 when m_ref = -inf
         l *= alpha;
         m_ref = m_new;
       }
-      // P = exp2(S * scale - m_ref) as bf16 pairs into this warpgroup's 32 columns of P_(j&1)
+      // P = exp2(S * scale - m_ref) as bf16 pairs over this half's first 32 S columns (already read)
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      const uint32_t pcol = tl + P_COL + (j & 1) * (TN / 2) + c0 / 2;
       const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_use, -m_use);
       float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
@@ -346,60 +345,75 @@ __global__ void __launch_bounds__(THREADS, 1)
           ls[u & 1] = __fadd2_rn(ls[u & 1], pp);
           pk[u] = pack_bf16(pp.x, pp.y);
         }
-        tmem_st16(pcol + hh * 16, pk);
+        tmem_st16(scol + hh * 16, pk);
       }
       l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
 #undef SV
-      // (after P, so that S is no longer live) the rescale must land before P V of this tile
+      // this warpgroup's P V of tile j-1 (issued a whole tile ago, so normally long
+      // complete): waited at every tile, phase after phase, before O_wg may be rescaled
+      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait_bounded(&pv_done[wg], (j - 1) & 1, a.err))) {
+        ok = false;
+        break;
+      }
       if (__any_sync(0xffffffffu, need && j > 0)) {
-        // O holds the sum up to tile j-1: wait for that P V, then rescale this
-        // warp's rows in this warpgroup's half of the O columns
-        if (!mbar_wait_bounded(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err)) *abort_s = 1;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < TD / 64; ++c) {
+        for (int c = 0; c < TD / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tl + O_COL + c0 + c * 32, o);
+          tmem_ld32(ocol + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tl + O_COL + c0 + c * 32, o);
+          tmem_st32(ocol + c * 32, o);
         }
-        tmem_wait_st();
       }
       tmem_wait_st();  // P (and any rescaled O) is in TMEM before the MMA may read it
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&p_full[j & 1]);
-        mbar_arrive(&s_free[j & 1]);
-      }
+      if (lane == 0) mbar_arrive(&p_full[wg * 2 + (j & 1)]);
     }
-    // ---- epilogue: O / l once the last P V has completed; l sums both halves of the keys
-    // row sums through the second S column of each half of buffer 0 (no S MMA is left)
+    // ---- epilogue: once every P V has completed (o_done has a single phase, so
+    // its wait is unambiguous), merge the two halves' (m, l, O) of each row
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(o_done, 0, a.err));
+    if (!ok) *abort_s = 1;
+    tc_fence_after();
+    // (m, l) through this half's first two columns of S buffer 0, free once its P V completed
+    tmem_st1(tl + c0, __float_as_uint(m_ref));
     tmem_st1(tl + c0 + 1, __float_as_uint(l));
     tmem_wait_st();
     tc_fence_before();
     named_barrier_sync(1, 2 * 4 * 32);
     tc_fence_after();
-    const float lt = l + __uint_as_float(tmem_ld1(tl + ((c0 + 1) ^ (TN / 2))));
-    tmem_wait_ld();
-    if (!*abort_s && T > 0 && mbar_wait_bounded(&p_free[(T - 1) & 1], ((T - 1) >> 1) & 1, a.err)) {
-      tc_fence_after();
+    if (!*abort_s && T > 0) {
+      const uint32_t pc = tl + (c0 ^ (TN / 2));
+      const float m_o = __uint_as_float(tmem_ld1(pc));
+      const float l_o = __uint_as_float(tmem_ld1(pc + 1));
+      tmem_wait_ld();
+      const float mA = wg ? m_o : m_ref, lA = wg ? l_o : l;  // keys [0, 64) of every tile
+      const float mB = wg ? m_ref : m_o, lB = wg ? l : l_o;  // keys [64, 128)
+      const float mm = fmaxf(mA, mB);
+      const float fA = mA == -INFINITY ? 0.f : exp2f(mA - mm);
+      const float fB = mB == -INFINITY ? 0.f : exp2f(mB - mm);
+      const float lt = lA * fA + lB * fB;
       const float inv = lt > 0.f ? 1.0f / lt : 0.f;
+      const float wA = fA * inv, wB = fB * inv;
       const int hq = h * G + g;
       const int t = blk * Bq + t_in;
+      // this warpgroup writes dims [64 wg, 64 wg + 64) of its rows
       float* dst = a.out + (((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t) * TD + c0;
 #pragma unroll
-      for (int c = 0; c < TD / 64; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tl + O_COL + c0 + c * 32, o);
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t oa[32], ob[32];
+        tmem_ld32(tl + O_COL + c0 + cc * 32, oa);
+        tmem_ld32(tl + O_COL + TD + c0 + cc * 32, ob);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dst + c * 32 + e) =
-              make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                          __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+          *reinterpret_cast<float4*>(dst + cc * 32 + e) =
+              make_float4(__uint_as_float(oa[e]) * wA + __uint_as_float(ob[e]) * wB,
+                          __uint_as_float(oa[e + 1]) * wA + __uint_as_float(ob[e + 1]) * wB,
+                          __uint_as_float(oa[e + 2]) * wA + __uint_as_float(ob[e + 2]) * wB,
+                          __uint_as_float(oa[e + 3]) * wA + __uint_as_float(ob[e + 3]) * wB);
       }
     }
   }
