@@ -70,9 +70,16 @@ def tensor_peak():
     return 1590.0, "fallback"
 
 
-def launches_per_step(w) -> int:
-    """Kernels libmsa launches for one route + attend step of workload w."""
-    rows_route = w.batch * (w.q_tokens // w.route_block)
+def launches_per_step(w, batch=None) -> int:
+    """Kernels libmsa launches for one route + attend step of workload w (over `batch`
+    sequences; msa_forward on a pinned-host bank runs micro-batches of up to 4 parts)."""
+    if batch is None and w.host_tier:
+        parts = min(w.batch, 4)
+        nb = -(-w.batch // parts)
+        sizes = [min(nb, w.batch - b0) for b0 in range(0, w.batch, nb)]
+        return sum(launches_per_step(w, b) for b in sizes)
+    batch = w.batch if batch is None else batch
+    rows_route = batch * (w.q_tokens // w.route_block)
     n = (0 if w.route_block <= 4 else 1) + (rows_route + 15) // 16 + 1     # qr_prep, router passes, top-k
     rows = (w.n_q_heads // w.n_kv_heads) * w.route_block
     tc = w.head_dim == 128 and w.route_block in (64, 128) and rows % 128 == 0
@@ -494,11 +501,13 @@ def run_route_only(args):
 
 def run_host_tier(args):
     """Decode steps on a bank whose K/V live in pinned host memory (69M / 100M tokens):
-    route on the device, copy the selected documents' K/V slabs over PCIe, attend."""
+    msa_forward routes on the device, copies the selected documents' K/V slabs over
+    PCIe and attends, pipelined over micro-batches of sequences. Also timed: the
+    routing alone, and routing then attention without the pipeline."""
     import torch
 
     import synth
-    from sparse_attention_routed_b200 import MSA_KV_PINNED_HOST, msa_attend, msa_route
+    from sparse_attention_routed_b200 import MSA_KV_PINNED_HOST, msa_attend, msa_forward, msa_route
     from sparse_attention_routed_b200.runner import Bank
     from synth.device import fill_normal, host_kv_pool, query_tensors
 
@@ -526,8 +535,9 @@ def run_host_tier(args):
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
     for _ in range(max(3, args.warmup)):
-        msa_route(bank.handle, qry, k, 0, idx.data_ptr(), 0, sh)
-        msa_attend(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
+        msa_forward(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
+    msa_route(bank.handle, qry, k, 0, idx.data_ptr(), 0, sh)
+    msa_attend(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
     torch.cuda.synchronize()
     assert bank.device_error() == 0
     sel = idx.cpu().numpy()
@@ -551,21 +561,30 @@ def run_host_tier(args):
     h2d_peak = (1 << 30) / (best / 1e3) / 1e9
     del hbuf, dbuf
     n = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
     clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
     time.sleep(0.4)
     torch.cuda.synchronize()
+    t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_begin.record(stream)
     for i in range(n):
+        msa_forward(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    step_ms = t_begin.elapsed_time(t_end) / n
+    assert bank.device_error() == 0
+    # the routing alone, and routing then attention without the pipeline (a few steps each)
+    n2 = max(3, n // 3)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n2)]
+    for i in range(n2):
         ev[i][0].record(stream)
         msa_route(bank.handle, qry, k, 0, idx.data_ptr(), 0, sh)
         ev[i][1].record(stream)
         msa_attend(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
         ev[i][2].record(stream)
     torch.cuda.synchronize()
-    clk = clocks.stop()
-    route_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / n
-    attend_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / n
-    step_ms = route_ms + attend_ms
+    route_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / n2
+    unpipelined_ms = sum(e[0].elapsed_time(e[2]) for e in ev) / n2
     router_bytes = Hkv * bank.info["n_chunks"] * d * 4
     peak, kind = peaks()
     line = {
@@ -576,12 +595,14 @@ def run_host_tier(args):
         "config": {"workload": args.workload, "batch": B, "q_heads": w.n_q_heads, "kv_heads": Hkv,
                    "head_dim": d, "bank_docs": w.n_docs, "bank_tokens": w.n_tokens, "local_len": w.local_len,
                    "top_k": k, "kv_slabs_pinned": w.kv_slabs, "pinned_kv_bytes": 2 * Kh.numel() * 2},
-        "roofline": {"kernel": "selected K/V slabs over PCIe (cudaMemcpyAsync per slab)", "bound": "pcie",
-                     "achieved": pcie_bytes / (attend_ms / 1e3) / 1e9, "peak": h2d_peak,
+        "roofline": {"kernel": "selected K/V slabs over PCIe (cudaMemcpyAsync per host-contiguous run of slabs), "
+                               "whole pipelined step", "bound": "pcie",
+                     "achieved": pcie_bytes / (step_ms / 1e3) / 1e9, "peak": h2d_peak,
                      "peak_kind": "measured pinned H2D copy, 1 GiB", "unit": "GB/s",
-                     "frac": pcie_bytes / (attend_ms / 1e3) / 1e9 / h2d_peak, "bytes_per_step": pcie_bytes},
+                     "frac": pcie_bytes / (step_ms / 1e3) / 1e9 / h2d_peak, "bytes_per_step": pcie_bytes},
         "router": {"ms": route_ms, "bytes": router_bytes, "GBps": router_bytes / (route_ms / 1e3) / 1e9,
                    "frac_of_hbm_peak": router_bytes / (route_ms / 1e3) / 1e9 / peak},
+        "unpipelined_ms_per_step": unpipelined_ms,
         "planted_recall": recall, "setup_s": setup_s, "clocks": clk,
         "gpu_launches": launches_per_step(w) * n,
     }

@@ -130,8 +130,16 @@ struct msa_bank {
   RouteMaps route_maps{};
   // pinned-host K/V tier: selected slabs are copied into a device staging pool
   static constexpr int kSide = 4;    // copies round-robin over several streams (copy engines)
+#ifndef MSA_HOST_MICRO
+#define MSA_HOST_MICRO 2
+#endif
+  static constexpr int kMicro = MSA_HOST_MICRO;  // micro-batches of msa_forward's fetch / attention pipeline
   cudaStream_t side[kSide] = {};
   cudaEvent_t ev_fetch[kSide] = {};
+  cudaStream_t att = nullptr;        // attention stream of the pipelined forward
+  cudaStream_t rb = nullptr;         // selection read-back, kept apart from the copy queues
+  cudaEvent_t ev_route[kMicro] = {};
+  cudaEvent_t ev_att = nullptr;
   int32_t* h_idx = nullptr;   // pinned copy of the selection
   int64_t* h_base = nullptr;  // pinned staging row of every selection entry
   int64_t* d_base = nullptr;  // device copy of h_base
@@ -151,6 +159,11 @@ void free_bank(msa_bank* b) {
     if (b->side[i]) cudaStreamDestroy(b->side[i]);
     if (b->ev_fetch[i]) cudaEventDestroy(b->ev_fetch[i]);
   }
+  for (int i = 0; i < msa_bank::kMicro; ++i)
+    if (b->ev_route[i]) cudaEventDestroy(b->ev_route[i]);
+  if (b->att) cudaStreamDestroy(b->att);
+  if (b->rb) cudaStreamDestroy(b->rb);
+  if (b->ev_att) cudaEventDestroy(b->ev_att);
   if (b->h_idx) cudaFreeHost(b->h_idx);
   if (b->h_base) cudaFreeHost(b->h_base);
   if (b->d_base) cudaFree(b->d_base);
@@ -330,21 +343,27 @@ msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, co
 
 // Pinned-host tier ("MSA (Memory Sparse Attention)", robocikowo.com, Komponenty:
 // K_r in GPU memory, full K/V in CPU RAM; Pułapki implementacyjne: pinned memory
-// and asynchronous prefetch). The selection is read back, every distinct
+// and asynchronous prefetch). A step's selection is read back, every distinct
 // (document, KV head) slab it names is copied from pinned host memory into the
-// device staging pool on the bank's side streams (one cudaMemcpyAsync per slab
-// and per K/V, round-robin over the streams so that copy engines overlap their
-// per-copy costs), and `st` waits for the copies. Returns the staging row of every
-// selection entry in bank->d_base. Host-synchronising: not capturable.
-msa_status host_fetch(msa_bank* bank, const StepShape& s, const int32_t* idx_dev, cudaStream_t st) {
-  const size_t n = (size_t)s.P * s.k;
+// device staging pool on the bank's side streams with cudaMemcpyAsync, and the
+// attention kernels read the pool. Slabs that are neighbours in host memory (the
+// same head, one document right after the other) get neighbouring staging rows
+// and travel as one copy. Host-synchronising: not capturable.
+
+// Side streams, events, the attention stream and the pinned selection buffers.
+msa_status ensure_host_tier(msa_bank* bank, size_t entries) {
   if (!bank->side[0]) {
     for (int i = 0; i < msa_bank::kSide; ++i) {
       MSA_CUDA(cudaStreamCreateWithFlags(&bank->side[i], cudaStreamNonBlocking));
       MSA_CUDA(cudaEventCreateWithFlags(&bank->ev_fetch[i], cudaEventDisableTiming));
     }
+    for (int i = 0; i < msa_bank::kMicro; ++i)
+      MSA_CUDA(cudaEventCreateWithFlags(&bank->ev_route[i], cudaEventDisableTiming));
+    MSA_CUDA(cudaStreamCreateWithFlags(&bank->att, cudaStreamNonBlocking));
+    MSA_CUDA(cudaStreamCreateWithFlags(&bank->rb, cudaStreamNonBlocking));
+    MSA_CUDA(cudaEventCreateWithFlags(&bank->ev_att, cudaEventDisableTiming));
   }
-  if (n > bank->sel_cap) {
+  if (entries > bank->sel_cap) {
     MSA_CUDA(cudaDeviceSynchronize());
     if (bank->h_idx) cudaFreeHost(bank->h_idx);
     if (bank->h_base) cudaFreeHost(bank->h_base);
@@ -353,70 +372,116 @@ msa_status host_fetch(msa_bank* bank, const StepShape& s, const int32_t* idx_dev
     bank->h_base = nullptr;
     bank->d_base = nullptr;
     bank->sel_cap = 0;
-    if (cudaHostAlloc(&bank->h_idx, n * 4, cudaHostAllocDefault) != cudaSuccess) return MSA_ERR_HOST_TIER;
-    if (cudaHostAlloc(&bank->h_base, n * 8, cudaHostAllocDefault) != cudaSuccess) return MSA_ERR_HOST_TIER;
-    MSA_CUDA(cudaMalloc(&bank->d_base, n * 8));
-    bank->sel_cap = n;
+    if (cudaHostAlloc(&bank->h_idx, entries * 4, cudaHostAllocDefault) != cudaSuccess) return MSA_ERR_HOST_TIER;
+    if (cudaHostAlloc(&bank->h_base, entries * 8, cudaHostAllocDefault) != cudaSuccess) return MSA_ERR_HOST_TIER;
+    MSA_CUDA(cudaMalloc(&bank->d_base, entries * 8));
+    bank->sel_cap = entries;
   }
-  MSA_CUDA(cudaMemcpyAsync(bank->h_idx, idx_dev, n * 4, cudaMemcpyDeviceToHost, st));
-  MSA_CUDA(cudaStreamSynchronize(st));  // also retires every earlier step that read the staging pool
-  std::unordered_map<int64_t, int64_t> slot;
-  slot.reserve(n * 2);
-  std::vector<std::pair<int64_t, int64_t>> uniq;  // (doc * Hkv + head, staging row)
-  int64_t rows = 0;
-  for (size_t e = 0; e < n; ++e) {
-    const int p = (int)(e / s.k);
-    const int h = p % bank->hkv;
-    const int j = bank->h_idx[e];
-    if (j < 0 || j >= bank->n_docs) return MSA_ERR_INVALID_ARG;
-    const int64_t key = (int64_t)j * bank->hkv + h;
-    auto it = slot.find(key);
-    if (it == slot.end()) {
-      it = slot.emplace(key, rows).first;
-      uniq.emplace_back(key, rows);
-      rows += bank->doc_lens[j];
-    }
-    bank->h_base[e] = it->second;
-  }
-  if (rows >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
-  if (rows > bank->stage_cap) {
-    if (capturing(st)) return MSA_ERR_INVALID_ARG;
-    if (bank->stage_k) cudaFree(bank->stage_k);
-    if (bank->stage_v) cudaFree(bank->stage_v);
-    bank->stage_k = bank->stage_v = nullptr;
-    bank->stage_cap = 0;
-    const size_t bytes = (size_t)rows * bank->d * 2;
-    if (cudaMalloc(&bank->stage_k, bytes) != cudaSuccess || cudaMalloc(&bank->stage_v, bytes) != cudaSuccess)
-      return MSA_ERR_OOM;
-    bank->stage_cap = rows;
-  }
-  const size_t row_bytes = (size_t)bank->d * 2;
-  const uint16_t* hk = static_cast<const uint16_t*>(bank->k);
-  const uint16_t* hv = static_cast<const uint16_t*>(bank->v);
-  int64_t bytes = 0;
-  int c = 0;
-  for (const auto& u : uniq) {
-    const int j = (int)(u.first / bank->hkv), h = (int)(u.first % bank->hkv);
-    const int64_t src = ((int64_t)h * bank->kv_rows + bank->doc_rows[j]) * bank->d;
-    const size_t len = (size_t)bank->doc_lens[j] * row_bytes;
-    if (cudaMemcpyAsync(bank->stage_k + u.second * bank->d, hk + src, len, cudaMemcpyHostToDevice,
-                        bank->side[c++ % msa_bank::kSide]) != cudaSuccess ||
-        cudaMemcpyAsync(bank->stage_v + u.second * bank->d, hv + src, len, cudaMemcpyHostToDevice,
-                        bank->side[c++ % msa_bank::kSide]) != cudaSuccess)
-      return MSA_ERR_HOST_TIER;
-    bytes += 2 * (int64_t)len;
-  }
-  MSA_CUDA(cudaMemcpyAsync(bank->d_base, bank->h_base, n * 8, cudaMemcpyHostToDevice, bank->side[0]));
-  for (int i = 0; i < msa_bank::kSide; ++i) {
-    MSA_CUDA(cudaEventRecord(bank->ev_fetch[i], bank->side[i]));
-    MSA_CUDA(cudaStreamWaitEvent(st, bank->ev_fetch[i], 0));
-  }
-  bank->last_fetch_bytes = bytes;
   return MSA_OK;
 }
 
+// Staging pool of at least `rows` rows for K and for V (grows only; the caller
+// has made sure no kernel still reads the old pool).
+msa_status ensure_stage(msa_bank* bank, int64_t rows, cudaStream_t st) {
+  if (rows >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  if (rows <= bank->stage_cap) return MSA_OK;
+  if (capturing(st)) return MSA_ERR_INVALID_ARG;
+  MSA_CUDA(cudaDeviceSynchronize());
+  if (bank->stage_k) cudaFree(bank->stage_k);
+  if (bank->stage_v) cudaFree(bank->stage_v);
+  bank->stage_k = bank->stage_v = nullptr;
+  bank->stage_cap = 0;
+  const size_t bytes = (size_t)rows * bank->d * 2;
+  if (cudaMalloc(&bank->stage_k, bytes) != cudaSuccess || cudaMalloc(&bank->stage_v, bytes) != cudaSuccess)
+    return MSA_ERR_OOM;
+  bank->stage_cap = rows;
+  return MSA_OK;
+}
+
+// Staging plan of one stretch of selection entries [e0, e1) (bank->h_idx holds
+// them): slabs not staged earlier in the step get rows in host-address order,
+// runs of host-contiguous slabs are copied as one, and h_base[e] receives each
+// entry's first staging row. `slot` and `rows` carry the step's earlier plans.
+msa_status stage_entries(msa_bank* bank, int k, size_t e0, size_t e1, std::unordered_map<int64_t, int64_t>& slot,
+                         int64_t& rows, int& stream_rr) {
+  std::vector<std::pair<int64_t, int64_t>> fresh;  // (host row of the slab's first token, doc * Hkv + head)
+  for (size_t e = e0; e < e1; ++e) {
+    const int h = (int)((e / k) % bank->hkv);
+    const int j = bank->h_idx[e];
+    if (j < 0 || j >= bank->n_docs) return MSA_ERR_INVALID_ARG;
+    const int64_t key = (int64_t)j * bank->hkv + h;
+    if (slot.emplace(key, -1).second) fresh.emplace_back((int64_t)h * bank->kv_rows + bank->doc_rows[j], key);
+  }
+  std::sort(fresh.begin(), fresh.end());
+  const size_t row_bytes = (size_t)bank->d * 2;
+  const uint16_t* hk = static_cast<const uint16_t*>(bank->k);
+  const uint16_t* hv = static_cast<const uint16_t*>(bank->v);
+  size_t i = 0;
+  while (i < fresh.size()) {
+    // a run: each next slab starts where the previous one ends, inside the same head
+    const int64_t src0 = fresh[i].first, dst0 = rows;
+    int64_t len = 0;
+    size_t r = i;
+    for (; r < fresh.size(); ++r) {
+      const int64_t key = fresh[r].second;
+      const int j = (int)(key / bank->hkv), h = (int)(key % bank->hkv);
+      if (r > i && (fresh[r].first != src0 + len || (src0 / bank->kv_rows) != h)) break;
+      slot[key] = dst0 + len;
+      len += bank->doc_lens[j];
+    }
+    if (rows + len > bank->stage_cap) return MSA_ERR_HOST_TIER;
+    const size_t bytes = (size_t)len * row_bytes;
+    if (cudaMemcpyAsync(bank->stage_k + dst0 * bank->d, hk + src0 * bank->d, bytes, cudaMemcpyHostToDevice,
+                        bank->side[stream_rr++ % msa_bank::kSide]) != cudaSuccess ||
+        cudaMemcpyAsync(bank->stage_v + dst0 * bank->d, hv + src0 * bank->d, bytes, cudaMemcpyHostToDevice,
+                        bank->side[stream_rr++ % msa_bank::kSide]) != cudaSuccess)
+      return MSA_ERR_HOST_TIER;
+    bank->last_fetch_bytes += 2 * (int64_t)bytes;
+    rows += len;
+    i = r;
+  }
+  for (size_t e = e0; e < e1; ++e) {
+    const int h = (int)((e / k) % bank->hkv);
+    bank->h_base[e] = slot[(int64_t)bank->h_idx[e] * bank->hkv + h];
+  }
+  return MSA_OK;
+}
+
+// Upper bound of the staging rows a step can need (every entry a different slab).
+int64_t stage_bound(const msa_bank* bank, const StepShape& s) { return (int64_t)s.P * s.k * bank->max_len; }
+
+// `to` waits for everything issued so far on the side streams.
+msa_status join_side(msa_bank* bank, cudaStream_t to) {
+  for (int i = 0; i < msa_bank::kSide; ++i) {
+    MSA_CUDA(cudaEventRecord(bank->ev_fetch[i], bank->side[i]));
+    MSA_CUDA(cudaStreamWaitEvent(to, bank->ev_fetch[i], 0));
+  }
+  return MSA_OK;
+}
+
+// Whole-step fetch for msa_attend: returns the staging row of every selection
+// entry in bank->d_base; `st` waits for the copies.
+msa_status host_fetch(msa_bank* bank, const StepShape& s, const int32_t* idx_dev, cudaStream_t st) {
+  const size_t n = (size_t)s.P * s.k;
+  msa_status rc = ensure_host_tier(bank, n);
+  if (rc != MSA_OK) return rc;
+  MSA_CUDA(cudaMemcpyAsync(bank->h_idx, idx_dev, n * 4, cudaMemcpyDeviceToHost, st));
+  MSA_CUDA(cudaStreamSynchronize(st));  // also retires every earlier step that read the staging pool
+  if ((rc = ensure_stage(bank, stage_bound(bank, s), st)) != MSA_OK) return rc;
+  std::unordered_map<int64_t, int64_t> slot;
+  slot.reserve(n * 2);
+  int64_t rows = 0;
+  int rr = 0;
+  bank->last_fetch_bytes = 0;
+  if ((rc = stage_entries(bank, s.k, 0, n, slot, rows, rr)) != MSA_OK) return rc;
+  MSA_CUDA(cudaMemcpyAsync(bank->d_base, bank->h_base, n * 8, cudaMemcpyHostToDevice, bank->side[0]));
+  return join_side(bank, st);
+}
+
+// `staged`: for a pinned-host bank whose selection the caller has already staged,
+// the device table of staging rows (one per selection entry); NULL fetches here.
 msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, int splits, const Workspace& w,
-                       const int32_t* idx, float* out, cudaStream_t st) {
+                       const int32_t* idx, float* out, cudaStream_t st, const int64_t* staged = nullptr) {
   const bool prefill = s.rows > kMaxRows;
   const bool tc = prefill && attend_prefill_tc_supported(bank->d, s.G, s.Bq);
   const int box = tc ? attend_prefill_tc_tile_rows() : prefill ? attend_prefill_tile_rows() : attend_tile_rows();
@@ -424,11 +489,14 @@ msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, i
   AttendMaps maps;
   const int64_t* sel_base = nullptr;
   if (bank->kv_loc == MSA_KV_PINNED_HOST) {
-    msa_status rf = host_fetch(bank, s, idx, st);
-    if (rf != MSA_OK) return rf;
+    msa_status rf = MSA_OK;
+    if (!staged) {
+      if ((rf = host_fetch(bank, s, idx, st)) != MSA_OK) return rf;
+      staged = bank->d_base;
+    }
     if ((rf = make_map(&maps.bank_k, bank->stage_k, bank->stage_cap, bank->d, box)) != MSA_OK) return rf;
     if ((rf = make_map(&maps.bank_v, bank->stage_v, bank->stage_cap, bank->d, box)) != MSA_OK) return rf;
-    sel_base = bank->d_base;
+    sel_base = staged;
   } else {
     maps.bank_k = tc ? bank->map_k128 : prefill ? bank->map_k64 : bank->map_k;
     maps.bank_v = tc ? bank->map_v128 : prefill ? bank->map_v64 : bank->map_v;
@@ -488,6 +556,88 @@ void msa_bank_route_view(const msa_bank* bank, msa::BankRouteView* v) {
   v->n_docs = bank->n_docs;
   v->n_kv_heads = bank->hkv;
   v->route_dim = bank->dr;
+}
+
+// msa_forward on a pinned-host bank: the batch runs as up to kMicro
+// micro-batches of sequences, so that the PCIe fetch overlaps the GPU work
+// ("MSA (Memory Sparse Attention)", robocikowo.com, Pułapki implementacyjne:
+// pinned memory and asynchronous prefetch). Every micro-batch's routing is
+// queued on `st` at once; the host then takes the micro-batches in order: it
+// reads one's selection back as soon as its routing is done (the next
+// micro-batch's routing runs meanwhile), stages its slabs on the side streams,
+// and queues its attention on the attention stream behind those copies, so that
+// attention of micro-batch i runs while micro-batch i+1 is being copied. A slab
+// selected by several micro-batches is copied once. `st` waits for the last
+// attention.
+msa_status forward_host(msa_bank* bank, const msa_query* q, const StepShape& s, int32_t* topk_idx, float* out,
+                        cudaStream_t st) {
+  const int M = std::min(s.B, msa_bank::kMicro);
+  const int nb = (s.B + M - 1) / M;  // sequences per micro-batch (the last may hold fewer)
+  StepShape sm = s;
+  sm.B = nb;
+  sm.P = nb * s.nblk * bank->hkv;
+  const int splits = choose_splits(bank, sm);
+  Workspace w = layout(bank, sm, splits, nullptr);
+  msa_status rc = ensure_workspace(bank, w.bytes, st);
+  if (rc != MSA_OK) return rc;
+  if ((rc = ensure_gtab(bank, (int64_t)s.k * bank->max_len, s.Lc, st)) != MSA_OK) return rc;
+  w = layout(bank, sm, splits, bank->ws);
+  const size_t n = (size_t)s.P * s.k;
+  if ((rc = ensure_host_tier(bank, n)) != MSA_OK) return rc;
+  if ((rc = ensure_stage(bank, stage_bound(bank, s), st)) != MSA_OK) return rc;
+  if (capturing(st)) return MSA_ERR_INVALID_ARG;
+
+  const size_t d = bank->d;
+  auto sub = [&](int b0, int bn, msa_query* qm, StepShape* sh) {
+    *qm = *q;
+    qm->batch = bn;
+    qm->q = static_cast<const uint16_t*>(q->q) + (size_t)b0 * s.Hq * s.Tq * d;
+    qm->qr = static_cast<const uint16_t*>(q->qr) + (size_t)b0 * bank->hkv * s.Tq * bank->dr;
+    qm->local_k = static_cast<const uint16_t*>(q->local_k) + (size_t)b0 * bank->hkv * s.Lc * d;
+    qm->local_v = static_cast<const uint16_t*>(q->local_v) + (size_t)b0 * bank->hkv * s.Lc * d;
+    *sh = s;
+    sh->B = bn;
+    sh->P = bn * s.nblk * bank->hkv;
+  };
+  const size_t per_seq = (size_t)s.nblk * bank->hkv * s.k;  // selection entries per sequence
+  for (int m = 0; m < M; ++m) {
+    const int b0 = m * nb, bn = std::min(nb, s.B - b0);
+    if (bn <= 0) break;
+    msa_query qm;
+    StepShape sh;
+    sub(b0, bn, &qm, &sh);
+    if ((rc = route_impl(bank, &qm, sh, w, nullptr, topk_idx + b0 * per_seq, nullptr, st)) != MSA_OK) return rc;
+    MSA_CUDA(cudaEventRecord(bank->ev_route[m], st));
+  }
+  std::unordered_map<int64_t, int64_t> slot;
+  slot.reserve(n * 2);
+  int64_t rows = 0;
+  int rr = 0;
+  bank->last_fetch_bytes = 0;
+  for (int m = 0; m < M; ++m) {
+    const int b0 = m * nb, bn = std::min(nb, s.B - b0);
+    if (bn <= 0) break;
+    msa_query qm;
+    StepShape sh;
+    sub(b0, bn, &qm, &sh);
+    const size_t e0 = (size_t)b0 * per_seq, e1 = e0 + (size_t)bn * per_seq;
+    // the selection of micro-batch m (its routing is the last thing ev_route[m] waits for;
+    // for m = 0 it also follows every earlier step's attention, which read the pool)
+    MSA_CUDA(cudaStreamWaitEvent(bank->rb, bank->ev_route[m], 0));
+    MSA_CUDA(cudaMemcpyAsync(bank->h_idx + e0, topk_idx + e0, (e1 - e0) * 4, cudaMemcpyDeviceToHost, bank->rb));
+    MSA_CUDA(cudaStreamSynchronize(bank->rb));
+    if ((rc = stage_entries(bank, s.k, e0, e1, slot, rows, rr)) != MSA_OK) return rc;
+    MSA_CUDA(cudaMemcpyAsync(bank->d_base + e0, bank->h_base + e0, (e1 - e0) * 8, cudaMemcpyHostToDevice,
+                             bank->side[0]));
+    if ((rc = join_side(bank, bank->att)) != MSA_OK) return rc;
+    MSA_CUDA(cudaStreamWaitEvent(bank->att, bank->ev_route[m], 0));
+    if ((rc = attend_impl(bank, &qm, sh, splits, w, topk_idx + e0, out + (size_t)b0 * s.Hq * s.Tq * d, bank->att,
+                          bank->d_base + e0)) != MSA_OK)
+      return rc;
+  }
+  MSA_CUDA(cudaEventRecord(bank->ev_att, bank->att));
+  MSA_CUDA(cudaStreamWaitEvent(st, bank->ev_att, 0));
+  return MSA_OK;
 }
 
 extern "C" {
@@ -711,6 +861,7 @@ msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_
   if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->max_len, s.Lc, (cudaStream_t)stream)) != MSA_OK) return rc;
   w = layout(bank, s, splits, bank->ws);
   cudaStream_t st = (cudaStream_t)stream;
+  if (bank->kv_loc == MSA_KV_PINNED_HOST) return forward_host(bank, q, s, topk_idx, out, st);
   if ((rc = route_impl(bank, q, s, w, nullptr, topk_idx, nullptr, st)) != MSA_OK) return rc;
   return attend_impl(bank, q, s, splits, w, topk_idx, out, st);
 }

@@ -22,6 +22,10 @@ HOST = {
     # 256-row problems (tcgen05 prefill) reading the staging pool
     "host_prefill": Workload("host_prefill", 33, 1, 8, 2, 128, 16, 0, 256, 128, 64, 3, ragged=(100, 900),
                              host_tier=True, kv_slabs=4),
+    # 5 sequences: msa_forward runs micro-batches of 2, 2 and 1 sequences; 12 equal-length
+    # documents over 6 slabs, so sequences share slabs across micro-batches and slabs that
+    # are neighbours in host memory are copied as one
+    "host_micro": Workload("host_micro", 34, 5, 8, 2, 128, 12, 300, 200, 1, 1, 4, host_tier=True, kv_slabs=6),
 }
 
 
@@ -74,8 +78,10 @@ def test_host_tier_parity(name):
                  ref["doc_scores"].reshape(-1, w.n_docs), w.top_k)
     ref2 = O.forward(inp, w.doc_lens(), w.top_k, w.route_block, w.rope_base, selection=g["idx"])
     P.check_out(g["out"], ref2["out"])
+    # msa_forward pipelines micro-batches of sequences (its split-KV partition may differ
+    # from msa_attend's on the whole batch, so its output is checked against the oracle)
     np.testing.assert_array_equal(g["idx2"], g["idx"])
-    np.testing.assert_array_equal(g["out2"], g["out"])
+    P.check_out(g["out2"], ref2["out"])
     import sparse_attention_routed_b200 as msa
     assert g["bad_status"] == msa.MSA_ERR_INVALID_ARG
 
