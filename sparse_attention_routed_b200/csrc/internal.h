@@ -60,10 +60,16 @@ struct RouteArgs {
 // Largest routing block for which the router computes q_r itself.
 constexpr int kRouteFuseMaxBlock = 4;
 struct RouteMaps {
-  CUtensorMap k_hat_hi, k_hat_lo;  // boxes of route_tile_rows() chunks x 64 dims
+  CUtensorMap k_hat_hi, k_hat_lo;        // boxes of route_tile_rows() chunks x 64 dims
+  CUtensorMap k_hat_hi128, k_hat_lo128;  // boxes of route_tc_tile_rows() chunks x 64 dims
 };
 cudaError_t launch_route(const RouteArgs& a, const RouteMaps& m, cudaStream_t s);
 int route_tile_rows();
+// tcgen05 router for more than 16 routing rows at d_r = 128 (q_r and 1/|q_r|
+// precomputed by launch_qr_prep); same results up to summation order.
+bool route_tc_supported(int route_dim, int rows);
+int route_tc_tile_rows();
+cudaError_t launch_route_tc(const RouteArgs& a, const RouteMaps& m, int sms, cudaStream_t s);
 
 // Top-k per row of doc_scores, ordered (score desc, index asc).
 struct TopkArgs {
@@ -117,7 +123,7 @@ struct BankRouteView {
   RouteMaps maps;
   const int32_t* chunk_off;
   int64_t nch;
-  int32_t n_docs, n_kv_heads, route_dim;
+  int32_t n_docs, n_kv_heads, route_dim, sms;
 };
 
 // Host-side helpers.

@@ -316,7 +316,8 @@ msa_status ensure_gtab(msa_bank* bank, int64_t koff, int lc, cudaStream_t s) {
 msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, const Workspace& w,
                       float* doc_scores, int32_t* idx, float* top_scores, cudaStream_t st) {
   RouteArgs ra{};
-  const bool fuse = s.Bq <= kRouteFuseMaxBlock;  // the router forms q_r itself
+  const bool tc = route_tc_supported(bank->dr, s.B * s.nblk);
+  const bool fuse = !tc && s.Bq <= kRouteFuseMaxBlock;  // the router forms q_r itself
   if (!fuse) {
     QrArgs qa{(const uint16_t*)q->qr, w.q_r, w.q_r_inv, s.B, bank->hkv, s.Tq, s.Bq, bank->dr};
     MSA_CUDA(launch_qr_prep(qa, st));
@@ -335,7 +336,11 @@ msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, co
   ra.n_docs = bank->n_docs;
   ra.route_dim = bank->dr;
   ra.err = bank->d_err;
-  MSA_CUDA(launch_route(ra, bank->route_maps, st));
+  if (tc) {
+    MSA_CUDA(launch_route_tc(ra, bank->route_maps, bank->sms, st));
+  } else {
+    MSA_CUDA(launch_route(ra, bank->route_maps, st));
+  }
   TopkArgs ta{ra.doc_scores, idx, top_scores, s.P, bank->n_docs, s.k};
   MSA_CUDA(launch_topk(ta, st));
   return MSA_OK;
@@ -556,6 +561,7 @@ void msa_bank_route_view(const msa_bank* bank, msa::BankRouteView* v) {
   v->n_docs = bank->n_docs;
   v->n_kv_heads = bank->hkv;
   v->route_dim = bank->dr;
+  v->sms = bank->sms;
 }
 
 // msa_forward on a pinned-host bank: the batch runs as up to kMicro
@@ -743,6 +749,12 @@ msa_status msa_bank_create(const msa_bank_config* cfg, msa_bank** out) {
   if ((rc = make_map(&b->route_maps.k_hat_hi, b->d_khi, (int64_t)b->hkv * b->nch, b->dr, route_tile_rows())) != MSA_OK)
     return fail(rc);
   if ((rc = make_map(&b->route_maps.k_hat_lo, b->d_klo, (int64_t)b->hkv * b->nch, b->dr, route_tile_rows())) != MSA_OK)
+    return fail(rc);
+  if ((rc = make_map(&b->route_maps.k_hat_hi128, b->d_khi, (int64_t)b->hkv * b->nch, b->dr,
+                     route_tc_tile_rows())) != MSA_OK)
+    return fail(rc);
+  if ((rc = make_map(&b->route_maps.k_hat_lo128, b->d_klo, (int64_t)b->hkv * b->nch, b->dr,
+                     route_tc_tile_rows())) != MSA_OK)
     return fail(rc);
   if (cudaMalloc(&b->d_err, sizeof(int)) != cudaSuccess) return fail(MSA_ERR_OOM);
   if (cudaMemset(b->d_err, 0, sizeof(int)) != cudaSuccess) return fail(MSA_ERR_CUDA);

@@ -88,7 +88,10 @@ extern "C" msa_status msa_route_noalloc(msa_bank* bank, const msa_query* q, int3
   ra.n_kv_heads = v.n_kv_heads;
   ra.n_docs = v.n_docs;
   ra.route_dim = v.route_dim;
-  if (msa::launch_route(ra, v.maps, s) != cudaSuccess) return MSA_ERR_CUDA;
+  // the same router msa_route takes for this shape
+  const cudaError_t e = msa::route_tc_supported(v.route_dim, (int)rows) ? msa::launch_route_tc(ra, v.maps, v.sms, s)
+                                                                          : msa::launch_route(ra, v.maps, s);
+  if (e != cudaSuccess) return MSA_ERR_CUDA;
   msa::TopkArgs ta{scores, topk_idx, topk_scores, (int32_t)(rows * v.n_kv_heads), v.n_docs, top_k};
   if (msa::launch_topk(ta, s) != cudaSuccess) return MSA_ERR_CUDA;
   return MSA_OK;

@@ -29,6 +29,10 @@ SMALL = {
     # 3 heads x 48 tokens = 144 rows (a 16-row tail CTA), ragged docs, queries not at the local start
     "prefill_ragged": Workload("prefill_ragged", 18, 2, 6, 2, 128, 20, 0, 300, 96, 48, 4, ragged=(1, 900)),
     "prefill_d64": Workload("prefill_d64", 19, 1, 4, 1, 64, 12, 0, 200, 64, 32, 12, ragged=(50, 400)),
+    # more than 16 routing rows per KV head: the tcgen05 router (64 rows, ragged documents)
+    "route_tc_rows": Workload("route_tc_rows", 20, 2, 8, 2, 128, 30, 0, 300, 32, 1, 5, ragged=(1, 900)),
+    # 160 routing rows: two passes of the tcgen05 router (128 + 32 rows)
+    "route_tc_passes": Workload("route_tc_passes", 22, 5, 4, 4, 128, 20, 520, 64, 32, 1, 3),
 }
 
 
