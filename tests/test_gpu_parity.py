@@ -33,6 +33,11 @@ SMALL = {
     "route_tc_rows": Workload("route_tc_rows", 20, 2, 8, 2, 128, 30, 0, 300, 32, 1, 5, ragged=(1, 900)),
     # 160 routing rows: two passes of the tcgen05 router (128 + 32 rows)
     "route_tc_passes": Workload("route_tc_passes", 22, 5, 4, 4, 128, 20, 520, 64, 32, 1, 3),
+    # tcgen05 prefill with 128-token routing blocks and G = 1 (one 128-row CTA per problem);
+    # the queries are the whole local context (Lc = Tq)
+    "prefill_bq128": Workload("prefill_bq128", 23, 1, 2, 2, 128, 10, 0, 256, 256, 128, 3, ragged=(60, 700)),
+    # the largest top_k (64) over 80 short documents, decode kernel with G = 2
+    "topk64": Workload("topk64", 24, 2, 4, 2, 128, 80, 0, 130, 1, 1, 64, ragged=(1, 200)),
 }
 
 
