@@ -55,6 +55,18 @@ constexpr float kLazy = 8.0f;         // rescale O only when a row max grows by 
 #define MSA_PF_POLY 1                 // of every 4 key pairs, how many take exp2 on the FMA pipe
 #endif
 constexpr int kPolyPairs = MSA_PF_POLY;
+#ifndef MSA_PF_OPTIMISTIC
+#define MSA_PF_OPTIMISTIC 1
+#endif
+// Full half-tiles skip the row-max pass: P is taken against the current
+// reference max and the tile is kept while every P stays below 2^64 (bf16 and
+// the fp32 accumulators hold such values with their full relative precision);
+// otherwise, and for the first and the masked tiles, the exact path runs.
+constexpr bool kOptimistic = MSA_PF_OPTIMISTIC != 0;
+#ifndef MSA_PF_PMAX
+#define MSA_PF_PMAX 18446744073709551616.f  // 2^64
+#endif
+constexpr float kPMax = MSA_PF_PMAX;
 
 // 2^x on the FMA and integer pipes, to share the exponentials of a tile between
 // them and the special-function unit. Range reduction x = n + f with n the
@@ -304,50 +316,76 @@ __global__ void __launch_bounds__(THREADS, 1)
 #define SV(e) __uint_as_float((e) < 32 ? v0[(e) & 31] : v1[(e) & 31])
       // every key of this half visible for every row of the warp: no per-key masks
       const bool full = __all_sync(0xffffffffu, vis_end >= c0 + TN / 2);
-      float mt;
-      if (full) {
-        float m4[4] = {SV(0), SV(1), SV(2), SV(3)};
-#pragma unroll
-        for (int pr = 2; pr < TN / 4; ++pr) m4[pr & 3] = max3f(m4[pr & 3], SV(2 * pr), SV(2 * pr + 1));
-        mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale_log2;
-      } else {
-        mt = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < TN / 2; ++e)
-          if (c0 + e < vis_end) mt = fmaxf(mt, SV(e));
-        mt = (mt == -INFINITY) ? mt : mt * a.scale_log2;
-      }
-      const float m_new = fmaxf(m_ref, mt);
-      const bool need = m_new > m_ref + kLazy;  // also true when m_ref = -inf and the half-tile has a key
+      bool need = false;  // the reference max moved (O and l rescaled by alpha)
       float alpha = 1.f;
-      if (need) {
-        alpha = exp2f(m_ref - m_new);  // 0 when m_ref = -inf
-        l *= alpha;
-        m_ref = m_new;
-      }
-      // P = exp2(S * scale - m_ref) as bf16 pairs over this half's first 32 S columns (already read)
-      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_use, -m_use);
-      float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      bool done = false;
+      if (kOptimistic && full && __all_sync(0xffffffffu, m_ref != -INFINITY)) {
+        // fast path: P = exp2(S * scale - m_ref) with the current reference, no max pass
+        const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_ref, -m_ref);
+        float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t pk[16];
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int e = hh * 32 + 2 * u;
-          const bool poly = (u & 3) >= 4 - kPolyPairs;
-          const float2 x = __ffma2_rn(make_float2(SV(e), SV(e + 1)), sc2, nm2);
-          float2 pp = poly ? exp2_poly3x2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          if (!full) {
-            pp.x = (c0 + e < vis_end) ? pp.x : 0.f;
-            pp.y = (c0 + e + 1 < vis_end) ? pp.y : 0.f;
+          for (int u = 0; u < 16; ++u) {
+            const int e = hh * 32 + 2 * u;
+            const float2 x = __ffma2_rn(make_float2(SV(e), SV(e + 1)), sc2, nm2);
+            const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));  // +inf past 2^128
+            ls[u & 1] = __fadd2_rn(ls[u & 1], pp);
+            pk[u] = pack_bf16(pp.x, pp.y);
           }
-          ls[u & 1] = __fadd2_rn(ls[u & 1], pp);
-          pk[u] = pack_bf16(pp.x, pp.y);
+          tmem_st16(scol + hh * 16, pk);
         }
-        tmem_st16(scol + hh * 16, pk);
+        const float lt = (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+        done = __all_sync(0xffffffffu, lt < kPMax);  // false for +inf and NaN as well
+        if (done) l += lt;
       }
-      l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+      if (!done) {
+        // exact path: the (masked) half-row max, the lazy reference update, P over the S columns
+        float mt;
+        if (full) {
+          float m4[4] = {SV(0), SV(1), SV(2), SV(3)};
+#pragma unroll
+          for (int pr = 2; pr < TN / 4; ++pr) m4[pr & 3] = max3f(m4[pr & 3], SV(2 * pr), SV(2 * pr + 1));
+          mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale_log2;
+        } else {
+          mt = -INFINITY;
+#pragma unroll
+          for (int e = 0; e < TN / 2; ++e)
+            if (c0 + e < vis_end) mt = fmaxf(mt, SV(e));
+          mt = (mt == -INFINITY) ? mt : mt * a.scale_log2;
+        }
+        const float m_new = fmaxf(m_ref, mt);
+        need = m_new > m_ref + kLazy;  // also true when m_ref = -inf and the half-tile has a key
+        if (need) {
+          alpha = exp2f(m_ref - m_new);  // 0 when m_ref = -inf
+          l *= alpha;
+          m_ref = m_new;
+        }
+        // P = exp2(S * scale - m_ref) as bf16 pairs over this half's first 32 S columns (already read)
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_use, -m_use);
+        float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int e = hh * 32 + 2 * u;
+            const bool poly = (u & 3) >= 4 - kPolyPairs;
+            const float2 x = __ffma2_rn(make_float2(SV(e), SV(e + 1)), sc2, nm2);
+            float2 pp = poly ? exp2_poly3x2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if (!full) {
+              pp.x = (c0 + e < vis_end) ? pp.x : 0.f;
+              pp.y = (c0 + e + 1 < vis_end) ? pp.y : 0.f;
+            }
+            ls[u & 1] = __fadd2_rn(ls[u & 1], pp);
+            pk[u] = pack_bf16(pp.x, pp.y);
+          }
+          tmem_st16(scol + hh * 16, pk);
+        }
+        l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+      }
 #undef SV
       // this warpgroup's P V of tile j-1 (issued a whole tile ago, so normally long
       // complete): waited at every tile, phase after phase, before O_wg may be rescaled
