@@ -63,6 +63,10 @@ constexpr int kPolyPairs = MSA_PF_POLY;
 // the fp32 accumulators hold such values with their full relative precision);
 // otherwise, and for the first and the masked tiles, the exact path runs.
 constexpr bool kOptimistic = MSA_PF_OPTIMISTIC != 0;
+#ifndef MSA_PF_FAST_POLY
+#define MSA_PF_FAST_POLY 0            // of every 4 key pairs of the fast path, how many take the polynomial
+#endif
+constexpr int kFastPoly = MSA_PF_FAST_POLY;
 #ifndef MSA_PF_PMAX
 #define MSA_PF_PMAX 18446744073709551616.f  // 2^64
 #endif
@@ -74,12 +78,13 @@ constexpr float kPMax = MSA_PF_PMAX;
 // f in [-1/2, 1/2]; 2^f from a cubic whose coefficients are a Remez
 // (equioscillating relative error) fit on that interval, max relative error
 // 7.5e-5 -- far below the 2^-9 of the bf16 rounding P gets next; 2^n is
-// added to the exponent field. x is clamped at -125 so the result stays normal
-// (its weight next to the row max is then below 2^-125 anyway).
+// added to the exponent field.
 // Two lanes at once with the packed fp32x2 FMA/add of sm_100.
 __device__ __forceinline__ float2 exp2_poly3x2(float2 x) {
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
+  // [-125, 64]: the result stays normal, and above 2^64 it saturates there (which the
+  // fast path's row-sum check rejects, as it rejects ex2's +inf)
+  x.x = fminf(fmaxf(x.x, -125.f), 64.f);
+  x.y = fminf(fmaxf(x.y, -125.f), 64.f);
   const float2 big = make_float2(12582912.f, 12582912.f), nbig = make_float2(-12582912.f, -12582912.f);
   const float2 j = __fadd2_rn(x, big);
   const float2 f = __ffma2_rn(__fadd2_rn(j, nbig), make_float2(-1.f, -1.f), x);  // x - (j - big)
@@ -329,8 +334,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             const int e = hh * 32 + 2 * u;
+            const bool poly = (u & 3) >= 4 - kFastPoly;
             const float2 x = __ffma2_rn(make_float2(SV(e), SV(e + 1)), sc2, nm2);
-            const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));  // +inf past 2^128
+            // ex2: +inf past 2^128; the polynomial: 2^64 at most
+            const float2 pp = poly ? exp2_poly3x2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
             ls[u & 1] = __fadd2_rn(ls[u & 1], pp);
             pk[u] = pack_bf16(pp.x, pp.y);
           }
