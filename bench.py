@@ -295,13 +295,23 @@ def run_ours(args):
     torch.cuda.synchronize()
     del R
     torch.cuda.empty_cache()
-    Q, Qr, LK, LV = query_tensors(w)
+    # the step's inputs and outputs live in a few contiguous device buffers (queries and
+    # routing queries together, local K and V together, output and selection together),
+    # so that the end-to-end run moves each group with one copy
+    Q0, Qr0, LK0, LV0 = query_tensors(w)
+    qin = torch.cat([Q0.reshape(-1), Qr0.reshape(-1)])
+    Q, Qr = qin[:Q0.numel()].view(Q0.shape), qin[Q0.numel():].view(Qr0.shape)
+    kvloc = torch.stack([LK0, LV0])
+    LK, LV = kvloc[0], kvloc[1]
+    del Q0, Qr0, LK0, LV0
     qry = bank.query(Q, Qr, LK, LV, w.route_block)
     bank.reserve(qry, w.top_k)
     B, k, Hkv, d = w.batch, w.top_k, w.n_kv_heads, w.head_dim
     nblk = w.q_tokens // w.route_block
-    idx = torch.empty((B, nblk, Hkv, k), dtype=torch.int32, device="cuda")
-    out = torch.empty((B, w.n_q_heads, w.q_tokens, d), dtype=torch.float32, device="cuda")
+    n_out, n_idx = B * w.n_q_heads * w.q_tokens * d, B * nblk * Hkv * k
+    outbuf = torch.empty(4 * (n_out + n_idx), dtype=torch.uint8, device="cuda")
+    out = outbuf[:4 * n_out].view(torch.float32).view(B, w.n_q_heads, w.q_tokens, d)
+    idx = outbuf[4 * n_out:].view(torch.int32).view(B, nblk, Hkv, k)
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
 
@@ -362,27 +372,19 @@ def run_ours(args):
     # e2e: pinned host inputs of each step copied in -- decode: queries, routing
     # queries and the newest local token's K/V; prefill: queries, routing queries
     # and the whole local K/V (the prompt) -- the step run, output + selection copied out.
-    q_h = Q.cpu().pin_memory()
-    qr_h = Qr.cpu().pin_memory()
-    kv_h = (torch.stack([LK, LV]) if prefill else torch.stack([LK[:, :, -1], LV[:, :, -1]])).cpu().pin_memory()
-    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    idx_h = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
-    h2d = q_h.numel() * 2 + qr_h.numel() * 2 + kv_h.numel() * 2
-    d2h = out_h.numel() * 4 + idx_h.numel() * 4
+    qin_h = qin.cpu().pin_memory()
+    new_kv = kvloc if prefill else kvloc[:, :, :, -1]   # decode: the newest local token's K and V
+    kv_h = new_kv.cpu().pin_memory()
+    out_h = torch.empty(outbuf.shape, dtype=outbuf.dtype, pin_memory=True)
+    h2d = qin_h.numel() * 2 + kv_h.numel() * 2
+    d2h = out_h.numel()
     n_e2e = max(10, n // 2)
 
     def e2e_step():
-        Q.copy_(q_h, non_blocking=True)
-        Qr.copy_(qr_h, non_blocking=True)
-        if prefill:
-            LK.copy_(kv_h[0], non_blocking=True)
-            LV.copy_(kv_h[1], non_blocking=True)
-        else:
-            LK[:, :, -1].copy_(kv_h[0], non_blocking=True)
-            LV[:, :, -1].copy_(kv_h[1], non_blocking=True)
+        qin.copy_(qin_h, non_blocking=True)
+        new_kv.copy_(kv_h, non_blocking=True)
         step()
-        out_h.copy_(out, non_blocking=True)
-        idx_h.copy_(idx, non_blocking=True)
+        out_h.copy_(outbuf, non_blocking=True)
 
     for _ in range(3):
         e2e_step()
