@@ -46,6 +46,10 @@ def parse():
     ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "decode_512k", "prefill", "prefill_64docs", "ragged_planted", "bank_100m"],
                     help="decode_512k: the same step on a 128-document bank (profiling captures); "
                          "prefill: 4096 query tokens in 64-token routing blocks (tensor-bound)")
+    ap.add_argument("--kv-cache-gb", type=float, default=0.0,
+                    help="host-tier workloads: device-resident slab cache of this many GB (msa_set_kv_cache); "
+                         "each step then takes one of --query-pool query batches at random")
+    ap.add_argument("--query-pool", type=int, default=4)
     ap.add_argument("--route-only", action="store_true",
                     help="time msa_route alone on the full bank's K_r with a stand-in 1-document K/V "
                          "(routing keys streamed in slices; a few GB on the device, for profiling captures)")
@@ -530,6 +534,8 @@ def run_host_tier(args):
         del R
     torch.cuda.synchronize()
     setup_s = time.time() - t0
+    if args.kv_cache_gb > 0:
+        return run_host_cache(args, w, bank, setup_s, Kh)
     Q, Qr, LK, LV = query_tensors(w)
     qry = bank.query(Q, Qr, LK, LV, w.route_block)
     idx = torch.empty((B, 1, Hkv, k), dtype=torch.int32, device="cuda")
@@ -607,6 +613,71 @@ def run_host_tier(args):
         "unpipelined_ms_per_step": unpipelined_ms,
         "planted_recall": recall, "setup_s": setup_s, "clocks": clk,
         "gpu_launches": launches_per_step(w) * n,
+    }
+    print(json.dumps(line), flush=True)
+    bank.close()
+
+
+def run_host_cache(args, w, bank, setup_s, Kh):
+    """Host-tier decode with a device-resident slab cache: each step takes one of
+    --query-pool seeded query batches uniformly at random, so the cache sees the
+    locality of a pool of recurring queries; hit rate and PCIe bytes per step are
+    reported with the throughput."""
+    import torch
+
+    import synth
+    from sparse_attention_routed_b200 import msa_forward
+    from synth.device import fill_normal, query_tensors
+
+    B, Hkv, d, k = w.batch, w.n_kv_heads, w.head_dim, w.top_k
+    bank.set_kv_cache(int(args.kv_cache_gb * 1e9))
+    pool = []
+    for i in range(args.query_pool):
+        Q, Qr, LK, LV = query_tensors(w)
+        if i:
+            for t, tid in ((Q, synth.T_Q), (Qr, synth.T_QR), (LK, synth.T_LK), (LV, synth.T_LV)):
+                fill_normal(t, w.seed + 7919 * i, tid)
+        pool.append((bank.query(Q, Qr, LK, LV, w.route_block), (Q, Qr, LK, LV)))
+    idx = torch.empty((B, 1, Hkv, k), dtype=torch.int32, device="cuda")
+    out = torch.empty((B, w.n_q_heads, 1, d), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    rng = np.random.RandomState(w.seed)
+    for _ in range(max(3, args.warmup)):
+        msa_forward(bank.handle, pool[rng.randint(len(pool))][0], k, idx.data_ptr(), out.data_ptr(), sh)
+    torch.cuda.synchronize()
+    assert bank.device_error() == 0
+    n = args.steps
+    picks = rng.randint(len(pool), size=n)
+    slabs = hits = copied = 0
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    time.sleep(0.4)
+    torch.cuda.synchronize()
+    t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_begin.record(stream)
+    for i in range(n):
+        msa_forward(bank.handle, pool[picks[i]][0], k, idx.data_ptr(), out.data_ptr(), sh)
+        st = bank.cache_stats()  # host-side figures of the step just planned
+        slabs += st["slabs"]
+        hits += st["hits"]
+        copied += st["bytes_copied"]
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    assert bank.device_error() == 0
+    step_ms = t_begin.elapsed_time(t_end) / n
+    slab_bytes = 2 * w.max_len * d * 2
+    line = {
+        "metric": f"decode queries/s, pinned-host K/V tier with a device slab cache ({w.n_tokens / 1e6:.1f}M-token bank)",
+        "value": B / (step_ms / 1e3), "unit": "queries/s", "n_gpus": 1, "steps": n, "warmup": args.warmup,
+        "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": f"synthetic; each step one of {len(pool)} seeded query batches, uniform at random",
+        "config": dict(base_config(w), bank_tokens=w.n_tokens, kv_slabs_pinned=w.kv_slabs,
+                       kv_cache_bytes=int(args.kv_cache_gb * 1e9),
+                       kv_cache_slots=int(args.kv_cache_gb * 1e9) // slab_bytes, query_pool=len(pool)),
+        "cache": {"hit_rate": hits / max(1, slabs), "slabs_per_step": slabs / n,
+                  "pcie_bytes_per_step": copied / n, "pcie_GBps": copied / n / (step_ms / 1e3) / 1e9},
+        "setup_s": setup_s, "clocks": clk, "gpu_launches": launches_per_step(w) * n,
     }
     print(json.dumps(line), flush=True)
     bank.close()

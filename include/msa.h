@@ -194,6 +194,26 @@ msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_
 msa_status msa_route_noalloc(msa_bank* bank, const msa_query* q, int32_t top_k, float* doc_scores,
                              int32_t* topk_idx, float* topk_scores, void* stream);
 
+/* Device-resident cache of selected K/V slabs for a pinned-host bank: the hot tier
+ * of a hot/cold split ("MSA (Memory Sparse Attention)", robocikowo.com, Komponenty:
+ * K_r in GPU memory, K/V in CPU RAM; "MSA：大模型高效推理的新突破，仅需2张A800显卡驱动1亿Token",
+ * yicaiai.com: a hierarchical KV cache pool). `bytes` is the device memory budget
+ * for K and V together; it is split into slots of max_doc_len rows (one (document,
+ * KV head) slab each). With the cache on, msa_attend and msa_forward copy over PCIe
+ * only the selected slabs that are not resident; a slab is replaced least recently
+ * used first, never while the current step uses it. A step that selects more
+ * distinct slabs than there are slots returns MSA_ERR_UNSUPPORTED. bytes = 0 turns
+ * the cache off (the default: every step copies its selection). Synchronises the
+ * device. MSA_ERR_INVALID_ARG for a NULL or device-tier bank or bytes < 0, MSA_ERR_OOM
+ * if the slots cannot be allocated. */
+msa_status msa_set_kv_cache(msa_bank* bank, int64_t bytes);
+
+/* Host-tier statistics of the most recent msa_attend / msa_forward on a
+ * pinned-host bank (any pointer may be NULL): distinct (document, KV head) slabs
+ * the step selected, how many of them were already resident in the cache, and
+ * the bytes copied over PCIe. */
+msa_status msa_kv_cache_stats(const msa_bank* bank, int64_t* slabs, int64_t* hits, int64_t* bytes_copied);
+
 /* Failure-detection check of the device-side bounded waits (the pages describe
  * no such call): launches one small kernel on `stream` whose thread waits on an
  * mbarrier phase that nothing ever completes, with the same poll limit every

@@ -72,6 +72,8 @@ def _load():
         "msa_forward": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp], ctypes.c_int),
         "msa_get_device_error": ([vp, vp], ctypes.c_int),
         "msa_route_noalloc": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp, vp], ctypes.c_int),
+        "msa_set_kv_cache": ([vp, i64], ctypes.c_int),
+        "msa_kv_cache_stats": ([vp, ctypes.POINTER(i64), ctypes.POINTER(i64), ctypes.POINTER(i64)], ctypes.c_int),
         "msa_check_wait_timeout": ([vp, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
@@ -99,8 +101,8 @@ def __getattr__(name):
 
 # Every symbol include/msa.h declares, in declaration order.
 EXPORTED = ["msa_bank_create", "msa_bank_destroy", "msa_build_bank", "msa_bank_info", "msa_reserve",
-            "msa_route", "msa_attend", "msa_forward", "msa_route_noalloc", "msa_check_wait_timeout",
-            "msa_get_device_error", "msa_status_string"]
+            "msa_route", "msa_attend", "msa_forward", "msa_route_noalloc", "msa_set_kv_cache",
+            "msa_kv_cache_stats", "msa_check_wait_timeout", "msa_get_device_error", "msa_status_string"]
 
 
 def msa_status_string(status: int) -> str:
@@ -205,6 +207,19 @@ def msa_route_noalloc(bank, query: msa_query, top_k: int, doc_scores: int, topk_
     if check:
         _check(st, "msa_route_noalloc")
     return st
+
+
+def msa_set_kv_cache(bank, nbytes: int, check=True) -> int:
+    st = lib().msa_set_kv_cache(bank, int(nbytes))
+    if check:
+        _check(st, "msa_set_kv_cache")
+    return st
+
+
+def msa_kv_cache_stats(bank) -> dict:
+    vals = [ctypes.c_int64() for _ in range(3)]
+    _check(lib().msa_kv_cache_stats(bank, *[ctypes.byref(v) for v in vals]), "msa_kv_cache_stats")
+    return {"slabs": vals[0].value, "hits": vals[1].value, "bytes_copied": vals[2].value}
 
 
 def msa_check_wait_timeout(bank, stream=0) -> None:

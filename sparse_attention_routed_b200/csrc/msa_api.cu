@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <list>
 #include <mutex>
 #include <new>
 #include <unordered_map>
@@ -148,6 +149,17 @@ struct msa_bank {
   uint16_t* stage_v = nullptr;
   int64_t stage_cap = 0;      // rows of stage_k / stage_v
   int64_t last_fetch_bytes = 0;
+  // device-resident slab cache (msa_set_kv_cache): stage_k / stage_v become slots of
+  // max_len rows that keep their slab across steps
+  bool cache_on = false;
+  int64_t cache_slots = 0;
+  std::unordered_map<int64_t, int64_t> cache_map;  // doc * Hkv + head -> slot
+  std::vector<int64_t> slot_key;                   // -1: free
+  std::vector<int64_t> slot_use;                   // step that last used the slot
+  std::list<int64_t> lru;                          // slots, least recently used first
+  std::vector<std::list<int64_t>::iterator> slot_it;
+  int64_t step_no = 0;
+  int64_t st_slabs = 0, st_hits = 0;  // the last step's distinct slabs and cache hits
 };
 
 namespace {
@@ -417,6 +429,7 @@ msa_status stage_entries(msa_bank* bank, int k, size_t e0, size_t e1, std::unord
     const int64_t key = (int64_t)j * bank->hkv + h;
     if (slot.emplace(key, -1).second) fresh.emplace_back((int64_t)h * bank->kv_rows + bank->doc_rows[j], key);
   }
+  bank->st_slabs += (int64_t)fresh.size();
   std::sort(fresh.begin(), fresh.end());
   const size_t row_bytes = (size_t)bank->d * 2;
   const uint16_t* hk = static_cast<const uint16_t*>(bank->k);
@@ -452,6 +465,62 @@ msa_status stage_entries(msa_bank* bank, int k, size_t e0, size_t e1, std::unord
   return MSA_OK;
 }
 
+// Cache-mode plan of selection entries [e0, e1): a slab resident in a slot is a
+// hit; a missing one takes the least recently used slot that the current step has
+// not used and is copied into it. `step` maps the slabs already placed in this step.
+msa_status stage_entries_cached(msa_bank* bank, int k, size_t e0, size_t e1,
+                                std::unordered_map<int64_t, int64_t>& step, int& stream_rr) {
+  const size_t row_bytes = (size_t)bank->d * 2;
+  const uint16_t* hk = static_cast<const uint16_t*>(bank->k);
+  const uint16_t* hv = static_cast<const uint16_t*>(bank->v);
+  for (size_t e = e0; e < e1; ++e) {
+    const int h = (int)((e / k) % bank->hkv);
+    const int j = bank->h_idx[e];
+    if (j < 0 || j >= bank->n_docs) return MSA_ERR_INVALID_ARG;
+    const int64_t key = (int64_t)j * bank->hkv + h;
+    auto placed = step.find(key);
+    if (placed != step.end()) {
+      bank->h_base[e] = placed->second;
+      continue;
+    }
+    ++bank->st_slabs;
+    int64_t slot;
+    auto c = bank->cache_map.find(key);
+    if (c != bank->cache_map.end()) {
+      slot = c->second;
+      ++bank->st_hits;
+    } else {
+      slot = bank->lru.front();
+      if (bank->slot_use[slot] == bank->step_no) return MSA_ERR_UNSUPPORTED;  // more slabs than slots
+      if (bank->slot_key[slot] >= 0) bank->cache_map.erase(bank->slot_key[slot]);
+      bank->cache_map[key] = slot;
+      bank->slot_key[slot] = key;
+      const int64_t src = (int64_t)h * bank->kv_rows + bank->doc_rows[j];
+      const int64_t dst = slot * bank->max_len;
+      const size_t bytes = (size_t)bank->doc_lens[j] * row_bytes;
+      if (cudaMemcpyAsync(bank->stage_k + dst * bank->d, hk + src * bank->d, bytes, cudaMemcpyHostToDevice,
+                          bank->side[stream_rr++ % msa_bank::kSide]) != cudaSuccess ||
+          cudaMemcpyAsync(bank->stage_v + dst * bank->d, hv + src * bank->d, bytes, cudaMemcpyHostToDevice,
+                          bank->side[stream_rr++ % msa_bank::kSide]) != cudaSuccess)
+        return MSA_ERR_HOST_TIER;
+      bank->last_fetch_bytes += 2 * (int64_t)bytes;
+    }
+    bank->slot_use[slot] = bank->step_no;
+    bank->lru.splice(bank->lru.end(), bank->lru, bank->slot_it[slot]);
+    const int64_t base = slot * bank->max_len;
+    step[key] = base;
+    bank->h_base[e] = base;
+  }
+  return MSA_OK;
+}
+
+// A new host-tier step: statistics restart, and the cache's "used by this step" marks.
+void begin_host_step(msa_bank* bank) {
+  ++bank->step_no;
+  bank->st_slabs = bank->st_hits = 0;
+  bank->last_fetch_bytes = 0;
+}
+
 // Upper bound of the staging rows a step can need (every entry a different slab).
 int64_t stage_bound(const msa_bank* bank, const StepShape& s) { return (int64_t)s.P * s.k * bank->max_len; }
 
@@ -472,13 +541,14 @@ msa_status host_fetch(msa_bank* bank, const StepShape& s, const int32_t* idx_dev
   if (rc != MSA_OK) return rc;
   MSA_CUDA(cudaMemcpyAsync(bank->h_idx, idx_dev, n * 4, cudaMemcpyDeviceToHost, st));
   MSA_CUDA(cudaStreamSynchronize(st));  // also retires every earlier step that read the staging pool
-  if ((rc = ensure_stage(bank, stage_bound(bank, s), st)) != MSA_OK) return rc;
+  if (!bank->cache_on && (rc = ensure_stage(bank, stage_bound(bank, s), st)) != MSA_OK) return rc;
   std::unordered_map<int64_t, int64_t> slot;
   slot.reserve(n * 2);
   int64_t rows = 0;
   int rr = 0;
-  bank->last_fetch_bytes = 0;
-  if ((rc = stage_entries(bank, s.k, 0, n, slot, rows, rr)) != MSA_OK) return rc;
+  begin_host_step(bank);
+  rc = bank->cache_on ? stage_entries_cached(bank, s.k, 0, n, slot, rr) : stage_entries(bank, s.k, 0, n, slot, rows, rr);
+  if (rc != MSA_OK) return rc;
   MSA_CUDA(cudaMemcpyAsync(bank->d_base, bank->h_base, n * 8, cudaMemcpyHostToDevice, bank->side[0]));
   return join_side(bank, st);
 }
@@ -590,7 +660,7 @@ msa_status forward_host(msa_bank* bank, const msa_query* q, const StepShape& s, 
   w = layout(bank, sm, splits, bank->ws);
   const size_t n = (size_t)s.P * s.k;
   if ((rc = ensure_host_tier(bank, n)) != MSA_OK) return rc;
-  if ((rc = ensure_stage(bank, stage_bound(bank, s), st)) != MSA_OK) return rc;
+  if (!bank->cache_on && (rc = ensure_stage(bank, stage_bound(bank, s), st)) != MSA_OK) return rc;
   if (capturing(st)) return MSA_ERR_INVALID_ARG;
 
   const size_t d = bank->d;
@@ -619,7 +689,7 @@ msa_status forward_host(msa_bank* bank, const msa_query* q, const StepShape& s, 
   slot.reserve(n * 2);
   int64_t rows = 0;
   int rr = 0;
-  bank->last_fetch_bytes = 0;
+  begin_host_step(bank);
   for (int m = 0; m < M; ++m) {
     const int b0 = m * nb, bn = std::min(nb, s.B - b0);
     if (bn <= 0) break;
@@ -632,7 +702,9 @@ msa_status forward_host(msa_bank* bank, const msa_query* q, const StepShape& s, 
     MSA_CUDA(cudaStreamWaitEvent(bank->rb, bank->ev_route[m], 0));
     MSA_CUDA(cudaMemcpyAsync(bank->h_idx + e0, topk_idx + e0, (e1 - e0) * 4, cudaMemcpyDeviceToHost, bank->rb));
     MSA_CUDA(cudaStreamSynchronize(bank->rb));
-    if ((rc = stage_entries(bank, s.k, e0, e1, slot, rows, rr)) != MSA_OK) return rc;
+    rc = bank->cache_on ? stage_entries_cached(bank, s.k, e0, e1, slot, rr)
+                        : stage_entries(bank, s.k, e0, e1, slot, rows, rr);
+    if (rc != MSA_OK) return rc;
     MSA_CUDA(cudaMemcpyAsync(bank->d_base + e0, bank->h_base + e0, (e1 - e0) * 8, cudaMemcpyHostToDevice,
                              bank->side[0]));
     if ((rc = join_side(bank, bank->att)) != MSA_OK) return rc;
@@ -876,6 +948,51 @@ msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_
   if (bank->kv_loc == MSA_KV_PINNED_HOST) return forward_host(bank, q, s, topk_idx, out, st);
   if ((rc = route_impl(bank, q, s, w, nullptr, topk_idx, nullptr, st)) != MSA_OK) return rc;
   return attend_impl(bank, q, s, splits, w, topk_idx, out, st);
+}
+
+msa_status msa_set_kv_cache(msa_bank* bank, int64_t bytes) {
+  if (!bank || bank->kv_loc != MSA_KV_PINNED_HOST || bytes < 0) return MSA_ERR_INVALID_ARG;
+  MSA_CUDA(cudaDeviceSynchronize());
+  if (bank->stage_k) cudaFree(bank->stage_k);
+  if (bank->stage_v) cudaFree(bank->stage_v);
+  bank->stage_k = bank->stage_v = nullptr;
+  bank->stage_cap = 0;
+  bank->cache_on = false;
+  bank->cache_slots = 0;
+  bank->cache_map.clear();
+  bank->slot_key.clear();
+  bank->slot_use.clear();
+  bank->lru.clear();
+  bank->slot_it.clear();
+  if (bytes == 0) return MSA_OK;
+  const int64_t slot_bytes = 2 * bank->max_len * bank->d * 2;
+  const int64_t slots = bytes / slot_bytes;
+  if (slots < 1) return MSA_ERR_INVALID_ARG;
+  const int64_t rows = slots * bank->max_len;
+  if (rows >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  const size_t b = (size_t)rows * bank->d * 2;
+  if (cudaMalloc(&bank->stage_k, b) != cudaSuccess || cudaMalloc(&bank->stage_v, b) != cudaSuccess) {
+    if (bank->stage_k) cudaFree(bank->stage_k);
+    bank->stage_k = nullptr;
+    return MSA_ERR_OOM;
+  }
+  bank->stage_cap = rows;
+  bank->cache_slots = slots;
+  bank->slot_key.assign(slots, -1);
+  bank->slot_use.assign(slots, -1);
+  bank->slot_it.resize(slots);
+  for (int64_t i = 0; i < slots; ++i) bank->slot_it[i] = bank->lru.insert(bank->lru.end(), i);
+  bank->cache_map.reserve((size_t)slots * 2);
+  bank->cache_on = true;
+  return MSA_OK;
+}
+
+msa_status msa_kv_cache_stats(const msa_bank* bank, int64_t* slabs, int64_t* hits, int64_t* bytes_copied) {
+  if (!bank) return MSA_ERR_INVALID_ARG;
+  if (slabs) *slabs = bank->st_slabs;
+  if (hits) *hits = bank->st_hits;
+  if (bytes_copied) *bytes_copied = bank->last_fetch_bytes;
+  return MSA_OK;
 }
 
 msa_status msa_check_wait_timeout(msa_bank* bank, void* stream) {

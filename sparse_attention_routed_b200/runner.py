@@ -10,7 +10,8 @@ import numpy as np
 import torch
 
 from . import (MSA_KV_DEVICE, make_query, msa_attend, msa_bank_create, msa_bank_destroy, msa_bank_info,
-               msa_build_bank, msa_forward, msa_get_device_error, msa_reserve, msa_route, ptr)
+               msa_build_bank, msa_forward, msa_get_device_error, msa_kv_cache_stats, msa_reserve, msa_route,
+               msa_set_kv_cache, ptr)
 
 
 class _DeviceArray:
@@ -104,6 +105,14 @@ class Bank:
                               dtype=torch.float32, device="cuda")
         msa_forward(self.handle, query, top_k, ptr(idx, torch.int32), ptr(out), _stream(stream))
         return idx, out
+
+    def set_kv_cache(self, nbytes: int):
+        """Device-resident slab cache of a pinned-host bank (0 turns it off)."""
+        msa_set_kv_cache(self.handle, nbytes)
+
+    def cache_stats(self) -> dict:
+        """Distinct slabs, cache hits and PCIe bytes of the last host-tier step."""
+        return msa_kv_cache_stats(self.handle)
 
     def device_error(self, stream=None) -> int:
         return msa_get_device_error(self.handle, _stream(stream))
