@@ -50,6 +50,9 @@ def parse():
                     help="host-tier workloads: device-resident slab cache of this many GB (msa_set_kv_cache); "
                          "each step then takes one of --query-pool query batches at random")
     ap.add_argument("--query-pool", type=int, default=4)
+    ap.add_argument("--build-only", action="store_true",
+                    help="time msa_build_bank (chunk-mean pooling of the routing keys + Parallel RoPE of the "
+                         "bank keys, in place) over the whole bank of --workload")
     ap.add_argument("--route-only", action="store_true",
                     help="time msa_route alone on the full bank's K_r with a stand-in 1-document K/V "
                          "(routing keys streamed in slices; a few GB on the device, for profiling captures)")
@@ -683,10 +686,58 @@ def run_host_cache(args, w, bank, setup_s, Kh):
     bank.close()
 
 
+def run_build(args):
+    """The offline bank build over a whole device bank, timed with CUDA events:
+    reads the routing keys (2 d_r bytes per token per KV head) and reads and
+    rewrites the keys (2 x 2 d bytes), writes K_r (small)."""
+    import torch
+
+    import synth
+    from sparse_attention_routed_b200.runner import Bank
+    from synth.device import bank_tensors
+
+    w = synth.WORKLOADS[args.workload]
+    K, V, R = bank_tensors(w)
+    bank = Bank(K, V, w.doc_lens(), w.rope_base)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        bank.build(R)
+    torch.cuda.synchronize()
+    n = args.steps
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    time.sleep(0.4)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        bank.build(R)  # RoPE turns the keys again each time: the same bytes and work
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / n
+    tok = w.n_tokens * w.n_kv_heads
+    nbytes = tok * (w.route_dim + 2 * w.head_dim) * 2 + w.n_kv_heads * bank.info["n_chunks"] * w.route_dim * (4 + 4)
+    peak, kind = peaks()
+    line = {
+        "metric": "bank build HBM GB/s (pooling + Parallel RoPE, in place)", "value": nbytes / (ms / 1e3) / 1e9,
+        "unit": "GB/s", "n_gpus": 1, "steps": n, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(base_config(w), bank_tokens=w.n_tokens),
+        "roofline": {"kernel": "bank_build_kernel", "bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9,
+                     "peak": peak, "peak_kind": kind, "unit": "GB/s",
+                     "frac": nbytes / (ms / 1e3) / 1e9 / peak, "algorithmic_bytes_per_launch": nbytes},
+        "clocks": clk, "gpu_launches": n,
+    }
+    print(json.dumps(line), flush=True)
+    bank.close()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.build_only:
+        run_build(args)
     elif args.route_only:
         run_route_only(args)
     elif args.workload in ("ragged_planted", "bank_100m"):
