@@ -39,6 +39,12 @@
  *     msa_get_device_error() (MSA_ERR_TIMEOUT).
  *   - There is no CPU fallback: without a usable sm_100 device the calls that
  *     launch work return MSA_ERR_CUDA or MSA_ERR_UNSUPPORTED.
+ *   - A bank belongs to the CUDA device that was current at msa_bank_create;
+ *     make that device current for every call on it. A bank is not safe for
+ *     concurrent use: calls on one bank must not overlap in time (several banks
+ *     may be used from several threads). The bank's workspace is shared by its
+ *     calls, which are ordered on their streams; calls on one bank issued to two
+ *     unordered streams may race on it.
  *   - Supported shapes: head_dim = route_dim in {64, 128}; n_q_heads a
  *     multiple of n_kv_heads; 1 <= top_k <= min(n_docs, 64); q_tokens a
  *     multiple of route_block; batch * (q_tokens / route_block) * n_kv_heads
