@@ -314,3 +314,111 @@ def forward(inputs: Dict[str, np.ndarray], doc_lens: Sequence[int], top_k: int,
                                                      LK[b, h], LV[b, h])
     return {"K_r": K_r, "K_rot": K_rot, "q_r": q_r, "doc_scores": scores, "topk": topk,
             "out": out, "k_off": k_off}
+
+
+# --------------------------------------------------------------------------
+# backward of the routed attention (the selection is fixed: top-k routing is
+# not differentiated), for training the layer end to end
+#   -- "MSA (Memory Sparse Attention)" (robocikowo.com), Komponenty: the memory
+#      sparse attention layer is trained end to end on top of a fixed router
+#      selection per step.
+# --------------------------------------------------------------------------
+
+def rope_adjoint(g: np.ndarray, pos, base: float) -> np.ndarray:
+    """Adjoint (transpose) of rope at the same positions: the inverse rotation,
+    i.e. a turn by -pos * theta_i (each pair's rotation matrix is orthogonal)."""
+    return rope(g, -np.asarray(pos, dtype=np.float64), base)
+
+
+def routed_attention_row_backward(q: np.ndarray, q_index: int, k_off: int, base: float,
+                                  mem_k_rot: np.ndarray, mem_v: np.ndarray,
+                                  local_k: np.ndarray, local_v: np.ndarray, d_out: np.ndarray):
+    """Gradients of sum(d_out * o) for one query row o = routed_attention_row(...).
+
+    With s_j = q_rot . k_j / sqrt(d), p = softmax(s), o = sum_j p_j v_j:
+      dv_j = p_j d_out;  dp_j = d_out . v_j;  ds_j = p_j (dp_j - d_out . o);
+      dq_rot = sum_j ds_j k_j / sqrt(d);  dk_j = ds_j q_rot / sqrt(d);
+    rotated quantities go back through the RoPE adjoint.
+    Returns dq (un-rotated), d_mem_k_rot [M, d] (with respect to the rotated bank
+    keys), d_mem_v [M, d], d_local_k [vis, d] (un-rotated), d_local_v [vis, d].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    d = q.shape[-1]
+    M = len(mem_k_rot)
+    q_rot = rope(q, k_off + q_index, base)
+    vis = q_index + 1
+    loc_pos = k_off + np.arange(vis)
+    loc_k_rot = rope(local_k[:vis], loc_pos, base)
+    keys = np.concatenate([np.asarray(mem_k_rot, dtype=np.float64), loc_k_rot], axis=0)
+    values = np.concatenate([np.asarray(mem_v, dtype=np.float64),
+                             np.asarray(local_v[:vis], dtype=np.float64)], axis=0)
+    s = keys @ q_rot / math.sqrt(d)
+    w = np.exp(s - s.max())
+    p = w / w.sum()
+    o = p @ values
+    d_out = np.asarray(d_out, dtype=np.float64)
+    dp = values @ d_out
+    ds = p * (dp - d_out @ o)
+    dq_rot = ds @ keys / math.sqrt(d)
+    dkeys = np.outer(ds, q_rot) / math.sqrt(d)
+    dvalues = np.outer(p, d_out)
+    dq = rope_adjoint(dq_rot, k_off + q_index, base)
+    d_local_k = rope_adjoint(dkeys[M:], loc_pos, base)
+    return dq, dkeys[:M], dvalues[:M], d_local_k, dvalues[M:]
+
+
+def backward(inputs: Dict[str, np.ndarray], doc_lens: Sequence[int], top_k: int, route_block: int,
+             d_out: np.ndarray, base: float = 10000.0, chunk: int = CHUNK, selection=None) -> Dict[str, np.ndarray]:
+    """Gradients of L = sum(d_out * out) with respect to Q, the bank keys K and
+    values V (K before Parallel RoPE, as msa_build_bank takes them), and the
+    local keys LK (before Global RoPE) and values LV, with the step's selection
+    held fixed (the oracle's own top-k, or `selection`).
+
+    Returns dQ [B, Hq, Tq, d], dK / dV [Hkv, Ntok, d], dLK / dLV [B, Hkv, Lc, d]
+    and the selection used."""
+    fwd = forward(inputs, doc_lens, top_k, route_block, base, chunk, selection)
+    sel = fwd["topk"] if selection is None else np.asarray(selection, dtype=np.int64)
+    K_rot = fwd["K_rot"]
+    k_off = fwd["k_off"]
+    V = np.asarray(inputs["V"], dtype=np.float64)
+    Q = np.asarray(inputs["Q"], dtype=np.float64)
+    LK = np.asarray(inputs["LK"], dtype=np.float64)
+    LV = np.asarray(inputs["LV"], dtype=np.float64)
+    d_out = np.asarray(d_out, dtype=np.float64)
+    Hkv, Ntok, d = K_rot.shape
+    B, Hq, Tq, _ = Q.shape
+    Lc = LK.shape[2]
+    G = Hq // Hkv
+    off = doc_offsets(doc_lens)
+
+    dQ = np.zeros_like(Q)
+    dK_rot = np.zeros((Hkv, Ntok, d))
+    dV = np.zeros((Hkv, Ntok, d))
+    dLK = np.zeros_like(LK)
+    dLV = np.zeros_like(LV)
+    for b in range(B):
+        for hq in range(Hq):
+            h = hq // G
+            for t in range(Tq):
+                docs = sel[b, t // route_block, h]
+                mk = np.concatenate([K_rot[h, off[j]:off[j + 1]] for j in docs], axis=0)
+                mv = np.concatenate([V[h, off[j]:off[j + 1]] for j in docs], axis=0)
+                i = Lc - Tq + t
+                dq, dmk, dmv, dlk, dlv = routed_attention_row_backward(
+                    Q[b, hq, t], i, k_off, base, mk, mv, LK[b, h], LV[b, h], d_out[b, hq, t])
+                dQ[b, hq, t] = dq
+                row = 0
+                for j in docs:
+                    L = off[j + 1] - off[j]
+                    dK_rot[h, off[j]:off[j + 1]] += dmk[row:row + L]
+                    dV[h, off[j]:off[j + 1]] += dmv[row:row + L]
+                    row += L
+                dLK[b, h, :i + 1] += dlk
+                dLV[b, h, :i + 1] += dlv
+    # the bank keys were turned by Parallel RoPE (positions restart in every document)
+    dK = np.empty_like(dK_rot)
+    for h in range(Hkv):
+        for j in range(len(doc_lens)):
+            L = off[j + 1] - off[j]
+            dK[h, off[j]:off[j + 1]] = rope_adjoint(dK_rot[h, off[j]:off[j + 1]], np.arange(L), base)
+    return {"dQ": dQ, "dK": dK, "dV": dV, "dLK": dLK, "dLV": dLV, "selection": sel, "out": fwd["out"]}
