@@ -50,6 +50,9 @@ def parse():
                     help="host-tier workloads: device-resident slab cache of this many GB (msa_set_kv_cache); "
                          "each step then takes one of --query-pool query batches at random")
     ap.add_argument("--query-pool", type=int, default=4)
+    ap.add_argument("--backward", action="store_true",
+                    help="time msa_attend_backward on --workload's selection (gradients of the queries, "
+                         "local K/V and bank K/V)")
     ap.add_argument("--build-only", action="store_true",
                     help="time msa_build_bank (chunk-mean pooling of the routing keys + Parallel RoPE of the "
                          "bank keys, in place) over the whole bank of --workload")
@@ -686,6 +689,81 @@ def run_host_cache(args, w, bank, setup_s, Kh):
     bank.close()
 
 
+def run_backward(args):
+    """The backward of the routed attention on the workload's own selection, timed
+    with CUDA events. Algorithmic FLOPs: 2.5 x the forward's (the five matmuls
+    S, dP, dV, dK, dQ of 2 d FLOP per (query row, visible key)), no credit for
+    recomputation."""
+    import torch
+
+    import synth
+    from sparse_attention_routed_b200 import msa_attend_backward
+    from sparse_attention_routed_b200.runner import Bank
+    from synth.device import bank_tensors, normal, query_tensors
+
+    w = synth.WORKLOADS[args.workload]
+    K, V, R = bank_tensors(w)
+    bank = Bank(K, V, w.doc_lens(), w.rope_base)
+    bank.build(R)
+    del R
+    Q, Qr, LK, LV = query_tensors(w)
+    qry = bank.query(Q, Qr, LK, LV, w.route_block)
+    idx, out = bank.forward(qry, w.top_k)
+    d_out = normal(tuple(out.shape), w.seed, 77).float()
+    dq = torch.empty_like(out)
+    dlk = torch.empty(LK.shape, dtype=torch.float32, device="cuda")
+    dlv = torch.empty(LV.shape, dtype=torch.float32, device="cuda")
+    dbk = torch.zeros(K.shape, dtype=torch.float32, device="cuda")
+    dbv = torch.zeros(V.shape, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    def step():
+        msa_attend_backward(bank.handle, qry, w.top_k, idx.data_ptr(), d_out.data_ptr(), dq.data_ptr(),
+                            dlk.data_ptr(), dlv.data_ptr(), dbk.data_ptr(), dbv.data_ptr(), sh)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert bank.device_error() == 0
+    sel = idx.cpu().numpy()
+    lens = w.doc_lens()
+    nblk = w.q_tokens // w.route_block
+    G = w.n_q_heads // w.n_kv_heads
+    mem_keys = sum(int(lens[j]) for b in range(w.batch) for blk in range(nblk) for h in range(w.n_kv_heads)
+                   for j in sel[b, blk, h]) * G * w.route_block
+    first = w.local_len - w.q_tokens
+    loc_keys = w.batch * w.n_q_heads * sum(first + t + 1 for t in range(w.q_tokens))
+    flops = 10 * w.head_dim * (mem_keys + loc_keys)
+    n = args.steps
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    time.sleep(0.4)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / n
+    tpeak, tkind = tensor_peak()
+    achieved = flops / (ms / 1e3) / 1e12
+    units = w.batch * w.q_tokens
+    line = {
+        "metric": "routed attention backward, query tokens/s", "value": units / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": 1, "steps": n, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(base_config(w), parallelism="replicas x1"),
+        "roofline": {"kernel": "bwd_dq_kernel + bwd_dkdv_kernel (mma.sync)", "bound": "tensor", "achieved": achieved,
+                     "peak": tpeak, "peak_kind": tkind, "unit": "TFLOP/s", "frac": achieved / tpeak,
+                     "algorithmic_flops_per_launch": flops},
+        "clocks": clk, "gpu_launches": 4 * n,
+    }
+    print(json.dumps(line), flush=True)
+    bank.close()
+
+
 def run_build(args):
     """The offline bank build over a whole device bank, timed with CUDA events:
     reads the routing keys (2 d_r bytes per token per KV head) and reads and
@@ -738,6 +816,8 @@ def main():
         run_reference(args)
     elif args.build_only:
         run_build(args)
+    elif args.backward:
+        run_backward(args)
     elif args.route_only:
         run_route_only(args)
     elif args.workload in ("ragged_planted", "bank_100m"):

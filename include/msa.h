@@ -177,6 +177,26 @@ msa_status msa_route(msa_bank* bank, const msa_query* q, int32_t top_k, float* d
 msa_status msa_attend(msa_bank* bank, const msa_query* q, int32_t top_k,
                       const int32_t* topk_idx, float* out, void* stream);
 
+/* Backward of msa_attend for the selection in topk_idx (the top-k routing is not
+ * differentiated: the layer trains end to end on each step's selection,
+ * "MSA (Memory Sparse Attention)", robocikowo.com, Komponenty). Gradients of
+ * sum(d_out * out), with out = msa_attend(q, top_k, topk_idx):
+ *   dq        [B, Hq, Tq, d]   fp32, written: the queries as msa_query takes them
+ *                              (before Global RoPE);
+ *   dlocal_k  [B, Hkv, Lc, d]  fp32, written: the local keys (before Global RoPE);
+ *   dlocal_v  [B, Hkv, Lc, d]  fp32, written: the local values;
+ *   dbank_k   [Hkv, kv_rows, d] fp32, ADDED TO: the bank keys before Parallel RoPE
+ *                              (as msa_build_bank takes them); rows that several
+ *                              documents share receive the sum;
+ *   dbank_v   [Hkv, kv_rows, d] fp32, added to: the bank values.
+ * d_out: [B, Hq, Tq, d] fp32. The call recomputes each row's softmax statistics
+ * (it does not need the forward's output) and uses workspace for the RoPE'd
+ * queries and local keys. Device-tier banks only (MSA_ERR_UNSUPPORTED for a
+ * pinned-host bank). Pointers must be 16-byte aligned. */
+msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k, const int32_t* topk_idx,
+                               const float* d_out, float* dq, float* dlocal_k, float* dlocal_v,
+                               float* dbank_k, float* dbank_v, void* stream);
+
 /* msa_route followed by msa_attend on one stream; topk_idx receives the selection. */
 msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_t* topk_idx,
                        float* out, void* stream);

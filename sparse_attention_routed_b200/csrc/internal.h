@@ -136,6 +136,27 @@ size_t attend_smem_bytes(int head_dim);
 // raises kErrTimeout in *err.
 cudaError_t launch_wait_timeout(int* err, cudaStream_t s);
 
+// Backward of the routed attention (selection fixed). Row statistics and dQ by
+// one kernel (it re-runs the forward for the log-sum-exp and dO . O), dK and
+// dV by a second one (accumulated into the outputs with atomics).
+struct AttendBwdArgs {
+  AttendArgs a;              // as for the forward; maps: the bank K/V and the RoPE'd local K / local V
+  const float* dout;         // [B, Hq, Tq, d]
+  float* dq;                 // [B, Hq, Tq, d] written: gradient of the un-rotated queries
+  float* lse2;               // [P][rows] log2-domain log-sum-exp of each row's scaled logits
+  float* drow;               // [P][rows] dO . O of each row
+  const uint16_t* q_rot;     // [B, Hq, Tq, d] queries with Global RoPE
+  const float2* ptab;        // [max_doc_len][d/2] Parallel RoPE (cos, sin)
+  float* dk_bank;            // [Hkv, kv_rows, d] += gradient of the bank keys before Parallel RoPE
+  float* dv_bank;            // [Hkv, kv_rows, d] += gradient of the bank values
+  float* dk_loc;             // [B, Hkv, Lc, d] += gradient of the local keys before Global RoPE
+  float* dv_loc;             // [B, Hkv, Lc, d] += gradient of the local values
+};
+cudaError_t launch_attend_bwd_dq(const AttendBwdArgs& g, const AttendMaps& m, int head_dim, cudaStream_t s);
+cudaError_t launch_attend_bwd_dkdv(const AttendBwdArgs& g, const AttendMaps& m, int head_dim, int max_tiles,
+                                   cudaStream_t s);
+int attend_bwd_tile_rows();  // keys per TMA box of both backward kernels
+
 }  // namespace msa
 
 struct msa_bank;

@@ -950,6 +950,75 @@ msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_
   return attend_impl(bank, q, s, splits, w, topk_idx, out, st);
 }
 
+msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k, const int32_t* topk_idx,
+                               const float* d_out, float* dq, float* dlocal_k, float* dlocal_v,
+                               float* dbank_k, float* dbank_v, void* stream) {
+  StepShape s;
+  msa_status rc = check_query(bank, q, top_k, &s, true);
+  if (rc != MSA_OK) return rc;
+  if (!topk_idx || !d_out || !dq || !dlocal_k || !dlocal_v || !dbank_k || !dbank_v) return MSA_ERR_INVALID_ARG;
+  for (const void* p : {(const void*)d_out, (const void*)dq, (const void*)dlocal_k, (const void*)dlocal_v,
+                        (const void*)dbank_k, (const void*)dbank_v})
+    if (!aligned16(p)) return MSA_ERR_INVALID_ARG;
+  if (bank->kv_loc != MSA_KV_DEVICE) return MSA_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  // workspace after the split counters: RoPE'd queries and local keys, row statistics
+  const size_t qrot = align_up((size_t)s.B * s.Hq * s.Tq * bank->d * 2);
+  const size_t lrot = align_up((size_t)s.B * bank->hkv * s.Lc * bank->d * 2);
+  const size_t stats = align_up((size_t)s.P * s.rows * 4);
+  if ((rc = ensure_workspace(bank, kCounterBytes + qrot + lrot + 2 * stats, st)) != MSA_OK) return rc;
+  if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->max_len, s.Lc, st)) != MSA_OK) return rc;
+  uint8_t* ws = bank->ws + kCounterBytes;
+  uint16_t* q_rot = reinterpret_cast<uint16_t*>(ws);
+  uint16_t* l_rot = reinterpret_cast<uint16_t*>(ws + qrot);
+  float* lse2 = reinterpret_cast<float*>(ws + qrot + lrot);
+  float* drow = reinterpret_cast<float*>(ws + qrot + lrot + stats);
+  const int64_t qrows = (int64_t)s.B * s.Hq * s.Tq, lrows = (int64_t)s.B * bank->hkv * s.Lc;
+  MSA_CUDA(launch_rope_rows((const uint16_t*)q->q, q_rot, bank->d_gtab, qrows, s.Tq, s.Lc - s.Tq, bank->d, st));
+  MSA_CUDA(launch_rope_rows((const uint16_t*)q->local_k, l_rot, bank->d_gtab, lrows, s.Lc, 0, bank->d, st));
+  MSA_CUDA(cudaMemsetAsync(dlocal_k, 0, (size_t)lrows * bank->d * 4, st));
+  MSA_CUDA(cudaMemsetAsync(dlocal_v, 0, (size_t)lrows * bank->d * 4, st));
+  const int box = attend_bwd_tile_rows();
+  AttendMaps maps;
+  if ((rc = make_map(&maps.bank_k, bank->k, (int64_t)bank->hkv * bank->kv_rows, bank->d, box)) != MSA_OK) return rc;
+  if ((rc = make_map(&maps.bank_v, bank->v, (int64_t)bank->hkv * bank->kv_rows, bank->d, box)) != MSA_OK) return rc;
+  if ((rc = make_map(&maps.loc_k, l_rot, lrows, bank->d, box)) != MSA_OK) return rc;
+  if ((rc = make_map(&maps.loc_v, q->local_v, lrows, bank->d, box)) != MSA_OK) return rc;
+  AttendBwdArgs g{};
+  AttendArgs& a = g.a;
+  a.q = (const uint16_t*)q->q;
+  a.sel = topk_idx;
+  a.doc_row = bank->d_doc_row;
+  a.doc_len = bank->d_doc_len;
+  a.gtab = bank->d_gtab;
+  a.err = bank->d_err;
+  a.kv_rows = bank->kv_rows;
+  a.batch = s.B;
+  a.n_q_heads = s.Hq;
+  a.n_kv_heads = bank->hkv;
+  a.q_tokens = s.Tq;
+  a.local_len = s.Lc;
+  a.route_block = s.Bq;
+  a.top_k = s.k;
+  a.n_docs = bank->n_docs;
+  a.n_splits = 1;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)bank->d));
+  g.dout = d_out;
+  g.dq = dq;
+  g.lse2 = lse2;
+  g.drow = drow;
+  g.q_rot = q_rot;
+  g.ptab = bank->d_ptab;
+  g.dk_bank = dbank_k;
+  g.dv_bank = dbank_v;
+  g.dk_loc = dlocal_k;
+  g.dv_loc = dlocal_v;
+  MSA_CUDA(launch_attend_bwd_dq(g, maps, bank->d, st));
+  const int max_tiles = s.k * (int)((bank->max_len + box - 1) / box) + (s.Lc + box - 1) / box;
+  MSA_CUDA(launch_attend_bwd_dkdv(g, maps, bank->d, max_tiles, st));
+  return MSA_OK;
+}
+
 msa_status msa_set_kv_cache(msa_bank* bank, int64_t bytes) {
   if (!bank || bank->kv_loc != MSA_KV_PINNED_HOST || bytes < 0) return MSA_ERR_INVALID_ARG;
   MSA_CUDA(cudaDeviceSynchronize());
