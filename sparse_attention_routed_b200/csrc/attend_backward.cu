@@ -397,7 +397,7 @@ __global__ void __launch_bounds__((BW + 1) * 32, 1)
 
 constexpr int KW = 4;                // consumer warps of the dK/dV kernel (16 keys each)
 constexpr int KSTAGES = 2;
-constexpr int KROWS = 128;           // query rows per dK/dV CTA (a slice of the problem's rows)
+constexpr int KROWS = 256;           // query rows per dK/dV CTA (a slice of the problem's rows)
 constexpr int KGROUP = 16;           // key tiles per dK/dV CTA
 
 template <int D>
