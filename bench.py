@@ -43,7 +43,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "decode_512k", "prefill", "prefill_64docs", "ragged_planted", "bank_100m"],
+    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "decode_512k", "prefill", "prefill_64docs", "prefill_short_docs", "ragged_planted", "bank_100m"],
                     help="decode_512k: the same step on a 128-document bank (profiling captures); "
                          "prefill: 4096 query tokens in 64-token routing blocks (tensor-bound)")
     ap.add_argument("--kv-cache-gb", type=float, default=0.0,
@@ -750,15 +750,21 @@ def run_backward(args):
     tpeak, tkind = tensor_peak()
     achieved = flops / (ms / 1e3) / 1e12
     units = w.batch * w.q_tokens
+    # head_dim 128 with routing blocks of a multiple of 64 tokens takes the key-tile tcgen05 dK/dV
+    # (plus the dO conversion and the selection index); other shapes the mma.sync one
+    if w.head_dim == 128 and w.route_block % 64 == 0:
+        kernels, launches = "bwd_dq_kernel (mma.sync) + bwd_dkdv_tc_kernel (tcgen05)", 6
+    else:
+        kernels, launches = "bwd_dq_kernel + bwd_dkdv_kernel (mma.sync)", 4
     line = {
         "metric": "routed attention backward, query tokens/s", "value": units / (ms / 1e3), "unit": "tokens/s",
         "n_gpus": 1, "steps": n, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(base_config(w), parallelism="replicas x1"),
-        "roofline": {"kernel": "bwd_dq_kernel + bwd_dkdv_kernel (mma.sync)", "bound": "tensor", "achieved": achieved,
+        "roofline": {"kernel": kernels, "bound": "tensor", "achieved": achieved,
                      "peak": tpeak, "peak_kind": tkind, "unit": "TFLOP/s", "frac": achieved / tpeak,
                      "algorithmic_flops_per_launch": flops},
-        "clocks": clk, "gpu_launches": 4 * n,
+        "clocks": clk, "gpu_launches": launches * n,
     }
     print(json.dumps(line), flush=True)
     bank.close()

@@ -92,6 +92,8 @@ struct AttendArgs {
   float* part_o;            // [P][S][rows][d]   rows = G * route_block
   float* part_ml;           // [P][S][rows][2]   (running max in log2 units, sum)
   float* out;               // [B, Hq, Tq, d] fp32
+  float* lse2;              // [P][rows] or nullptr: log2-domain log-sum-exp of each row's scaled logits
+                            // (written by the tcgen05 prefill kernel only)
   int* counters;            // [P] split-completion counters, zero between calls
   int* err;
   int64_t kv_rows;          // rows per head in the bank tensor map
@@ -151,11 +153,44 @@ struct AttendBwdArgs {
   float* dv_bank;            // [Hkv, kv_rows, d] += gradient of the bank values
   float* dk_loc;             // [B, Hkv, Lc, d] += gradient of the local keys before Global RoPE
   float* dv_loc;             // [B, Hkv, Lc, d] += gradient of the local values
+  // key-tile (tcgen05) dK/dV kernel only
+  const int* idx_nitems;     // [Hkv] bank key tiles of the head's selected documents
+  const int4* idx_items;     // [Hkv][idx_item_cap] {first K/V row, t | keys << 16, place in idx_prob, problems}
+  const int* idx_prob;       // [Hkv][idx_cap] the problems that selected each document, ascending
+  int idx_item_cap;          // bound on the key tiles of one head
+  int idx_cap;               // selections per head (problems per head x top_k)
+};
+// fp32 gradient tensors [rows, 128] in boxes of 32 columns x 128 rows, 128-byte swizzle
+struct AttendGradMaps {
+  CUtensorMap dk_bank, dv_bank, dk_loc, dv_loc;
 };
 cudaError_t launch_attend_bwd_dq(const AttendBwdArgs& g, const AttendMaps& m, int head_dim, cudaStream_t s);
 cudaError_t launch_attend_bwd_dkdv(const AttendBwdArgs& g, const AttendMaps& m, int head_dim, int max_tiles,
                                    cudaStream_t s);
 int attend_bwd_tile_rows();  // keys per TMA box of both backward kernels
+// tcgen05 dK/dV for head_dim 128 and routing blocks a multiple of 64 tokens: the
+// maps take boxes of attend_bwd_tc_tile_rows() keys, q_map / do_map (RoPE'd
+// queries, dO in bf16) boxes of attend_bwd_tc_chunk_rows() rows. The gradient
+// outputs are added to (the local ones must be zeroed first); rows of a key tile
+// past its document or context receive +0.
+bool attend_bwd_tc_supported(int head_dim, int route_block, int top_k);
+int attend_bwd_tc_tile_rows();
+int attend_bwd_tc_chunk_rows();
+cudaError_t launch_attend_bwd_index(const int32_t* sel, const int32_t* doc_len, const int64_t* doc_row,
+                                    int64_t kv_rows, int* cnt, int* idx_nitems, int4* idx_items, int* idx_prob,
+                                    int n_docs, int n_kv_heads, int problems_per_head, int top_k, int item_cap,
+                                    int cap, int* err, cudaStream_t s);
+cudaError_t launch_to_bf16(const float* in, uint16_t* out, int64_t n, int sms, cudaStream_t s);
+// tcgen05 dQ for the shapes of attend_prefill_tc_supported (top_k <= 64), given
+// lse2 and drow; maps as for launch_attend_prefill_tc, do_map like q_map over dO (bf16).
+cudaError_t launch_attend_bwd_dq_tc(const AttendBwdArgs& g, const AttendMaps& m, const CUtensorMap& q_map,
+                                    const CUtensorMap& do_map, cudaStream_t s);
+// dO (fp32) -> bf16 and drow[p][r] = dO . O of every query row (head_dim 128).
+cudaError_t launch_attend_bwd_prep(const float* dout, const float* out, uint16_t* dout_bf, float* drow, int batch,
+                                   int n_q_heads, int n_kv_heads, int q_tokens, int route_block, int sms,
+                                   cudaStream_t s);
+cudaError_t launch_attend_bwd_dkdv_tc(const AttendBwdArgs& g, const AttendMaps& m, const CUtensorMap& q_map,
+                                      const CUtensorMap& do_map, const AttendGradMaps& gm, int sms, cudaStream_t s);
 
 }  // namespace msa
 

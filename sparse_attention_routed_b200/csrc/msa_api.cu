@@ -67,6 +67,21 @@ msa_status make_map(CUtensorMap* map, const void* base, int64_t rows, int d, int
   return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
 }
 
+// fp32 [rows, d] in boxes of 32 columns x box_rows rows, 128-byte swizzle (TMA reduce-add targets)
+msa_status make_map_f32(CUtensorMap* map, void* base, int64_t rows, int d, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return MSA_ERR_CUDA;
+  if (!aligned16(base) || rows <= 0 || rows >= (int64_t(1) << 31)) return MSA_ERR_INVALID_ARG;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 4};
+  cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
+}
+
 // (cos, sin) of pos * base^(-2i/d) for positions p0 .. p0+n-1, angles in fp64
 // reduced mod 2*pi before the fp32 rounding.
 std::vector<float2> rope_table(int64_t p0, int64_t n, int d, double base) {
@@ -966,13 +981,39 @@ msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k
   const size_t qrot = align_up((size_t)s.B * s.Hq * s.Tq * bank->d * 2);
   const size_t lrot = align_up((size_t)s.B * bank->hkv * s.Lc * bank->d * 2);
   const size_t stats = align_up((size_t)s.P * s.rows * 4);
-  if ((rc = ensure_workspace(bank, kCounterBytes + qrot + lrot + 2 * stats, st)) != MSA_OK) return rc;
+  // the key-tile (tcgen05) dK/dV path: dO in bf16 and the per-head index of who selected what
+  const bool tc = attend_bwd_tc_supported(bank->d, s.Bq, s.k);
+  // the whole step on the tensor cores: the tcgen05 forward gives O and each row's
+  // log-sum-exp, then the tcgen05 dQ and dK/dV kernels
+  const bool tc_all = tc && attend_prefill_tc_supported(bank->d, s.G, s.Bq) && s.k <= 64;
+  const size_t otmp = tc_all ? align_up((size_t)s.B * s.Hq * s.Tq * bank->d * 4) : 0;
+  const int64_t ph = (int64_t)s.B * (s.Tq / s.Bq);           // problems per KV head
+  const int64_t cap = ph * s.k;                              // selections per KV head
+  const int64_t rb = std::min<int64_t>(bank->n_docs, cap);    // documents one head can have selected
+  const int kt = attend_bwd_tc_tile_rows();
+  const int64_t item_cap = rb * ((bank->max_len + kt - 1) / kt);  // their key tiles, at most
+  const size_t dob = tc ? align_up((size_t)s.B * s.Hq * s.Tq * bank->d * 2) : 0;
+  const size_t i_cnt = tc ? align_up((size_t)bank->hkv * bank->n_docs * 4) : 0;
+  const size_t i_nit = tc ? align_up((size_t)bank->hkv * 4) : 0;
+  const size_t i_items = tc ? align_up((size_t)bank->hkv * item_cap * 16) : 0;
+  const size_t i_prob = tc ? align_up((size_t)bank->hkv * cap * 4) : 0;
+  if (tc && (cap >= (int64_t(1) << 31) || item_cap >= (int64_t(1) << 31) || bank->hkv > 64))
+    return MSA_ERR_UNSUPPORTED;
+  const size_t base_ws = kCounterBytes + qrot + lrot + 2 * stats;
+  if ((rc = ensure_workspace(bank, base_ws + dob + i_cnt + i_nit + i_items + i_prob + otmp, st)) != MSA_OK) return rc;
   if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->max_len, s.Lc, st)) != MSA_OK) return rc;
   uint8_t* ws = bank->ws + kCounterBytes;
   uint16_t* q_rot = reinterpret_cast<uint16_t*>(ws);
   uint16_t* l_rot = reinterpret_cast<uint16_t*>(ws + qrot);
   float* lse2 = reinterpret_cast<float*>(ws + qrot + lrot);
   float* drow = reinterpret_cast<float*>(ws + qrot + lrot + stats);
+  uint8_t* wtc = bank->ws + base_ws;
+  uint16_t* do_bf = reinterpret_cast<uint16_t*>(wtc);
+  int* idx_cnt = reinterpret_cast<int*>(wtc + dob);
+  int* idx_nitems = reinterpret_cast<int*>(wtc + dob + i_cnt);
+  int4* idx_items = reinterpret_cast<int4*>(wtc + dob + i_cnt + i_nit);
+  int* idx_prob = reinterpret_cast<int*>(wtc + dob + i_cnt + i_nit + i_items);
+  float* o_tmp = reinterpret_cast<float*>(wtc + dob + i_cnt + i_nit + i_items + i_prob);
   const int64_t qrows = (int64_t)s.B * s.Hq * s.Tq, lrows = (int64_t)s.B * bank->hkv * s.Lc;
   MSA_CUDA(launch_rope_rows((const uint16_t*)q->q, q_rot, bank->d_gtab, qrows, s.Tq, s.Lc - s.Tq, bank->d, st));
   MSA_CUDA(launch_rope_rows((const uint16_t*)q->local_k, l_rot, bank->d_gtab, lrows, s.Lc, 0, bank->d, st));
@@ -1013,7 +1054,44 @@ msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k
   g.dv_bank = dbank_v;
   g.dk_loc = dlocal_k;
   g.dv_loc = dlocal_v;
-  MSA_CUDA(launch_attend_bwd_dq(g, maps, bank->d, st));
+  if (!tc_all) MSA_CUDA(launch_attend_bwd_dq(g, maps, bank->d, st));
+  if (tc) {
+    if (!tc_all) MSA_CUDA(launch_to_bf16(d_out, do_bf, qrows * bank->d, bank->sms, st));
+    MSA_CUDA(launch_attend_bwd_index(topk_idx, bank->d_doc_len, bank->d_doc_row, bank->kv_rows, idx_cnt, idx_nitems,
+                                     idx_items, idx_prob, bank->n_docs, bank->hkv, (int)ph, s.k, (int)item_cap,
+                                     (int)cap, bank->d_err, st));
+    const int rc_rows = attend_bwd_tc_chunk_rows();
+    AttendMaps m2;
+    m2.bank_k = bank->map_k128;
+    m2.bank_v = bank->map_v128;
+    if (kt != attend_prefill_tc_tile_rows()) return MSA_ERR_UNSUPPORTED;
+    if ((rc = make_map(&m2.loc_k, l_rot, lrows, bank->d, kt)) != MSA_OK) return rc;
+    if ((rc = make_map(&m2.loc_v, q->local_v, lrows, bank->d, kt)) != MSA_OK) return rc;
+    CUtensorMap q_map{}, do_map{};
+    if ((rc = make_map(&q_map, q_rot, qrows, bank->d, rc_rows)) != MSA_OK) return rc;
+    if ((rc = make_map(&do_map, do_bf, qrows, bank->d, rc_rows)) != MSA_OK) return rc;
+    if (tc_all) {
+      // forward (O into the workspace, log-sum-exp per row), dO . O, then dQ
+      AttendArgs fa = a;
+      fa.out = o_tmp;
+      fa.lse2 = lse2;
+      MSA_CUDA(launch_attend_prefill_tc(fa, m2, q_map, st));
+      MSA_CUDA(launch_attend_bwd_prep(d_out, o_tmp, do_bf, drow, s.B, s.Hq, bank->hkv, s.Tq, s.Bq, bank->sms, st));
+      MSA_CUDA(launch_attend_bwd_dq_tc(g, m2, q_map, do_map, st));
+    }
+    AttendGradMaps gm;
+    if ((rc = make_map_f32(&gm.dk_bank, dbank_k, (int64_t)bank->hkv * bank->kv_rows, bank->d, kt)) != MSA_OK) return rc;
+    if ((rc = make_map_f32(&gm.dv_bank, dbank_v, (int64_t)bank->hkv * bank->kv_rows, bank->d, kt)) != MSA_OK) return rc;
+    if ((rc = make_map_f32(&gm.dk_loc, dlocal_k, lrows, bank->d, kt)) != MSA_OK) return rc;
+    if ((rc = make_map_f32(&gm.dv_loc, dlocal_v, lrows, bank->d, kt)) != MSA_OK) return rc;
+    g.idx_nitems = idx_nitems;
+    g.idx_items = idx_items;
+    g.idx_prob = idx_prob;
+    g.idx_item_cap = (int)item_cap;
+    g.idx_cap = (int)cap;
+    MSA_CUDA(launch_attend_bwd_dkdv_tc(g, m2, q_map, do_map, gm, bank->sms, st));
+    return MSA_OK;
+  }
   const int max_tiles = s.k * (int)((bank->max_len + box - 1) / box) + (s.Lc + box - 1) / box;
   MSA_CUDA(launch_attend_bwd_dkdv(g, maps, bank->d, max_tiles, st));
   return MSA_OK;

@@ -219,6 +219,9 @@ WORKLOADS = {
     "prefill": Workload("prefill", 2, 1, 32, 8, 128, 256, 8192, 4096, 4096, 64, 8),
     # the prefill step on a 64-document bank: same work per CTA, 2 GB of K/V (hardware-counter captures)
     "prefill_64docs": Workload("prefill_64docs", 2, 1, 32, 8, 128, 64, 8192, 4096, 4096, 64, 8),
+    # the prefill step with 1024-token documents: a document draws as many problems as in
+    # prefill (the backward's key tiles see the same rows), 1 GB of K/V (hardware-counter captures)
+    "prefill_short_docs": Workload("prefill_short_docs", 2, 1, 32, 8, 128, 256, 1024, 4096, 4096, 64, 8),
     # K/V of these two banks (283 GB, 410 GB) exceed host RAM: the pinned pool holds
     # kv_slabs distinct slabs and document j reads slab j mod kv_slabs (routing keys
     # stay distinct per document; the bytes each step moves over PCIe are unchanged)

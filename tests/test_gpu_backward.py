@@ -30,6 +30,12 @@ CASES = {
     "bwd_d64_all": Workload("bwd_d64_all", 64, 1, 4, 1, 64, 6, 0, 40, 4, 2, 6, ragged=(5, 90)),
     # one-token documents, Lc = Tq = 1
     "bwd_tiny_docs": Workload("bwd_tiny_docs", 65, 2, 2, 2, 128, 4, 0, 1, 1, 1, 2, ragged=(1, 3)),
+    # key-tile tcgen05 dK/dV: 128-token routing blocks, G = 2, queries after 44 local tokens
+    # (local tiles that only some blocks reach, a ragged third local tile)
+    "bwd_tc_bq128": Workload("bwd_tc_bq128", 67, 1, 4, 2, 128, 6, 0, 300, 256, 128, 3, ragged=(60, 500)),
+    # key-tile tcgen05 dK/dV: 6 problems per KV head choosing 2 of 3 documents, so
+    # most key tiles gather the rows of several problems
+    "bwd_tc_hot": Workload("bwd_tc_hot", 68, 2, 8, 2, 128, 3, 0, 192, 192, 64, 2, ragged=(100, 400)),
 }
 
 
@@ -75,11 +81,12 @@ def test_backward_parity(name):
     bank.close()
 
 
-def test_backward_adds_to_the_bank_gradients_and_refuses_a_host_bank():
+@pytest.mark.parametrize("name", ["bwd_decode", "bwd_tc_hot"])
+def test_backward_adds_to_the_bank_gradients_and_refuses_a_host_bank(name):
     import sparse_attention_routed_b200 as msa
     from sparse_attention_routed_b200.runner import Bank
     from synth.device import bank_tensors, normal, query_tensors
-    w = CASES["bwd_decode"]
+    w = CASES[name]
     K, V, R = bank_tensors(w)
     Q, Qr, LK, LV = query_tensors(w)
     bank = Bank(K, V, w.doc_lens(), w.rope_base)
