@@ -31,11 +31,14 @@
 //              P = exp2(S scale - lse) and dS = P (dP - D) / sqrt(d) (zero for
 //              keys past the document, and for local keys after the row's
 //              position), and writes both back as packed bf16 over the columns
-//              it read. At the end of an item they move dK and dV out of TMEM
-//              (freeing it for the next item at once), apply the RoPE adjoint
-//              to dK and stage both, 64 KB at a time, in the item's K/V slot,
-//              from where TMA reduce-adds them into the gradients (the
-//              additions run in L2).
+//              it read. At the end of an item they stage its dV in the item's
+//              K/V slot (64 KB), take its dK into registers -- TMEM is free for
+//              the next item from here -- and apply the RoPE adjoint; the dK
+//              follows into the slot two chunks into the next item, once the
+//              dV has left it.
+//   warp 10    reducer: adds each staged half to the gradients with TMA
+//              reduce-add (the additions run in L2) and frees the slot; the
+//              waits for those copies fall on this warp alone.
 // Every mbarrier parity wait targets the phase right after one the same waiter
 // saw complete, so no wait can be satisfied by an older phase.
 #include "common.cuh"
@@ -53,7 +56,7 @@ constexpr int CBOX = RC * 128;        // 64 dims of a chunk (8 KB)
 constexpr int CTILE = 2 * CBOX;       // 64 x 128 bf16 (16 KB)
 constexpr int KVSLOT = 2;
 constexpr int CSLOT = 3;
-constexpr int THREADS = 320;          // producer, MMA, 8 elementwise warps
+constexpr int THREADS = 352;          // producer, MMA, 8 elementwise warps, reducer
 constexpr int TMEM_COLS = 512;
 constexpr int S_COL = 0;              // S^T[buf]  = S_COL + 64 buf   (P^T over its columns)
 constexpr int DP_COL = 128;           // dP^T[buf] = DP_COL + 64 buf  (dS^T over its columns)
@@ -65,7 +68,7 @@ constexpr int OFF_KV = 0;                                  // slot s: K at OFF_K
 constexpr int OFF_C = OFF_KV + KVSLOT * 2 * KTILE;         // slot c: Q at OFF_C + c * 2 CTILE, dO after it
 constexpr int OFF_ST = OFF_C + CSLOT * 2 * CTILE;          // slot c: lse2[64], D[64] at OFF_ST + c * 512
 constexpr int OFF_BAR = OFF_ST + CSLOT * 2 * RC * 4;
-constexpr int N_BAR = 2 * KVSLOT + 2 * CSLOT + 2 + 2 + 4 + 3;
+constexpr int N_BAR = 2 * KVSLOT + 2 * CSLOT + 2 + 2 + 4 + 5;
 constexpr int OFF_TMEM = OFF_BAR + N_BAR * 8;
 
 // One item: 128 keys and the problems whose rows attend them.
@@ -169,6 +172,20 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// 16 / 8 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 // This thread's 32 fp32 values of row r into box c of the staging area: four boxes
 // of [128 rows][32 floats], 128-byte swizzled as the gradient tensor maps expect.
 __device__ __forceinline__ void stage_row(uint8_t* stg, int c, int r, const float (&v)[32]) {
@@ -182,7 +199,6 @@ constexpr int OFF_PRE = OFF_TMEM + 16;                     // item prefix over K
 constexpr int MAX_HKV = 64;
 constexpr size_t SMEM_TOTAL = 1024 + OFF_PRE + (MAX_HKV + 1) * 4;
 static_assert(SMEM_TOTAL <= 232448, "shared memory");
-constexpr int EPI_TID = 64;                                // first elementwise thread: issues the reductions
 
 __global__ void __launch_bounds__(THREADS, 1)
     bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -204,7 +220,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* p_full = s_free + 2;                 // [buf * 2 + half]  one arrival per warp of the warpgroup
   uint64_t* acc_full = p_full + 4;               // one phase per item: its dK / dV are complete
   uint64_t* acc_free = acc_full + 1;             // one phase per item: the elementwise warps have read them
-  uint64_t* epi_bar = acc_free + 1;              // the elementwise warps' own barrier (bounded waits)
+  uint64_t* staged_v = acc_free + 1;             // one phase per item: its dV is in the staging area
+  uint64_t* staged_k = staged_v + 1;             // one phase per item: its dK is in the staging area
+  uint64_t* vread = staged_k + 1;                // one phase per item: its dV left the staging area
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
   int* pre = reinterpret_cast<int*>(sm + OFF_PRE);
 
@@ -221,7 +239,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = 0; i < N_BAR; ++i) {
       uint32_t cnt = 1;
       if (bars + i >= p_full && bars + i < acc_full) cnt = 4;
-      if (bars + i == acc_free || bars + i == epi_bar) cnt = 8;
+      if (bars + i == acc_free || bars + i == staged_v || bars + i == staged_k) cnt = 8;
       mbar_init(&bars[i], cnt);
     }
     fence_barrier_init();
@@ -366,7 +384,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (ok && have) grads(pv);
     }
-  } else {
+  } else if (warp < 10) {
     // ------------------------------------------------------------ elementwise warps
     const int q4 = warp & 3;                       // TMEM lane quadrant
     const int hh = (warp - 2) >> 2;                // half of the chunk's rows / of the dims in the epilogue
@@ -374,15 +392,23 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
     const float scale_log2 = a.scale_log2;
     const float inv_sqrt_d = a.scale_log2 * 0.693147180559945309f;
-    uint32_t n_it = 0, cc = 0, ep = 0;
+    uint32_t n_it = 0, cc = 0;
     bool ok = true;
-    // all 8 warps meet; false (and the error flag) if the others did not come in time
-    auto epi_sync = [&]() -> bool {
+    // dK of the previous item (through the RoPE adjoint), held until the staging area is free
+    float klo[32], khi[32];
+    bool pend = false;
+    uint32_t pend_it = 0, pend_slot = 0;
+    // stage the held dK once the reducer has read the item's dV out of its slot
+    auto flush_dk = [&]() -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(vread, pend_it & 1, a.err))) return false;
+      uint8_t* stg = sm + OFF_KV + pend_slot * 2 * KTILE;
+      stage_row(stg, hh, key, klo);
+      stage_row(stg, 2 + hh, key, khi);
+      fence_proxy_async();
       __syncwarp();
-      if (lane == 0) mbar_arrive(epi_bar);
-      const bool w = mbar_wait_bounded(epi_bar, ep & 1, a.err);
-      ++ep;
-      return __all_sync(0xffffffffu, w);
+      if (lane == 0) mbar_arrive(staged_k);
+      pend = false;
+      return true;
     };
     Item it;
     int nidx = 0;
@@ -406,87 +432,115 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int blk = it.blk0 + q / CH;
           lim0 = a.local_len - a.q_tokens + blk * Bq + ((q % CH) * RC) % Bq + 32 * hh;
         }
-        uint32_t sv[32], dv[32];
-        tmem_ld32(lane_base + S_COL + buf * 64 + 32 * hh, sv);
-        tmem_ld32(lane_base + DP_COL + buf * 64 + 32 * hh, dv);
-        tmem_wait_ld();
         const float* st = reinterpret_cast<const float*>(sm + OFF_ST + cs * 2 * RC * 4) + 32 * hh;
-        uint32_t pp[16], ds[16];
+        const uint32_t scol = lane_base + S_COL + buf * 64 + 32 * hh, dcol = lane_base + DP_COL + buf * 64 + 32 * hh;
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          float pr[2], dr[2];
+        for (int rr = 0; rr < 2; ++rr) {           // 16 rows at a time; P / dS over columns already read
+          uint32_t sv[16], dv[16], pp[8], ds[8];
+          tmem_ld16(scol + 16 * rr, sv);
+          tmem_ld16(dcol + 16 * rr, dv);
+          tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const bool vis = kvalid && u <= lim0 + j + e;
-            const float pe = vis ? ex2_approx(__uint_as_float(sv[j + e]) * scale_log2 - st[j + e]) : 0.f;
-            pr[e] = pe;
-            dr[e] = pe * (__uint_as_float(dv[j + e]) - st[RC + j + e]) * inv_sqrt_d;
+          for (int j = 0; j < 16; j += 2) {
+            float pr[2], dr[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int row = 16 * rr + j + e;
+              const bool vis = kvalid && u <= lim0 + row;
+              const float pe = vis ? ex2_approx(__uint_as_float(sv[j + e]) * scale_log2 - st[row]) : 0.f;
+              pr[e] = pe;
+              dr[e] = pe * (__uint_as_float(dv[j + e]) - st[RC + row]) * inv_sqrt_d;
+            }
+            pp[j >> 1] = pack_bf16(pr[0], pr[1]);
+            ds[j >> 1] = pack_bf16(dr[0], dr[1]);
           }
-          pp[j >> 1] = pack_bf16(pr[0], pr[1]);
-          ds[j >> 1] = pack_bf16(dr[0], dr[1]);
+          tmem_st8(scol + 8 * rr, pp);
+          tmem_st8(dcol + 8 * rr, ds);
         }
-        tmem_st16(lane_base + S_COL + buf * 64 + 32 * hh, pp);
-        tmem_st16(lane_base + DP_COL + buf * 64 + 32 * hh, ds);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[buf * 2 + hh]);
+        // the previous item's dK goes out after this item's second chunk (its dV has had time to leave)
+        if (pend && q == min(1, nch - 1) && !flush_dk()) { ok = false; break; }
       }
       if (!ok) break;
-      // ---- the item's dK and dV, dims [32 hh, 32 hh + 32) and their RoPE partners + 64,
-      // out of TMEM and, through the item's K/V slot as staging, into the gradients
+      if (pend && !flush_dk()) { ok = false; break; }
+      // ---- the item's dV, dims [32 hh, 32 hh + 32) and [64 + 32 hh, 96 + 32 hh): staged in the
+      // item's K/V slot for the reducer; then its dK, held in registers, and TMEM is free
       const uint32_t kvs = n_it % KVSLOT;
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(acc_full, n_it & 1, a.err))) { ok = false; break; }
       tc_fence_after();
-      float vlo[32], vhi[32], klo[32], khi[32];
-      tmem_ld32(lane_base + DV_COL + 32 * hh, reinterpret_cast<uint32_t(&)[32]>(vlo));
-      tmem_ld32(lane_base + DV_COL + 64 + 32 * hh, reinterpret_cast<uint32_t(&)[32]>(vhi));
+      {
+        float vlo[32], vhi[32];
+        tmem_ld32(lane_base + DV_COL + 32 * hh, reinterpret_cast<uint32_t(&)[32]>(vlo));
+        tmem_ld32(lane_base + DV_COL + 64 + 32 * hh, reinterpret_cast<uint32_t(&)[32]>(vhi));
+        tmem_wait_ld();
+        // keys past the document / context hold exact zeros (P = dS = 0): adding them is harmless
+        uint8_t* stg = sm + OFF_KV + kvs * 2 * KTILE;
+        stage_row(stg, hh, key, vlo);
+        stage_row(stg, 2 + hh, key, vhi);
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(staged_v);
+      }
       tmem_ld32(lane_base + DK_COL + 32 * hh, reinterpret_cast<uint32_t(&)[32]>(klo));
       tmem_ld32(lane_base + DK_COL + 64 + 32 * hh, reinterpret_cast<uint32_t(&)[32]>(khi));
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_free);
-      ++n_it;
-      uint8_t* stg = sm + OFF_KV + kvs * 2 * KTILE;
-      const CUtensorMap* mdv = it.local ? &tm_dvl : &tm_dvb;
-      const CUtensorMap* mdk = it.local ? &tm_dkl : &tm_dkb;
-      // keys past the document / context hold exact zeros (P = dS = 0): adding them is harmless
-      stage_row(stg, hh, key, vlo);
-      stage_row(stg, 2 + hh, key, vhi);
-      fence_proxy_async();
-      if (!epi_sync()) { ok = false; break; }
-      if (tid == EPI_TID) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tma_reduce_add_2d(mdv, stg + c * (KT * 128), 32 * c, it.kv_row);
-        bulk_commit();
-      }
-      // dK through the RoPE adjoint: Global RoPE at k_off + u (local keys), Parallel RoPE at u (bank)
+      // dK through the RoPE adjoint: Global RoPE at k_off + u (local keys), Parallel RoPE at u (bank);
+      // the transposed tables put consecutive keys (positions) next to each other
       if (kvalid) {
-        const float2* cs2 = (it.local ? a.gtab : g.ptab) + (int64_t)u * (DH / 2) + 32 * hh;
+        const int64_t stride = it.local ? g.gtab_t_len : g.ptab_t_len;
+        const float2* cs2 = (it.local ? g.gtab_t : g.ptab_t) + (int64_t)(32 * hh) * stride + u;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float2 c2 = __ldg(cs2 + j);
+          const float2 c2 = __ldg(cs2 + j * stride);
           const float x = klo[j], y = khi[j];
           klo[j] = x * c2.x + y * c2.y;
           khi[j] = y * c2.x - x * c2.y;
         }
       }
-      if (tid == EPI_TID) bulk_wait_read0();
-      if (!epi_sync()) { ok = false; break; }     // the dV boxes have been read: reuse the staging
-      stage_row(stg, hh, key, klo);
-      stage_row(stg, 2 + hh, key, khi);
-      fence_proxy_async();
-      if (!epi_sync()) { ok = false; break; }
-      if (tid == EPI_TID) {
+      pend = true;
+      pend_it = n_it;
+      pend_slot = kvs;
+      ++n_it;
+    }
+    if (ok && pend) flush_dk();
+  } else {
+    // ------------------------------------------------------------ reducer: the gradients out of the staging area
+    if (lane == 0) {
+      uint32_t n_it = 0;
+      bool ok = true;
+      Item it;
+      int nidx = 0;
+      int4 rec = item_record(g, blockIdx.x, NL, total, pre, a.n_kv_heads), nrec;
+      for (int idx = blockIdx.x; ok && idx < total; idx = nidx, rec = nrec) {
+        nidx = idx + step;
+        nrec = item_record(g, nidx, NL, total, pre, a.n_kv_heads);
+        if (!make_item(g, idx, NL, LT, pre, rec, it)) continue;
+        const uint32_t kvs = n_it % KVSLOT;
+        const uint8_t* stg = sm + OFF_KV + kvs * 2 * KTILE;
+        const CUtensorMap* mdv = it.local ? &tm_dvl : &tm_dvb;
+        const CUtensorMap* mdk = it.local ? &tm_dkl : &tm_dkb;
+        if (!mbar_wait_bounded(staged_v, n_it & 1, a.err)) { ok = false; break; }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tma_reduce_add_2d(mdv, stg + c * (KT * 128), 32 * c, it.kv_row);
+        bulk_commit();
+        bulk_wait_read0();
+        mbar_arrive(vread);
+        if (!mbar_wait_bounded(staged_k, n_it & 1, a.err)) { ok = false; break; }
 #pragma unroll
         for (int c = 0; c < 4; ++c) tma_reduce_add_2d(mdk, stg + c * (KT * 128), 32 * c, it.kv_row);
         bulk_commit();
         bulk_wait_read0();
         mbar_arrive(&kv_empty[kvs]);               // the producer may refill the slot
+        ++n_it;
       }
+      bulk_wait0();
     }
-    if (tid == EPI_TID) bulk_wait0();
   }
   tc_fence_before();
   __syncthreads();
@@ -578,6 +632,15 @@ __global__ void __launch_bounds__(IDX_THREADS)
   }
 }
 
+// out[i][pos] = in[pos][i] for a [n][half_d] RoPE table.
+__global__ void rope_transpose_kernel(const float2* __restrict__ in, float2* __restrict__ out, int64_t n, int half_d) {
+  const int64_t total = n * half_d;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = e / n, pos = e % n;
+    out[e] = in[pos * half_d + i];
+  }
+}
+
 __global__ void to_bf16_kernel(const float4* __restrict__ in, uint2* __restrict__ out, int64_t n4) {
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
     const float4 v = in[i];
@@ -601,6 +664,13 @@ cudaError_t launch_attend_bwd_index(const int32_t* sel, const int32_t* doc_len, 
   bwd_index_kernel<<<n_kv_heads, IDX_THREADS, 0, s>>>(sel, doc_len, doc_row, kv_rows, cnt, idx_nitems, idx_items,
                                                       idx_prob, n_docs, n_kv_heads, problems_per_head, top_k,
                                                       item_cap, cap, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_transpose(const float2* in, float2* out, int64_t n, int half_d, int sms, cudaStream_t s) {
+  const int64_t want = (n * half_d + 255) / 256;
+  const int blocks = (int)std::min<int64_t>(want, (int64_t)sms * 8);
+  rope_transpose_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, s>>>(in, out, n, half_d);
   return cudaGetLastError();
 }
 
