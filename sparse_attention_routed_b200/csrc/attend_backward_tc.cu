@@ -32,13 +32,13 @@
 //              keys past the document, and for local keys after the row's
 //              position), and writes both back as packed bf16 over the columns
 //              it read. At the end of an item they stage its dV in the item's
-//              K/V slot (64 KB), take its dK into registers -- TMEM is free for
-//              the next item from here -- and apply the RoPE adjoint; the dK
-//              follows into the slot two chunks into the next item, once the
-//              dV has left it.
-//   warp 10    reducer: adds each staged half to the gradients with TMA
-//              reduce-add (the additions run in L2) and frees the slot; the
-//              waits for those copies fall on this warp alone.
+//              K/V slot (64 KB) and take its dK into registers -- TMEM is free
+//              for the next item from here; the dK follows into the slot two
+//              chunks into the next item, once the dV has left it.
+//   warps 10-11 reducers: turn the staged dK through the RoPE adjoint in
+//              place (64 keys each), and warp 10 adds each staged half to the
+//              gradients with TMA reduce-add (the additions run in L2) and
+//              frees the slot; the waits for those copies fall on it alone.
 // Every mbarrier parity wait targets the phase right after one the same waiter
 // saw complete, so no wait can be satisfied by an older phase.
 #include "common.cuh"
@@ -56,7 +56,7 @@ constexpr int CBOX = RC * 128;        // 64 dims of a chunk (8 KB)
 constexpr int CTILE = 2 * CBOX;       // 64 x 128 bf16 (16 KB)
 constexpr int KVSLOT = 2;
 constexpr int CSLOT = 3;
-constexpr int THREADS = 352;          // producer, MMA, 8 elementwise warps, reducer
+constexpr int THREADS = 384;          // producer, MMA, 8 elementwise warps, 2 reducer warps
 constexpr int TMEM_COLS = 512;
 constexpr int S_COL = 0;              // S^T[buf]  = S_COL + 64 buf   (P^T over its columns)
 constexpr int DP_COL = 128;           // dP^T[buf] = DP_COL + 64 buf  (dS^T over its columns)
@@ -68,7 +68,7 @@ constexpr int OFF_KV = 0;                                  // slot s: K at OFF_K
 constexpr int OFF_C = OFF_KV + KVSLOT * 2 * KTILE;         // slot c: Q at OFF_C + c * 2 CTILE, dO after it
 constexpr int OFF_ST = OFF_C + CSLOT * 2 * CTILE;          // slot c: lse2[64], D[64] at OFF_ST + c * 512
 constexpr int OFF_BAR = OFF_ST + CSLOT * 2 * RC * 4;
-constexpr int N_BAR = 2 * KVSLOT + 2 * CSLOT + 2 + 2 + 4 + 5;
+constexpr int N_BAR = 2 * KVSLOT + 2 * CSLOT + 2 + 2 + 4 + 6;
 constexpr int OFF_TMEM = OFF_BAR + N_BAR * 8;
 
 // One item: 128 keys and the problems whose rows attend them.
@@ -223,6 +223,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* staged_v = acc_free + 1;             // one phase per item: its dV is in the staging area
   uint64_t* staged_k = staged_v + 1;             // one phase per item: its dK is in the staging area
   uint64_t* vread = staged_k + 1;                // one phase per item: its dV left the staging area
+  uint64_t* rope_done = vread + 1;               // one phase per item: the second reducer warp turned its keys
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
   int* pre = reinterpret_cast<int*>(sm + OFF_PRE);
 
@@ -394,7 +395,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const float inv_sqrt_d = a.scale_log2 * 0.693147180559945309f;
     uint32_t n_it = 0, cc = 0;
     bool ok = true;
-    // dK of the previous item (through the RoPE adjoint), held until the staging area is free
+    // dK of the previous item, held until the staging area is free
     float klo[32], khi[32];
     bool pend = false;
     uint32_t pend_it = 0, pend_slot = 0;
@@ -434,25 +435,39 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         const float* st = reinterpret_cast<const float*>(sm + OFF_ST + cs * 2 * RC * 4) + 32 * hh;
         const uint32_t scol = lane_base + S_COL + buf * 64 + 32 * hh, dcol = lane_base + DP_COL + buf * 64 + 32 * hh;
+        // rows [vstart, 32) of this half see the key: all of them (bank keys), from the row whose
+        // position reaches the key (local keys), none (keys past the document or context)
+        const int vstart = !kvalid ? 32 : (it.local ? max(0, u - lim0) : 0);
+        const bool dense = __all_sync(0xffffffffu, vstart == 0);
+        const float2 sc2 = make_float2(scale_log2, scale_log2), c2 = make_float2(inv_sqrt_d, inv_sqrt_d);
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {           // 16 rows at a time; P / dS over columns already read
           uint32_t sv[16], dv[16], pp[8], ds[8];
           tmem_ld16(scol + 16 * rr, sv);
           tmem_ld16(dcol + 16 * rr, dv);
+          float4 l4[4], d4[4];                     // the rows' log-sum-exp and D
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            l4[v] = *reinterpret_cast<const float4*>(st + 16 * rr + 4 * v);
+            d4[v] = *reinterpret_cast<const float4*>(st + RC + 16 * rr + 4 * v);
+          }
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 16; j += 2) {
-            float pr[2], dr[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int row = 16 * rr + j + e;
-              const bool vis = kvalid && u <= lim0 + row;
-              const float pe = vis ? ex2_approx(__uint_as_float(sv[j + e]) * scale_log2 - st[row]) : 0.f;
-              pr[e] = pe;
-              dr[e] = pe * (__uint_as_float(dv[j + e]) - st[RC + row]) * inv_sqrt_d;
+            const float4 lv = l4[j >> 2], dvv = d4[j >> 2];
+            const float2 nl = (j & 2) ? make_float2(-lv.z, -lv.w) : make_float2(-lv.x, -lv.y);
+            const float2 nd = (j & 2) ? make_float2(-dvv.z, -dvv.w) : make_float2(-dvv.x, -dvv.y);
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), sc2, nl);
+            float2 pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if (!dense) {
+              const int row = 16 * rr + j;
+              pe.x = row >= vstart ? pe.x : 0.f;
+              pe.y = row + 1 >= vstart ? pe.y : 0.f;
             }
-            pp[j >> 1] = pack_bf16(pr[0], pr[1]);
-            ds[j >> 1] = pack_bf16(dr[0], dr[1]);
+            const float2 dd = __fadd2_rn(make_float2(__uint_as_float(dv[j]), __uint_as_float(dv[j + 1])), nd);
+            const float2 dsv = __fmul2_rn(__fmul2_rn(pe, dd), c2);
+            pp[j >> 1] = pack_bf16(pe.x, pe.y);
+            ds[j >> 1] = pack_bf16(dsv.x, dsv.y);
           }
           tmem_st8(scol + 8 * rr, pp);
           tmem_st8(dcol + 8 * rr, ds);
@@ -490,19 +505,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_free);
-      // dK through the RoPE adjoint: Global RoPE at k_off + u (local keys), Parallel RoPE at u (bank);
-      // the transposed tables put consecutive keys (positions) next to each other
-      if (kvalid) {
-        const int64_t stride = it.local ? g.gtab_t_len : g.ptab_t_len;
-        const float2* cs2 = (it.local ? g.gtab_t : g.ptab_t) + (int64_t)(32 * hh) * stride + u;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float2 c2 = __ldg(cs2 + j * stride);
-          const float x = klo[j], y = khi[j];
-          klo[j] = x * c2.x + y * c2.y;
-          khi[j] = y * c2.x - x * c2.y;
-        }
-      }
       pend = true;
       pend_it = n_it;
       pend_slot = kvs;
@@ -510,37 +512,106 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (ok && pend) flush_dk();
   } else {
-    // ------------------------------------------------------------ reducer: the gradients out of the staging area
-    if (lane == 0) {
-      uint32_t n_it = 0;
-      bool ok = true;
-      Item it;
-      int nidx = 0;
-      int4 rec = item_record(g, blockIdx.x, NL, total, pre, a.n_kv_heads), nrec;
-      for (int idx = blockIdx.x; ok && idx < total; idx = nidx, rec = nrec) {
-        nidx = idx + step;
-        nrec = item_record(g, nidx, NL, total, pre, a.n_kv_heads);
-        if (!make_item(g, idx, NL, LT, pre, rec, it)) continue;
-        const uint32_t kvs = n_it % KVSLOT;
-        const uint8_t* stg = sm + OFF_KV + kvs * 2 * KTILE;
-        const CUtensorMap* mdv = it.local ? &tm_dvl : &tm_dvb;
-        const CUtensorMap* mdk = it.local ? &tm_dkl : &tm_dkb;
-        if (!mbar_wait_bounded(staged_v, n_it & 1, a.err)) { ok = false; break; }
+    // ------------------------------------------------------------ reducers: the gradients out of the staging area
+    // warp 10 issues the copies (and alone waits for them); both turn dK through the RoPE adjoint,
+    // warp 10 keys [0, 64) of the tile and warp 11 keys [64, 128)
+    const bool lead = warp == 10;
+    const int kr0 = lead ? 0 : 64;
+    // offset of dim l (this lane) of a row r with r % 8 == e inside a swizzled box, minus 32 r
+    int swz[8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tma_reduce_add_2d(mdv, stg + c * (KT * 128), 32 * c, it.kv_row);
-        bulk_commit();
-        bulk_wait_read0();
-        mbar_arrive(vread);
-        if (!mbar_wait_bounded(staged_k, n_it & 1, a.err)) { ok = false; break; }
+    for (int e = 0; e < 8; ++e) swz[e] = (((lane >> 2) ^ e) << 2) + (lane & 3);
+    uint32_t n_it = 0;
+    bool ok = true;
+    Item it;
+    int nidx = 0;
+    int4 rec = item_record(g, blockIdx.x, NL, total, pre, a.n_kv_heads), nrec;
+    for (int idx = blockIdx.x; ok && idx < total; idx = nidx, rec = nrec) {
+      nidx = idx + step;
+      nrec = item_record(g, nidx, NL, total, pre, a.n_kv_heads);
+      if (!make_item(g, idx, NL, LT, pre, rec, it)) continue;
+      const uint32_t kvs = n_it % KVSLOT;
+      uint8_t* stg = sm + OFF_KV + kvs * 2 * KTILE;
+      const CUtensorMap* mdv = it.local ? &tm_dvl : &tm_dvb;
+      const CUtensorMap* mdk = it.local ? &tm_dkl : &tm_dkb;
+      if (lead) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(staged_v, n_it & 1, a.err))) { ok = false; break; }
+        if (lane == 0) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tma_reduce_add_2d(mdk, stg + c * (KT * 128), 32 * c, it.kv_row);
-        bulk_commit();
-        bulk_wait_read0();
-        mbar_arrive(&kv_empty[kvs]);               // the producer may refill the slot
-        ++n_it;
+          for (int c = 0; c < 4; ++c) tma_reduce_add_2d(mdv, stg + c * (KT * 128), 32 * c, it.kv_row);
+          bulk_commit();
+          bulk_wait_read0();
+          mbar_arrive(vread);
+        }
+        __syncwarp();
       }
-      bulk_wait0();
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(staged_k, n_it & 1, a.err))) { ok = false; break; }
+      // dK through the RoPE adjoint, in place: Global RoPE at k_off + u (local keys), Parallel
+      // RoPE at the position u in the document (bank keys). Lane l turns the dim pairs (l, l + 64)
+      // and (l + 32, l + 96) of every key. The (cos, sin) of a key come from the table every 16
+      // keys and in between from the previous key's by the one-position rotation
+      // R(1) = R(u + 1) R(u)^-1 (fp32 rounding of 15 steps, ~1e-6).
+      if (kr0 < it.nvalid) {
+        const float2* tab = it.local ? a.gtab : g.ptab;
+        const int64_t u0 = (int64_t)it.t * KT + kr0;
+        const int nv = it.nvalid - kr0;          // keys of this warp's half inside the tile (> 0)
+        float* box0 = reinterpret_cast<float*>(stg) + kr0 * 32;
+        float2 sa[4], sb[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int64_t u = u0 + min(16 * k, nv - 1);
+          sa[k] = __ldg(tab + u * (DH / 2) + lane);
+          sb[k] = __ldg(tab + u * (DH / 2) + 32 + lane);
+        }
+        float2 ra = make_float2(1.f, 0.f), rb = make_float2(1.f, 0.f);
+        if (nv > 1) {
+          const float2 a1 = __ldg(tab + (u0 + 1) * (DH / 2) + lane), b1 = __ldg(tab + (u0 + 1) * (DH / 2) + 32 + lane);
+          ra = make_float2(a1.x * sa[0].x + a1.y * sa[0].y, a1.y * sa[0].x - a1.x * sa[0].y);
+          rb = make_float2(b1.x * sb[0].x + b1.y * sb[0].y, b1.y * sb[0].x - b1.x * sb[0].y);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (16 * k >= nv) break;
+          float2 ca = sa[k], cb = sb[k];
+#pragma unroll
+          for (int h8 = 0; h8 < 2; ++h8)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int r = 16 * k + 8 * h8 + e;     // r % 8 == e (kr0 is a multiple of 8)
+              if (r < nv) {
+                float* x0 = box0 + r * 32 + swz[e];    // dim l        (box 0)
+                float* x1 = x0 + KT * 32;              // dim l + 32   (box 1)
+                float* y0 = x0 + 2 * KT * 32;          // dim l + 64   (box 2)
+                float* y1 = x0 + 3 * KT * 32;          // dim l + 96   (box 3)
+                const float a0 = *x0, b0 = *y0, a1 = *x1, b1 = *y1;
+                *x0 = a0 * ca.x + b0 * ca.y;
+                *y0 = b0 * ca.x - a0 * ca.y;
+                *x1 = a1 * cb.x + b1 * cb.y;
+                *y1 = b1 * cb.x - a1 * cb.y;
+              }
+              ca = make_float2(ca.x * ra.x - ca.y * ra.y, ca.y * ra.x + ca.x * ra.y);
+              cb = make_float2(cb.x * rb.x - cb.y * rb.y, cb.y * rb.x + cb.x * rb.y);
+            }
+        }
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (!lead) {
+        if (lane == 0) mbar_arrive(rope_done);
+      } else {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(rope_done, n_it & 1, a.err))) { ok = false; break; }
+        if (lane == 0) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tma_reduce_add_2d(mdk, stg + c * (KT * 128), 32 * c, it.kv_row);
+          bulk_commit();
+          bulk_wait_read0();
+          mbar_arrive(&kv_empty[kvs]);             // the producer may refill the slot
+        }
+        __syncwarp();
+      }
+      ++n_it;
     }
+    if (lead && lane == 0) bulk_wait0();
   }
   tc_fence_before();
   __syncthreads();
@@ -632,15 +703,6 @@ __global__ void __launch_bounds__(IDX_THREADS)
   }
 }
 
-// out[i][pos] = in[pos][i] for a [n][half_d] RoPE table.
-__global__ void rope_transpose_kernel(const float2* __restrict__ in, float2* __restrict__ out, int64_t n, int half_d) {
-  const int64_t total = n * half_d;
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t i = e / n, pos = e % n;
-    out[e] = in[pos * half_d + i];
-  }
-}
-
 __global__ void to_bf16_kernel(const float4* __restrict__ in, uint2* __restrict__ out, int64_t n4) {
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
     const float4 v = in[i];
@@ -664,13 +726,6 @@ cudaError_t launch_attend_bwd_index(const int32_t* sel, const int32_t* doc_len, 
   bwd_index_kernel<<<n_kv_heads, IDX_THREADS, 0, s>>>(sel, doc_len, doc_row, kv_rows, cnt, idx_nitems, idx_items,
                                                       idx_prob, n_docs, n_kv_heads, problems_per_head, top_k,
                                                       item_cap, cap, err);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_rope_transpose(const float2* in, float2* out, int64_t n, int half_d, int sms, cudaStream_t s) {
-  const int64_t want = (n * half_d + 255) / 256;
-  const int blocks = (int)std::min<int64_t>(want, (int64_t)sms * 8);
-  rope_transpose_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, s>>>(in, out, n, half_d);
   return cudaGetLastError();
 }
 

@@ -159,9 +159,6 @@ struct AttendBwdArgs {
   const int* idx_prob;       // [Hkv][idx_cap] the problems that selected each document, ascending
   int idx_item_cap;          // bound on the key tiles of one head
   int idx_cap;               // selections per head (problems per head x top_k)
-  const float2* ptab_t;      // [d/2][ptab_t_len] Parallel RoPE table, transposed
-  const float2* gtab_t;      // [d/2][gtab_t_len] Global RoPE table, transposed
-  int64_t ptab_t_len, gtab_t_len;
 };
 // fp32 gradient tensors [rows, 128] in boxes of 32 columns x 128 rows, 128-byte swizzle
 struct AttendGradMaps {
@@ -184,8 +181,6 @@ cudaError_t launch_attend_bwd_index(const int32_t* sel, const int32_t* doc_len, 
                                     int n_docs, int n_kv_heads, int problems_per_head, int top_k, int item_cap,
                                     int cap, int* err, cudaStream_t s);
 cudaError_t launch_to_bf16(const float* in, uint16_t* out, int64_t n, int sms, cudaStream_t s);
-// out[i][pos] = in[pos][i] for a [n][half_d] RoPE table
-cudaError_t launch_rope_transpose(const float2* in, float2* out, int64_t n, int half_d, int sms, cudaStream_t s);
 // tcgen05 dQ for the shapes of attend_prefill_tc_supported (top_k <= 64), given
 // lse2 and drow; maps as for launch_attend_prefill_tc, do_map like q_map over dO (bf16).
 cudaError_t launch_attend_bwd_dq_tc(const AttendBwdArgs& g, const AttendMaps& m, const CUtensorMap& q_map,

@@ -987,8 +987,6 @@ msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k
   // log-sum-exp, then the tcgen05 dQ and dK/dV kernels
   const bool tc_all = tc && attend_prefill_tc_supported(bank->d, s.G, s.Bq) && s.k <= 64;
   const size_t otmp = tc_all ? align_up((size_t)s.B * s.Hq * s.Tq * bank->d * 4) : 0;
-  const size_t ptt = tc ? align_up((size_t)bank->max_len * bank->d / 2 * 8) : 0;
-  const size_t gtt = tc ? align_up((size_t)s.Lc * bank->d / 2 * 8) : 0;
   const int64_t ph = (int64_t)s.B * (s.Tq / s.Bq);           // problems per KV head
   const int64_t cap = ph * s.k;                              // selections per KV head
   const int64_t rb = std::min<int64_t>(bank->n_docs, cap);    // documents one head can have selected
@@ -1002,8 +1000,7 @@ msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k
   if (tc && (cap >= (int64_t(1) << 31) || item_cap >= (int64_t(1) << 31) || bank->hkv > 64))
     return MSA_ERR_UNSUPPORTED;
   const size_t base_ws = kCounterBytes + qrot + lrot + 2 * stats;
-  if ((rc = ensure_workspace(bank, base_ws + dob + i_cnt + i_nit + i_items + i_prob + otmp + ptt + gtt, st)) != MSA_OK)
-    return rc;
+  if ((rc = ensure_workspace(bank, base_ws + dob + i_cnt + i_nit + i_items + i_prob + otmp, st)) != MSA_OK) return rc;
   if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->max_len, s.Lc, st)) != MSA_OK) return rc;
   uint8_t* ws = bank->ws + kCounterBytes;
   uint16_t* q_rot = reinterpret_cast<uint16_t*>(ws);
@@ -1017,8 +1014,6 @@ msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k
   int4* idx_items = reinterpret_cast<int4*>(wtc + dob + i_cnt + i_nit);
   int* idx_prob = reinterpret_cast<int*>(wtc + dob + i_cnt + i_nit + i_items);
   float* o_tmp = reinterpret_cast<float*>(wtc + dob + i_cnt + i_nit + i_items + i_prob);
-  float2* ptab_t = reinterpret_cast<float2*>(wtc + dob + i_cnt + i_nit + i_items + i_prob + otmp);
-  float2* gtab_t = reinterpret_cast<float2*>(wtc + dob + i_cnt + i_nit + i_items + i_prob + otmp + ptt);
   const int64_t qrows = (int64_t)s.B * s.Hq * s.Tq, lrows = (int64_t)s.B * bank->hkv * s.Lc;
   MSA_CUDA(launch_rope_rows((const uint16_t*)q->q, q_rot, bank->d_gtab, qrows, s.Tq, s.Lc - s.Tq, bank->d, st));
   MSA_CUDA(launch_rope_rows((const uint16_t*)q->local_k, l_rot, bank->d_gtab, lrows, s.Lc, 0, bank->d, st));
@@ -1094,12 +1089,6 @@ msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k
     g.idx_prob = idx_prob;
     g.idx_item_cap = (int)item_cap;
     g.idx_cap = (int)cap;
-    MSA_CUDA(launch_rope_transpose(bank->d_ptab, ptab_t, bank->max_len, bank->d / 2, bank->sms, st));
-    MSA_CUDA(launch_rope_transpose(bank->d_gtab, gtab_t, s.Lc, bank->d / 2, bank->sms, st));
-    g.ptab_t = ptab_t;
-    g.gtab_t = gtab_t;
-    g.ptab_t_len = bank->max_len;
-    g.gtab_t_len = s.Lc;
     MSA_CUDA(launch_attend_bwd_dkdv_tc(g, m2, q_map, do_map, gm, bank->sms, st));
     return MSA_OK;
   }
