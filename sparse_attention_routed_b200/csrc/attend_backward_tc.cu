@@ -574,24 +574,37 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (16 * k >= nv) break;
           float2 ca = sa[k], cb = sb[k];
 #pragma unroll
-          for (int h8 = 0; h8 < 2; ++h8)
+          for (int h8 = 0; h8 < 2; ++h8) {
+            // 8 keys at a time: all loads, then the turns, then all stores (r % 8 == e, kr0 a multiple of 8);
+            // dim l of row r: box 0, dim l + 32: box 1, their partners + 64: boxes 2 and 3
+            const int rb8 = 16 * k + 8 * h8;
+            float v[8][4];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const int r = 16 * k + 8 * h8 + e;     // r % 8 == e (kr0 is a multiple of 8)
-              if (r < nv) {
-                float* x0 = box0 + r * 32 + swz[e];    // dim l        (box 0)
-                float* x1 = x0 + KT * 32;              // dim l + 32   (box 1)
-                float* y0 = x0 + 2 * KT * 32;          // dim l + 64   (box 2)
-                float* y1 = x0 + 3 * KT * 32;          // dim l + 96   (box 3)
-                const float a0 = *x0, b0 = *y0, a1 = *x1, b1 = *y1;
-                *x0 = a0 * ca.x + b0 * ca.y;
-                *y0 = b0 * ca.x - a0 * ca.y;
-                *x1 = a1 * cb.x + b1 * cb.y;
-                *y1 = b1 * cb.x - a1 * cb.y;
-              }
+              const float* x = box0 + (rb8 + e) * 32 + swz[e];
+              const bool in = rb8 + e < nv;
+#pragma unroll
+              for (int c = 0; c < 4; ++c) v[e][c] = in ? x[c * KT * 32] : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float a0 = v[e][0], a1 = v[e][1], b0 = v[e][2], b1 = v[e][3];
+              v[e][0] = a0 * ca.x + b0 * ca.y;
+              v[e][2] = b0 * ca.x - a0 * ca.y;
+              v[e][1] = a1 * cb.x + b1 * cb.y;
+              v[e][3] = b1 * cb.x - a1 * cb.y;
               ca = make_float2(ca.x * ra.x - ca.y * ra.y, ca.y * ra.x + ca.x * ra.y);
               cb = make_float2(cb.x * rb.x - cb.y * rb.y, cb.y * rb.x + cb.x * rb.y);
             }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              float* x = box0 + (rb8 + e) * 32 + swz[e];
+              if (rb8 + e < nv) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) x[c * KT * 32] = v[e][c];
+              }
+            }
+          }
         }
       }
       fence_proxy_async();
