@@ -298,6 +298,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t dcol = tl + DP_COL + (j & 1) * 128 + c0;
+      // every key of this half visible for every row of the warp: no per-key masks
+      const bool dense = __all_sync(0xffffffffu, vis_end >= c0 + TN / 2);
+      const float2 sc2 = make_float2(scale_log2, scale_log2), nl2 = make_float2(-lse, -lse);
+      const float2 nd2 = make_float2(-drow, -drow), c2 = make_float2(inv_sqrt_d, inv_sqrt_d);
 #pragma unroll
       for (int rr = 0; rr < 2; ++rr) {
         uint32_t dv[32], pk[16];
@@ -305,14 +309,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          float ds2[2];
-#pragma unroll
-          for (int f = 0; f < 2; ++f) {
-            const int kk = 32 * rr + e + f;
-            const float pe = (c0 + kk < vis_end) ? ex2_approx(__uint_as_float(sv[kk]) * scale_log2 - lse) : 0.f;
-            ds2[f] = pe * (__uint_as_float(dv[e + f]) - drow) * inv_sqrt_d;
+          const int kk = 32 * rr + e;
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[kk]), __uint_as_float(sv[kk + 1])), sc2, nl2);
+          float2 pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          if (!dense) {
+            pe.x = (c0 + kk < vis_end) ? pe.x : 0.f;
+            pe.y = (c0 + kk + 1 < vis_end) ? pe.y : 0.f;
           }
-          pk[e >> 1] = pack_bf16(ds2[0], ds2[1]);
+          const float2 dd = __fadd2_rn(make_float2(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), nd2);
+          const float2 ds2 = __fmul2_rn(__fmul2_rn(pe, dd), c2);
+          pk[e >> 1] = pack_bf16(ds2.x, ds2.y);
         }
         tmem_st16(dcol + 16 * rr, pk);           // columns already read (this round or the last)
       }
