@@ -195,6 +195,24 @@ def chunk_cosines(q_r: np.ndarray, K_r: np.ndarray) -> np.ndarray:
     return (K @ q) / np.maximum(den, 1e-30)
 
 
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """fp64 -> the nearest bf16 value (8 significant bits, ties to even), as fp64.
+    x = m 2^e with 1/2 <= |m| < 1; m 2^8 rounded to an integer (half to even)."""
+    m, e = np.frexp(np.asarray(x, dtype=np.float64))
+    return np.ldexp(np.rint(m * 256.0), e - 8)
+
+
+def chunk_cosines_bf16_keys(q_r: np.ndarray, K_r: np.ndarray) -> np.ndarray:
+    """Chunk cosines with the normalised routing keys stored in bf16 (the reduced-
+    precision router variant): q^ . bf16(k^), q^ = q_r / |q_r| and k^ = K_r / |K_r|
+    exact. Differs from the exact cosine by at most 2^-8 sum_i |q^_i k^_i| <= 2^-8."""
+    q = np.asarray(q_r, dtype=np.float64)
+    K = np.asarray(K_r, dtype=np.float64)
+    qh = q / max(math.sqrt(float(q @ q)), 1e-30)
+    kh = K / np.maximum(np.sqrt(np.einsum("cd,cd->c", K, K)), 1e-30)[:, None]
+    return round_bf16(kh) @ qh
+
+
 def doc_max(chunk_scores: np.ndarray, chunk_doc: np.ndarray, n_docs: int) -> np.ndarray:
     out = np.full(n_docs, -np.inf, dtype=np.float64)
     np.maximum.at(out, chunk_doc, chunk_scores)
@@ -249,7 +267,7 @@ def routed_attention_row(q: np.ndarray, q_index: int, k_off: int, base: float,
 
 def forward(inputs: Dict[str, np.ndarray], doc_lens: Sequence[int], top_k: int,
             route_block: int, base: float = 10000.0, chunk: int = CHUNK,
-            selection=None) -> Dict[str, np.ndarray]:
+            selection=None, router_keys: str = "f32") -> Dict[str, np.ndarray]:
     """The routed sparse-attention step on fully materialised inputs.
 
     inputs (all real-valued arrays, converted to fp64):
@@ -260,6 +278,8 @@ def forward(inputs: Dict[str, np.ndarray], doc_lens: Sequence[int], top_k: int,
       LK, LV [B, Hkv, Lc, d] un-rotated local keys / values
     selection: optional [B, nblk, Hkv, k] document indices to attend over
       instead of the oracle's own top-k (used when several sets are correct).
+    router_keys: "f32" (the exact cosine) or "bf16" (the reduced-precision router
+      variant: normalised routing keys rounded to bf16, chunk_cosines_bf16_keys).
 
     Returns K_r [Hkv, Nch, d_r], K_rot [Hkv, Ntok, d], q_r [B, nblk, Hkv, d_r],
     doc_scores [B, nblk, Hkv, n], topk [B, nblk, Hkv, k], out [B, Hq, Tq, d].
@@ -296,7 +316,10 @@ def forward(inputs: Dict[str, np.ndarray], doc_lens: Sequence[int], top_k: int,
             qb = block_mean_query(Qr[b, h], route_block)
             for blk in range(nblk):
                 q_r[b, blk, h] = qb[blk]
-                scores[b, blk, h] = route_doc_scores(qb[blk], K_r[h], chunk_doc, n)
+                if router_keys == "bf16":
+                    scores[b, blk, h] = doc_max(chunk_cosines_bf16_keys(qb[blk], K_r[h]), chunk_doc, n)
+                else:
+                    scores[b, blk, h] = route_doc_scores(qb[blk], K_r[h], chunk_doc, n)
                 topk[b, blk, h] = select_top_k(scores[b, blk, h], top_k)
     sel = topk if selection is None else np.asarray(selection, dtype=np.int64)
 
