@@ -56,6 +56,9 @@ def parse():
     ap.add_argument("--build-only", action="store_true",
                     help="time msa_build_bank (chunk-mean pooling of the routing keys + Parallel RoPE of the "
                          "bank keys, in place) over the whole bank of --workload")
+    ap.add_argument("--kr-bf16", action="store_true",
+                    help="the reduced-precision router: read only the bf16 high part of the normalised K_r "
+                         "(msa_set_router_precision(MSA_KR_BF16)), half the router's bytes")
     ap.add_argument("--route-only", action="store_true",
                     help="time msa_route alone on the full bank's K_r with a stand-in 1-document K/V "
                          "(routing keys streamed in slices; a few GB on the device, for profiling captures)")
@@ -285,7 +288,7 @@ def run_ours(args):
     import torch.distributed as dist
 
     import synth
-    from sparse_attention_routed_b200 import msa_attend, msa_route, ptr
+    from sparse_attention_routed_b200 import MSA_KR_BF16, msa_attend, msa_route, ptr
     from sparse_attention_routed_b200.runner import Bank
     from synth.device import bank_tensors, query_tensors
 
@@ -302,6 +305,8 @@ def run_ours(args):
     K, V, R = bank_tensors(w)
     bank = Bank(K, V, w.doc_lens(), w.rope_base)
     bank.build(R)
+    if args.kr_bf16:
+        bank.set_router_precision(MSA_KR_BF16)
     torch.cuda.synchronize()
     del R
     torch.cuda.empty_cache()
@@ -342,7 +347,7 @@ def run_ours(args):
     kv_local = B * Hkv * w.local_len * d * 2 * 2
     q_out = B * w.n_q_heads * w.q_tokens * d * (2 + 4)
     nch = bank.info["n_chunks"]
-    router = Hkv * nch * (d * 4) + B * nblk * Hkv * w.n_docs * 4 * 2 + B * Hkv * w.q_tokens * d * 2
+    router = Hkv * nch * (d * (2 if args.kr_bf16 else 4)) + B * nblk * Hkv * w.n_docs * 4 * 2 + B * Hkv * w.q_tokens * d * 2
     attn_bytes = kv_sel + kv_local + q_out
     step_bytes = attn_bytes + router
     G = w.n_q_heads // w.n_kv_heads
@@ -472,7 +477,8 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(base_config(w), parallelism=f"replicas x{world}",
-                           l2=f"inputs larger than L2: {step_bytes / 1e9:.2f} GB of HBM per step vs 126 MB L2"),
+                           l2=f"inputs larger than L2: {step_bytes / 1e9:.2f} GB of HBM per step vs 126 MB L2",
+                           router_keys="bf16" if args.kr_bf16 else "f32"),
             "router_attn_hbm": {"bytes_per_step": step_bytes, "GBps": step_bytes / (ms_step / 1000.0) / 1e9,
                                 "frac_of_peak": step_bytes / (ms_step / 1000.0) / 1e9 / peak,
                                 "route_ms": route_ms, "attend_ms": attend_ms},

@@ -84,6 +84,12 @@ typedef enum {
   MSA_KV_PINNED_HOST = 1  /* bank K/V in pinned (page-locked) host memory */
 } msa_kv_location;
 
+/* Precision of the routing keys the router reads (msa_set_router_precision). */
+typedef enum {
+  MSA_KR_F32 = 0,         /* normalised K_r as a bf16 high part + bf16 remainder (~16 significant bits) */
+  MSA_KR_BF16 = 1         /* the bf16 high part only: half the router's bytes */
+} msa_kr_precision;
+
 /* Opaque bank handle. Owns: K_r (fp32) and its inverse norms, document and
  * chunk offsets, RoPE tables, workspace, and (host tier) the device staging
  * pool, side stream and events. */
@@ -240,10 +246,22 @@ msa_status msa_set_kv_cache(msa_bank* bank, int64_t bytes);
  * the bytes copied over PCIe. */
 msa_status msa_kv_cache_stats(const msa_bank* bank, int64_t* slabs, int64_t* hits, int64_t* bytes_copied);
 
+/* Precision of the routing keys the router reads (a 16-bit memory bank: the
+ * nxmr.cn article "MSA技术解析为什么它能引爆AI社区", §2.2). MSA_KR_F32 (the
+ * default): the normalised K_r is read as a bf16 high part plus a bf16
+ * remainder, about 16 significant bits, so scores are the fp32 cosine to ~1e-5.
+ * MSA_KR_BF16: only the bf16 high part, half the router's bytes; a score then
+ * differs from the exact cosine by at most 2^-8 sum_i |q^_i k^_i| (the query
+ * keeps full precision). Applies to every later msa_route / msa_forward /
+ * msa_route_noalloc call on the bank. Returns MSA_ERR_INVALID_ARG for a NULL
+ * bank or another value. */
+msa_status msa_set_router_precision(msa_bank* bank, msa_kr_precision precision);
+
 /* Failure-detection check of the device-side bounded waits (the pages describe
  * no such call): launches one small kernel on `stream` whose thread waits on an
- * mbarrier phase that nothing ever completes, with the same poll limit every
- * kernel of this library uses (2^22 polls of mbarrier.try_wait). The wait gives
+ * mbarrier phase that nothing ever completes, with the same limit every kernel
+ * of this library uses (mbarrier.try_wait polls that suspend up to 1 us each,
+ * about 1.1 s in all). The wait gives
  * up, raises the bank's device error flag and the kernel returns normally: no
  * fault, and the context stays usable. A following msa_get_device_error()
  * returns MSA_ERR_TIMEOUT (and clears the flag). Returns MSA_ERR_INVALID_ARG for

@@ -29,6 +29,8 @@ MSA_ERR_HOST_TIER = 6
 
 MSA_KV_DEVICE = 0
 MSA_KV_PINNED_HOST = 1
+MSA_KR_F32 = 0
+MSA_KR_BF16 = 1
 
 
 class MsaError(RuntimeError):
@@ -75,6 +77,7 @@ def _load():
         "msa_attend_backward": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "msa_set_kv_cache": ([vp, i64], ctypes.c_int),
         "msa_kv_cache_stats": ([vp, ctypes.POINTER(i64), ctypes.POINTER(i64), ctypes.POINTER(i64)], ctypes.c_int),
+        "msa_set_router_precision": ([vp, ctypes.c_int], ctypes.c_int),
         "msa_check_wait_timeout": ([vp, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
@@ -103,7 +106,8 @@ def __getattr__(name):
 # Every symbol include/msa.h declares, in declaration order.
 EXPORTED = ["msa_bank_create", "msa_bank_destroy", "msa_build_bank", "msa_bank_info", "msa_reserve",
             "msa_route", "msa_attend", "msa_attend_backward", "msa_forward", "msa_route_noalloc", "msa_set_kv_cache",
-            "msa_kv_cache_stats", "msa_check_wait_timeout", "msa_get_device_error", "msa_status_string"]
+            "msa_kv_cache_stats", "msa_set_router_precision", "msa_check_wait_timeout", "msa_get_device_error",
+            "msa_status_string"]
 
 
 def msa_status_string(status: int) -> str:
@@ -231,6 +235,11 @@ def msa_kv_cache_stats(bank) -> dict:
     vals = [ctypes.c_int64() for _ in range(3)]
     _check(lib().msa_kv_cache_stats(bank, *[ctypes.byref(v) for v in vals]), "msa_kv_cache_stats")
     return {"slabs": vals[0].value, "hits": vals[1].value, "bytes_copied": vals[2].value}
+
+
+def msa_set_router_precision(bank, precision: int) -> None:
+    """MSA_KR_F32 (default: K_r hi + lo, ~16 significant bits) or MSA_KR_BF16 (the bf16 high part only)."""
+    _check(lib().msa_set_router_precision(bank, int(precision)), "msa_set_router_precision")
 
 
 def msa_check_wait_timeout(bank, stream=0) -> None:

@@ -56,6 +56,7 @@ struct RouteArgs {
   const uint16_t* qr;
   int32_t q_tokens, route_block;
   int* err;                // device error flag for expired waits, or nullptr
+  int32_t kr_bf16;         // 1: read only the bf16 high part of the normalised K_r (half the bytes)
 };
 // Largest routing block for which the router computes q_r itself.
 constexpr int kRouteFuseMaxBlock = 4;
@@ -126,6 +127,7 @@ struct BankRouteView {
   const int32_t* chunk_off;
   int64_t nch;
   int32_t n_docs, n_kv_heads, route_dim, sms;
+  int32_t kr_bf16;
 };
 
 // Host-side helpers.

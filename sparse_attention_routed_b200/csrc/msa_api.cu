@@ -174,6 +174,7 @@ struct msa_bank {
   std::list<int64_t> lru;                          // slots, least recently used first
   std::vector<std::list<int64_t>::iterator> slot_it;
   int64_t step_no = 0;
+  bool kr_bf16 = false;     // router reads only the bf16 high part of the normalised K_r
   int64_t st_slabs = 0, st_hits = 0;  // the last step's distinct slabs and cache hits
 };
 
@@ -363,6 +364,7 @@ msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, co
   ra.n_docs = bank->n_docs;
   ra.route_dim = bank->dr;
   ra.err = bank->d_err;
+  ra.kr_bf16 = bank->kr_bf16 ? 1 : 0;
   if (tc) {
     MSA_CUDA(launch_route_tc(ra, bank->route_maps, bank->sms, st));
   } else {
@@ -647,6 +649,7 @@ void msa_bank_route_view(const msa_bank* bank, msa::BankRouteView* v) {
   v->n_kv_heads = bank->hkv;
   v->route_dim = bank->dr;
   v->sms = bank->sms;
+  v->kr_bf16 = bank->kr_bf16 ? 1 : 0;
 }
 
 // msa_forward on a pinned-host bank: the batch runs as up to kMicro
@@ -1139,6 +1142,12 @@ msa_status msa_kv_cache_stats(const msa_bank* bank, int64_t* slabs, int64_t* hit
   if (slabs) *slabs = bank->st_slabs;
   if (hits) *hits = bank->st_hits;
   if (bytes_copied) *bytes_copied = bank->last_fetch_bytes;
+  return MSA_OK;
+}
+
+msa_status msa_set_router_precision(msa_bank* bank, msa_kr_precision precision) {
+  if (!bank || (precision != MSA_KR_F32 && precision != MSA_KR_BF16)) return MSA_ERR_INVALID_ARG;
+  bank->kr_bf16 = precision == MSA_KR_BF16;
   return MSA_OK;
 }
 

@@ -48,7 +48,9 @@ __global__ void qr_prep_kernel(QrArgs a) {
 //   S^T[chunk, row] = sum_d Khat[chunk, d] * Qhat[row, d],
 // with Khat = K_r/|K_r| and Qhat = q_r/|q_r| each split into bf16 hi + lo and
 // the products lo*hi + hi*lo + hi*hi accumulated in fp32 by mma.sync m16n8k16
-// (chunks as M, query rows as N). The score is then the cosine itself.
+// (chunks as M, query rows as N). The score is then the cosine itself. With
+// LO = false (the bf16 K_r variant) only Khat_hi is streamed, half the bytes,
+// and the score is Khat_hi . Qhat (the query keeps its hi + lo split).
 // Khat tiles of RITEM chunks arrive by 2-D TMA (128-byte swizzle) into a ring
 // whose slots each consumer warp owns; CTA (x, h) owns documents
 // x, x + gridDim.x, ... of KV head h, its j-th document going to warp
@@ -72,7 +74,7 @@ struct RouteShape {
   }
 };
 
-template <int DR, int NT>
+template <int DR, int NT, bool LO>
 __global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
     route_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo,
                  const RouteArgs a, int row0) {
@@ -170,11 +172,11 @@ __global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
             ++qw[w];
             uint8_t* dst = ring + slot * SH::SLOT_BYTES;
             const int y = (int)((int64_t)h * a.nch + cs);
-            mbar_arrive_expect_tx(&full[slot], SH::SLOT_BYTES);
+            mbar_arrive_expect_tx(&full[slot], LO ? SH::SLOT_BYTES : SH::MAT_BYTES);
 #pragma unroll
             for (int bx = 0; bx < SH::BOXES; ++bx) {
               tma_load_2d(dst + bx * SH::BOX_BYTES, &tm_hi, bx * 64, y, &full[slot], pol);
-              tma_load_2d(dst + SH::MAT_BYTES + bx * SH::BOX_BYTES, &tm_lo, bx * 64, y, &full[slot], pol);
+              if (LO) tma_load_2d(dst + SH::MAT_BYTES + bx * SH::BOX_BYTES, &tm_lo, bx * 64, y, &full[slot], pol);
             }
           }
         }
@@ -230,10 +232,10 @@ __global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
         const uint32_t off = (col >> 6) * SH::BOX_BYTES + swz128(arow, (col & 63) >> 3);
         uint32_t ah[4], al[4];
         ldmatrix_x4(ah, hbase + off);
-        ldmatrix_x4(al, lbase + off);
+        if (LO) ldmatrix_x4(al, lbase + off);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          mma_bf16_16816(acc[nt], al, bh[ks][nt][0], bh[ks][nt][1]);
+          if (LO) mma_bf16_16816(acc[nt], al, bh[ks][nt][0], bh[ks][nt][1]);
           mma_bf16_16816(acc[nt], ah, bl[ks][nt][0], bl[ks][nt][1]);
           mma_bf16_16816(acc[nt], ah, bh[ks][nt][0], bh[ks][nt][1]);
         }
@@ -267,7 +269,7 @@ __global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
 
 template <int DR, int NT>
 cudaError_t launch_route_t(const RouteArgs& a, const RouteMaps& m, int row0, int sms, cudaStream_t s) {
-  auto kern = route_kernel<DR, NT>;
+  auto kern = a.kr_bf16 ? route_kernel<DR, NT, false> : route_kernel<DR, NT, true>;
   const size_t smem = RouteShape<DR, NT>::bytes();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

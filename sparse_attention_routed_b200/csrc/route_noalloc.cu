@@ -88,6 +88,7 @@ extern "C" msa_status msa_route_noalloc(msa_bank* bank, const msa_query* q, int3
   ra.n_kv_heads = v.n_kv_heads;
   ra.n_docs = v.n_docs;
   ra.route_dim = v.route_dim;
+  ra.kr_bf16 = v.kr_bf16;
   // the same router msa_route takes for this shape
   const cudaError_t e = msa::route_tc_supported(v.route_dim, (int)rows) ? msa::launch_route_tc(ra, v.maps, v.sms, s)
                                                                           : msa::launch_route(ra, v.maps, s);

@@ -8,8 +8,9 @@
 // score(row, chunk) = cos(q_r[row], K_r[chunk]) = q^ . k^ with both sides
 // normalised and split into a bf16 high part and a bf16 remainder, the product
 // taken as q_lo.k_hi + q_hi.k_lo + q_hi.k_hi (about 16 significant bits on each
-// side; the dropped lo.lo term is below 2^-16 relative). A document's score is
-// the max over its chunks.
+// side; the dropped lo.lo term is below 2^-16 relative). With the bf16 K_r
+// variant only k^_hi is streamed and the product is q_lo.k_hi + q_hi.k_hi. A
+// document's score is the max over its chunks.
 //
 // One CTA per (range of whole documents, KV head, pass of up to 128 rows):
 //   warp 0     TMA: 128-chunk tiles of k^_hi and k^_lo into a 2-stage ring.
@@ -121,11 +122,13 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         // rows past c1 belong to other CTAs (or past the end: zero-filled) and are ignored
         const int y = (int)((int64_t)h * a.nch + c0 + t * RT_N);
         uint8_t* dst = sm + OFF_B0 + st * 2 * RT_TILE;
-        mbar_arrive_expect_tx(&b_full[st], 2 * RT_TILE);
+        mbar_arrive_expect_tx(&b_full[st], a.kr_bf16 ? RT_TILE : 2 * RT_TILE);
         tma_load_2d(dst, &tm_hi, 0, y, &b_full[st], pol);
         tma_load_2d(dst + RT_BOX, &tm_hi, 64, y, &b_full[st], pol);
-        tma_load_2d(dst + RT_TILE, &tm_lo, 0, y, &b_full[st], pol);
-        tma_load_2d(dst + RT_TILE + RT_BOX, &tm_lo, 64, y, &b_full[st], pol);
+        if (!a.kr_bf16) {
+          tma_load_2d(dst + RT_TILE, &tm_lo, 0, y, &b_full[st], pol);
+          tma_load_2d(dst + RT_TILE + RT_BOX, &tm_lo, 64, y, &b_full[st], pol);
+        }
       }
     }
   } else if (warp == 1) {
@@ -147,7 +150,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         for (int ks = 0; ks < RT_D / 16; ++ks) {
           const uint64_t o = (uint64_t)(((ks >> 2) * RT_BOX + (ks & 3) * 32) >> 4);
           umma_bf16_ss(dt, alo + o, bhi + o, idesc, ks > 0 ? 1u : 0u);
-          umma_bf16_ss(dt, ahi + o, blo + o, idesc, 1u);
+          if (!a.kr_bf16) umma_bf16_ss(dt, ahi + o, blo + o, idesc, 1u);
           umma_bf16_ss(dt, ahi + o, bhi + o, idesc, 1u);
         }
         umma_commit(&d_full[buf]);

@@ -11,7 +11,7 @@ import torch
 
 from . import (MSA_KV_DEVICE, make_query, msa_attend, msa_bank_create, msa_bank_destroy, msa_bank_info,
                msa_build_bank, msa_forward, msa_get_device_error, msa_kv_cache_stats, msa_reserve, msa_route,
-               msa_set_kv_cache, ptr)
+               msa_set_kv_cache, ptr, msa_set_router_precision)
 
 
 class _DeviceArray:
@@ -109,6 +109,10 @@ class Bank:
     def set_kv_cache(self, nbytes: int):
         """Device-resident slab cache of a pinned-host bank (0 turns it off)."""
         msa_set_kv_cache(self.handle, nbytes)
+
+    def set_router_precision(self, precision: int):
+        """MSA_KR_F32 (default) or MSA_KR_BF16: the precision of the routing keys the router reads."""
+        msa_set_router_precision(self.handle, precision)
 
     def cache_stats(self) -> dict:
         """Distinct slabs, cache hits and PCIe bytes of the last host-tier step."""
