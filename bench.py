@@ -787,9 +787,16 @@ def run_backward(args):
     tpeak, tkind = tensor_peak()
     achieved = flops / (ms / 1e3) / 1e12
     units = w.batch * w.q_tokens
-    # head_dim 128 with routing blocks of a multiple of 64 tokens takes the key-tile tcgen05 dK/dV
-    # (plus the dO conversion and the selection index); other shapes the mma.sync one
-    if w.head_dim == 128 and w.route_block % 64 == 0:
+    # kernels per step: two RoPE passes (queries, local keys), then
+    #   head_dim 128, 64- or 128-token blocks, G * Bq a multiple of 128: the tcgen05 forward
+    #     (O and log-sum-exp), bwd_prep, bwd_index, bwd_dq_tc, bwd_dkdv_tc;
+    #   other blocks of a multiple of 64 tokens at head_dim 128: bwd_dq (mma.sync), to_bf16,
+    #     bwd_index, bwd_dkdv_tc;
+    #   anything else: bwd_dq and bwd_dkdv (mma.sync)
+    G_ = w.n_q_heads // w.n_kv_heads
+    if w.head_dim == 128 and w.route_block in (64, 128) and (G_ * w.route_block) % 128 == 0 and w.top_k <= 64:
+        kernels, launches = "bwd_dq_tc_kernel + bwd_dkdv_tc_kernel (tcgen05; forward recompute on tcgen05)", 7
+    elif w.head_dim == 128 and w.route_block % 64 == 0:
         kernels, launches = "bwd_dq_kernel (mma.sync) + bwd_dkdv_tc_kernel (tcgen05)", 6
     else:
         kernels, launches = "bwd_dq_kernel + bwd_dkdv_kernel (mma.sync)", 4
