@@ -261,6 +261,22 @@ def routed_attention_row(q: np.ndarray, q_index: int, k_off: int, base: float,
     return softmax_attention(q_rot, keys, values)
 
 
+def routed_attention_row_lse(q: np.ndarray, q_index: int, k_off: int, base: float,
+                             mem_k_rot: np.ndarray, local_k: np.ndarray) -> float:
+    """log sum_j exp(s_j) (natural log) over one query row's key set, with
+    s_j = q_rot . k_j / sqrt(d) -- the normaliser of routed_attention_row's softmax
+    (out = sum_j exp(s_j - lse) v_j). Same key set and RoPE positions; evaluated as
+    m + log sum_j exp(s_j - m), m = max_j s_j."""
+    q_rot = rope(q, k_off + q_index, base)
+    d = q_rot.shape[-1]
+    vis = q_index + 1
+    loc_k_rot = rope(local_k[:vis], k_off + np.arange(vis), base)
+    keys = np.concatenate([np.asarray(mem_k_rot, dtype=np.float64), loc_k_rot], axis=0)
+    s = keys @ q_rot / math.sqrt(d)
+    m = s.max()
+    return float(m + math.log(np.exp(s - m).sum()))
+
+
 # --------------------------------------------------------------------------
 # the whole step on explicit (small) tensors
 # --------------------------------------------------------------------------
