@@ -183,6 +183,15 @@ msa_status msa_route(msa_bank* bank, const msa_query* q, int32_t top_k, float* d
 msa_status msa_attend(msa_bank* bank, const msa_query* q, int32_t top_k,
                       const int32_t* topk_idx, float* out, void* stream);
 
+/* msa_attend that also writes each row's log-sum-exp, the state a training step
+ * keeps for msa_attend_backward_saved:
+ *   lse [B, Hq, Tq] fp32: log sum_j exp(s_j), natural log, over the row's key
+ *   set, s_j = q_rot . k_j / sqrt(d) (so out = sum_j exp(s_j - lse) v_j).
+ * out is bit for bit what msa_attend writes. Same shapes, errors and device-side
+ * checks as msa_attend; MSA_ERR_INVALID_ARG for a NULL lse. */
+msa_status msa_attend_lse(msa_bank* bank, const msa_query* q, int32_t top_k,
+                          const int32_t* topk_idx, float* out, float* lse, void* stream);
+
 /* Backward of msa_attend for the selection in topk_idx (the top-k routing is not
  * differentiated: the layer trains end to end on each step's selection,
  * "MSA (Memory Sparse Attention)", robocikowo.com, Komponenty). Gradients of
@@ -202,6 +211,18 @@ msa_status msa_attend(msa_bank* bank, const msa_query* q, int32_t top_k,
 msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k, const int32_t* topk_idx,
                                const float* d_out, float* dq, float* dlocal_k, float* dlocal_v,
                                float* dbank_k, float* dbank_v, void* stream);
+
+/* msa_attend_backward given the forward's state: out and lse as msa_attend_lse
+ * wrote them for the same q, top_k and topk_idx (both read, not written). Where
+ * the backward runs on the tcgen05 tensor cores (head_dim 128, routing blocks of
+ * 64 or 128 tokens, Hq / Hkv * route_block a multiple of 128, top_k <= 64) they
+ * replace the forward recompute that msa_attend_backward performs; other shapes
+ * recompute as msa_attend_backward does. Same outputs, layouts, errors and
+ * accumulation; MSA_ERR_INVALID_ARG for a NULL or unaligned out or a NULL lse. */
+msa_status msa_attend_backward_saved(msa_bank* bank, const msa_query* q, int32_t top_k, const int32_t* topk_idx,
+                                     const float* out, const float* lse, const float* d_out, float* dq,
+                                     float* dlocal_k, float* dlocal_v, float* dbank_k, float* dbank_v,
+                                     void* stream);
 
 /* msa_route followed by msa_attend on one stream; topk_idx receives the selection. */
 msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_t* topk_idx,

@@ -74,7 +74,10 @@ def _load():
         "msa_forward": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp], ctypes.c_int),
         "msa_get_device_error": ([vp, vp], ctypes.c_int),
         "msa_route_noalloc": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp, vp], ctypes.c_int),
+        "msa_attend_lse": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp, vp], ctypes.c_int),
         "msa_attend_backward": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+        "msa_attend_backward_saved": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+                                      ctypes.c_int),
         "msa_set_kv_cache": ([vp, i64], ctypes.c_int),
         "msa_kv_cache_stats": ([vp, ctypes.POINTER(i64), ctypes.POINTER(i64), ctypes.POINTER(i64)], ctypes.c_int),
         "msa_set_router_precision": ([vp, ctypes.c_int], ctypes.c_int),
@@ -105,7 +108,8 @@ def __getattr__(name):
 
 # Every symbol include/msa.h declares, in declaration order.
 EXPORTED = ["msa_bank_create", "msa_bank_destroy", "msa_build_bank", "msa_bank_info", "msa_reserve",
-            "msa_route", "msa_attend", "msa_attend_backward", "msa_forward", "msa_route_noalloc", "msa_set_kv_cache",
+            "msa_route", "msa_attend", "msa_attend_lse", "msa_attend_backward", "msa_attend_backward_saved",
+            "msa_forward", "msa_route_noalloc", "msa_set_kv_cache",
             "msa_kv_cache_stats", "msa_set_router_precision", "msa_check_wait_timeout", "msa_get_device_error",
             "msa_status_string"]
 
@@ -197,6 +201,15 @@ def msa_attend(bank, query: msa_query, top_k: int, topk_idx: int, out: int, stre
     return st
 
 
+def msa_attend_lse(bank, query: msa_query, top_k: int, topk_idx: int, out: int, lse: int, stream=0,
+                   check=True) -> int:
+    st = lib().msa_attend_lse(bank, ctypes.byref(query), top_k, topk_idx or None, out or None, lse or None,
+                              stream or None)
+    if check:
+        _check(st, "msa_attend_lse")
+    return st
+
+
 def msa_forward(bank, query: msa_query, top_k: int, topk_idx: int, out: int, stream=0, check=True) -> int:
     st = lib().msa_forward(bank, ctypes.byref(query), top_k, topk_idx or None, out or None, stream or None)
     if check:
@@ -221,6 +234,17 @@ def msa_attend_backward(bank, query: msa_query, top_k: int, topk_idx: int, d_out
                                    stream or None)
     if check:
         _check(st, "msa_attend_backward")
+    return st
+
+
+def msa_attend_backward_saved(bank, query: msa_query, top_k: int, topk_idx: int, out: int, lse: int, d_out: int,
+                              dq: int, dlocal_k: int, dlocal_v: int, dbank_k: int, dbank_v: int, stream=0,
+                              check=True) -> int:
+    st = lib().msa_attend_backward_saved(bank, ctypes.byref(query), top_k, topk_idx or None, out or None,
+                                         lse or None, d_out or None, dq or None, dlocal_k or None, dlocal_v or None,
+                                         dbank_k or None, dbank_v or None, stream or None)
+    if check:
+        _check(st, "msa_attend_backward_saved")
     return st
 
 

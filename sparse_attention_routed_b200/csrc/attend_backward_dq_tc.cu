@@ -360,9 +360,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-// dO in bf16 and D = dO . O for every query row (one warp per row of 128 dims).
+// dO in bf16, D = dO . O and the log-sum-exp in the backward's units (log2, rows
+// of a problem) for every query row (one warp per row of 128 dims).
 __global__ void bwd_prep_kernel(const float* __restrict__ dout, const float* __restrict__ out,
-                                uint16_t* __restrict__ dout_bf, float* __restrict__ drow, int64_t n_rows,
+                                const float* __restrict__ lse, uint16_t* __restrict__ dout_bf,
+                                float* __restrict__ drow, float* __restrict__ lse2, int64_t n_rows,
                                 int n_q_heads, int n_kv_heads, int q_tokens, int route_block) {
   const int lane = threadIdx.x & 31;
   const int64_t wpb = blockDim.x >> 5;
@@ -380,7 +382,9 @@ __global__ void bwd_prep_kernel(const float* __restrict__ dout, const float* __r
       const int64_t bb = row / ((int64_t)q_tokens * n_q_heads);
       const int G = n_q_heads / n_kv_heads, nblk = q_tokens / route_block;
       const int64_t p = (bb * nblk + t / route_block) * n_kv_heads + hq / G;
-      drow[p * (G * route_block) + (hq % G) * route_block + t % route_block] = s;
+      const int64_t pr = p * (G * route_block) + (hq % G) * route_block + t % route_block;
+      drow[pr] = s;
+      lse2[pr] = lse[row] * 1.4426950408889634f;
     }
   }
 }
@@ -400,14 +404,14 @@ cudaError_t launch_attend_bwd_dq_tc(const AttendBwdArgs& g, const AttendMaps& m,
   return cudaGetLastError();
 }
 
-cudaError_t launch_attend_bwd_prep(const float* dout, const float* out, uint16_t* dout_bf, float* drow, int batch,
-                                   int n_q_heads, int n_kv_heads, int q_tokens, int route_block, int sms,
-                                   cudaStream_t s) {
+cudaError_t launch_attend_bwd_prep(const float* dout, const float* out, const float* lse, uint16_t* dout_bf,
+                                   float* drow, float* lse2, int batch, int n_q_heads, int n_kv_heads, int q_tokens,
+                                   int route_block, int sms, cudaStream_t s) {
   const int64_t n_rows = (int64_t)batch * n_q_heads * q_tokens;
   const int64_t want = (n_rows + 7) / 8;
   const int blocks = (int)std::min<int64_t>(want, (int64_t)sms * 16);
-  bwd_prep_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, s>>>(dout, out, dout_bf, drow, n_rows, n_q_heads, n_kv_heads,
-                                                          q_tokens, route_block);
+  bwd_prep_kernel<<<blocks < 1 ? 1 : blocks, 256, 0, s>>>(dout, out, lse, dout_bf, drow, lse2, n_rows, n_q_heads,
+                                                          n_kv_heads, q_tokens, route_block);
   return cudaGetLastError();
 }
 

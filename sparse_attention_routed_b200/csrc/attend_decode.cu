@@ -515,6 +515,9 @@ __global__ void __launch_bounds__(S::THREADS, S::MINB)
     }
     const float inv = (L > 0.f) ? 1.0f / L : 0.f;
     for (int sp = 0; sp < nS; ++sp) wgt_s[sp * kRowsMax + i] *= inv;
+    if (a.lse_out)
+      a.lse_out[((int64_t)b * a.n_q_heads + h * G + i % G) * a.q_tokens + blk * a.route_block + i / G] =
+          L > 0.f ? (M + log2f(L)) * 0.693147180559945309f : -INFINITY;
   }
   named_barrier_sync(1, CT);
   const float* po = a.part_o + (int64_t)p * nS * rows * D;

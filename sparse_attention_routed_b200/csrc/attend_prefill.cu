@@ -323,6 +323,9 @@ __global__ void __launch_bounds__((PW + 1) * 32, 1)
     if (r >= rows) continue;
     const int hq = h * G + r / a.route_block;
     const int t = blk * a.route_block + r % a.route_block;
+    if (a.lse_out && c == 0)
+      a.lse_out[((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t] =
+          l > 0.f ? (m_run[hf] + log2f(l)) * 0.693147180559945309f : -INFINITY;
     float* dst = a.out + (((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t) * D;
 #pragma unroll
     for (int nd = 0; nd < D / 8; ++nd)

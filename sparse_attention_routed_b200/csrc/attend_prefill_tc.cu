@@ -442,9 +442,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float lt = lA * fA + lB * fB;
       const float inv = lt > 0.f ? 1.0f / lt : 0.f;
       const float wA = fA * inv, wB = fB * inv;
-      if (a.lse2 && wg == 0) a.lse2[(int64_t)p * (G * Bq) + R] = lt > 0.f ? mm + log2f(lt) : -INFINITY;
       const int hq = h * G + g;
       const int t = blk * Bq + t_in;
+      if (a.lse_out && wg == 0)
+        a.lse_out[((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t] =
+            lt > 0.f ? (mm + log2f(lt)) * 0.693147180559945309f : -INFINITY;
       // this warpgroup writes dims [64 wg, 64 wg + 64) of its rows
       float* dst = a.out + (((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t) * TD + c0;
 #pragma unroll

@@ -93,8 +93,8 @@ struct AttendArgs {
   float* part_o;            // [P][S][rows][d]   rows = G * route_block
   float* part_ml;           // [P][S][rows][2]   (running max in log2 units, sum)
   float* out;               // [B, Hq, Tq, d] fp32
-  float* lse2;              // [P][rows] or nullptr: log2-domain log-sum-exp of each row's scaled logits
-                            // (written by the tcgen05 prefill kernel only)
+  float* lse_out;           // [B, Hq, Tq] or nullptr: each row's log-sum-exp (natural log) of its
+                            // logits q_rot . k / sqrt(d) over the row's key set
   int* counters;            // [P] split-completion counters, zero between calls
   int* err;
   int64_t kv_rows;          // rows per head in the bank tensor map
@@ -187,10 +187,11 @@ cudaError_t launch_to_bf16(const float* in, uint16_t* out, int64_t n, int sms, c
 // lse2 and drow; maps as for launch_attend_prefill_tc, do_map like q_map over dO (bf16).
 cudaError_t launch_attend_bwd_dq_tc(const AttendBwdArgs& g, const AttendMaps& m, const CUtensorMap& q_map,
                                     const CUtensorMap& do_map, cudaStream_t s);
-// dO (fp32) -> bf16 and drow[p][r] = dO . O of every query row (head_dim 128).
-cudaError_t launch_attend_bwd_prep(const float* dout, const float* out, uint16_t* dout_bf, float* drow, int batch,
-                                   int n_q_heads, int n_kv_heads, int q_tokens, int route_block, int sms,
-                                   cudaStream_t s);
+// dO (fp32) -> bf16, drow[p][r] = dO . O and lse2[p][r] = lse[b, hq, t] * log2(e) of every
+// query row (head_dim 128; lse is the forward's natural-log log-sum-exp).
+cudaError_t launch_attend_bwd_prep(const float* dout, const float* out, const float* lse, uint16_t* dout_bf,
+                                   float* drow, float* lse2, int batch, int n_q_heads, int n_kv_heads, int q_tokens,
+                                   int route_block, int sms, cudaStream_t s);
 cudaError_t launch_attend_bwd_dkdv_tc(const AttendBwdArgs& g, const AttendMaps& m, const CUtensorMap& q_map,
                                       const CUtensorMap& do_map, const AttendGradMaps& gm, int sms, cudaStream_t s);
 

@@ -573,7 +573,8 @@ msa_status host_fetch(msa_bank* bank, const StepShape& s, const int32_t* idx_dev
 // `staged`: for a pinned-host bank whose selection the caller has already staged,
 // the device table of staging rows (one per selection entry); NULL fetches here.
 msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, int splits, const Workspace& w,
-                       const int32_t* idx, float* out, cudaStream_t st, const int64_t* staged = nullptr) {
+                       const int32_t* idx, float* out, cudaStream_t st, const int64_t* staged = nullptr,
+                       float* lse_out = nullptr) {
   const bool prefill = s.rows > kMaxRows;
   const bool tc = prefill && attend_prefill_tc_supported(bank->d, s.G, s.Bq);
   const int box = tc ? attend_prefill_tc_tile_rows() : prefill ? attend_prefill_tile_rows() : attend_tile_rows();
@@ -629,6 +630,7 @@ msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, i
   a.n_docs = bank->n_docs;
   a.n_splits = splits;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)bank->d));
+  a.lse_out = lse_out;
   if (tc) {
     MSA_CUDA(launch_attend_prefill_tc(a, maps, q_map, st));
   } else if (prefill) {
@@ -951,6 +953,20 @@ msa_status msa_attend(msa_bank* bank, const msa_query* q, int32_t top_k, const i
   return attend_impl(bank, q, s, splits, w, topk_idx, out, (cudaStream_t)stream);
 }
 
+msa_status msa_attend_lse(msa_bank* bank, const msa_query* q, int32_t top_k, const int32_t* topk_idx, float* out,
+                          float* lse, void* stream) {
+  StepShape s;
+  msa_status rc = check_query(bank, q, top_k, &s, true);
+  if (rc != MSA_OK) return rc;
+  if (!topk_idx || !out || !lse) return MSA_ERR_INVALID_ARG;
+  const int splits = choose_splits(bank, s);
+  Workspace w = layout(bank, s, splits, nullptr);
+  if ((rc = ensure_workspace(bank, w.bytes, (cudaStream_t)stream)) != MSA_OK) return rc;
+  if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->max_len, s.Lc, (cudaStream_t)stream)) != MSA_OK) return rc;
+  w = layout(bank, s, splits, bank->ws);
+  return attend_impl(bank, q, s, splits, w, topk_idx, out, (cudaStream_t)stream, nullptr, lse);
+}
+
 msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_t* topk_idx, float* out,
                        void* stream) {
   StepShape s;
@@ -968,9 +984,11 @@ msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_
   return attend_impl(bank, q, s, splits, w, topk_idx, out, st);
 }
 
-msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k, const int32_t* topk_idx,
-                               const float* d_out, float* dq, float* dlocal_k, float* dlocal_v,
-                               float* dbank_k, float* dbank_v, void* stream) {
+namespace {
+// saved_out / saved_lse: the forward's output and log-sum-exp, or both NULL (recomputed)
+msa_status backward_impl(msa_bank* bank, const msa_query* q, int32_t top_k, const int32_t* topk_idx,
+                         const float* saved_out, const float* saved_lse, const float* d_out, float* dq,
+                         float* dlocal_k, float* dlocal_v, float* dbank_k, float* dbank_v, void* stream) {
   StepShape s;
   msa_status rc = check_query(bank, q, top_k, &s, true);
   if (rc != MSA_OK) return rc;
@@ -989,7 +1007,9 @@ msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k
   // the whole step on the tensor cores: the tcgen05 forward gives O and each row's
   // log-sum-exp, then the tcgen05 dQ and dK/dV kernels
   const bool tc_all = tc && attend_prefill_tc_supported(bank->d, s.G, s.Bq) && s.k <= 64;
-  const size_t otmp = tc_all ? align_up((size_t)s.B * s.Hq * s.Tq * bank->d * 4) : 0;
+  const bool saved = saved_out && saved_lse;
+  const size_t otmp = tc_all && !saved ? align_up((size_t)s.B * s.Hq * s.Tq * bank->d * 4) : 0;
+  const size_t ltmp = tc_all && !saved ? align_up((size_t)s.B * s.Hq * s.Tq * 4) : 0;
   const int64_t ph = (int64_t)s.B * (s.Tq / s.Bq);           // problems per KV head
   const int64_t cap = ph * s.k;                              // selections per KV head
   const int64_t rb = std::min<int64_t>(bank->n_docs, cap);    // documents one head can have selected
@@ -1003,7 +1023,8 @@ msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k
   if (tc && (cap >= (int64_t(1) << 31) || item_cap >= (int64_t(1) << 31) || bank->hkv > 64))
     return MSA_ERR_UNSUPPORTED;
   const size_t base_ws = kCounterBytes + qrot + lrot + 2 * stats;
-  if ((rc = ensure_workspace(bank, base_ws + dob + i_cnt + i_nit + i_items + i_prob + otmp, st)) != MSA_OK) return rc;
+  if ((rc = ensure_workspace(bank, base_ws + dob + i_cnt + i_nit + i_items + i_prob + otmp + ltmp, st)) != MSA_OK)
+    return rc;
   if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->max_len, s.Lc, st)) != MSA_OK) return rc;
   uint8_t* ws = bank->ws + kCounterBytes;
   uint16_t* q_rot = reinterpret_cast<uint16_t*>(ws);
@@ -1017,6 +1038,7 @@ msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k
   int4* idx_items = reinterpret_cast<int4*>(wtc + dob + i_cnt + i_nit);
   int* idx_prob = reinterpret_cast<int*>(wtc + dob + i_cnt + i_nit + i_items);
   float* o_tmp = reinterpret_cast<float*>(wtc + dob + i_cnt + i_nit + i_items + i_prob);
+  float* lse_tmp = reinterpret_cast<float*>(wtc + dob + i_cnt + i_nit + i_items + i_prob + otmp);
   const int64_t qrows = (int64_t)s.B * s.Hq * s.Tq, lrows = (int64_t)s.B * bank->hkv * s.Lc;
   MSA_CUDA(launch_rope_rows((const uint16_t*)q->q, q_rot, bank->d_gtab, qrows, s.Tq, s.Lc - s.Tq, bank->d, st));
   MSA_CUDA(launch_rope_rows((const uint16_t*)q->local_k, l_rot, bank->d_gtab, lrows, s.Lc, 0, bank->d, st));
@@ -1074,12 +1096,20 @@ msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k
     if ((rc = make_map(&q_map, q_rot, qrows, bank->d, rc_rows)) != MSA_OK) return rc;
     if ((rc = make_map(&do_map, do_bf, qrows, bank->d, rc_rows)) != MSA_OK) return rc;
     if (tc_all) {
-      // forward (O into the workspace, log-sum-exp per row), dO . O, then dQ
-      AttendArgs fa = a;
-      fa.out = o_tmp;
-      fa.lse2 = lse2;
-      MSA_CUDA(launch_attend_prefill_tc(fa, m2, q_map, st));
-      MSA_CUDA(launch_attend_bwd_prep(d_out, o_tmp, do_bf, drow, s.B, s.Hq, bank->hkv, s.Tq, s.Bq, bank->sms, st));
+      // the forward's O and log-sum-exp (saved by the caller, else recomputed into the
+      // workspace), dO . O, then dQ
+      const float* o_use = saved_out;
+      const float* lse_use = saved_lse;
+      if (!saved) {
+        AttendArgs fa = a;
+        fa.out = o_tmp;
+        fa.lse_out = lse_tmp;
+        MSA_CUDA(launch_attend_prefill_tc(fa, m2, q_map, st));
+        o_use = o_tmp;
+        lse_use = lse_tmp;
+      }
+      MSA_CUDA(launch_attend_bwd_prep(d_out, o_use, lse_use, do_bf, drow, lse2, s.B, s.Hq, bank->hkv, s.Tq, s.Bq,
+                                      bank->sms, st));
       MSA_CUDA(launch_attend_bwd_dq_tc(g, m2, q_map, do_map, st));
     }
     AttendGradMaps gm;
@@ -1098,6 +1128,23 @@ msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k
   const int max_tiles = s.k * (int)((bank->max_len + box - 1) / box) + (s.Lc + box - 1) / box;
   MSA_CUDA(launch_attend_bwd_dkdv(g, maps, bank->d, max_tiles, st));
   return MSA_OK;
+}
+
+}  // namespace
+
+msa_status msa_attend_backward(msa_bank* bank, const msa_query* q, int32_t top_k, const int32_t* topk_idx,
+                               const float* d_out, float* dq, float* dlocal_k, float* dlocal_v,
+                               float* dbank_k, float* dbank_v, void* stream) {
+  return backward_impl(bank, q, top_k, topk_idx, nullptr, nullptr, d_out, dq, dlocal_k, dlocal_v, dbank_k, dbank_v,
+                       stream);
+}
+
+msa_status msa_attend_backward_saved(msa_bank* bank, const msa_query* q, int32_t top_k, const int32_t* topk_idx,
+                                     const float* out, const float* lse, const float* d_out, float* dq,
+                                     float* dlocal_k, float* dlocal_v, float* dbank_k, float* dbank_v,
+                                     void* stream) {
+  if (!out || !lse || !aligned16(out)) return MSA_ERR_INVALID_ARG;
+  return backward_impl(bank, q, top_k, topk_idx, out, lse, d_out, dq, dlocal_k, dlocal_v, dbank_k, dbank_v, stream);
 }
 
 msa_status msa_set_kv_cache(msa_bank* bank, int64_t bytes) {
