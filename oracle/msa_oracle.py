@@ -34,14 +34,16 @@ a time, in the order the method states its steps:
       implementacyjne (Global RoPE with a k-offset for the active context),
       Paradygmat wykonania (only the k selected documents take part).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 the document score is the max over its chunks; a ragged last chunk is the mean
 over its actual tokens; q_r is the unnormalised block mean; a zero-norm cosine
 is 0; RoPE is rotate-half with theta_i = base^(-2i/d); the softmax scale is
 1/sqrt(d); query head hq reads KV head hq // (Hq/Hkv); the Tq queries are the
 last Tq local tokens and local key u is visible to local query i iff u <= i.
 
-Parity pins: every function here is pinned in tests/test_oracle_pins.py
+Parity pins: every function here is pinned -- tests/test_oracle_pins.py (the
+step), tests/test_oracle_backward.py (the backward), tests/test_oracle_router_bf16.py
+(the bf16-key router variant) and tests/test_oracle_lse.py (the row log-sum-exp) --
 against closed forms, invariants, library special cases or brute force.
 """
 from __future__ import annotations

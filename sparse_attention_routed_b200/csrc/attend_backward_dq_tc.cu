@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const float2 ds2 = __fmul2_rn(__fmul2_rn(pe, dd), c2);
           pk[e >> 1] = pack_bf16(ds2.x, ds2.y);
         }
-        tmem_st16(dcol + 16 * rr, pk);           // columns already read (this round or the last)
+        tmem_st16(dcol + 16 * rr, pk);           // columns already read (this pass of 32 keys or the last)
       }
       tmem_wait_st();
       tc_fence_before();
