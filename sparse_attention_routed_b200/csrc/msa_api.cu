@@ -145,7 +145,10 @@ struct msa_bank {
   CUtensorMap map_k128{}, map_v128{};  // boxes of the tcgen05 prefill kernel's tile
   RouteMaps route_maps{};
   // pinned-host K/V tier: selected slabs are copied into a device staging pool
-  static constexpr int kSide = 4;    // copies round-robin over several streams (copy engines)
+#ifndef MSA_HOST_SIDE
+#define MSA_HOST_SIDE 4
+#endif
+  static constexpr int kSide = MSA_HOST_SIDE;  // copies round-robin over several streams (copy engines)
 #ifndef MSA_HOST_MICRO
 #define MSA_HOST_MICRO 2
 #endif
