@@ -634,11 +634,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-// Per KV head h (one CTA each): the documents that some problem of head h
-// selected, in ascending order, the problems that selected each (idx_prob from
-// idx_off, ascending), and one record per 128-key tile of those documents:
-//   {first row of the tile in the K/V maps, t | keys << 16, place in idx_prob, problems},
-// idx_items[h][0 .. idx_nitems[h]). cnt is [Hkv][n_docs] scratch.
+// Per KV head h (one CTA each), over the documents some problem of head h
+// selected (ascending): the problems that selected each document, ascending and
+// contiguous in idx_prob[h], and one record per 128-key tile of those documents,
+//   {first row of the tile in the K/V maps, t | keys << 16, place of the
+//    document's problems in idx_prob[h], number of problems},
+// in idx_items[h][0 .. idx_nitems[h]). cnt is [Hkv][n_docs] scratch.
 constexpr int IDX_THREADS = 1024;
 
 __global__ void __launch_bounds__(IDX_THREADS)
