@@ -1,9 +1,11 @@
 """Full-size parity of the pinned-host tier on the bank_100m workload (24414 documents
 x 4096 tokens = 100M tokens, K/V in pinned host memory over 1024 slabs, 16 decode
-sequences, 32/8 heads, top_k 16) -- the launch bench.py --workload bank_100m times --
-on outputs the oracle computes one by one:
+sequences, 32/8 heads, top_k 16) and the ragged_planted workload (8192 documents of
+512-16384 tokens = 69M tokens, 4 sequences, 64/8 heads, top_k 32, planted routing
+queries) -- the launches bench.py --workload bank_100m / ragged_planted time -- on
+outputs the oracle computes one by one:
   - the top-k of every (sequence, KV head) row is exactly the top-k of the GPU's own
-    scores (index work, all 24414 documents);
+    scores (index work, every document of the bank);
   - for one row, the oracle's scores of the selected documents and of 48 random other
     documents (pooling their routing keys afresh) match the GPU's, and no sampled
     unselected document beats a selected one by more than the near-tie window;
@@ -24,12 +26,12 @@ def _f64(bits):
     return synth.bf16_bits_to_f32(bits).astype(np.float64)
 
 
-@pytest.fixture(scope="module")
-def run():
+@pytest.fixture(scope="module", params=["bank_100m", "ragged_planted"])
+def run(request):
     import sparse_attention_routed_b200 as msa
     from sparse_attention_routed_b200.runner import Bank
     from synth.device import fill_normal, host_kv_pool, query_tensors
-    w = synth.WORKLOADS["bank_100m"]
+    w = synth.WORKLOADS[request.param]
     Hkv, d, B, k = w.n_kv_heads, w.head_dim, w.batch, w.top_k
     Kh, Vh = host_kv_pool(w)
     bank = Bank(Kh, Vh, w.doc_lens(), w.rope_base, kv_location=msa.MSA_KV_PINNED_HOST, doc_rows=w.doc_kv_rows())
@@ -75,11 +77,14 @@ def test_host_full_topk_exact_on_own_scores(run):
 
 def test_host_full_router_sample(run):
     w = run["w"]
-    b, h = 11, 6
+    b, h = w.batch - 1, 6
     rng = np.random.default_rng(7)
     sel = [int(j) for j in run["idx"][b, 0, h]]
     others = [int(j) for j in rng.choice(np.setdiff1d(np.arange(w.n_docs), sel), size=48, replace=False)]
-    Qr = _f64(synth.query_bits(w, synth.T_QR, (w.batch, w.n_kv_heads, w.q_tokens, w.route_dim)))
+    if w.planted:
+        Qr = _f64(synth.planted_qr_bits(w))
+    else:
+        Qr = _f64(synth.query_bits(w, synth.T_QR, (w.batch, w.n_kv_heads, w.q_tokens, w.route_dim)))
     q = O.block_mean_query(Qr[b, h], w.route_block)[0]
     off = run["off"]
     ref = {}
