@@ -50,6 +50,9 @@ def parse():
                     help="host-tier workloads: device-resident slab cache of this many GB (msa_set_kv_cache); "
                          "each step then takes one of --query-pool query batches at random")
     ap.add_argument("--query-pool", type=int, default=4)
+    ap.add_argument("--host-fetch", default="gather", choices=["gather", "copy"],
+                    help="host-tier workloads: move the selected slabs with the SM gather kernel through the "
+                         "mapped pinned K/V (default) or with cudaMemcpyAsync copies (msa_set_host_fetch)")
     ap.add_argument("--backward", action="store_true",
                     help="time msa_attend_backward on --workload's selection (gradients of the queries, "
                          "local K/V and bank K/V)")
@@ -83,14 +86,15 @@ def tensor_peak():
     return 1590.0, "fallback"
 
 
-def launches_per_step(w, batch=None) -> int:
+def launches_per_step(w, batch=None, gather=False) -> int:
     """Kernels libmsa launches for one route + attend step of workload w (over `batch`
-    sequences; msa_forward on a pinned-host bank runs micro-batches of up to 4 parts)."""
+    sequences; msa_forward on a pinned-host bank runs micro-batches of up to 2 parts,
+    each with one slab-gather launch when the SM gather moves the slabs)."""
     if batch is None and w.host_tier:
-        parts = min(w.batch, 4)
+        parts = min(w.batch, 2)
         nb = -(-w.batch // parts)
         sizes = [min(nb, w.batch - b0) for b0 in range(0, w.batch, nb)]
-        return sum(launches_per_step(w, b) for b in sizes)
+        return sum(launches_per_step(w, b) + (1 if gather else 0) for b in sizes)
     batch = w.batch if batch is None else batch
     rows_route = batch * (w.q_tokens // w.route_block)
     n = (0 if w.route_block <= 4 else 1) + (rows_route + 15) // 16 + 1     # qr_prep, router passes, top-k
@@ -556,7 +560,8 @@ def run_host_tier(args):
     import torch
 
     import synth
-    from sparse_attention_routed_b200 import MSA_KV_PINNED_HOST, msa_attend, msa_forward, msa_route
+    from sparse_attention_routed_b200 import (MSA_FETCH_COPY_ENGINE, MSA_FETCH_SM_GATHER, MSA_KV_PINNED_HOST,
+                                              msa_attend, msa_forward, msa_route)
     from sparse_attention_routed_b200.runner import Bank
     from synth.device import fill_normal, host_kv_pool, query_tensors
 
@@ -577,6 +582,7 @@ def run_host_tier(args):
         del R
     torch.cuda.synchronize()
     setup_s = time.time() - t0
+    bank.set_host_fetch(MSA_FETCH_SM_GATHER if args.host_fetch == "gather" else MSA_FETCH_COPY_ENGINE)
     if args.kv_cache_gb > 0:
         return run_host_cache(args, w, bank, setup_s, Kh)
     Q, Qr, LK, LV = query_tensors(w)
@@ -645,8 +651,9 @@ def run_host_tier(args):
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": args.workload, "batch": B, "q_heads": w.n_q_heads, "kv_heads": Hkv,
                    "head_dim": d, "bank_docs": w.n_docs, "bank_tokens": w.n_tokens, "local_len": w.local_len,
-                   "top_k": k, "kv_slabs_pinned": w.kv_slabs, "pinned_kv_bytes": 2 * Kh.numel() * 2},
-        "roofline": {"kernel": "selected K/V slabs over PCIe (cudaMemcpyAsync per host-contiguous run of slabs), "
+                   "top_k": k, "kv_slabs_pinned": w.kv_slabs, "pinned_kv_bytes": 2 * Kh.numel() * 2,
+                   "host_fetch": args.host_fetch},
+        "roofline": {"kernel": "selected K/V slabs over PCIe (" + FETCH_DESC[args.host_fetch] + "), "
                                "whole pipelined step", "bound": "pcie",
                      "achieved": pcie_bytes / (step_ms / 1e3) / 1e9, "peak": h2d_peak,
                      "peak_kind": "measured pinned H2D copy, 1 GiB", "unit": "GB/s",
@@ -655,10 +662,14 @@ def run_host_tier(args):
                    "frac_of_hbm_peak": router_bytes / (route_ms / 1e3) / 1e9 / peak},
         "unpipelined_ms_per_step": unpipelined_ms,
         "planted_recall": recall, "setup_s": setup_s, "clocks": clk,
-        "gpu_launches": launches_per_step(w) * n,
+        "gpu_launches": launches_per_step(w, gather=args.host_fetch == "gather") * n,
     }
     print(json.dumps(line), flush=True)
     bank.close()
+
+
+FETCH_DESC = {"gather": "host_gather_kernel: the SMs read the mapped pinned K/V, one launch per micro-batch",
+              "copy": "cudaMemcpyAsync per host-contiguous run of slabs"}
 
 
 def run_host_cache(args, w, bank, setup_s, Kh):
@@ -717,10 +728,12 @@ def run_host_cache(args, w, bank, setup_s, Kh):
         "dtype": "bf16", "data": f"synthetic; each step one of {len(pool)} seeded query batches, uniform at random",
         "config": dict(base_config(w), bank_tokens=w.n_tokens, kv_slabs_pinned=w.kv_slabs,
                        kv_cache_bytes=int(args.kv_cache_gb * 1e9),
-                       kv_cache_slots=int(args.kv_cache_gb * 1e9) // slab_bytes, query_pool=len(pool)),
+                       kv_cache_slots=int(args.kv_cache_gb * 1e9) // slab_bytes, query_pool=len(pool),
+                       host_fetch=args.host_fetch),
         "cache": {"hit_rate": hits / max(1, slabs), "slabs_per_step": slabs / n,
                   "pcie_bytes_per_step": copied / n, "pcie_GBps": copied / n / (step_ms / 1e3) / 1e9},
-        "setup_s": setup_s, "clocks": clk, "gpu_launches": launches_per_step(w) * n,
+        "setup_s": setup_s, "clocks": clk,
+        "gpu_launches": launches_per_step(w, gather=args.host_fetch == "gather") * n,
     }
     print(json.dumps(line), flush=True)
     bank.close()

@@ -54,11 +54,14 @@
  *     kernel when head_dim = 128, route_block is 64 or 128 and G * route_block
  *     is a multiple of 128; an mma.sync kernel otherwise).
  *   - Bank K/V may live in pinned host memory (MSA_KV_PINNED_HOST): msa_attend
- *     and msa_forward then read the step's selection back to the host, copy
+ *     and msa_forward then read the step's selection back to the host, move
  *     every distinct selected (document, KV head) slab into a device staging
- *     pool with cudaMemcpyAsync on side streams, and attend from there. Those
- *     two calls synchronise the stream once per call and cannot be captured
- *     into a CUDA graph; msa_route never touches host K/V.
+ *     pool (by default with one gather kernel that reads the page-locked K/V
+ *     through its device mapping; else cudaMemcpyAsync on side streams, see
+ *     msa_set_host_fetch), and attend from there. The whole K and V ranges must
+ *     be page-locked (cudaHostAlloc, or cudaHostRegister'd). Those two calls
+ *     synchronise the stream once per call and cannot be captured into a CUDA
+ *     graph; msa_route never touches host K/V.
  */
 #ifndef MSA_H_
 #define MSA_H_
@@ -89,6 +92,12 @@ typedef enum {
   MSA_KR_F32 = 0,         /* normalised K_r as a bf16 high part + bf16 remainder (~16 significant bits) */
   MSA_KR_BF16 = 1         /* the bf16 high part only: half the router's bytes */
 } msa_kr_precision;
+
+/* How a pinned-host bank moves its selected slabs to the device (msa_set_host_fetch). */
+typedef enum {
+  MSA_FETCH_COPY_ENGINE = 0, /* cudaMemcpyAsync per run of host-contiguous slabs, on side streams */
+  MSA_FETCH_SM_GATHER = 1    /* one kernel per stretch reads the mapped host K/V (the default) */
+} msa_host_fetch;
 
 /* Opaque bank handle. Owns: K_r (fp32) and its inverse norms, document and
  * chunk offsets, RoPE tables, workspace, and (host tier) the device staging
@@ -266,6 +275,22 @@ msa_status msa_set_kv_cache(msa_bank* bank, int64_t bytes);
  * the step selected, how many of them were already resident in the cache, and
  * the bytes copied over PCIe. */
 msa_status msa_kv_cache_stats(const msa_bank* bank, int64_t* slabs, int64_t* hits, int64_t* bytes_copied);
+
+/* Transport of a pinned-host bank's slab fetch ("MSA (Memory Sparse Attention)",
+ * robocikowo.com, Pułapki implementacyjne: pinned memory and asynchronous
+ * prefetch). MSA_FETCH_SM_GATHER (the default when msa_bank_create finds the
+ * whole K and V ranges page-locked and mapped into the device's address space):
+ * per planned stretch of slabs, one kernel on a side stream reads the host rows
+ * with 16-byte loads through that mapping and writes the staging pool, so a step
+ * of many small slabs pays no per-transfer cost. MSA_FETCH_COPY_ENGINE: one
+ * cudaMemcpyAsync of K and one of V per run of host-contiguous slabs, round-robin
+ * over the side streams. Both move the same bytes to the same staging rows, so
+ * outputs are identical. Applies to later msa_attend / msa_forward calls;
+ * synchronises the device. Returns MSA_ERR_INVALID_ARG for a NULL or device-tier
+ * bank or another value, MSA_ERR_UNSUPPORTED for MSA_FETCH_SM_GATHER when the host
+ * K/V is not mapped. msa_get_host_fetch reports the current transport. */
+msa_status msa_set_host_fetch(msa_bank* bank, msa_host_fetch mode);
+msa_status msa_get_host_fetch(const msa_bank* bank, msa_host_fetch* mode);
 
 /* Precision of the routing keys the router reads (a 16-bit memory bank: the
  * nxmr.cn article "MSA技术解析为什么它能引爆AI社区", §2.2). MSA_KR_F32 (the

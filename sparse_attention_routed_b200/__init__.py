@@ -31,6 +31,8 @@ MSA_KV_DEVICE = 0
 MSA_KV_PINNED_HOST = 1
 MSA_KR_F32 = 0
 MSA_KR_BF16 = 1
+MSA_FETCH_COPY_ENGINE = 0
+MSA_FETCH_SM_GATHER = 1
 
 
 class MsaError(RuntimeError):
@@ -80,6 +82,8 @@ def _load():
                                       ctypes.c_int),
         "msa_set_kv_cache": ([vp, i64], ctypes.c_int),
         "msa_kv_cache_stats": ([vp, ctypes.POINTER(i64), ctypes.POINTER(i64), ctypes.POINTER(i64)], ctypes.c_int),
+        "msa_set_host_fetch": ([vp, ctypes.c_int], ctypes.c_int),
+        "msa_get_host_fetch": ([vp, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
         "msa_set_router_precision": ([vp, ctypes.c_int], ctypes.c_int),
         "msa_check_wait_timeout": ([vp, vp], ctypes.c_int),
     }
@@ -110,7 +114,7 @@ def __getattr__(name):
 EXPORTED = ["msa_bank_create", "msa_bank_destroy", "msa_build_bank", "msa_bank_info", "msa_reserve",
             "msa_route", "msa_attend", "msa_attend_lse", "msa_attend_backward", "msa_attend_backward_saved",
             "msa_forward", "msa_route_noalloc", "msa_set_kv_cache",
-            "msa_kv_cache_stats", "msa_set_router_precision", "msa_check_wait_timeout", "msa_get_device_error",
+            "msa_kv_cache_stats", "msa_set_host_fetch", "msa_get_host_fetch", "msa_set_router_precision", "msa_check_wait_timeout", "msa_get_device_error",
             "msa_status_string"]
 
 
@@ -259,6 +263,20 @@ def msa_kv_cache_stats(bank) -> dict:
     vals = [ctypes.c_int64() for _ in range(3)]
     _check(lib().msa_kv_cache_stats(bank, *[ctypes.byref(v) for v in vals]), "msa_kv_cache_stats")
     return {"slabs": vals[0].value, "hits": vals[1].value, "bytes_copied": vals[2].value}
+
+
+def msa_set_host_fetch(bank, mode: int, check=True) -> int:
+    """MSA_FETCH_SM_GATHER (default where the host K/V is mapped) or MSA_FETCH_COPY_ENGINE."""
+    st = lib().msa_set_host_fetch(bank, int(mode))
+    if check:
+        _check(st, "msa_set_host_fetch")
+    return st
+
+
+def msa_get_host_fetch(bank) -> int:
+    v = ctypes.c_int()
+    _check(lib().msa_get_host_fetch(bank, ctypes.byref(v)), "msa_get_host_fetch")
+    return v.value
 
 
 def msa_set_router_precision(bank, precision: int) -> None:

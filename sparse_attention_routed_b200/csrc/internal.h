@@ -195,6 +195,20 @@ cudaError_t launch_attend_bwd_prep(const float* dout, const float* out, const fl
 cudaError_t launch_attend_bwd_dkdv_tc(const AttendBwdArgs& g, const AttendMaps& m, const CUtensorMap& q_map,
                                       const CUtensorMap& do_map, const AttendGradMaps& gm, int sms, cudaStream_t s);
 
+// Pinned-host tier: one run of host-contiguous K/V rows and the staging rows it goes
+// to; jobs ascend in piece0, the index of their first piece (host_gather_piece_rows
+// rows of K and of V each) among all pieces of a launch.
+struct HostGatherJob {
+  int64_t src_row;  // first row in the host K / V ([Hkv * kv_rows, d])
+  int64_t dst_row;  // first row in the staging pool
+  int64_t rows;
+  int64_t piece0;
+};
+int64_t host_gather_piece_rows(int head_dim);
+// hk / hv: device mappings of the page-locked host K / V; dk / dv: the staging pool.
+cudaError_t launch_host_gather(const HostGatherJob* jobs, int njobs, int64_t npieces, const void* hk, const void* hv,
+                               void* dk, void* dv, int head_dim, int ctas, cudaStream_t s);
+
 }  // namespace msa
 
 struct msa_bank;

@@ -106,6 +106,24 @@ msa_status upload(T** dst, const std::vector<T>& src) {
   return MSA_OK;
 }
 
+// Device address of page-locked host memory [p, p + bytes), mapped as one range, or
+// nullptr.
+const void* mapped_host(const void* p, size_t bytes) {
+  int dev = 0, can = 0;
+  cudaGetDevice(&dev);
+  if (cudaDeviceGetAttribute(&can, cudaDevAttrCanMapHostMemory, dev) != cudaSuccess || !can) return nullptr;
+  cudaPointerAttributes a{}, z{};
+  const char* last = static_cast<const char*>(p) + bytes - 1;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess || cudaPointerGetAttributes(&z, last) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (a.type != cudaMemoryTypeHost || z.type != cudaMemoryTypeHost || !a.devicePointer ||
+      static_cast<const char*>(z.devicePointer) != static_cast<const char*>(a.devicePointer) + bytes - 1)
+    return nullptr;
+  return a.devicePointer;
+}
+
 }  // namespace
 
 struct msa_bank {
@@ -163,6 +181,17 @@ struct msa_bank {
   int64_t* h_base = nullptr;  // pinned staging row of every selection entry
   int64_t* d_base = nullptr;  // device copy of h_base
   size_t sel_cap = 0;         // entries of h_idx / h_base / d_base
+  // slabs move by an SM gather through the device mapping of the page-locked K/V
+  // (MSA_FETCH_SM_GATHER) or by copy-engine transfers (MSA_FETCH_COPY_ENGINE)
+#ifndef MSA_HOST_FETCH_DEFAULT
+#define MSA_HOST_FETCH_DEFAULT MSA_FETCH_SM_GATHER
+#endif
+  const void* k_map = nullptr;  // device addresses of the host K / V, or nullptr: not mapped
+  const void* v_map = nullptr;
+  bool gather = false;
+  msa::HostGatherJob* h_jobs = nullptr;  // pinned, sel_cap entries: the jobs of selection entries [e0, e1) start at e0
+  msa::HostGatherJob* d_jobs = nullptr;
+  std::vector<msa::HostGatherJob> jobs;  // the stretch being planned
   uint16_t* stage_k = nullptr;
   uint16_t* stage_v = nullptr;
   int64_t stage_cap = 0;      // rows of stage_k / stage_v
@@ -198,6 +227,8 @@ void free_bank(msa_bank* b) {
   if (b->h_idx) cudaFreeHost(b->h_idx);
   if (b->h_base) cudaFreeHost(b->h_base);
   if (b->d_base) cudaFree(b->d_base);
+  if (b->h_jobs) cudaFreeHost(b->h_jobs);
+  if (b->d_jobs) cudaFree(b->d_jobs);
   if (b->stage_k) cudaFree(b->stage_k);
   if (b->stage_v) cudaFree(b->stage_v);
   void* ptrs[] = {b->d_doc_row, b->d_doc_len, b->d_chunk_off, b->d_chunk_tok, b->d_chunk_len,
@@ -405,13 +436,21 @@ msa_status ensure_host_tier(msa_bank* bank, size_t entries) {
     if (bank->h_idx) cudaFreeHost(bank->h_idx);
     if (bank->h_base) cudaFreeHost(bank->h_base);
     if (bank->d_base) cudaFree(bank->d_base);
+    if (bank->h_jobs) cudaFreeHost(bank->h_jobs);
+    if (bank->d_jobs) cudaFree(bank->d_jobs);
     bank->h_idx = nullptr;
     bank->h_base = nullptr;
     bank->d_base = nullptr;
+    bank->h_jobs = bank->d_jobs = nullptr;
     bank->sel_cap = 0;
     if (cudaHostAlloc(&bank->h_idx, entries * 4, cudaHostAllocDefault) != cudaSuccess) return MSA_ERR_HOST_TIER;
     if (cudaHostAlloc(&bank->h_base, entries * 8, cudaHostAllocDefault) != cudaSuccess) return MSA_ERR_HOST_TIER;
     MSA_CUDA(cudaMalloc(&bank->d_base, entries * 8));
+    if (bank->k_map) {
+      const size_t jb = entries * sizeof(msa::HostGatherJob);
+      if (cudaHostAlloc(&bank->h_jobs, jb, cudaHostAllocDefault) != cudaSuccess) return MSA_ERR_HOST_TIER;
+      MSA_CUDA(cudaMalloc(&bank->d_jobs, jb));
+    }
     bank->sel_cap = entries;
   }
   return MSA_OK;
@@ -435,6 +474,51 @@ msa_status ensure_stage(msa_bank* bank, int64_t rows, cudaStream_t st) {
   return MSA_OK;
 }
 
+// One run of `rows` host-contiguous K/V rows, host row `src` to staging row `dst`:
+// a job of the stretch's gather launch, or a copy-engine transfer each of K and V.
+msa_status issue_rows(msa_bank* bank, int64_t src, int64_t dst, int64_t rows, int& stream_rr) {
+  const size_t bytes = (size_t)rows * bank->d * 2;
+  bank->last_fetch_bytes += 2 * (int64_t)bytes;
+  if (bank->gather) {
+    bank->jobs.push_back({src, dst, rows, 0});
+    return MSA_OK;
+  }
+  const uint16_t* hk = static_cast<const uint16_t*>(bank->k);
+  const uint16_t* hv = static_cast<const uint16_t*>(bank->v);
+  if (cudaMemcpyAsync(bank->stage_k + dst * bank->d, hk + src * bank->d, bytes, cudaMemcpyHostToDevice,
+                      bank->side[stream_rr++ % msa_bank::kSide]) != cudaSuccess ||
+      cudaMemcpyAsync(bank->stage_v + dst * bank->d, hv + src * bank->d, bytes, cudaMemcpyHostToDevice,
+                      bank->side[stream_rr++ % msa_bank::kSide]) != cudaSuccess)
+    return MSA_ERR_HOST_TIER;
+  return MSA_OK;
+}
+
+// Launches the gather of the jobs just planned for the stretch of selection entries
+// that starts at e0, on side stream 0. The stretch has at least as many entries as
+// jobs, so its jobs go to the job buffers' entries from e0 on, which no other stretch
+// of the step uses; the previous step's launches are over before any plan is made.
+msa_status flush_jobs(msa_bank* bank, size_t e0) {
+  if (!bank->gather || bank->jobs.empty()) {
+    bank->jobs.clear();
+    return MSA_OK;
+  }
+  const int64_t pr = host_gather_piece_rows(bank->d);
+  const int nj = (int)bank->jobs.size();
+  msa::HostGatherJob* hj = bank->h_jobs + e0;
+  int64_t pieces = 0;
+  for (int i = 0; i < nj; ++i) {
+    hj[i] = bank->jobs[i];
+    hj[i].piece0 = pieces;
+    pieces += (hj[i].rows + pr - 1) / pr;
+  }
+  bank->jobs.clear();
+  MSA_CUDA(cudaMemcpyAsync(bank->d_jobs + e0, hj, nj * sizeof(msa::HostGatherJob), cudaMemcpyHostToDevice,
+                           bank->side[0]));
+  MSA_CUDA(launch_host_gather(bank->d_jobs + e0, nj, pieces, bank->k_map, bank->v_map, bank->stage_k, bank->stage_v,
+                              bank->d, bank->sms, bank->side[0]));
+  return MSA_OK;
+}
+
 // Staging plan of one stretch of selection entries [e0, e1) (bank->h_idx holds
 // them): slabs not staged earlier in the step get rows in host-address order,
 // runs of host-contiguous slabs are copied as one, and h_base[e] receives each
@@ -451,9 +535,6 @@ msa_status stage_entries(msa_bank* bank, int k, size_t e0, size_t e1, std::unord
   }
   bank->st_slabs += (int64_t)fresh.size();
   std::sort(fresh.begin(), fresh.end());
-  const size_t row_bytes = (size_t)bank->d * 2;
-  const uint16_t* hk = static_cast<const uint16_t*>(bank->k);
-  const uint16_t* hv = static_cast<const uint16_t*>(bank->v);
   size_t i = 0;
   while (i < fresh.size()) {
     // a run: each next slab starts where the previous one ends, inside the same head
@@ -468,13 +549,8 @@ msa_status stage_entries(msa_bank* bank, int k, size_t e0, size_t e1, std::unord
       len += bank->doc_lens[j];
     }
     if (rows + len > bank->stage_cap) return MSA_ERR_HOST_TIER;
-    const size_t bytes = (size_t)len * row_bytes;
-    if (cudaMemcpyAsync(bank->stage_k + dst0 * bank->d, hk + src0 * bank->d, bytes, cudaMemcpyHostToDevice,
-                        bank->side[stream_rr++ % msa_bank::kSide]) != cudaSuccess ||
-        cudaMemcpyAsync(bank->stage_v + dst0 * bank->d, hv + src0 * bank->d, bytes, cudaMemcpyHostToDevice,
-                        bank->side[stream_rr++ % msa_bank::kSide]) != cudaSuccess)
-      return MSA_ERR_HOST_TIER;
-    bank->last_fetch_bytes += 2 * (int64_t)bytes;
+    const msa_status rc = issue_rows(bank, src0, dst0, len, stream_rr);
+    if (rc != MSA_OK) return rc;
     rows += len;
     i = r;
   }
@@ -490,9 +566,6 @@ msa_status stage_entries(msa_bank* bank, int k, size_t e0, size_t e1, std::unord
 // not used and is copied into it. `step` maps the slabs already placed in this step.
 msa_status stage_entries_cached(msa_bank* bank, int k, size_t e0, size_t e1,
                                 std::unordered_map<int64_t, int64_t>& step, int& stream_rr) {
-  const size_t row_bytes = (size_t)bank->d * 2;
-  const uint16_t* hk = static_cast<const uint16_t*>(bank->k);
-  const uint16_t* hv = static_cast<const uint16_t*>(bank->v);
   for (size_t e = e0; e < e1; ++e) {
     const int h = (int)((e / k) % bank->hkv);
     const int j = bank->h_idx[e];
@@ -516,14 +589,8 @@ msa_status stage_entries_cached(msa_bank* bank, int k, size_t e0, size_t e1,
       bank->cache_map[key] = slot;
       bank->slot_key[slot] = key;
       const int64_t src = (int64_t)h * bank->kv_rows + bank->doc_rows[j];
-      const int64_t dst = slot * bank->max_len;
-      const size_t bytes = (size_t)bank->doc_lens[j] * row_bytes;
-      if (cudaMemcpyAsync(bank->stage_k + dst * bank->d, hk + src * bank->d, bytes, cudaMemcpyHostToDevice,
-                          bank->side[stream_rr++ % msa_bank::kSide]) != cudaSuccess ||
-          cudaMemcpyAsync(bank->stage_v + dst * bank->d, hv + src * bank->d, bytes, cudaMemcpyHostToDevice,
-                          bank->side[stream_rr++ % msa_bank::kSide]) != cudaSuccess)
-        return MSA_ERR_HOST_TIER;
-      bank->last_fetch_bytes += 2 * (int64_t)bytes;
+      const msa_status rc = issue_rows(bank, src, slot * bank->max_len, bank->doc_lens[j], stream_rr);
+      if (rc != MSA_OK) return rc;
     }
     bank->slot_use[slot] = bank->step_no;
     bank->lru.splice(bank->lru.end(), bank->lru, bank->slot_it[slot]);
@@ -567,7 +634,11 @@ msa_status host_fetch(msa_bank* bank, const StepShape& s, const int32_t* idx_dev
   int64_t rows = 0;
   int rr = 0;
   begin_host_step(bank);
+  bank->jobs.clear();
   rc = bank->cache_on ? stage_entries_cached(bank, s.k, 0, n, slot, rr) : stage_entries(bank, s.k, 0, n, slot, rows, rr);
+  // what was planned is moved even when the plan stops early: the cache already lists it
+  const msa_status rg = flush_jobs(bank, 0);
+  if (rc == MSA_OK) rc = rg;
   if (rc != MSA_OK) return rc;
   MSA_CUDA(cudaMemcpyAsync(bank->d_base, bank->h_base, n * 8, cudaMemcpyHostToDevice, bank->side[0]));
   return join_side(bank, st);
@@ -725,8 +796,11 @@ msa_status forward_host(msa_bank* bank, const msa_query* q, const StepShape& s, 
     MSA_CUDA(cudaStreamWaitEvent(bank->rb, bank->ev_route[m], 0));
     MSA_CUDA(cudaMemcpyAsync(bank->h_idx + e0, topk_idx + e0, (e1 - e0) * 4, cudaMemcpyDeviceToHost, bank->rb));
     MSA_CUDA(cudaStreamSynchronize(bank->rb));
+    bank->jobs.clear();
     rc = bank->cache_on ? stage_entries_cached(bank, s.k, e0, e1, slot, rr)
                         : stage_entries(bank, s.k, e0, e1, slot, rows, rr);
+    const msa_status rg = flush_jobs(bank, e0);
+    if (rc == MSA_OK) rc = rg;
     if (rc != MSA_OK) return rc;
     MSA_CUDA(cudaMemcpyAsync(bank->d_base + e0, bank->h_base + e0, (e1 - e0) * 8, cudaMemcpyHostToDevice,
                              bank->side[0]));
@@ -812,6 +886,13 @@ msa_status msa_bank_create(const msa_bank_config* cfg, msa_bank** out) {
   int dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&b->sms, cudaDevAttrMultiProcessorCount, dev);
+  if (b->kv_loc == MSA_KV_PINNED_HOST) {
+    const size_t kv_bytes = (size_t)b->hkv * b->kv_rows * b->d * 2;
+    b->k_map = mapped_host(b->k, kv_bytes);
+    b->v_map = b->k_map ? mapped_host(b->v, kv_bytes) : nullptr;
+    if (!b->v_map) b->k_map = nullptr;
+    b->gather = MSA_HOST_FETCH_DEFAULT == MSA_FETCH_SM_GATHER && b->k_map;
+  }
 
   // chunk table
   std::vector<int64_t> ctok(b->nch);
@@ -1192,6 +1273,21 @@ msa_status msa_kv_cache_stats(const msa_bank* bank, int64_t* slabs, int64_t* hit
   if (slabs) *slabs = bank->st_slabs;
   if (hits) *hits = bank->st_hits;
   if (bytes_copied) *bytes_copied = bank->last_fetch_bytes;
+  return MSA_OK;
+}
+
+msa_status msa_set_host_fetch(msa_bank* bank, msa_host_fetch mode) {
+  if (!bank || bank->kv_loc != MSA_KV_PINNED_HOST) return MSA_ERR_INVALID_ARG;
+  if (mode != MSA_FETCH_COPY_ENGINE && mode != MSA_FETCH_SM_GATHER) return MSA_ERR_INVALID_ARG;
+  if (mode == MSA_FETCH_SM_GATHER && !bank->k_map) return MSA_ERR_UNSUPPORTED;
+  MSA_CUDA(cudaDeviceSynchronize());
+  bank->gather = mode == MSA_FETCH_SM_GATHER;
+  return MSA_OK;
+}
+
+msa_status msa_get_host_fetch(const msa_bank* bank, msa_host_fetch* mode) {
+  if (!bank || !mode || bank->kv_loc != MSA_KV_PINNED_HOST) return MSA_ERR_INVALID_ARG;
+  *mode = bank->gather ? MSA_FETCH_SM_GATHER : MSA_FETCH_COPY_ENGINE;
   return MSA_OK;
 }
 

@@ -11,7 +11,7 @@ import torch
 
 from . import (MSA_KV_DEVICE, make_query, msa_attend, msa_bank_create, msa_bank_destroy, msa_bank_info,
                msa_build_bank, msa_forward, msa_get_device_error, msa_kv_cache_stats, msa_reserve, msa_route,
-               msa_set_kv_cache, ptr, msa_set_router_precision)
+               msa_set_kv_cache, ptr, msa_set_router_precision, msa_set_host_fetch, msa_get_host_fetch)
 
 
 class _DeviceArray:
@@ -113,6 +113,13 @@ class Bank:
     def set_router_precision(self, precision: int):
         """MSA_KR_F32 (default) or MSA_KR_BF16: the precision of the routing keys the router reads."""
         msa_set_router_precision(self.handle, precision)
+
+    def set_host_fetch(self, mode: int):
+        """MSA_FETCH_SM_GATHER or MSA_FETCH_COPY_ENGINE: how a pinned-host bank moves its slabs."""
+        msa_set_host_fetch(self.handle, mode)
+
+    def host_fetch(self) -> int:
+        return msa_get_host_fetch(self.handle)
 
     def cache_stats(self) -> dict:
         """Distinct slabs, cache hits and PCIe bytes of the last host-tier step."""

@@ -29,7 +29,7 @@ HOST = {
 }
 
 
-def _run(w, host: bool):
+def _run(w, host: bool, fetch=None):
     import sparse_attention_routed_b200 as msa
     from sparse_attention_routed_b200.runner import Bank
     from synth.device import bank_tensors, host_kv_pool, query_tensors
@@ -47,6 +47,8 @@ def _run(w, host: bool):
     Q, Qr, LK, LV = query_tensors(w)
     bank = Bank(K, V, w.doc_lens(), w.rope_base, kv_location=kv_loc, doc_rows=w.doc_kv_rows())
     bank.build(R, rope=False)
+    if fetch is not None:
+        bank.set_host_fetch(fetch)
     qry = bank.query(Q, Qr, LK, LV, w.route_block)
     idx, tsc, scores = bank.route(qry, w.top_k)
     out = bank.attend(qry, w.top_k, idx)
@@ -62,6 +64,8 @@ def _run(w, host: bool):
         st = msa.msa_attend(bank.handle, qry, w.top_k, bad.data_ptr(), out.data_ptr(),
                             torch.cuda.current_stream().cuda_stream, check=False)
         res["bad_status"] = st
+        res["fetch"] = bank.host_fetch()
+        res["stats"] = bank.cache_stats()
     bank.close()
     return res
 
@@ -92,3 +96,38 @@ def test_host_tier_equals_device_bank():
     gd = _run(w, host=False)
     np.testing.assert_array_equal(gh["idx"], gd["idx"])
     np.testing.assert_array_equal(gh["out"], gd["out"])
+
+
+@pytest.mark.parametrize("name", list(HOST))
+def test_host_fetch_transports_agree(name):
+    """The SM gather (the default: torch's pinned memory is mapped) and the copy-engine
+    transfers stage the same bytes: routing and outputs bit for bit equal."""
+    import sparse_attention_routed_b200 as msa
+    w = HOST[name]
+    gd = _run(w, host=True)
+    assert gd["fetch"] == msa.MSA_FETCH_SM_GATHER
+    gc = _run(w, host=True, fetch=msa.MSA_FETCH_COPY_ENGINE)
+    assert gc["fetch"] == msa.MSA_FETCH_COPY_ENGINE
+    for key in ("idx", "out", "idx2", "out2"):
+        np.testing.assert_array_equal(gd[key], gc[key], err_msg=key)
+    assert gd["bad_status"] == gc["bad_status"] == msa.MSA_ERR_INVALID_ARG
+
+
+def test_host_fetch_arguments():
+    import sparse_attention_routed_b200 as msa
+    from sparse_attention_routed_b200.runner import Bank
+    from synth.device import bank_tensors
+    w = HOST["host_decode"]
+    K, V, R = bank_tensors(w)
+    bank = Bank(K, V, w.doc_lens(), w.rope_base, doc_rows=w.doc_kv_rows())
+    assert msa.msa_set_host_fetch(bank.handle, msa.MSA_FETCH_SM_GATHER, check=False) == msa.MSA_ERR_INVALID_ARG
+    bank.close()
+    from synth.device import host_kv_pool
+    Kh, Vh = host_kv_pool(w)
+    hb = Bank(Kh, Vh, w.doc_lens(), w.rope_base, kv_location=msa.MSA_KV_PINNED_HOST, doc_rows=w.doc_kv_rows())
+    assert msa.msa_set_host_fetch(hb.handle, 2, check=False) == msa.MSA_ERR_INVALID_ARG
+    hb.set_host_fetch(msa.MSA_FETCH_COPY_ENGINE)
+    assert hb.host_fetch() == msa.MSA_FETCH_COPY_ENGINE
+    hb.set_host_fetch(msa.MSA_FETCH_SM_GATHER)
+    assert hb.host_fetch() == msa.MSA_FETCH_SM_GATHER
+    hb.close()

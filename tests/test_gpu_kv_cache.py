@@ -67,8 +67,10 @@ def test_resident_slabs_are_not_copied_again():
         b.close()
 
 
-def test_evictions_keep_every_step_correct():
+@pytest.mark.parametrize("fetch", [1, 0], ids=["sm_gather", "copy_engine"])
+def test_evictions_keep_every_step_correct(fetch):
     (plain, cached), keep = _banks(44)  # room for any one step, not for the steps' union
+    cached.set_host_fetch(fetch)         # the uncached bank keeps the default SM gather
     hits = copied = 0
     for step in range(6):
         q0, k0 = _query(plain, step)
