@@ -17,7 +17,13 @@ namespace msa {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
+#ifndef MSA_GATHER_UNROLL
+#define MSA_GATHER_UNROLL 4
+#endif
+#ifndef MSA_GATHER_CTAS_PER_SM
+#define MSA_GATHER_CTAS_PER_SM 1
+#endif
+constexpr int kUnroll = MSA_GATHER_UNROLL;
 constexpr int64_t kPieceBytes = 64 * 1024;
 constexpr int64_t kPieceVec = kPieceBytes / 16;
 
@@ -70,6 +76,7 @@ int64_t host_gather_piece_rows(int head_dim) { return kPieceBytes / ((int64_t)he
 cudaError_t launch_host_gather(const HostGatherJob* jobs, int njobs, int64_t npieces, const void* hk, const void* hv,
                                void* dk, void* dv, int head_dim, int ctas, cudaStream_t s) {
   if (njobs <= 0 || npieces <= 0) return cudaSuccess;
+  ctas *= MSA_GATHER_CTAS_PER_SM;
   const int grid = (int)(npieces < ctas ? npieces : ctas);
   host_gather_kernel<<<grid, kThreads, 0, s>>>(jobs, njobs, npieces, static_cast<const uint4*>(hk),
                                                static_cast<const uint4*>(hv), static_cast<uint4*>(dk),
