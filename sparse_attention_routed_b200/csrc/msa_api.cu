@@ -412,11 +412,12 @@ msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, co
 // Pinned-host tier ("MSA (Memory Sparse Attention)", robocikowo.com, Komponenty:
 // K_r in GPU memory, full K/V in CPU RAM; Pułapki implementacyjne: pinned memory
 // and asynchronous prefetch). A step's selection is read back, every distinct
-// (document, KV head) slab it names is copied from pinned host memory into the
-// device staging pool on the bank's side streams with cudaMemcpyAsync, and the
-// attention kernels read the pool. Slabs that are neighbours in host memory (the
-// same head, one document right after the other) get neighbouring staging rows
-// and travel as one copy. Host-synchronising: not capturable.
+// (document, KV head) slab it names is moved from pinned host memory into the
+// device staging pool on the bank's side streams -- by host_gather_kernel reading
+// the mapped host K/V, or by cudaMemcpyAsync -- and the attention kernels read the
+// pool. Slabs that are neighbours in host memory (the same head, one document
+// right after the other) get neighbouring staging rows and travel as one run.
+// Host-synchronising: not capturable.
 
 // Side streams, events, the attention stream and the pinned selection buffers.
 msa_status ensure_host_tier(msa_bank* bank, size_t entries) {
