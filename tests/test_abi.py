@@ -28,6 +28,18 @@ def test_header_declarations_are_exported():
         assert hasattr(lib, n), n
 
 
+def test_header_enum_values_match_the_binding():
+    """Every enumerator include/msa.h declares has the same value in the Python binding."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    found = {}
+    for body in re.findall(r"typedef\s+enum\s*\{(.*?)\}", text, flags=re.S):
+        for name, val in re.findall(r"(MSA_\w+)\s*=\s*(\d+)", body):
+            found[name] = int(val)
+    assert len(found) >= 13
+    for name, val in found.items():
+        assert getattr(msa, name) == val, name
+
+
 def test_status_strings():
     for s in range(7):
         assert msa.msa_status_string(s) and msa.msa_status_string(s) != "unknown status"
