@@ -282,7 +282,8 @@ msa_status msa_kv_cache_stats(const msa_bank* bank, int64_t* slabs, int64_t* hit
  * whole K and V ranges page-locked and mapped into the device's address space):
  * per planned stretch of slabs, one kernel on a side stream reads the host rows
  * with 16-byte loads through that mapping and writes the staging pool, so a step
- * of many small slabs pays no per-transfer cost. MSA_FETCH_COPY_ENGINE: one
+ * of many small slabs pays no per-transfer cost (the bank keeps a job list of 32
+ * bytes per selection entry, pinned and on the device). MSA_FETCH_COPY_ENGINE: one
  * cudaMemcpyAsync of K and one of V per run of host-contiguous slabs, round-robin
  * over the side streams. Both move the same bytes to the same staging rows, so
  * outputs are identical. Applies to later msa_attend / msa_forward calls;
