@@ -131,3 +131,33 @@ def test_host_fetch_arguments():
     hb.set_host_fetch(msa.MSA_FETCH_SM_GATHER)
     assert hb.host_fetch() == msa.MSA_FETCH_SM_GATHER
     hb.close()
+
+
+def test_unmapped_host_kv_falls_back_to_copy_engines():
+    """Host K/V that is not page-locked (so not mapped for the device): the bank moves
+    its slabs with copy-engine transfers, refuses the SM gather, and attends exactly as
+    over page-locked K/V."""
+    import sparse_attention_routed_b200 as msa
+    from sparse_attention_routed_b200.runner import Bank
+    from synth.device import bank_tensors, host_kv_pool, query_tensors
+    w = HOST["host_decode"]
+    Kp, Vp = host_kv_pool(w)
+    Ku, Vu = Kp.clone(), Vp.clone()          # ordinary (pageable) host memory
+    assert not Ku.is_pinned()
+    _, _, R = bank_tensors(w)
+    Q, Qr, LK, LV = query_tensors(w)
+    outs = []
+    for K, V in ((Kp, Vp), (Ku, Vu)):
+        bank = Bank(K, V, w.doc_lens(), w.rope_base, kv_location=msa.MSA_KV_PINNED_HOST, doc_rows=w.doc_kv_rows())
+        bank.build(R, rope=False)
+        qry = bank.query(Q, Qr, LK, LV, w.route_block)
+        idx, out = bank.forward(qry, w.top_k)
+        torch.cuda.synchronize()
+        assert bank.device_error() == 0
+        outs.append((bank.host_fetch(), idx.cpu().numpy(), out.cpu().numpy()))
+        if K is Ku:
+            assert msa.msa_set_host_fetch(bank.handle, msa.MSA_FETCH_SM_GATHER, check=False) == msa.MSA_ERR_UNSUPPORTED
+        bank.close()
+    assert outs[0][0] == msa.MSA_FETCH_SM_GATHER and outs[1][0] == msa.MSA_FETCH_COPY_ENGINE
+    np.testing.assert_array_equal(outs[0][1], outs[1][1])
+    np.testing.assert_array_equal(outs[0][2], outs[1][2])
