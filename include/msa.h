@@ -40,7 +40,10 @@
  *   - There is no CPU fallback: without a usable sm_100 device the calls that
  *     launch work return MSA_ERR_CUDA or MSA_ERR_UNSUPPORTED.
  *   - A bank belongs to the CUDA device that was current at msa_bank_create;
- *     make that device current for every call on it. A bank is not safe for
+ *     make that device current for every call on it. Every call that launches
+ *     work, waits or allocates returns MSA_ERR_INVALID_ARG, before touching any
+ *     device, when another device is current (msa_bank_destroy switches to the
+ *     bank's device itself and back). A bank is not safe for
  *     concurrent use: calls on one bank must not overlap in time (several banks
  *     may be used from several threads). The bank's workspace is shared by its
  *     calls, which are ordered on their streams; calls on one bank issued to two
@@ -148,7 +151,13 @@ msa_status msa_build_bank(msa_bank* bank, int32_t doc_begin, int32_t doc_end,
                           void* k_slice, int64_t k_head_stride, void* stream);
 
 /* Sizes and device pointers owned by the bank: K_r fp32 [Hkv, n_chunks, d_r],
- * inverse norms fp32 [Hkv, n_chunks]. Any output pointer may be NULL. */
+ * inverse norms fp32 [Hkv, n_chunks] -- the compressed routing keys that stay in
+ * GPU memory while the full K/V may live elsewhere ("MSA (Memory Sparse
+ * Attention)", robocikowo.com, Komponenty: Router K_r in VRAM; "MSA架构…",
+ * §2.1 item 2: one pooled key per 256-token chunk). n_chunks = sum over
+ * documents of ceil(L_j / 256). Any output pointer may be NULL; the device
+ * pointers stay valid until msa_bank_destroy. Host-only: MSA_ERR_INVALID_ARG for
+ * a NULL bank, nothing else. */
 msa_status msa_bank_info(const msa_bank* bank, int64_t* n_tokens, int64_t* n_chunks,
                          int64_t* max_doc_len, const float** k_r, const float** k_r_inv_norm);
 
@@ -167,20 +176,38 @@ typedef struct {
 
 /* Pre-allocates the workspace and Global-RoPE table for steps up to the given
  * sizes, so that later calls allocate nothing (required before capturing
- * calls into a CUDA graph). */
+ * calls into a CUDA graph). The pages describe no such call: it serves the
+ * per-step routing + attention of "MSA (Memory Sparse Attention)",
+ * robocikowo.com, Paradygmat wykonania, run back to back. `shape` carries the
+ * step's sizes; its q / local_k / local_v may be NULL (routing only: the
+ * attention workspace is not reserved). Same argument checks as msa_route /
+ * msa_attend; MSA_ERR_OOM when the device memory cannot be allocated.
+ * Synchronises the device when it has to grow the workspace. */
 msa_status msa_reserve(msa_bank* bank, const msa_query* shape, int32_t top_k);
 
-/* Router: q_r per (sequence, routing block, KV head) = mean of the block's
- * routing queries; score of chunk c = cos(q_r, K_r[h, c]); document score =
- * max over its chunks; selection = top_k documents, ordered by (score desc,
- * index asc).
+/* Router ("MSA架构…", §2.1 item 1: cosine top-k over the pooled routing keys;
+ * robocikowo.com, Komponenty: Router / Routing Projector, and Hiperparametry:
+ * top-k documents): q_r per (sequence, routing block, KV head) = mean of the
+ * block's routing queries; score of chunk c = cos(q_r, K_r[h, c]); document
+ * score = max over its chunks; selection = top_k documents, ordered by (score
+ * desc, index asc). Scores are computed in fp32 with the normalised K_r read
+ * as a bf16 high part plus remainder (msa_set_router_precision). q, local_k and
+ * local_v of `q` are not read and may be NULL; qr must be 16-byte aligned.
+ * MSA_ERR_INVALID_ARG for a NULL bank, q, qr or topk_idx, a shape outside the
+ * supported set, or 1 <= top_k <= n_docs violated; MSA_ERR_UNSUPPORTED for
+ * top_k > 64. Grows the bank's workspace on first use of a larger shape.
  * doc_scores:  [B, nblk, Hkv, n_docs] fp32, or NULL.
  * topk_idx:    [B, nblk, Hkv, top_k] int32 (required).
  * topk_scores: [B, nblk, Hkv, top_k] fp32, or NULL.  (nblk = Tq / Bq) */
 msa_status msa_route(msa_bank* bank, const msa_query* q, int32_t top_k, float* doc_scores,
                      int32_t* topk_idx, float* topk_scores, void* stream);
 
-/* Routed attention: for query head hq at local index i = Lc - Tq + t,
+/* Routed attention ("MSA (Memory Sparse Attention)", robocikowo.com,
+ * Komponenty: Memory Sparse Attention Layer -- the selected documents' K/V are
+ * appended to the local context and one softmax runs over both; Pułapki
+ * implementacyjne: Global RoPE with a k-offset for the active context;
+ * Paradygmat wykonania: only the k selected documents take part):
+ * for query head hq at local index i = Lc - Tq + t,
  * out[b, hq, t] = softmax over { all tokens of the documents in
  * topk_idx[b, t / Bq, hq / G] (bank keys, Parallel RoPE) } and { local keys
  * u <= i with Global RoPE at k_off + u }, query with Global RoPE at k_off + i,
@@ -193,7 +220,8 @@ msa_status msa_attend(msa_bank* bank, const msa_query* q, int32_t top_k,
                       const int32_t* topk_idx, float* out, void* stream);
 
 /* msa_attend that also writes each row's log-sum-exp, the state a training step
- * keeps for msa_attend_backward_saved:
+ * keeps for msa_attend_backward_saved (the layer trains end to end:
+ * robocikowo.com, Komponenty):
  *   lse [B, Hq, Tq] fp32: log sum_j exp(s_j), natural log, over the row's key
  *   set, s_j = q_rot . k_j / sqrt(d) (so out = sum_j exp(s_j - lse) v_j).
  * out is bit for bit what msa_attend writes. Same shapes, errors and device-side
@@ -233,15 +261,23 @@ msa_status msa_attend_backward_saved(msa_bank* bank, const msa_query* q, int32_t
                                      float* dlocal_k, float* dlocal_v, float* dbank_k, float* dbank_v,
                                      void* stream);
 
-/* msa_route followed by msa_attend on one stream; topk_idx receives the selection. */
+/* One routed step as the pages run it per decoding step -- score the bank,
+ * select top-k, fetch and attend ("MSA (Memory Sparse Attention)",
+ * robocikowo.com, Paradygmat wykonania; Równoległość: selection then K/V fetch
+ * in sequence within a step): msa_route followed by msa_attend on one stream;
+ * topk_idx [B, nblk, Hkv, top_k] receives the selection, out [B, Hq, Tq, d]
+ * fp32 the attention. On a pinned-host bank the fetch overlaps the routing of
+ * the next micro-batch of sequences. Errors as msa_route and msa_attend. */
 msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_t* topk_idx,
                        float* out, void* stream);
 
 /* msa_route without any allocation, for callers that must not allocate device
- * memory while they run (inside a CUDA-graph capture, under a fixed memory
- * budget or pool, or where a cudaMalloc's implicit synchronisation is not
- * acceptable). The pages describe no such entry point; it exists for those
- * callers only. Same arguments, outputs and results as msa_route.
+ * memory while they run: a process held to a fixed device-memory budget or
+ * pool it may not grow, or a host that cannot accept the implicit device
+ * synchronisation a cudaMalloc can bring. The pages describe no such entry
+ * point; it exists for those callers only. Same arguments, checks, kernels,
+ * device error flag and results as msa_route (the one routing path of the
+ * library, given this scratch instead of the bank's workspace).
  * Scratch: q_r, 1/|q_r| and (when doc_scores is NULL) the document scores live
  * in one 4 MiB device array that libmsa defines at file scope; every GPU that
  * loads the library holds it until the process exits. A step needing more than

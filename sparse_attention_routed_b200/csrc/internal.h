@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/msa.h"
+
 namespace msa {
 
 // Chunk-mean pooling of routing keys and in-place Parallel RoPE of bank keys
@@ -121,15 +123,6 @@ int attend_prefill_tc_tile_rows();
 cudaError_t launch_attend_prefill_tc(const AttendArgs& a, const AttendMaps& m, const CUtensorMap& q_map,
                                      cudaStream_t s);
 
-// Device pointers and sizes of a bank that the routing kernels read.
-struct BankRouteView {
-  RouteMaps maps;
-  const int32_t* chunk_off;
-  int64_t nch;
-  int32_t n_docs, n_kv_heads, route_dim, sms;
-  int32_t kr_bf16;
-};
-
 // Host-side helpers.
 int attend_tile_rows();               // keys per TMA tile of the decode attention kernel
 int attend_max_splits();              // upper bound on n_splits
@@ -211,6 +204,12 @@ cudaError_t launch_host_gather(const HostGatherJob* jobs, int njobs, int64_t npi
 
 }  // namespace msa
 
-struct msa_bank;
-// Fills `v` from a bank handle (no allocation, no CUDA call).
-void msa_bank_route_view(const msa_bank* bank, msa::BankRouteView* v);
+// msa_route with its scratch supplied by the caller instead of the bank's workspace:
+// `scratch` (256-byte aligned, `scratch_bytes` long) receives q_r [rows][Hkv][d_r],
+// 1/|q_r| [rows][Hkv] and, when doc_scores is NULL, the document scores
+// [rows][Hkv][n_docs], each part rounded up to 256 bytes (rows = B * Tq / Bq).
+// The same checks, router choice and kernels as msa_route; MSA_ERR_UNSUPPORTED
+// before any launch when the parts do not fit.
+msa_status msa_route_with_scratch(msa_bank* bank, const msa_query* q, int32_t top_k, float* doc_scores,
+                                  int32_t* topk_idx, float* topk_scores, void* scratch, size_t scratch_bytes,
+                                  cudaStream_t st);

@@ -136,6 +136,7 @@ struct msa_bank {
   std::vector<int64_t> doc_lens, doc_off, doc_rows;
   std::vector<int32_t> chunk_off;
   int sms = 148;
+  int device = 0;  // the CUDA device current at msa_bank_create; every launch happens there
   // device, owned
   int64_t* d_doc_row = nullptr;
   int32_t* d_doc_len = nullptr;
@@ -242,8 +243,17 @@ struct StepShape {
   int B, Hq, Tq, Lc, Bq, G, nblk, rows, P, k;
 };
 
+// A bank's kernels, tensor maps and workspace belong to the device that was current
+// when it was created: a call made with another device current is refused before
+// anything is launched or allocated.
+bool on_bank_device(const msa_bank* bank) {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess && dev == bank->device;
+}
+
 msa_status check_query(const msa_bank* bank, const msa_query* q, int top_k, StepShape* s, bool need_attn) {
   if (!bank || !q) return MSA_ERR_INVALID_ARG;
+  if (!on_bank_device(bank)) return MSA_ERR_INVALID_ARG;
   if (q->batch < 1 || q->n_q_heads < 1 || q->q_tokens < 1 || q->local_len < 1 || q->route_block < 1)
     return MSA_ERR_INVALID_ARG;
   if (q->n_q_heads % bank->hkv) return MSA_ERR_INVALID_ARG;
@@ -375,13 +385,15 @@ msa_status ensure_gtab(msa_bank* bank, int64_t koff, int lc, cudaStream_t s) {
   return MSA_OK;
 }
 
-msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, const Workspace& w,
-                      float* doc_scores, int32_t* idx, float* top_scores, cudaStream_t st) {
+// The routing step. q_r / q_r_inv ([rows][Hkv][d_r], [rows][Hkv]) and score_scratch
+// ([rows][Hkv][n_docs], used when doc_scores is NULL) are the caller's scratch.
+msa_status route_into(msa_bank* bank, const msa_query* q, const StepShape& s, float* q_r, float* q_r_inv,
+                      float* score_scratch, float* doc_scores, int32_t* idx, float* top_scores, cudaStream_t st) {
   RouteArgs ra{};
   const bool tc = route_tc_supported(bank->dr, s.B * s.nblk);
   const bool fuse = !tc && s.Bq <= kRouteFuseMaxBlock;  // the router forms q_r itself
   if (!fuse) {
-    QrArgs qa{(const uint16_t*)q->qr, w.q_r, w.q_r_inv, s.B, bank->hkv, s.Tq, s.Bq, bank->dr};
+    QrArgs qa{(const uint16_t*)q->qr, q_r, q_r_inv, s.B, bank->hkv, s.Tq, s.Bq, bank->dr};
     MSA_CUDA(launch_qr_prep(qa, st));
   } else {
     ra.qr = (const uint16_t*)q->qr;
@@ -389,9 +401,9 @@ msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, co
     ra.route_block = s.Bq;
   }
   ra.chunk_off = bank->d_chunk_off;
-  ra.q_r = w.q_r;
-  ra.q_r_inv = w.q_r_inv;
-  ra.doc_scores = doc_scores ? doc_scores : w.scores;
+  ra.q_r = q_r;
+  ra.q_r_inv = q_r_inv;
+  ra.doc_scores = doc_scores ? doc_scores : score_scratch;
   ra.nch = bank->nch;
   ra.rows = s.B * s.nblk;
   ra.n_kv_heads = bank->hkv;
@@ -407,6 +419,11 @@ msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, co
   TopkArgs ta{ra.doc_scores, idx, top_scores, s.P, bank->n_docs, s.k};
   MSA_CUDA(launch_topk(ta, st));
   return MSA_OK;
+}
+
+msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, const Workspace& w,
+                      float* doc_scores, int32_t* idx, float* top_scores, cudaStream_t st) {
+  return route_into(bank, q, s, w.q_r, w.q_r_inv, w.scores, doc_scores, idx, top_scores, st);
 }
 
 // Pinned-host tier ("MSA (Memory Sparse Attention)", robocikowo.com, Komponenty:
@@ -718,15 +735,28 @@ msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, i
 
 }  // namespace
 
-void msa_bank_route_view(const msa_bank* bank, msa::BankRouteView* v) {
-  v->maps = bank->route_maps;
-  v->chunk_off = bank->d_chunk_off;
-  v->nch = bank->nch;
-  v->n_docs = bank->n_docs;
-  v->n_kv_heads = bank->hkv;
-  v->route_dim = bank->dr;
-  v->sms = bank->sms;
-  v->kr_bf16 = bank->kr_bf16 ? 1 : 0;
+static size_t route_scratch_bytes(const msa_bank* bank, const StepShape& s, bool with_scores) {
+  const size_t rows = (size_t)s.B * s.nblk;
+  return align_up(rows * bank->hkv * bank->dr * sizeof(float)) + align_up(rows * bank->hkv * sizeof(float)) +
+         (with_scores ? align_up(rows * bank->hkv * (size_t)bank->n_docs * sizeof(float)) : 0);
+}
+
+msa_status msa_route_with_scratch(msa_bank* bank, const msa_query* q, int32_t top_k, float* doc_scores,
+                                  int32_t* topk_idx, float* topk_scores, void* scratch, size_t scratch_bytes,
+                                  cudaStream_t st) {
+  StepShape s;
+  msa_status rc = check_query(bank, q, top_k, &s, false);
+  if (rc != MSA_OK) return rc;
+  if (!topk_idx) return MSA_ERR_INVALID_ARG;
+  if (route_scratch_bytes(bank, s, !doc_scores) > scratch_bytes) return MSA_ERR_UNSUPPORTED;
+  if (!scratch || (reinterpret_cast<uintptr_t>(scratch) & 255u)) return MSA_ERR_INVALID_ARG;
+  const size_t rows = (size_t)s.B * s.nblk;
+  uint8_t* p = static_cast<uint8_t*>(scratch);
+  float* q_r = reinterpret_cast<float*>(p);
+  float* q_inv = reinterpret_cast<float*>(p + align_up(rows * bank->hkv * bank->dr * sizeof(float)));
+  float* scores = reinterpret_cast<float*>(p + align_up(rows * bank->hkv * bank->dr * sizeof(float)) +
+                                           align_up(rows * bank->hkv * sizeof(float)));
+  return route_into(bank, q, s, q_r, q_inv, scores, doc_scores, topk_idx, topk_scores, st);
 }
 
 // msa_forward on a pinned-host bank: the batch runs as up to kMicro
@@ -885,7 +915,11 @@ msa_status msa_bank_create(const msa_bank_config* cfg, msa_bank** out) {
     return MSA_ERR_UNSUPPORTED;
   }
   int dev = 0;
-  cudaGetDevice(&dev);
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    delete b;
+    return MSA_ERR_CUDA;
+  }
+  b->device = dev;
   cudaDeviceGetAttribute(&b->sms, cudaDevAttrMultiProcessorCount, dev);
   if (b->kv_loc == MSA_KV_PINNED_HOST) {
     const size_t kv_bytes = (size_t)b->hkv * b->kv_rows * b->d * 2;
@@ -954,7 +988,13 @@ msa_status msa_bank_create(const msa_bank_config* cfg, msa_bank** out) {
 }
 
 msa_status msa_bank_destroy(msa_bank* bank) {
+  if (!bank) return MSA_OK;
+  // free on the bank's own device, whichever device the caller has current
+  int cur = -1;
+  const bool other = cudaGetDevice(&cur) == cudaSuccess && cur != bank->device;
+  if (other) cudaSetDevice(bank->device);
   free_bank(bank);
+  if (other) cudaSetDevice(cur);
   return MSA_OK;
 }
 
@@ -962,6 +1002,7 @@ msa_status msa_bank_destroy(msa_bank* bank) {
 msa_status msa_build_bank(msa_bank* bank, int32_t doc_begin, int32_t doc_end, const void* r_slice,
                           int64_t r_head_stride, void* k_slice, int64_t k_head_stride, void* stream) {
   if (!bank || (!r_slice && !k_slice)) return MSA_ERR_INVALID_ARG;
+  if (!on_bank_device(bank)) return MSA_ERR_INVALID_ARG;
   if (doc_begin < 0 || doc_end > bank->n_docs || doc_begin >= doc_end) return MSA_ERR_INVALID_ARG;
   const int64_t T = bank->doc_off[doc_end] - bank->doc_off[doc_begin];
   if (r_slice && (r_head_stride < T || !aligned16(r_slice))) return MSA_ERR_INVALID_ARG;
@@ -1234,6 +1275,7 @@ msa_status msa_attend_backward_saved(msa_bank* bank, const msa_query* q, int32_t
 
 msa_status msa_set_kv_cache(msa_bank* bank, int64_t bytes) {
   if (!bank || bank->kv_loc != MSA_KV_PINNED_HOST || bytes < 0) return MSA_ERR_INVALID_ARG;
+  if (!on_bank_device(bank)) return MSA_ERR_INVALID_ARG;
   MSA_CUDA(cudaDeviceSynchronize());
   if (bank->stage_k) cudaFree(bank->stage_k);
   if (bank->stage_v) cudaFree(bank->stage_v);
@@ -1281,6 +1323,7 @@ msa_status msa_set_host_fetch(msa_bank* bank, msa_host_fetch mode) {
   if (!bank || bank->kv_loc != MSA_KV_PINNED_HOST) return MSA_ERR_INVALID_ARG;
   if (mode != MSA_FETCH_COPY_ENGINE && mode != MSA_FETCH_SM_GATHER) return MSA_ERR_INVALID_ARG;
   if (mode == MSA_FETCH_SM_GATHER && !bank->k_map) return MSA_ERR_UNSUPPORTED;
+  if (!on_bank_device(bank)) return MSA_ERR_INVALID_ARG;
   MSA_CUDA(cudaDeviceSynchronize());
   bank->gather = mode == MSA_FETCH_SM_GATHER;
   return MSA_OK;
@@ -1299,13 +1342,13 @@ msa_status msa_set_router_precision(msa_bank* bank, msa_kr_precision precision) 
 }
 
 msa_status msa_check_wait_timeout(msa_bank* bank, void* stream) {
-  if (!bank) return MSA_ERR_INVALID_ARG;
+  if (!bank || !on_bank_device(bank)) return MSA_ERR_INVALID_ARG;
   MSA_CUDA(launch_wait_timeout(bank->d_err, (cudaStream_t)stream));
   return MSA_OK;
 }
 
 msa_status msa_get_device_error(msa_bank* bank, void* stream) {
-  if (!bank) return MSA_ERR_INVALID_ARG;
+  if (!bank || !on_bank_device(bank)) return MSA_ERR_INVALID_ARG;
   MSA_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
   int v = 0;
   MSA_CUDA(cudaMemcpy(&v, bank->d_err, sizeof(int), cudaMemcpyDeviceToHost));

@@ -42,4 +42,14 @@ def test_bounded_wait_expires_and_context_stays_usable():
     inp = P.oracle_inputs(w)
     ref = O.forward(inp, w.doc_lens(), w.top_k, w.route_block, w.rope_base, selection=idx.cpu().numpy())
     P.check_out(out.cpu().numpy(), ref["out"])
+
+    # the allocation-free router raises and clears the same flag: after another
+    # expired wait it reads MSA_ERR_TIMEOUT once, then routes exactly as msa_route
+    from sparse_attention_routed_b200 import msa_route_noalloc
+    msa_check_wait_timeout(bank.handle, torch.cuda.current_stream().cuda_stream)
+    assert bank.device_error() == MSA_ERR_TIMEOUT
+    idx2 = torch.full_like(idx, -1)
+    msa_route_noalloc(bank.handle, qry, w.top_k, 0, idx2.data_ptr(), 0, torch.cuda.current_stream().cuda_stream)
+    assert bank.device_error() == MSA_OK
+    assert torch.equal(idx2, idx)
     bank.close()

@@ -1,11 +1,13 @@
 """msa_route_noalloc: the routing step for callers that must not allocate device
-memory while they run (inside a CUDA-graph capture, under a fixed memory budget
-or pool, or where a cudaMalloc's implicit device synchronisation is not
-acceptable). Its scratch is the library's fixed 4 MiB device array.
+memory while they run (a process held to a fixed device-memory budget or pool,
+or a host that cannot accept the implicit device synchronisation a cudaMalloc
+can bring). Its scratch is the library's fixed 4 MiB device array.
 
 Checked through the C ABI against msa_route (the allocating entry point) on two
 calls in a row, so that a second call that reuses the shared array without
-clearing it would show; and the size limit is enforced before any launch.
+clearing it would show -- on a decode shape (the router that forms q_r itself)
+and on a shape with more than 16 routing rows (q_r formed first, then the
+tcgen05 router); the size limit is enforced before any launch.
 """
 import numpy as np
 import pytest
@@ -28,9 +30,14 @@ def _bank_and_query(w):
     return bank, bank.query(Q, Qr, LK, LV, w.route_block), keep
 
 
-def test_route_noalloc_matches_route_on_two_calls():
+@pytest.mark.parametrize("w", [
+    # 6 routing rows of 2-token blocks: q_r formed inside the mma.sync router
+    Workload("noalloc_check", 21, 3, 16, 4, 128, 70, 0, 64, 4, 2, 7, ragged=(1, 900)),
+    # 3 sequences x 8 one-token routing blocks = 24 routing rows (> 16): q_r kernel, then the tcgen05 router
+    Workload("noalloc_tc", 25, 3, 8, 2, 128, 40, 0, 96, 8, 1, 5, ragged=(1, 900)),
+], ids=lambda w: w.name)
+def test_route_noalloc_matches_route_on_two_calls(w):
     import sparse_attention_routed_b200 as msa
-    w = Workload("noalloc_check", 21, 3, 16, 4, 128, 70, 0, 64, 4, 2, 7, ragged=(1, 900))
     bank, qry, keep = _bank_and_query(w)
     stream = torch.cuda.current_stream().cuda_stream
     idx_ref, tsc_ref, sc_ref = bank.route(qry, w.top_k)
