@@ -42,7 +42,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="time only --workload (the default run also times prefill and the two host-tier banks)")
+    ap.add_argument("--cpu-steps", type=int, default=3,
+                    help="whole oracle steps timed for the cpu_baseline (after one untimed step)")
     ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "decode_512k", "prefill", "prefill_64docs", "prefill_short_docs", "ragged_planted", "bank_100m"],
                     help="decode_512k: the same step on a 128-document bank (profiling captures); "
                          "prefill: 4096 query tokens in 64-token routing blocks (tensor-bound)")
@@ -106,66 +109,173 @@ def launches_per_step(w, batch=None, gather=False) -> int:
 
 
 # ----------------------------------------------------------------- CPU oracle
-def oracle_sample(seconds: float):
-    """Times the oracle as it stands on a bounded sample of the decode workload.
+# The oracle as it stands, run on whole decode steps of the bench workload. One
+# step = every sequence of the batch: for each (sequence, KV head) the oracle's
+# router over every chunk of K_r, its top-k, and its attention for the G query
+# heads of that KV head. The (sequence, KV head) items are spread over worker
+# processes (spawned; each single-threaded: BLAS threads pinned to 1), so the
+# thread count is the worker count. K_r is pooled by the oracle from the
+# workload's routing keys, and the selected documents' keys carry the oracle's
+# Parallel RoPE: both are offline bank state, built before the first step.
 
-    Sample: whole decode queries (one sequence each): the oracle's router over
-    every chunk of the 4.19M-token bank for all 8 KV heads (per-chunk cosine
-    loop, per-document max, top-k by full sort), then the oracle's attention for
-    all 32 query heads over the 16 selected documents plus the 4096 local tokens.
-    K_r is offline state (built once per bank), so a stand-in K_r of the right
-    shape is drawn from the generator (the oracle's cost does not depend on
-    its values); the selected documents' K/V and the local K/V are regenerated
-    exactly. Queries run until `seconds` of oracle time are spent (>= 1 query).
-    """
+_ONE_THREAD = {v: "1" for v in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS",
+                                "NUMEXPR_NUM_THREADS", "VECLIB_MAXIMUM_THREADS")}
+# the workers allocate and free many multi-MB numpy temporaries: keep glibc from
+# returning each one to the kernel (mmap / munmap page-fault churn)
+_ONE_THREAD.update({"MALLOC_MMAP_THRESHOLD_": "33554432", "MALLOC_TRIM_THRESHOLD_": "2147483647"})
+
+
+def _oracle_worker(conn, wname, items):
+    """Serves oracle steps for a fixed list of (sequence, KV head) items."""
     import synth
     from oracle import msa_oracle as O
 
-    w = synth.WORKLOADS[WORKLOAD]
-    n, L, d, Hkv, G = w.n_docs, w.doc_len, w.head_dim, w.n_kv_heads, w.n_q_heads // w.n_kv_heads
-    nch_doc = L // 256
-    chunk_doc = np.repeat(np.arange(n), nch_doc)
-    kr = synth.normal_f32(99, 1, 0, Hkv * n * nch_doc * d).reshape(Hkv, n * nch_doc, d).astype(np.float64)
     f64 = lambda bits: synth.bf16_bits_to_f32(bits).astype(np.float64)
-    Qr = f64(synth.query_bits(w, synth.T_QR, (w.batch, Hkv, 1, d)))
-    Q = f64(synth.query_bits(w, synth.T_Q, (w.batch, w.n_q_heads, 1, d)))
-    k_off = O.k_offset(w.top_k, w.doc_lens())
-    b = 0  # the same query is repeated: the oracle's work per query does not depend on its values
+    w = synth.WORKLOADS[wname]
+    n, d, Hkv, Hq = w.n_docs, w.head_dim, w.n_kv_heads, w.n_q_heads
+    G, lens = Hq // Hkv, w.doc_lens()
+    off = np.concatenate([[0], np.cumsum(lens)])
+    t_setup = time.perf_counter()
+    kr, chunk_doc = {}, None
+    for h in sorted({h for _, h in items}):   # offline bank build: pooling of the routing keys
+        rows, owner = [], []
+        for j in range(n):
+            rows.append(O.chunk_mean_pool(f64(synth.bank_rows_bits(w, synth.T_R, h, int(off[j]), int(lens[j])))))
+            owner.extend([j] * rows[-1].shape[0])
+        kr[h], chunk_doc = np.concatenate(rows), np.asarray(owner, dtype=np.int64)
+    Qr = f64(synth.query_bits(w, synth.T_QR, (w.batch, Hkv, w.q_tokens, d)))
+    Q = f64(synth.query_bits(w, synth.T_Q, (w.batch, Hq, w.q_tokens, d)))
+    k_off = O.k_offset(w.top_k, lens)
+    conn.send(("ready", time.perf_counter() - t_setup))
     cache = {}
-    spent, queries = 0.0, 0
-    while queries == 0 or spent < seconds:
+    while True:
+        cmd = conn.recv()
+        if cmd is None:
+            break
+        misses, excluded = 0, 0.0
         t0 = time.perf_counter()
-        sel = []
-        for h in range(Hkv):
-            s = O.route_doc_scores(Qr[b, h, 0], kr[h], chunk_doc, n)
-            sel.append(O.select_top_k(s, w.top_k))
-        spent += time.perf_counter() - t0
-        for h in range(Hkv):
-            docs = sel[h]
-            if h not in cache:  # input regeneration, not timed
-                mk = np.concatenate([f64(synth.bank_rows_bits(w, synth.T_K, h, int(j) * L, L)) for j in docs])
-                mv = np.concatenate([f64(synth.bank_rows_bits(w, synth.T_V, h, int(j) * L, L)) for j in docs])
-                base = (b * Hkv + h) * w.local_len * d
-                lk = f64(synth.normal_bf16_bits(w.seed, synth.T_LK, base, w.local_len * d)).reshape(-1, d)
-                lv = f64(synth.normal_bf16_bits(w.seed, synth.T_LV, base, w.local_len * d)).reshape(-1, d)
-                cache[h] = (mk, mv, lk, lv)
-            mk, mv, lk, lv = cache[h]
-            t0 = time.perf_counter()
-            mk_rot = O.parallel_rope_bank(mk, [L] * len(docs), w.rope_base)
-            for g in range(G):
-                O.routed_attention_row(Q[b, h * G + g, 0], w.local_len - 1, k_off, w.rope_base,
-                                       mk_rot, mv, lk, lv)
-            spent += time.perf_counter() - t0
-        queries += 1
-    threads = int(os.environ.get("OMP_NUM_THREADS", "0")) or os.cpu_count()
-    return queries / spent, queries, spent, threads
+        for b, h in items:
+            for blk in range(w.q_tokens // w.route_block):
+                qb = O.block_mean_query(Qr[b, h], w.route_block)[blk]
+                sel = O.select_top_k(O.route_doc_scores(qb, kr[h], chunk_doc, n), w.top_k)
+                key = (b, h, tuple(int(j) for j in sel))
+                if key not in cache:
+                    # bank keys with Parallel RoPE and the values of the selected documents
+                    # (offline bank state), the local K/V: inputs, outside the step's time
+                    t_in = time.perf_counter()
+                    mk = np.concatenate([O.parallel_rope_bank(f64(synth.bank_rows_bits(w, synth.T_K, h, int(off[j]),
+                                                                                        int(lens[j]))),
+                                                              [int(lens[j])], w.rope_base) for j in sel])
+                    mv = np.concatenate([f64(synth.bank_rows_bits(w, synth.T_V, h, int(off[j]), int(lens[j])))
+                                         for j in sel])
+                    base = (b * Hkv + h) * w.local_len * d
+                    lk = f64(synth.normal_bf16_bits(w.seed, synth.T_LK, base, w.local_len * d)).reshape(-1, d)
+                    lv = f64(synth.normal_bf16_bits(w.seed, synth.T_LV, base, w.local_len * d)).reshape(-1, d)
+                    cache[key] = (mk, mv, lk, lv)
+                    misses += 1
+                    excluded += time.perf_counter() - t_in
+                mk, mv, lk, lv = cache[key]
+                for g in range(G):
+                    for t in range(blk * w.route_block, (blk + 1) * w.route_block):
+                        O.routed_attention_row(Q[b, h * G + g, t], w.local_len - w.q_tokens + t, k_off,
+                                               w.rope_base, mk, mv, lk, lv)
+        conn.send((time.perf_counter() - t0 - excluded, misses))
 
 
-def base_config(w) -> dict:
-    """The workload description both arms print."""
+class OracleSteps:
+    """Worker processes that run whole oracle steps of a workload on the host cores."""
+
+    def __init__(self, wname: str):
+        import multiprocessing as mp
+        import synth
+        w = synth.WORKLOADS[wname]
+        self.units = w.batch * w.q_tokens          # queries (decode) per step
+        items = [(b, h) for h in range(w.n_kv_heads) for b in range(w.batch)]
+        try:
+            avail = len(os.sched_getaffinity(0))
+        except AttributeError:
+            avail = os.cpu_count() or 1
+        self.workers = max(1, min(avail, len(items)))
+        ctx = mp.get_context("spawn")   # the parent may hold a CUDA context: never fork it
+        saved = {k: os.environ.get(k) for k in _ONE_THREAD}
+        os.environ.update(_ONE_THREAD)
+        self.procs, self.conns = [], []
+        try:
+            for i in range(self.workers):
+                a, b = ctx.Pipe()
+                # contiguous blocks of the head-major item list: a worker pools as few heads as possible
+                mine = items[i * len(items) // self.workers:(i + 1) * len(items) // self.workers]
+                p = ctx.Process(target=_oracle_worker, args=(b, wname, mine), daemon=True)
+                p.start()
+                self.procs.append(p)
+                self.conns.append(a)
+        finally:
+            for k, v in saved.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+        self.setup_s = max(c.recv()[1] for c in self.conns)
+
+    def step(self):
+        """One whole step; returns (wall seconds, cache misses)."""
+        t0 = time.perf_counter()
+        for c in self.conns:
+            c.send(1)
+        replies = [c.recv() for c in self.conns]
+        return time.perf_counter() - t0, sum(m for _, m in replies)
+
+    def close(self):
+        for c in self.conns:
+            c.send(None)
+        for p in self.procs:
+            p.join(timeout=30)
+
+
+def oracle_timed(wname: str, steps: int, warmup: int):
+    """Runs `warmup` untimed and `steps` timed whole oracle steps; returns a dict."""
+    runner = OracleSteps(wname)
+    try:
+        for _ in range(warmup):
+            runner.step()
+        walls, misses = [], 0
+        for _ in range(steps):
+            wall, m = runner.step()
+            walls.append(wall)
+            misses += m
+    finally:
+        runner.close()
+    mean = sum(walls) / len(walls)
+    return {"value": runner.units / mean, "ms_per_step": 1000.0 * mean, "steps": steps, "warmup": warmup,
+            "cores": runner.workers, "setup_s": runner.setup_s, "timed_misses": misses,
+            "total_s": sum(walls)}
+
+
+def oracle_sample_text(r: dict, w) -> str:
+    nch = int(sum(-(-int(L) // 256) for L in w.doc_lens()))
+    return (f"{r['steps']} whole decode steps of {w.batch} queries after {r['warmup']} untimed "
+            f"({r['total_s']:.1f} s timed): per (sequence, KV head) the oracle's router over all {nch} "
+            f"chunks of K_r (pooled by the oracle from the routing keys), its top-{w.top_k}, and its "
+            f"attention for the {w.n_q_heads // w.n_kv_heads} query heads; {r['cores']} single-threaded "
+            f"worker processes; bank build (pooling, Parallel RoPE) not timed")
+
+
+def step_bytes_estimate(w) -> float:
+    """HBM bytes a step reads at most (no shared documents): K_r once, the selected
+    documents' K/V per (sequence, routing block, KV head), the local K/V."""
+    nblk = w.q_tokens // w.route_block
+    nch = int(sum(-(-int(L) // 256) for L in w.doc_lens()))
+    return (w.n_kv_heads * nch * w.route_dim * 4 + w.batch * nblk * w.n_kv_heads * w.top_k * w.max_len * w.head_dim * 4
+            + w.batch * w.n_kv_heads * w.local_len * w.head_dim * 4)
+
+
+def base_config(w, world: int = 1) -> dict:
+    """The workload description both arms print (identical for the same workload and N)."""
     return {"workload": w.name, "batch": w.batch, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
             "head_dim": w.head_dim, "bank_docs": w.n_docs, "doc_len": w.doc_len, "local_len": w.local_len,
-            "q_tokens": w.q_tokens, "route_block": w.route_block, "top_k": w.top_k}
+            "q_tokens": w.q_tokens, "route_block": w.route_block, "top_k": w.top_k,
+            "parallelism": f"replicas x{world}",
+            "l2": f"inputs larger than L2: up to {step_bytes_estimate(w) / 1e9:.2f} GB read per step vs 126 MB L2"}
 
 
 def run_reference(args):
@@ -173,18 +283,19 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    qps, nq, spent, cores = oracle_sample(max(2.0, min(args.cpu_seconds, 5.0 * max(1, args.steps) / 100)))
+    w = synth.WORKLOADS[WORKLOAD]
+    r = oracle_timed(WORKLOAD, max(1, args.steps), max(0, args.warmup))
     line = {
-        "impl": "reference", "metric": METRIC, "value": qps, "unit": "queries/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * 8 / qps,
+        "impl": "reference", "metric": METRIC, "value": r["value"], "unit": "queries/s", "n_gpus": args.gpus,
+        "steps": r["steps"], "warmup": r["warmup"], "ms_per_step": r["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": dict(base_config(synth.WORKLOADS[WORKLOAD]), parallelism="oracle on host cores",
-                       l2="n/a (host cores)"),
-        "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{nq} decode queries (router over all 16384 chunks x 8 KV heads, "
-                                   f"top-16, attention for 32 heads), {spent:.1f} s of oracle time"},
-        "e2e": {"value": qps, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "config": base_config(w, args.gpus),
+        "cpu_baseline": {"value": r["value"], "unit": "queries/s", "cores": r["cores"], "kind": "oracle",
+                         "sample": oracle_sample_text(r, w)},
+        "e2e": {"value": r["value"], "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "reference_note": "the pages ship no code: the reference arm is the fp64 CPU oracle, timed as it stands",
+        "setup_s": r["setup_s"],
     }
     print(json.dumps(line), flush=True)
 
@@ -287,7 +398,10 @@ def job_throughput(world: int, units_per_step: float, steps: int, total_ms: floa
     return world * units_per_step * steps / (total_ms / 1000.0)
 
 
-def run_ours(args):
+def measure_device(args, wname: str, n: int, warmup: int, world: int, rank: int, local: int,
+                   with_e2e: bool = True):
+    """Times n steps (route + attend through the C ABI) of a device-resident workload
+    after `warmup` untimed ones; returns the JSON line on rank 0 (None elsewhere)."""
     import torch
     import torch.distributed as dist
 
@@ -296,16 +410,8 @@ def run_ours(args):
     from sparse_attention_routed_b200.runner import Bank
     from synth.device import bank_tensors, query_tensors
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-
-    w = synth.WORKLOADS[args.workload]
-    prefill = args.workload.startswith("prefill")
+    w = synth.WORKLOADS[wname]
+    prefill = wname.startswith("prefill")
     K, V, R = bank_tensors(w)
     bank = Bank(K, V, w.doc_lens(), w.rope_base)
     bank.build(R)
@@ -338,7 +444,7 @@ def run_ours(args):
         msa_route(bank.handle, qry, k, 0, idx.data_ptr(), 0, sh)
         msa_attend(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
 
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, warmup)):
         step()
     torch.cuda.synchronize()
     assert bank.device_error() == 0
@@ -366,7 +472,6 @@ def run_ours(args):
     torch.cuda.synchronize()
     clocks = ClockSampler(local)
     time.sleep(0.4)
-    n = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
     t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks.mark(True)
@@ -388,74 +493,76 @@ def run_ours(args):
     attend_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / n
     assert bank.device_error() == 0
 
-    # e2e: pinned host inputs of each step copied in -- decode: queries, routing
-    # queries and the newest local token's K/V; prefill: queries, routing queries
-    # and the whole local K/V (the prompt) -- the step run, output + selection copied out.
-    # Two buffer sets and two copy streams, as a server runs it: step i computes
-    # while step i+1's inputs come in and step i-1's result goes out; every step
-    # still moves its own bytes inside the timed region.
-    qin_h = qin.cpu().pin_memory()
-    kv_h = (kvloc if prefill else kvloc[:, :, :, -1]).cpu().pin_memory()  # decode: the newest token's K, V
-    sets = [(qin, kvloc, outbuf, qry, out, idx)]
-    qin1, kvloc1, outbuf1 = qin.clone(), kvloc.clone(), torch.empty_like(outbuf)
-    Q1, Qr1 = qin1[:Q.numel()].view(Q.shape), qin1[Q.numel():].view(Qr.shape)
-    qry1 = bank.query(Q1, Qr1, kvloc1[0], kvloc1[1], w.route_block)
-    sets.append((qin1, kvloc1, outbuf1, qry1, outbuf1[:4 * n_out].view(torch.float32).view(out.shape),
-                 outbuf1[4 * n_out:].view(torch.int32).view(idx.shape)))
-    out_h = [torch.empty(outbuf.shape, dtype=outbuf.dtype, pin_memory=True) for _ in range(2)]
-    h2d = qin_h.numel() * 2 + kv_h.numel() * 2
-    d2h = out_h[0].numel()
-    n_e2e = max(10, n // 2)
-    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_comp = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms, n_e2e, h2d, d2h = None, 0, 0, 0
+    if with_e2e:
+        # e2e: pinned host inputs of each step copied in -- decode: queries, routing
+        # queries and the newest local token's K/V; prefill: queries, routing queries
+        # and the whole local K/V (the prompt) -- the step run, output + selection copied out.
+        # Two buffer sets and two copy streams, as a server runs it: step i computes
+        # while step i+1's inputs come in and step i-1's result goes out; every step
+        # still moves its own bytes inside the timed region.
+        qin_h = qin.cpu().pin_memory()
+        kv_h = (kvloc if prefill else kvloc[:, :, :, -1]).cpu().pin_memory()  # decode: the newest token's K, V
+        sets = [(qin, kvloc, outbuf, qry, out, idx)]
+        qin1, kvloc1, outbuf1 = qin.clone(), kvloc.clone(), torch.empty_like(outbuf)
+        Q1, Qr1 = qin1[:Q.numel()].view(Q.shape), qin1[Q.numel():].view(Qr.shape)
+        qry1 = bank.query(Q1, Qr1, kvloc1[0], kvloc1[1], w.route_block)
+        sets.append((qin1, kvloc1, outbuf1, qry1, outbuf1[:4 * n_out].view(torch.float32).view(out.shape),
+                     outbuf1[4 * n_out:].view(torch.int32).view(idx.shape)))
+        out_h = [torch.empty(outbuf.shape, dtype=outbuf.dtype, pin_memory=True) for _ in range(2)]
+        h2d = qin_h.numel() * 2 + kv_h.numel() * 2
+        d2h = out_h[0].numel()
+        n_e2e = max(10, n // 2)
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-    def e2e_run(steps, timed):
-        if timed:
-            e0.record(stream)
-        s_in.wait_stream(stream)
-        s_out.wait_stream(stream)
-        for i in range(steps):
-            si = i % 2
-            q_d, kv_d, ob_d, qy, o_d, ix_d = sets[si]
-            with torch.cuda.stream(s_in):
+        def e2e_run(steps, timed):
+            if timed:
+                e0.record(stream)
+            s_in.wait_stream(stream)
+            s_out.wait_stream(stream)
+            for i in range(steps):
+                si = i % 2
+                q_d, kv_d, ob_d, qy, o_d, ix_d = sets[si]
+                with torch.cuda.stream(s_in):
+                    if i >= 2:
+                        s_in.wait_event(ev_comp[si])            # step i-2 has read this set's inputs
+                    q_d.copy_(qin_h, non_blocking=True)
+                    (kv_d if prefill else kv_d[:, :, :, -1]).copy_(kv_h, non_blocking=True)
+                    ev_in[si].record(s_in)
+                stream.wait_event(ev_in[si])
                 if i >= 2:
-                    s_in.wait_event(ev_comp[si])            # step i-2 has read this set's inputs
-                q_d.copy_(qin_h, non_blocking=True)
-                (kv_d if prefill else kv_d[:, :, :, -1]).copy_(kv_h, non_blocking=True)
-                ev_in[si].record(s_in)
-            stream.wait_event(ev_in[si])
-            if i >= 2:
-                stream.wait_event(ev_out[si])               # step i-2's result has left this set
-            msa_route(bank.handle, qy, k, 0, ix_d.data_ptr(), 0, sh)
-            msa_attend(bank.handle, qy, k, ix_d.data_ptr(), o_d.data_ptr(), sh)
-            ev_comp[si].record(stream)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(ev_comp[si])
-                out_h[si].copy_(ob_d, non_blocking=True)
-                ev_out[si].record(s_out)
-        stream.wait_stream(s_out)
-        if timed:
-            e1.record(stream)
+                    stream.wait_event(ev_out[si])               # step i-2's result has left this set
+                msa_route(bank.handle, qy, k, 0, ix_d.data_ptr(), 0, sh)
+                msa_attend(bank.handle, qy, k, ix_d.data_ptr(), o_d.data_ptr(), sh)
+                ev_comp[si].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_comp[si])
+                    out_h[si].copy_(ob_d, non_blocking=True)
+                    ev_out[si].record(s_out)
+            stream.wait_stream(s_out)
+            if timed:
+                e1.record(stream)
 
-    e2e_run(4, False)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e2e_run(n_e2e, True)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    assert bank.device_error() == 0
+        e2e_run(4, False)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e2e_run(n_e2e, True)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        assert bank.device_error() == 0
 
-    total_ms, e2e_ms, route_ms, attend_ms = max_over_ranks([total_ms, e2e_ms, route_ms, attend_ms], "cuda")
+    total_ms, e2e_ms, route_ms, attend_ms = max_over_ranks([total_ms, e2e_ms or 0.0, route_ms, attend_ms], "cuda")
     if world > 1:
         dist.barrier()
     ms_step = total_ms / n
     units = B * (w.q_tokens if prefill else 1)   # queries (decode) or query tokens (prefill) per step
     value = job_throughput(world, units, n, total_ms)
-    e2e_value = job_throughput(world, units, n_e2e, e2e_ms)
+    e2e_value = job_throughput(world, units, n_e2e, e2e_ms) if with_e2e else None
 
     if rank == 0:
         peak, peak_kind = peaks()
@@ -478,30 +585,73 @@ def run_ours(args):
             metric, unit = METRIC, "queries/s"
         line = {
             "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": n,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": dict(base_config(w), parallelism=f"replicas x{world}",
-                           l2=f"inputs larger than L2: {step_bytes / 1e9:.2f} GB of HBM per step vs 126 MB L2",
-                           router_keys="bf16" if args.kr_bf16 else "f32"),
+            "config": base_config(w, world),
+            "router_keys": "bf16" if args.kr_bf16 else "f32",
             "router_attn_hbm": {"bytes_per_step": step_bytes, "GBps": step_bytes / (ms_step / 1000.0) / 1e9,
                                 "frac_of_peak": step_bytes / (ms_step / 1000.0) / 1e9 / peak,
                                 "route_ms": route_ms, "attend_ms": attend_ms},
             "roofline": roofline,
             "clocks": clk,
-            "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step(w) * n,
         }
-        if world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
-            qps, nq, spent, cores = oracle_sample(args.cpu_seconds)
-            line["cpu_baseline"] = {
-                "value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
-                "sample": f"{nq} decode queries (router over all 16384 chunks x 8 KV heads, top-16, "
-                          f"attention for 32 heads), {spent:.1f} s of oracle time"}
-        print(json.dumps(line), flush=True)
+        if with_e2e:
+            line["e2e"] = {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     bank.close()
+    return line if rank == 0 else None
+
+
+# The other workloads the default run also times once (after the headline), so that
+# every configuration's figures come from the same run: (name, steps, warmup).
+EXTRA_WORKLOADS = (("prefill", 20, 3), ("ragged_planted", 5, 2), ("bank_100m", 5, 2))
+
+
+def extra_summary(line: dict) -> dict:
+    keep = ("metric", "value", "unit", "steps", "warmup", "ms_per_step", "config", "roofline", "router",
+            "router_attn_hbm", "planted_recall", "unpipelined_ms_per_step", "gpu_launches", "clocks", "setup_s")
+    return {k: line[k] for k in keep if k in line}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
     if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    line = measure_device(args, args.workload, args.steps, args.warmup, world, rank, local)
+    if world > 1:
+        dist.barrier()
         dist.destroy_process_group()
+    if rank != 0:
+        return
+    torch.cuda.empty_cache()
+    if world == 1 and args.workload == WORKLOAD and not args.no_extras:
+        extras = {}
+        for name, steps, warm in EXTRA_WORKLOADS:
+            try:
+                if synth.WORKLOADS[name].host_tier:
+                    r = measure_host(args, name, steps, warm)
+                else:
+                    r = measure_device(args, name, steps, warm, 1, 0, local, with_e2e=False)
+                extras[name] = extra_summary(r)
+            except Exception as e:  # reported in the line, never hidden
+                extras[name] = {"error": f"{type(e).__name__}: {e}"}
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+        line["workloads"] = extras
+    if world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
+        w = synth.WORKLOADS[WORKLOAD]
+        r = oracle_timed(WORKLOAD, args.cpu_steps, 1)
+        line["cpu_baseline"] = {"value": r["value"], "unit": "queries/s", "cores": r["cores"], "kind": "oracle",
+                                "sample": oracle_sample_text(r, w)}
+    print(json.dumps(line), flush=True)
 
 
 def run_route_only(args):
@@ -553,10 +703,16 @@ def run_route_only(args):
 
 
 def run_host_tier(args):
+    if args.kv_cache_gb > 0:
+        return measure_host(args, args.workload, args.steps, args.warmup, cache=True)
+    print(json.dumps(measure_host(args, args.workload, args.steps, args.warmup)), flush=True)
+
+
+def measure_host(args, wname: str, n: int, warmup: int, cache: bool = False):
     """Decode steps on a bank whose K/V live in pinned host memory (69M / 100M tokens):
     msa_forward routes on the device, copies the selected documents' K/V slabs over
     PCIe and attends, pipelined over micro-batches of sequences. Also timed: the
-    routing alone, and routing then attention without the pipeline."""
+    routing alone, and routing then attention without the pipeline. Returns the line."""
     import torch
 
     import synth
@@ -565,7 +721,7 @@ def run_host_tier(args):
     from sparse_attention_routed_b200.runner import Bank
     from synth.device import fill_normal, host_kv_pool, query_tensors
 
-    w = synth.WORKLOADS[args.workload]
+    w = synth.WORKLOADS[wname]
     Hkv, d, B, k = w.n_kv_heads, w.head_dim, w.batch, w.top_k
     t0 = time.time()
     Kh, Vh = host_kv_pool(w)
@@ -583,7 +739,7 @@ def run_host_tier(args):
     torch.cuda.synchronize()
     setup_s = time.time() - t0
     bank.set_host_fetch(MSA_FETCH_SM_GATHER if args.host_fetch == "gather" else MSA_FETCH_COPY_ENGINE)
-    if args.kv_cache_gb > 0:
+    if cache:
         return run_host_cache(args, w, bank, setup_s, Kh)
     Q, Qr, LK, LV = query_tensors(w)
     qry = bank.query(Q, Qr, LK, LV, w.route_block)
@@ -591,7 +747,7 @@ def run_host_tier(args):
     out = torch.empty((B, w.n_q_heads, 1, d), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(2, warmup)):
         msa_forward(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
     msa_route(bank.handle, qry, k, 0, idx.data_ptr(), 0, sh)
     msa_attend(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
@@ -617,7 +773,6 @@ def run_host_tier(args):
         best = min(best, a0.elapsed_time(a1))
     h2d_peak = (1 << 30) / (best / 1e3) / 1e9
     del hbuf, dbuf
-    n = args.steps
     clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
     time.sleep(0.4)
     torch.cuda.synchronize()
@@ -646,10 +801,10 @@ def run_host_tier(args):
     peak, kind = peaks()
     line = {
         "metric": f"decode queries/s, pinned-host K/V tier ({w.n_tokens / 1e6:.1f}M-token bank)",
-        "value": B / (step_ms / 1e3), "unit": "queries/s", "n_gpus": 1, "steps": n, "warmup": args.warmup,
+        "value": B / (step_ms / 1e3), "unit": "queries/s", "n_gpus": 1, "steps": n, "warmup": warmup,
         "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "batch": B, "q_heads": w.n_q_heads, "kv_heads": Hkv,
+        "config": {"workload": wname, "batch": B, "q_heads": w.n_q_heads, "kv_heads": Hkv,
                    "head_dim": d, "bank_docs": w.n_docs, "bank_tokens": w.n_tokens, "local_len": w.local_len,
                    "top_k": k, "kv_slabs_pinned": w.kv_slabs, "pinned_kv_bytes": 2 * Kh.numel() * 2,
                    "host_fetch": args.host_fetch},
@@ -664,8 +819,11 @@ def run_host_tier(args):
         "planted_recall": recall, "setup_s": setup_s, "clocks": clk,
         "gpu_launches": launches_per_step(w, gather=args.host_fetch == "gather") * n,
     }
-    print(json.dumps(line), flush=True)
     bank.close()
+    del Kh, Vh
+    if hasattr(torch._C, "_host_emptyCache"):
+        torch._C._host_emptyCache()   # hand the pinned pool back before the next workload pins its own
+    return line
 
 
 FETCH_DESC = {"gather": "host_gather_kernel: the SMs read the mapped pinned K/V, one launch per micro-batch",

@@ -86,6 +86,7 @@ def _load():
         "msa_get_host_fetch": ([vp, ctypes.POINTER(ctypes.c_int)], ctypes.c_int),
         "msa_set_router_precision": ([vp, ctypes.c_int], ctypes.c_int),
         "msa_check_wait_timeout": ([vp, vp], ctypes.c_int),
+        "msa_selftest_exp2_poly": ([vp, vp, vp, i64, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -110,12 +111,12 @@ def __getattr__(name):
         return lib()
     raise AttributeError(name)
 
-# Every symbol include/msa.h declares, in declaration order.
+# Every symbol include/msa.h and include/msa_selftest.h declare, in declaration order.
 EXPORTED = ["msa_bank_create", "msa_bank_destroy", "msa_build_bank", "msa_bank_info", "msa_reserve",
             "msa_route", "msa_attend", "msa_attend_lse", "msa_attend_backward", "msa_attend_backward_saved",
             "msa_forward", "msa_route_noalloc", "msa_set_kv_cache",
             "msa_kv_cache_stats", "msa_set_host_fetch", "msa_get_host_fetch", "msa_set_router_precision", "msa_check_wait_timeout", "msa_get_device_error",
-            "msa_status_string"]
+            "msa_status_string", "msa_selftest_exp2_poly"]
 
 
 def msa_status_string(status: int) -> str:
@@ -290,3 +291,9 @@ def msa_check_wait_timeout(bank, stream=0) -> None:
 
 def msa_get_device_error(bank, stream=0) -> int:
     return lib().msa_get_device_error(bank, stream or None)
+
+
+def msa_selftest_exp2_poly(x: int, y_poly: int, y_lib: int, n: int, stream=0) -> None:
+    """Self-test hook: the prefill kernel's polynomial 2^x and CUDA's exp2f over x [n] (device fp32)."""
+    _check(lib().msa_selftest_exp2_poly(x or None, y_poly or None, y_lib or None, int(n), stream or None),
+           "msa_selftest_exp2_poly")

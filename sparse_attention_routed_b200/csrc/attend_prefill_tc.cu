@@ -72,29 +72,6 @@ constexpr int kFastPoly = MSA_PF_FAST_POLY;
 #endif
 constexpr float kPMax = MSA_PF_PMAX;
 
-// 2^x on the FMA and integer pipes, to share the exponentials of a tile between
-// them and the special-function unit. Range reduction x = n + f with n the
-// nearest integer (adding 1.5 * 2^23 leaves n in the low mantissa bits) and
-// f in [-1/2, 1/2]; 2^f from a cubic whose coefficients are a Remez
-// (equioscillating relative error) fit on that interval, max relative error
-// 7.5e-5 -- far below the 2^-9 of the bf16 rounding P gets next; 2^n is
-// added to the exponent field.
-// Two lanes at once with the packed fp32x2 FMA/add of sm_100.
-__device__ __forceinline__ float2 exp2_poly3x2(float2 x) {
-  // [-125, 64]: the result stays normal, and above 2^64 it saturates there (which the
-  // fast path's row-sum check rejects, as it rejects ex2's +inf)
-  x.x = fminf(fmaxf(x.x, -125.f), 64.f);
-  x.y = fminf(fmaxf(x.y, -125.f), 64.f);
-  const float2 big = make_float2(12582912.f, 12582912.f), nbig = make_float2(-12582912.f, -12582912.f);
-  const float2 j = __fadd2_rn(x, big);
-  const float2 f = __ffma2_rn(__fadd2_rn(j, nbig), make_float2(-1.f, -1.f), x);  // x - (j - big)
-  float2 p = __ffma2_rn(make_float2(0.0551716685f, 0.0551716685f), f, make_float2(0.242611125f, 0.242611125f));
-  p = __ffma2_rn(p, f, make_float2(0.693260968f, 0.693260968f));
-  p = __ffma2_rn(p, f, make_float2(0.999928057f, 0.999928057f));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(j.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(j.y) << 23)));
-}
-
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;

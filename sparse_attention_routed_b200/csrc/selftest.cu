@@ -5,6 +5,7 @@
 // stays usable and the host reads MSA_ERR_TIMEOUT from msa_get_device_error.
 #include "common.cuh"
 #include "internal.h"
+#include "../../include/msa_selftest.h"
 
 namespace msa {
 namespace {
@@ -28,3 +29,36 @@ cudaError_t launch_wait_timeout(int* err, cudaStream_t s) {
 }
 
 }  // namespace msa
+
+// ---------------------------------------------------------------------------
+// Self-test of exp2_poly3x2, the polynomial 2^x that the tcgen05 prefill kernel
+// runs on the FMA pipe for part of its exponentials: y[i] = exp2_poly3x2(x[i])
+// and, beside it, CUDA's exp2f(x[i]), so a test can compare both against an
+// fp64 reference over the polynomial's whole domain.
+namespace msa {
+namespace {
+
+__global__ void exp2_poly_kernel(const float* x, float* y_poly, float* y_lib, int64_t n) {
+  const int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x1 = i + 1 < n ? x[i + 1] : 0.f;
+  const float2 p = exp2_poly3x2(make_float2(x[i], x1));
+  y_poly[i] = p.x;
+  y_lib[i] = exp2f(x[i]);
+  if (i + 1 < n) {
+    y_poly[i + 1] = p.y;
+    y_lib[i + 1] = exp2f(x1);
+  }
+}
+
+}  // namespace
+}  // namespace msa
+
+extern "C" msa_status msa_selftest_exp2_poly(const float* x, float* y_poly, float* y_lib, int64_t n,
+                                             void* stream) {
+  if (!x || !y_poly || !y_lib || n < 1 || n > (int64_t(1) << 30)) return MSA_ERR_INVALID_ARG;
+  const int threads = 256;
+  const int64_t blocks = ((n + 1) / 2 + threads - 1) / threads;
+  msa::exp2_poly_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_lib, n);
+  return cudaGetLastError() == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+}

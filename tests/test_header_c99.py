@@ -15,14 +15,19 @@ LIBDIR = os.path.join(ROOT, "sparse_attention_routed_b200")
 
 
 def _declared():
-    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
-    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(msa_\w+)\s*\(", text, flags=re.M)
+    names = []
+    for h in sorted(os.listdir(os.path.dirname(HEADER))):
+        if h.endswith(".h"):
+            text = re.sub(r"/\*.*?\*/", "", open(os.path.join(os.path.dirname(HEADER), h)).read(), flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(msa_\w+)\s*\(", text, flags=re.M)
+    return names
 
 
 PROGRAM = r"""
 #include <stdio.h>
 #include <string.h>
 #include "msa.h"
+#include "msa_selftest.h"
 
 typedef void (*any_fn)(void);
 
