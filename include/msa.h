@@ -29,8 +29,9 @@
  * theta_i = base^(-2i/d); query head hq reads KV head hq / (Hq/Hkv).
  *
  * Conventions for every entry point:
- *   - All tensors are caller-owned, row-major, densely packed, bf16 unless
- *     stated, and live in device memory unless the argument says "host".
+ *   - All tensors are caller-owned, row-major, densely packed, of the bank's
+ *     element type (msa_bank_config.dtype: bf16 unless stated) where no type is
+ *     named, and live in device memory unless the argument says "host".
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
  *     asynchronous on it; host arrays are read before the call returns.
  *   - Every call returns an msa_status and never throws. Argument errors are
@@ -102,6 +103,12 @@ typedef enum {
   MSA_FETCH_SM_GATHER = 1    /* one kernel per stretch reads the mapped host K/V (the default) */
 } msa_host_fetch;
 
+/* Element type of a bank's tensors and of its steps' inputs (msa_bank_config.dtype). */
+typedef enum {
+  MSA_DTYPE_BF16 = 0,     /* bf16 storage, tensor-core arithmetic with fp32 accumulation (the default) */
+  MSA_DTYPE_F32 = 1       /* fp32 storage and fp32 arithmetic throughout (CUDA cores; device-tier banks) */
+} msa_dtype;
+
 /* Opaque bank handle. Owns: K_r (fp32) and its inverse norms, document and
  * chunk offsets, RoPE tables, workspace, and (host tier) the device staging
  * pool, side stream and events. */
@@ -122,6 +129,13 @@ typedef struct {
   const int64_t* doc_rows; /* host [n_docs] or NULL: first row of document j inside
                               each head's k/v; NULL means the prefix sums of doc_lens.
                               Several documents may share rows (an aliased pool). */
+  int32_t dtype;           /* msa_dtype of k, v, the routing keys msa_build_bank pools and
+                              every msa_query tensor (q, qr, local_k, local_v). 0 = bf16.
+                              MSA_DTYPE_F32 keeps every value in fp32 end to end: Parallel
+                              RoPE is stored in fp32 and attention runs in fp32 on the CUDA
+                              cores (no bf16 rounding of the rotated query, keys or P);
+                              device-tier banks and the forward calls only (pinned-host
+                              banks and the backward return MSA_ERR_UNSUPPORTED). */
 } msa_bank_config;
 
 /* Creates a bank: validates the layout, computes document/chunk offsets and

@@ -33,6 +33,8 @@ MSA_KR_F32 = 0
 MSA_KR_BF16 = 1
 MSA_FETCH_COPY_ENGINE = 0
 MSA_FETCH_SM_GATHER = 1
+MSA_DTYPE_BF16 = 0
+MSA_DTYPE_F32 = 1
 
 
 class MsaError(RuntimeError):
@@ -47,6 +49,7 @@ class msa_bank_config(ctypes.Structure):
         ("route_dim", ctypes.c_int32), ("doc_lens", ctypes.POINTER(ctypes.c_int64)),
         ("rope_base", ctypes.c_float), ("kv_location", ctypes.c_int32), ("k", ctypes.c_void_p),
         ("v", ctypes.c_void_p), ("kv_rows", ctypes.c_int64), ("doc_rows", ctypes.POINTER(ctypes.c_int64)),
+        ("dtype", ctypes.c_int32),
     ]
 
 
@@ -146,14 +149,15 @@ def make_query(batch, n_q_heads, q_tokens, local_len, route_block, q=0, qr=0, lo
 
 def msa_bank_create(n_docs: int, n_kv_heads: int, head_dim: int, doc_lens, k: int, v: int,
                     rope_base: float = 10000.0, kv_location: int = MSA_KV_DEVICE, kv_rows: int = 0,
-                    doc_rows=None, route_dim: Optional[int] = None, check: bool = True):
+                    doc_rows=None, route_dim: Optional[int] = None, check: bool = True,
+                    dtype: int = MSA_DTYPE_BF16):
     """Returns (status, handle). doc_lens / doc_rows are host int64 sequences."""
     lens = np.ascontiguousarray(np.asarray(doc_lens, dtype=np.int64))
     rows = None if doc_rows is None else np.ascontiguousarray(np.asarray(doc_rows, dtype=np.int64))
     cfg = msa_bank_config(
         n_docs, n_kv_heads, head_dim, head_dim if route_dim is None else route_dim,
         lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), rope_base, kv_location, k or None, v or None,
-        kv_rows, None if rows is None else rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)))
+        kv_rows, None if rows is None else rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), dtype)
     handle = ctypes.c_void_p()
     st = lib().msa_bank_create(ctypes.byref(cfg), ctypes.byref(handle))
     if check:

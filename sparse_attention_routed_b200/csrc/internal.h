@@ -30,15 +30,19 @@ struct BankBuildArgs {
   int32_t n_chunks;         // chunks in the slice
   int32_t n_kv_heads;
   int32_t head_dim;
+  // fp32 banks: r32 / k32 take the place of r / k (same row numbering and strides)
+  const float* r32;
+  float* k32;
 };
 cudaError_t launch_bank_build(const BankBuildArgs& a, cudaStream_t s);
 
 // q_r = mean of each routing block's routing queries, plus 1/||q_r||.
 struct QrArgs {
-  const uint16_t* qr;  // [B, Hkv, Tq, d_r]
+  const uint16_t* qr;  // [B, Hkv, Tq, d_r] bf16 (or nullptr when qr32 is given)
   float* q_r;          // [B*nblk, Hkv, d_r]
   float* q_r_inv;      // [B*nblk, Hkv]
   int32_t batch, n_kv_heads, q_tokens, route_block, route_dim;
+  const float* qr32;   // [B, Hkv, Tq, d_r] fp32 routing queries (fp32 banks), or nullptr
 };
 cudaError_t launch_qr_prep(const QrArgs& a, cudaStream_t s);
 
@@ -187,6 +191,29 @@ cudaError_t launch_attend_bwd_prep(const float* dout, const float* out, const fl
                                    int route_block, int sms, cudaStream_t s);
 cudaError_t launch_attend_bwd_dkdv_tc(const AttendBwdArgs& g, const AttendMaps& m, const CUtensorMap& q_map,
                                       const CUtensorMap& do_map, const AttendGradMaps& gm, int sms, cudaStream_t s);
+
+// fp32 routed attention (banks of MSA_DTYPE_F32): the key set, masks and output of the
+// bf16 kernels, with every operand and product in fp32 on the CUDA cores. One CTA per
+// attend_f32_rows() query rows of a problem streams the problem's whole key list.
+struct AttendF32Args {
+  const float* q;           // [B, Hq, Tq, d], no RoPE
+  const float* local_k;     // [B, Hkv, Lc, d], no RoPE
+  const float* local_v;     // [B, Hkv, Lc, d]
+  const float* bank_k;      // [Hkv, kv_rows, d], Parallel RoPE applied
+  const float* bank_v;      // [Hkv, kv_rows, d]
+  const int32_t* sel;       // [P][top_k]
+  const int64_t* doc_row;   // [n_docs]
+  const int32_t* doc_len;   // [n_docs]
+  const float2* gtab;       // [Lc][d/2] Global RoPE (cos, sin) at k_off + u
+  float* out;               // [B, Hq, Tq, d]
+  float* lse_out;           // [B, Hq, Tq] or nullptr
+  int* err;
+  int64_t kv_rows;
+  int32_t batch, n_q_heads, n_kv_heads, q_tokens, local_len, route_block, top_k, n_docs;
+  float scale_log2;         // log2(e) / sqrt(d)
+};
+int attend_f32_rows();
+cudaError_t launch_attend_f32(const AttendF32Args& a, int head_dim, cudaStream_t s);
 
 // Pinned-host tier: one run of host-contiguous K/V rows and the staging rows it goes
 // to; jobs ascend in piece0, the index of their first piece (host_gather_piece_rows

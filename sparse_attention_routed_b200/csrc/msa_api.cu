@@ -129,6 +129,7 @@ const void* mapped_host(const void* p, size_t bytes) {
 struct msa_bank {
   // configuration
   int n_docs = 0, hkv = 0, d = 0, dr = 0, kv_loc = 0;
+  bool f32 = false;  // MSA_DTYPE_F32: fp32 tensors and fp32 arithmetic (attend_f32_kernel)
   double base = 10000.0;
   const void* k = nullptr;
   const void* v = nullptr;
@@ -333,9 +334,10 @@ Workspace layout(const msa_bank* bank, const StepShape& s, int splits, uint8_t* 
   w.q_r_inv = (float*)take(rows_route * bank->hkv * 4);
   w.scores = (float*)take(rows_route * bank->hkv * bank->n_docs * 4);
   w.idx = (int32_t*)take((size_t)s.P * s.k * 4);
-  const bool prefill = s.rows > kMaxRows;
-  w.part_o = (float*)take(prefill ? 0 : (size_t)s.P * splits * s.rows * bank->d * 4);
-  w.part_ml = (float*)take(prefill ? 0 : (size_t)s.P * splits * s.rows * 2 * 4);
+  const bool prefill = s.rows > kMaxRows && !bank->f32;
+  const bool decode = s.rows <= kMaxRows && !bank->f32;
+  w.part_o = (float*)take(decode ? (size_t)s.P * splits * s.rows * bank->d * 4 : 0);
+  w.part_ml = (float*)take(decode ? (size_t)s.P * splits * s.rows * 2 * 4 : 0);
   w.local_rot = (uint16_t*)take(prefill ? (size_t)s.B * bank->hkv * s.Lc * bank->d * 2 : 0);
   const bool tc = prefill && attend_prefill_tc_supported(bank->d, s.G, s.Bq);
   w.q_rot = (uint16_t*)take(tc ? (size_t)s.B * s.Hq * s.Tq * bank->d * 2 : 0);
@@ -391,9 +393,10 @@ msa_status route_into(msa_bank* bank, const msa_query* q, const StepShape& s, fl
                       float* score_scratch, float* doc_scores, int32_t* idx, float* top_scores, cudaStream_t st) {
   RouteArgs ra{};
   const bool tc = route_tc_supported(bank->dr, s.B * s.nblk);
-  const bool fuse = !tc && s.Bq <= kRouteFuseMaxBlock;  // the router forms q_r itself
+  const bool fuse = !tc && !bank->f32 && s.Bq <= kRouteFuseMaxBlock;  // the router forms q_r itself
   if (!fuse) {
-    QrArgs qa{(const uint16_t*)q->qr, q_r, q_r_inv, s.B, bank->hkv, s.Tq, s.Bq, bank->dr};
+    QrArgs qa{bank->f32 ? nullptr : (const uint16_t*)q->qr, q_r, q_r_inv, s.B, bank->hkv, s.Tq, s.Bq, bank->dr,
+              bank->f32 ? (const float*)q->qr : nullptr};
     MSA_CUDA(launch_qr_prep(qa, st));
   } else {
     ra.qr = (const uint16_t*)q->qr;
@@ -667,6 +670,33 @@ msa_status host_fetch(msa_bank* bank, const StepShape& s, const int32_t* idx_dev
 msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, int splits, const Workspace& w,
                        const int32_t* idx, float* out, cudaStream_t st, const int64_t* staged = nullptr,
                        float* lse_out = nullptr) {
+  if (bank->f32) {
+    AttendF32Args f{};
+    f.q = (const float*)q->q;
+    f.local_k = (const float*)q->local_k;
+    f.local_v = (const float*)q->local_v;
+    f.bank_k = (const float*)bank->k;
+    f.bank_v = (const float*)bank->v;
+    f.sel = idx;
+    f.doc_row = bank->d_doc_row;
+    f.doc_len = bank->d_doc_len;
+    f.gtab = bank->d_gtab;
+    f.out = out;
+    f.lse_out = lse_out;
+    f.err = bank->d_err;
+    f.kv_rows = bank->kv_rows;
+    f.batch = s.B;
+    f.n_q_heads = s.Hq;
+    f.n_kv_heads = bank->hkv;
+    f.q_tokens = s.Tq;
+    f.local_len = s.Lc;
+    f.route_block = s.Bq;
+    f.top_k = s.k;
+    f.n_docs = bank->n_docs;
+    f.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)bank->d));
+    MSA_CUDA(launch_attend_f32(f, bank->d, st));
+    return MSA_OK;
+  }
   const bool prefill = s.rows > kMaxRows;
   const bool tc = prefill && attend_prefill_tc_supported(bank->d, s.G, s.Bq);
   const int box = tc ? attend_prefill_tc_tile_rows() : prefill ? attend_prefill_tile_rows() : attend_tile_rows();
@@ -870,6 +900,8 @@ msa_status msa_bank_create(const msa_bank_config* cfg, msa_bank** out) {
   if (!(cfg->rope_base > 1.0f)) return MSA_ERR_INVALID_ARG;
   if (cfg->kv_location != MSA_KV_DEVICE && cfg->kv_location != MSA_KV_PINNED_HOST) return MSA_ERR_INVALID_ARG;
   if (!cfg->k || !cfg->v || !aligned16(cfg->k) || !aligned16(cfg->v)) return MSA_ERR_INVALID_ARG;
+  if (cfg->dtype != MSA_DTYPE_BF16 && cfg->dtype != MSA_DTYPE_F32) return MSA_ERR_INVALID_ARG;
+  if (cfg->dtype == MSA_DTYPE_F32 && cfg->kv_location != MSA_KV_DEVICE) return MSA_ERR_UNSUPPORTED;
 
   msa_bank* b = new (std::nothrow) msa_bank();
   if (!b) return MSA_ERR_OOM;
@@ -879,6 +911,7 @@ msa_status msa_bank_create(const msa_bank_config* cfg, msa_bank** out) {
   b->dr = cfg->route_dim;
   b->base = cfg->rope_base;
   b->kv_loc = cfg->kv_location;
+  b->f32 = cfg->dtype == MSA_DTYPE_F32;
   b->k = cfg->k;
   b->v = cfg->v;
   b->doc_lens.assign(cfg->doc_lens, cfg->doc_lens + cfg->n_docs);
@@ -969,7 +1002,7 @@ msa_status msa_bank_create(const msa_bank_config* cfg, msa_bank** out) {
     return fail(rc);
   if (cudaMalloc(&b->d_err, sizeof(int)) != cudaSuccess) return fail(MSA_ERR_OOM);
   if (cudaMemset(b->d_err, 0, sizeof(int)) != cudaSuccess) return fail(MSA_ERR_CUDA);
-  if (b->kv_loc == MSA_KV_DEVICE) {
+  if (b->kv_loc == MSA_KV_DEVICE && !b->f32) {  // bf16 tensor maps of the bank K/V
     if ((rc = make_map(&b->map_k, b->k, (int64_t)b->hkv * b->kv_rows, b->d, attend_tile_rows())) != MSA_OK) return fail(rc);
     if ((rc = make_map(&b->map_v, b->v, (int64_t)b->hkv * b->kv_rows, b->d, attend_tile_rows())) != MSA_OK) return fail(rc);
     if ((rc = make_map(&b->map_k64, b->k, (int64_t)b->hkv * b->kv_rows, b->d, attend_prefill_tile_rows())) != MSA_OK)
@@ -1010,9 +1043,14 @@ msa_status msa_build_bank(msa_bank* bank, int32_t doc_begin, int32_t doc_end, co
   const int64_t c0 = bank->chunk_off[doc_begin], c1 = bank->chunk_off[doc_end];
   if (c1 - c0 >= (int64_t(1) << 31) / bank->hkv) return MSA_ERR_UNSUPPORTED;
   BankBuildArgs a{};
-  a.r = (const uint16_t*)r_slice;
+  if (bank->f32) {
+    a.r32 = (const float*)r_slice;
+    a.k32 = (float*)k_slice;
+  } else {
+    a.r = (const uint16_t*)r_slice;
+    a.k = (uint16_t*)k_slice;
+  }
   a.r_head_stride = r_head_stride * bank->dr;
-  a.k = (uint16_t*)k_slice;
   a.tok_base = bank->doc_off[doc_begin];
   a.k_head_stride = k_head_stride * bank->d;
   a.chunk_tok = bank->d_chunk_tok + c0;
@@ -1122,7 +1160,7 @@ msa_status backward_impl(msa_bank* bank, const msa_query* q, int32_t top_k, cons
   for (const void* p : {(const void*)d_out, (const void*)dq, (const void*)dlocal_k, (const void*)dlocal_v,
                         (const void*)dbank_k, (const void*)dbank_v})
     if (!aligned16(p)) return MSA_ERR_INVALID_ARG;
-  if (bank->kv_loc != MSA_KV_DEVICE) return MSA_ERR_UNSUPPORTED;
+  if (bank->kv_loc != MSA_KV_DEVICE || bank->f32) return MSA_ERR_UNSUPPORTED;
   cudaStream_t st = (cudaStream_t)stream;
   // workspace after the split counters: RoPE'd queries and local keys, row statistics
   const size_t qrot = align_up((size_t)s.B * s.Hq * s.Tq * bank->d * 2);

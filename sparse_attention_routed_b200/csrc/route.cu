@@ -21,10 +21,14 @@ __global__ void qr_prep_kernel(QrArgs a) {
   __shared__ float red[32];
   float ss = 0.f;
   for (int i = threadIdx.x; i < a.route_dim; i += blockDim.x) {
-    const uint16_t* src =
-        a.qr + (((int64_t)b * a.n_kv_heads + h) * a.q_tokens + (int64_t)blk * a.route_block) * a.route_dim + i;
+    const int64_t off =
+        (((int64_t)b * a.n_kv_heads + h) * a.q_tokens + (int64_t)blk * a.route_block) * a.route_dim + i;
     float s = 0.f;
-    for (int t = 0; t < a.route_block; ++t) s += __uint_as_float((uint32_t)src[(int64_t)t * a.route_dim] << 16);
+    if (a.qr32) {
+      for (int t = 0; t < a.route_block; ++t) s += a.qr32[off + (int64_t)t * a.route_dim];
+    } else {
+      for (int t = 0; t < a.route_block; ++t) s += __uint_as_float((uint32_t)a.qr[off + (int64_t)t * a.route_dim] << 16);
+    }
     s /= (float)a.route_block;
     a.q_r[((int64_t)row * a.n_kv_heads + h) * a.route_dim + i] = s;
     ss += s * s;

@@ -9,7 +9,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (MSA_KV_DEVICE, make_query, msa_attend, msa_bank_create, msa_bank_destroy, msa_bank_info,
+from . import (MSA_DTYPE_BF16, MSA_DTYPE_F32, MSA_KV_DEVICE, make_query, msa_attend, msa_bank_create, msa_bank_destroy, msa_bank_info,
                msa_build_bank, msa_forward, msa_get_device_error, msa_kv_cache_stats, msa_reserve, msa_route,
                msa_set_kv_cache, ptr, msa_set_router_precision, msa_set_host_fetch, msa_get_host_fetch)
 
@@ -28,16 +28,19 @@ def _stream(stream=None) -> int:
 
 
 class Bank:
-    """A bank over [Hkv, rows, d] bf16 K/V tensors (K gets Parallel RoPE in place on build)."""
+    """A bank over [Hkv, rows, d] K/V tensors, bf16 or fp32 (the bank's element type
+    follows K; K gets Parallel RoPE in place on build)."""
 
     def __init__(self, K: torch.Tensor, V: torch.Tensor, doc_lens, rope_base: float = 10000.0,
                  kv_location: int = MSA_KV_DEVICE, doc_rows=None):
-        assert K.dtype == torch.bfloat16 and V.dtype == torch.bfloat16 and K.shape == V.shape
+        assert K.dtype in (torch.bfloat16, torch.float32) and V.dtype == K.dtype and K.shape == V.shape
         self.K, self.V = K, V
+        self.dtype = K.dtype
         self.n_kv_heads, self.kv_rows, self.head_dim = K.shape
         self.doc_lens = np.asarray(doc_lens, dtype=np.int64)
         _, self.handle = msa_bank_create(len(self.doc_lens), self.n_kv_heads, self.head_dim, self.doc_lens,
-                                         ptr(K), ptr(V), rope_base, kv_location, self.kv_rows, doc_rows)
+                                         ptr(K), ptr(V), rope_base, kv_location, self.kv_rows, doc_rows,
+                                         dtype=MSA_DTYPE_F32 if K.dtype == torch.float32 else MSA_DTYPE_BF16)
         self.info = msa_bank_info(self.handle)
 
     def build(self, R: torch.Tensor, doc_begin: int = 0, doc_end=None, K_slice=None, stream=None,
@@ -51,13 +54,13 @@ class Bank:
             k_ptr, k_stride = 0, 0
         elif K_slice is None:
             K_slice = self.K
-            k_ptr = self.K.data_ptr() + tok0 * self.head_dim * 2
+            k_ptr = self.K.data_ptr() + tok0 * self.head_dim * self.K.element_size()
             k_stride = self.kv_rows
         else:
-            k_ptr = ptr(K_slice, torch.bfloat16)
+            k_ptr = ptr(K_slice, self.dtype)
             k_stride = K_slice.shape[1]
         if R is not None:
-            assert R.is_contiguous() and R.dtype == torch.bfloat16
+            assert R.is_contiguous() and R.dtype == self.dtype
         msa_build_bank(self.handle, doc_begin, doc_end, 0 if R is None else R.data_ptr(),
                        0 if R is None else R.shape[1], k_ptr, k_stride, _stream(stream))
 
@@ -72,8 +75,8 @@ class Bank:
 
     def query(self, Q, Qr, LK, LV, route_block: int):
         B, Hq, Tq, _ = Q.shape
-        return make_query(B, Hq, Tq, LK.shape[2], route_block, ptr(Q, torch.bfloat16),
-                          ptr(Qr, torch.bfloat16), ptr(LK, torch.bfloat16), ptr(LV, torch.bfloat16))
+        return make_query(B, Hq, Tq, LK.shape[2], route_block, ptr(Q, self.dtype),
+                          ptr(Qr, self.dtype), ptr(LK, self.dtype), ptr(LV, self.dtype))
 
     def reserve(self, query, top_k):
         msa_reserve(self.handle, query, top_k)

@@ -103,6 +103,28 @@ def normal_f32(seed: int, tensor_id: int, start: int, count: int) -> np.ndarray:
     return NORMAL_TABLE_F32[(u64_at(key, idx) >> np.uint64(48)).astype(np.int64)]
 
 
+# fp32 workloads draw from streams of their own (tensor id + F32_STREAMS)
+F32_STREAMS = 100
+
+
+def gaussian_f32(seed: int, tensor_id: int, start: int, count: int) -> np.ndarray:
+    """Elements [start, start+count) of an fp32 N(0,1) tensor whose values use all
+    24 significant bits (unlike the table values, which are bf16 numbers).
+
+    Element i is the Box-Muller transform (Box & Muller, "A note on the generation
+    of random normal deviates", Ann. Math. Statist. 1958) of two 53-bit uniforms,
+    outputs 2i and 2i+1 of the tensor's SplitMix64 stream:
+    u1 = (top 53 bits + 1) / 2^53 in (0, 1], u2 = top 53 bits / 2^53 in [0, 1),
+    z = sqrt(-2 ln u1) cos(2 pi u2), computed in fp64 and rounded to fp32."""
+    key = stream_key(seed, tensor_id + F32_STREAMS)
+    idx = np.arange(start, start + count, dtype=np.uint64)
+    a = u64_at(key, idx * np.uint64(2)) >> np.uint64(11)
+    b = u64_at(key, idx * np.uint64(2) + np.uint64(1)) >> np.uint64(11)
+    u1 = (a.astype(np.float64) + 1.0) * 2.0 ** -53
+    u2 = b.astype(np.float64) * 2.0 ** -53
+    return (np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)).astype(np.float32)
+
+
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
@@ -137,6 +159,7 @@ class Workload:
     host_tier: bool = False
     kv_slabs: int = 0                # > 0: K/V of document j are the rows of slab (j mod kv_slabs)
     rope_base: float = 10000.0
+    dtype: str = "bf16"              # "f32": fp32 tensors from gaussian_f32 (device-tier banks)
     doc_lens_cache: Optional[np.ndarray] = field(default=None, repr=False)
 
     @property
@@ -212,6 +235,8 @@ def planted_targets(seed: int, batch: int, n_docs: int, count: int) -> np.ndarra
 
 WORKLOADS = {
     "tiny": Workload("tiny", 0, 1, 4, 4, 64, 16, 512, 256, 16, 16, 2),
+    # the tiny step with fp32 values (24 significant bits) and the fp32 path end to end
+    "tiny_f32": Workload("tiny_f32", 0, 1, 4, 4, 64, 16, 512, 256, 16, 16, 2, dtype="f32"),
     "decode_4m": Workload("decode_4m", 1, 8, 32, 8, 128, 1024, 4096, 4096, 1, 1, 16),
     # same step as decode_4m on a 128-document bank: identical attention bytes per
     # step, 2 GB of K/V on the device (for hardware-counter captures)
@@ -251,6 +276,11 @@ def doc_kv_bits(w: Workload, tensor_id: int, head: int, doc: int, t0: int = 0, n
     row = int(w.doc_kv_rows()[doc]) + t0
     start = (head * w.kv_rows + row) * d
     return normal_bf16_bits(w.seed, tensor_id, start, n * d).reshape(n, d)
+
+
+def f32_tensor(w: Workload, tensor_id: int, shape) -> np.ndarray:
+    """A whole fp32 tensor of an fp32 workload, flat index order (host)."""
+    return gaussian_f32(w.seed, tensor_id, 0, int(np.prod(shape))).reshape(shape)
 
 
 def query_bits(w: Workload, tensor_id: int, shape) -> np.ndarray:

@@ -8,7 +8,7 @@ import numpy as np
 import torch
 
 from . import (NORMAL_TABLE_BITS, T_K, T_LK, T_LV, T_Q, T_QR, T_R, T_V, Workload, device_normal_bf16,
-               planted_qr_bits)
+               f32_tensor, planted_qr_bits)
 
 _TABLES = {}
 
@@ -32,9 +32,18 @@ def normal(shape, seed: int, tensor_id: int, device="cuda", start: int = 0) -> t
     return fill_normal(torch.empty(shape, dtype=torch.bfloat16, device=device), seed, tensor_id, start)
 
 
+def _f32(w: Workload, tensor_id: int, shape, device) -> torch.Tensor:
+    return torch.from_numpy(f32_tensor(w, tensor_id, shape)).to(device)
+
+
 def bank_tensors(w: Workload, device="cuda", with_r: bool = True):
-    """K, V as [Hkv, kv_rows, d] and R as [Hkv, Ntok, d_r], bf16 (K without RoPE)."""
+    """K, V as [Hkv, kv_rows, d] and R as [Hkv, Ntok, d_r], bf16 (K without RoPE);
+    fp32 for an fp32 workload (generated on the host, copied)."""
     shape = (w.n_kv_heads, w.kv_rows, w.head_dim)
+    if w.dtype == "f32":
+        assert not w.kv_slabs and not w.planted
+        R = _f32(w, T_R, (w.n_kv_heads, w.n_tokens, w.route_dim), device) if with_r else None
+        return _f32(w, T_K, shape, device), _f32(w, T_V, shape, device), R
     K = normal(shape, w.seed, T_K, device)
     V = normal(shape, w.seed, T_V, device)
     R = normal((w.n_kv_heads, w.n_tokens, w.route_dim), w.seed, T_R, device) if with_r else None
@@ -42,7 +51,12 @@ def bank_tensors(w: Workload, device="cuda", with_r: bool = True):
 
 
 def query_tensors(w: Workload, device="cuda"):
-    """Q [B,Hq,Tq,d], Qr [B,Hkv,Tq,d_r], local K/V [B,Hkv,Lc,d], all bf16."""
+    """Q [B,Hq,Tq,d], Qr [B,Hkv,Tq,d_r], local K/V [B,Hkv,Lc,d], all bf16 (fp32 for an fp32 workload)."""
+    if w.dtype == "f32":
+        return (_f32(w, T_Q, (w.batch, w.n_q_heads, w.q_tokens, w.head_dim), device),
+                _f32(w, T_QR, (w.batch, w.n_kv_heads, w.q_tokens, w.route_dim), device),
+                _f32(w, T_LK, (w.batch, w.n_kv_heads, w.local_len, w.head_dim), device),
+                _f32(w, T_LV, (w.batch, w.n_kv_heads, w.local_len, w.head_dim), device))
     Q = normal((w.batch, w.n_q_heads, w.q_tokens, w.head_dim), w.seed, T_Q, device)
     if w.planted:
         bits = planted_qr_bits(w)

@@ -73,6 +73,12 @@ def test_bank_create_rejects_bad_arguments():
     assert st == msa.MSA_ERR_INVALID_ARG and not h
     st, h = msa.msa_bank_create(2, 1, 64, lens, fake, fake, kv_rows=25, check=False)   # rows too short
     assert st == msa.MSA_ERR_INVALID_ARG and not h
+    st, h = msa.msa_bank_create(2, 1, 64, lens, fake, fake, dtype=7, check=False)      # no such element type
+    assert st == msa.MSA_ERR_INVALID_ARG and not h
+    # fp32 banks are device-tier only
+    st, h = msa.msa_bank_create(2, 1, 64, lens, fake, fake, kv_location=msa.MSA_KV_PINNED_HOST,
+                                dtype=msa.MSA_DTYPE_F32, check=False)
+    assert st == msa.MSA_ERR_UNSUPPORTED and not h
 
 
 def test_null_handles_are_rejected():

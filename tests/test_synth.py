@@ -52,3 +52,14 @@ def test_workload_shapes():
     assert w.n_tokens == 1024 * 4096
     w5 = synth.WORKLOADS["bank_100m"]
     assert w5.n_tokens == 99_999_744
+
+
+def test_gaussian_f32_streams():
+    """The fp32 generator: deterministic, sliceable, N(0,1) moments, and values that
+    use more than bf16's 8 significant bits."""
+    x = synth.gaussian_f32(0, synth.T_K, 0, 200000)
+    assert x.dtype == np.float32
+    np.testing.assert_array_equal(x[1000:1500], synth.gaussian_f32(0, synth.T_K, 1000, 500))
+    assert abs(float(x.mean())) < 0.02 and abs(float(x.std()) - 1.0) < 0.02
+    assert np.mean((x.view(np.uint32) & 0xFFFF) == 0) < 1e-3
+    assert not np.array_equal(x[:100], synth.gaussian_f32(1, synth.T_K, 0, 100))
