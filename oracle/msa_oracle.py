@@ -43,8 +43,9 @@ last Tq local tokens and local key u is visible to local query i iff u <= i.
 
 Parity pins: every function here is pinned -- tests/test_oracle_pins.py (the
 step), tests/test_oracle_backward.py (the backward), tests/test_oracle_router_bf16.py
-(the bf16-key router variant) and tests/test_oracle_lse.py (the row log-sum-exp) --
-against closed forms, invariants, library special cases or brute force.
+(the bf16-key router variant), tests/test_oracle_lse.py (the row log-sum-exp) and
+tests/test_oracle_memory_parallel.py (the document-sharded step) -- against closed
+forms, invariants, library special cases or brute force.
 """
 from __future__ import annotations
 
@@ -463,3 +464,162 @@ def backward(inputs: Dict[str, np.ndarray], doc_lens: Sequence[int], top_k: int,
             L = off[j + 1] - off[j]
             dK[h, off[j]:off[j + 1]] = rope_adjoint(dK_rot[h, off[j]:off[j + 1]], np.arange(L), base)
     return {"dQ": dQ, "dK": dK, "dV": dV, "dLK": dLK, "dLV": dLV, "selection": sel, "out": fwd["out"]}
+
+
+# --------------------------------------------------------------------------
+# Memory Parallel: the bank's documents split into contiguous shards, one per
+# device; each shard scores its own documents, the shards' candidates are
+# gathered and merged into the one global top-k, each shard attends over the
+# selected documents it holds, and the partial attentions are combined
+#   -- "MSA架构：突破大模型记忆瓶颈的稀疏注意力技术", §2.1 item 3 (memory parallel:
+#      distributed memory retrieval across GPUs through an AllGather);
+#   -- "MSA (Memory Sparse Attention)" (robocikowo.com), Równoległość (the Memory
+#      Parallel engine scores the router across devices; the top-k selection and
+#      the K/V fetch that follows stay sequential within each decoding step).
+# Reading: the gathered items are each shard's own top-k candidates (score,
+# global document index); the merge keeps the top_k of their union under the
+# single-bank order (score desc, index asc); the partial of a shard is its
+# softmax over the keys it holds together with that softmax's log-sum-exp, and
+# the local context is attended by one shard (the owner of the sequence).
+# --------------------------------------------------------------------------
+
+def shard_ranges(n_docs: int, n_shards: int) -> List[Tuple[int, int]]:
+    """[lo, hi) document ranges of n_shards contiguous shards, sizes differing by at
+    most one (the first n_docs % n_shards shards hold the extra document)."""
+    if not 1 <= n_shards <= n_docs:
+        raise ValueError("1 <= n_shards <= n_docs")
+    q, r = divmod(n_docs, n_shards)
+    out, lo = [], 0
+    for s in range(n_shards):
+        hi = lo + q + (1 if s < r else 0)
+        out.append((lo, hi))
+        lo = hi
+    return out
+
+
+def merge_candidates(cand_scores: Sequence[np.ndarray], cand_idx: Sequence[np.ndarray],
+                     top_k: int) -> Tuple[np.ndarray, np.ndarray]:
+    """The global top_k from the shards' candidate lists: the top_k members of their
+    union ordered by (score desc, global index asc). Returns (indices, scores)."""
+    pairs = []
+    for sc, ix in zip(cand_scores, cand_idx):
+        for s, j in zip(np.asarray(sc, dtype=np.float64), np.asarray(ix)):
+            pairs.append((-float(s), int(j)))
+    if len(pairs) < top_k:
+        raise ValueError("fewer candidates than top_k")
+    pairs.sort()
+    chosen = pairs[:top_k]
+    return (np.asarray([j for _, j in chosen], dtype=np.int64),
+            np.asarray([-s for s, _ in chosen], dtype=np.float64))
+
+
+def attention_partial(q_rot: np.ndarray, keys: np.ndarray, values: np.ndarray) -> Tuple[np.ndarray, float]:
+    """Attention of one (already rotated) query row over a subset of its keys:
+    (softmax over the subset applied to its values, log sum_j exp(s_j) over the
+    subset) with s_j = q_rot . k_j / sqrt(d). An empty subset gives (0, -inf)."""
+    q = np.asarray(q_rot, dtype=np.float64)
+    keys = np.asarray(keys, dtype=np.float64).reshape(-1, q.shape[-1])
+    if keys.shape[0] == 0:
+        return np.zeros(q.shape[-1]), -math.inf
+    s = keys @ q / math.sqrt(q.shape[-1])
+    m = s.max()
+    w = np.exp(s - m)
+    return (w @ np.asarray(values, dtype=np.float64)) / w.sum(), float(m + math.log(w.sum()))
+
+
+def merge_partials(outs: Sequence[np.ndarray], lses: Sequence[float]) -> Tuple[np.ndarray, float]:
+    """One softmax over the union of disjoint key subsets from their partials:
+    L = log sum_s exp(lse_s), out = sum_s exp(lse_s - L) out_s. Parts with
+    lse = -inf (no keys) weigh nothing; if every part is empty, (0, -inf)."""
+    lses = [float(x) for x in lses]
+    finite = [x for x in lses if x != -math.inf]
+    if not finite:
+        return np.zeros_like(np.asarray(outs[0], dtype=np.float64)), -math.inf
+    m = max(finite)
+    total = sum(math.exp(x - m) for x in finite)
+    L = m + math.log(total)
+    out = np.zeros_like(np.asarray(outs[0], dtype=np.float64))
+    for o, x in zip(outs, lses):
+        if x != -math.inf:
+            out = out + math.exp(x - L) * np.asarray(o, dtype=np.float64)
+    return out, L
+
+
+def memory_parallel_forward(inputs: Dict[str, np.ndarray], doc_lens: Sequence[int], top_k: int,
+                            route_block: int, n_shards: int, base: float = 10000.0, owner: int = 0,
+                            chunk: int = CHUNK) -> Dict[str, np.ndarray]:
+    """The routed step of forward() with the documents in n_shards contiguous shards.
+
+    Per (sequence, routing block, KV head): every shard s routes over its own
+    documents only (K_r pooled from its routing keys, cosine, max over chunks) and
+    keeps its top min(top_k, n_s) (score, global index) candidates; the candidates of
+    all shards are merged (merge_candidates). Per query row: every shard attends over
+    the merged selection's documents it holds, the owner shard also over the causal
+    local context, each giving (out_s, lse_s) (attention_partial); the row's output
+    is merge_partials of those. Returns topk [B, nblk, Hkv, k], the candidates
+    ([n_shards] lists of [B, nblk, Hkv, k_s] scores / indices), partial outputs and
+    log-sum-exps [n_shards, B, Hq, Tq, (d)], and out [B, Hq, Tq, d]."""
+    K = np.asarray(inputs["K"], dtype=np.float64)
+    V = np.asarray(inputs["V"], dtype=np.float64)
+    R = np.asarray(inputs["R"], dtype=np.float64)
+    Q = np.asarray(inputs["Q"], dtype=np.float64)
+    Qr = np.asarray(inputs["Qr"], dtype=np.float64)
+    LK = np.asarray(inputs["LK"], dtype=np.float64)
+    LV = np.asarray(inputs["LV"], dtype=np.float64)
+    Hkv, _, d = K.shape
+    B, Hq, Tq, _ = Q.shape
+    Lc = LK.shape[2]
+    G = Hq // Hkv
+    nblk = Tq // route_block
+    n = len(doc_lens)
+    off = doc_offsets(doc_lens)
+    k_off = k_offset(top_k, doc_lens)          # the whole bank's longest document
+    shards = shard_ranges(n, n_shards)
+
+    # each shard's candidates, from its own documents' routing keys
+    cand_sc = [np.empty((B, nblk, Hkv, min(top_k, hi - lo))) for lo, hi in shards]
+    cand_ix = [np.empty((B, nblk, Hkv, min(top_k, hi - lo)), dtype=np.int64) for lo, hi in shards]
+    for s, (lo, hi) in enumerate(shards):
+        lens_s = list(doc_lens[lo:hi])
+        for h in range(Hkv):
+            kr, chunk_doc = build_routing_keys(R[h, off[lo]:off[hi]], lens_s, chunk)
+            for b in range(B):
+                qb = block_mean_query(Qr[b, h], route_block)
+                for blk in range(nblk):
+                    sc = route_doc_scores(qb[blk], kr, chunk_doc, hi - lo)
+                    loc = select_top_k(sc, min(top_k, hi - lo))
+                    cand_ix[s][b, blk, h] = loc + lo
+                    cand_sc[s][b, blk, h] = sc[loc]
+    topk = np.empty((B, nblk, Hkv, top_k), dtype=np.int64)
+    for b in range(B):
+        for blk in range(nblk):
+            for h in range(Hkv):
+                topk[b, blk, h] = merge_candidates([c[b, blk, h] for c in cand_sc],
+                                                   [c[b, blk, h] for c in cand_ix], top_k)[0]
+
+    K_rot = np.empty_like(K)
+    for h in range(Hkv):
+        K_rot[h] = parallel_rope_bank(K[h], doc_lens, base)
+    part_out = np.zeros((n_shards, B, Hq, Tq, d))
+    part_lse = np.full((n_shards, B, Hq, Tq), -math.inf)
+    out = np.empty((B, Hq, Tq, d))
+    for b in range(B):
+        for hq in range(Hq):
+            h = hq // G
+            for t in range(Tq):
+                i = Lc - Tq + t
+                q_rot = rope(Q[b, hq, t], k_off + i, base)
+                docs = topk[b, t // route_block, h]
+                for s, (lo, hi) in enumerate(shards):
+                    mine = [int(j) for j in docs if lo <= j < hi]
+                    ks = [K_rot[h, off[j]:off[j + 1]] for j in mine]
+                    vs = [V[h, off[j]:off[j + 1]] for j in mine]
+                    if s == owner:
+                        ks.append(rope(LK[b, h, :i + 1], k_off + np.arange(i + 1), base))
+                        vs.append(LV[b, h, :i + 1])
+                    keys = np.concatenate(ks, axis=0) if ks else np.zeros((0, d))
+                    vals = np.concatenate(vs, axis=0) if vs else np.zeros((0, d))
+                    part_out[s, b, hq, t], part_lse[s, b, hq, t] = attention_partial(q_rot, keys, vals)
+                out[b, hq, t] = merge_partials(part_out[:, b, hq, t], part_lse[:, b, hq, t])[0]
+    return {"topk": topk, "cand_scores": cand_sc, "cand_idx": cand_ix, "part_out": part_out,
+            "part_lse": part_lse, "out": out, "shards": shards, "k_off": k_off}
