@@ -43,8 +43,9 @@ last Tq local tokens and local key u is visible to local query i iff u <= i.
 
 Parity pins: every function here is pinned -- tests/test_oracle_pins.py (the
 step), tests/test_oracle_backward.py (the backward), tests/test_oracle_router_bf16.py
-(the bf16-key router variant), tests/test_oracle_lse.py (the row log-sum-exp) and
-tests/test_oracle_memory_parallel.py (the document-sharded step) -- against closed
+(the bf16-key router variant), tests/test_oracle_lse.py (the row log-sum-exp),
+tests/test_oracle_memory_parallel.py (the document-sharded step) and
+tests/test_oracle_interleave.py (multi-hop Memory Interleave) -- against closed
 forms, invariants, library special cases or brute force.
 """
 from __future__ import annotations
@@ -623,3 +624,99 @@ def memory_parallel_forward(inputs: Dict[str, np.ndarray], doc_lens: Sequence[in
                 out[b, hq, t] = merge_partials(part_out[:, b, hq, t], part_lse[:, b, hq, t])[0]
     return {"topk": topk, "cand_scores": cand_sc, "cand_idx": cand_ix, "part_out": part_out,
             "part_lse": part_lse, "out": out, "shards": shards, "k_off": k_off}
+
+
+# --------------------------------------------------------------------------
+# Memory Interleave: several hops of routing, each expanding the context
+#   -- "MSA (Memory Sparse Attention)" (robocikowo.com), Komponenty (Memory
+#      Interleave: generation of document identifiers and context expansion
+#      alternate, so retrieval proceeds in several steps over scattered memory);
+#   -- "MSA架构：突破大模型记忆瓶颈的稀疏注意力技术", §3.2 (several retrieval rounds,
+#      each building on the previous one).
+# Reading (there is no generating model here, so the "next identifiers" come from
+# a stated routing-space update): hop t routes with its routing query q_t over the
+# documents not yet in the context, keeps top_k of them and appends them to the
+# context; the next hop's query is q_{t+1} = q_t/|q_t| + (1/top_k) sum over the
+# hop's documents of kbar_j/|kbar_j|, kbar_j being document j's routing key (the
+# mean of its per-token routing keys); after hop t the attention runs over every
+# document retrieved so far (t * top_k of them, Global-RoPE offset
+# t * top_k * max length) plus the local context.
+# --------------------------------------------------------------------------
+
+def doc_routing_key(R_doc: np.ndarray) -> np.ndarray:
+    """A document's routing key: the mean of its per-token routing keys [L, d_r]."""
+    R_doc = np.asarray(R_doc, dtype=np.float64)
+    total = np.zeros(R_doc.shape[1], dtype=np.float64)
+    for t in range(R_doc.shape[0]):
+        total += R_doc[t]
+    return total / R_doc.shape[0]
+
+
+def interleave_next_query(q_r: np.ndarray, chosen_keys: Sequence[np.ndarray]) -> np.ndarray:
+    """The next hop's routing query: q/|q| + (1/k) sum_j kbar_j/|kbar_j| over the hop's k documents."""
+    q = np.asarray(q_r, dtype=np.float64)
+    out = q / max(math.sqrt(float(q @ q)), 1e-30)
+    for kb in chosen_keys:
+        kb = np.asarray(kb, dtype=np.float64)
+        out = out + kb / max(math.sqrt(float(kb @ kb)), 1e-30) / len(chosen_keys)
+    return out
+
+
+def select_top_k_excluding(doc_scores: np.ndarray, top_k: int, exclude) -> np.ndarray:
+    """select_top_k over the documents not in `exclude` (the context already holds them)."""
+    s = np.asarray(doc_scores, dtype=np.float64).copy()
+    ex = [int(j) for j in exclude]
+    if len(s) - len(set(ex)) < top_k:
+        raise ValueError("fewer documents outside the context than top_k")
+    s[ex] = -np.inf
+    return select_top_k(s, top_k)
+
+
+def memory_interleave(inputs: Dict[str, np.ndarray], doc_lens: Sequence[int], top_k: int, route_block: int,
+                      hops: int, base: float = 10000.0, chunk: int = CHUNK) -> Dict[str, list]:
+    """Memory Interleave over `hops` hops on explicit inputs (forward()'s layout).
+
+    Per (sequence, routing block, KV head): q_1 = the block mean of the routing
+    queries; hop t scores every document (cosine, max over chunks), keeps the top_k
+    not yet selected, and forms q_{t+1} = interleave_next_query(q_t, their keys).
+    After hop t, each query row attends over all t * top_k documents selected so far
+    (hop order, then rank) plus its local context, with k_off = t * top_k * max L.
+    Returns per hop: q_r [B, nblk, Hkv, d_r] (the query it routed with), topk
+    [B, nblk, Hkv, k] (its new documents), selection [B, nblk, Hkv, t*k] (all so
+    far), out [B, Hq, Tq, d]."""
+    R = np.asarray(inputs["R"], dtype=np.float64)
+    Qr = np.asarray(inputs["Qr"], dtype=np.float64)
+    Hkv = R.shape[0]
+    B, _, Tq, dr = Qr.shape
+    nblk = Tq // route_block
+    n = len(doc_lens)
+    off = doc_offsets(doc_lens)
+    K_r, chunk_doc = [], None
+    for h in range(Hkv):
+        kr, chunk_doc = build_routing_keys(R[h], doc_lens, chunk)
+        K_r.append(kr)
+    dkeys = np.stack([np.stack([doc_routing_key(R[h, off[j]:off[j + 1]]) for j in range(n)])
+                      for h in range(Hkv)])
+    q = np.empty((B, nblk, Hkv, dr))
+    for b in range(B):
+        for h in range(Hkv):
+            q[b, :, h] = block_mean_query(Qr[b, h], route_block)
+    res = {"q_r": [], "topk": [], "selection": [], "out": []}
+    sel = np.zeros((B, nblk, Hkv, 0), dtype=np.int64)
+    for t in range(hops):
+        new = np.empty((B, nblk, Hkv, top_k), dtype=np.int64)
+        nxt = np.empty_like(q)
+        for b in range(B):
+            for blk in range(nblk):
+                for h in range(Hkv):
+                    sc = route_doc_scores(q[b, blk, h], K_r[h], chunk_doc, n)
+                    new[b, blk, h] = select_top_k_excluding(sc, top_k, sel[b, blk, h])
+                    nxt[b, blk, h] = interleave_next_query(q[b, blk, h], [dkeys[h, j] for j in new[b, blk, h]])
+        sel = np.concatenate([sel, new], axis=-1)
+        out = forward(inputs, doc_lens, sel.shape[-1], route_block, base, chunk, selection=sel)["out"]
+        res["q_r"].append(q.copy())
+        res["topk"].append(new)
+        res["selection"].append(sel.copy())
+        res["out"].append(out)
+        q = nxt
+    return res
