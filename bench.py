@@ -65,6 +65,10 @@ def parse():
     ap.add_argument("--kr-bf16", action="store_true",
                     help="the reduced-precision router: read only the bf16 high part of the normalised K_r "
                          "(msa_set_router_precision(MSA_KR_BF16)), half the router's bytes")
+    ap.add_argument("--memory-parallel", type=int, default=0, metavar="S",
+                    help="Memory Parallel: the bank split into document shards. With one process, S shard banks "
+                         "on one GPU (stacks in place of the all-gathers); under torchrun, one shard per rank and "
+                         "NCCL all-gathers (S is then the world size)")
     ap.add_argument("--route-only", action="store_true",
                     help="time msa_route alone on the full bank's K_r with a stand-in 1-document K/V "
                          "(routing keys streamed in slices; a few GB on the device, for profiling captures)")
@@ -654,6 +658,128 @@ def run_ours(args):
     print(json.dumps(line), flush=True)
 
 
+def shard_tensors(w, lo: int, hi: int, device="cuda"):
+    """K, V, R of documents [lo, hi) of a device workload, generated directly (each
+    head's rows are one slice of the whole tensor's stream)."""
+    import torch
+
+    import synth
+    from synth.device import fill_normal
+    off = np.concatenate([[0], np.cumsum(w.doc_lens())])
+    a, b = int(off[lo]), int(off[hi])
+    out = []
+    for tid, rows, dim in ((synth.T_K, w.kv_rows, w.head_dim), (synth.T_V, w.kv_rows, w.head_dim),
+                           (synth.T_R, w.n_tokens, w.route_dim)):
+        t = torch.empty((w.n_kv_heads, b - a, dim), dtype=torch.bfloat16, device=device)
+        for h in range(w.n_kv_heads):
+            fill_normal(t[h], w.seed, tid, (h * rows + a) * dim)
+        out.append(t)
+    return out
+
+
+def run_memory_parallel(args):
+    """The decode step with the bank split into document shards (Memory Parallel):
+    every shard routes its own documents, the candidates are merged into the global
+    top-k, every shard attends over the selected documents it holds (shard 0 also
+    over the local context) and the partials are merged. One process: S shards on
+    one GPU, timed against the single bank on the same GPU. Under torchrun: one
+    shard per rank, NCCL all-gathers, max-over-ranks time (the bank is fixed and
+    split: strong scaling)."""
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    from sparse_attention_routed_b200.parallel import MemoryParallelStep, ShardedStep, shard_ranges
+    from sparse_attention_routed_b200.runner import Bank
+    from synth.device import query_tensors
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    w = synth.WORKLOADS[args.workload]
+    assert not w.host_tier and w.q_tokens == w.route_block, "Memory Parallel bench: device-tier decode workloads"
+    S = world if world > 1 else max(1, args.memory_parallel)
+    ranges = shard_ranges(w.n_docs, S)
+    lens, max_len = w.doc_lens(), int(w.doc_lens().max())
+    mine = [rank] if world > 1 else list(range(S))
+    banks, keep = [], []
+    for s in mine:
+        lo, hi = ranges[s]
+        K, V, R = shard_tensors(w, lo, hi)
+        bank = Bank(K, V, lens[lo:hi], w.rope_base)
+        bank.set_shard(lo, w.n_docs, max_len)
+        bank.build(R)
+        torch.cuda.synchronize()
+        del R
+        banks.append(bank)
+        keep += [K, V]
+    Q, Qr, LK, LV = query_tensors(w)
+    queries = [b.query(Q, Qr, LK, LV, w.route_block) for b in banks]
+    step = (MemoryParallelStep(banks[0], owner=0) if world > 1 else ShardedStep(banks, owner=0))
+    run = (lambda: step(queries[0], w.top_k)) if world > 1 else (lambda: step(queries, w.top_k))
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        run()
+    torch.cuda.synchronize()
+    for b in banks:
+        assert b.device_error() == 0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    time.sleep(0.4)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    (total_ms,) = max_over_ranks([e0.elapsed_time(e1)], "cuda")
+    line = None
+    if rank == 0:
+        ms = total_ms / args.steps
+        line = {"metric": f"decode queries/s, Memory Parallel over {S} document shards",
+                "value": w.batch / (ms / 1e3), "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "strong" if world > 1 else "n/a (shards share one GPU)", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": dict(base_config(w, world), parallelism=f"memory parallel, {S} shards"),
+                "clocks": clk}
+    if world > 1:
+        dist.destroy_process_group()
+    else:
+        # the same step on one bank holding every document, same GPU, same inputs
+        for b in banks:
+            b.close()
+        banks.clear()
+        keep.clear()
+        torch.cuda.empty_cache()
+        K, V, R = shard_tensors(w, 0, w.n_docs)
+        whole = Bank(K, V, lens, w.rope_base)
+        whole.build(R)
+        del R
+        qry = whole.query(Q, Qr, LK, LV, w.route_block)
+        for _ in range(max(3, args.warmup)):
+            whole.forward(qry, w.top_k)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            whole.forward(qry, w.top_k)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        line["single_bank_ms_per_step"] = e0.elapsed_time(e1) / args.steps
+        whole.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_route_only(args):
     """msa_route alone over the full K_r of the workload (profiling aid, not the headline)."""
     import torch
@@ -1059,6 +1185,8 @@ def main():
         run_backward(args)
     elif args.route_only:
         run_route_only(args)
+    elif args.memory_parallel:
+        run_memory_parallel(args)
     elif args.workload in ("ragged_planted", "bank_100m"):
         run_host_tier(args)
     else:

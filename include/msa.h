@@ -306,6 +306,95 @@ msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_
 msa_status msa_route_noalloc(msa_bank* bank, const msa_query* q, int32_t top_k, float* doc_scores,
                              int32_t* topk_idx, float* topk_scores, void* stream);
 
+/* ---- Memory Parallel: the bank's documents split into contiguous shards, one per
+ * device ("MSA架构：突破大模型记忆瓶颈的稀疏注意力技术", §2.1 item 3: distributed
+ * memory retrieval across GPUs through an AllGather; "MSA (Memory Sparse
+ * Attention)", robocikowo.com, Równoległość: router scoring spread over devices,
+ * then top-k and the K/V fetch in sequence). A step on S shards:
+ *   1. each shard: msa_route -> its own top_k candidates (scores + GLOBAL indices);
+ *   2. all-gather the candidates (NCCL, or plain copies when the shards share a GPU);
+ *   3. every shard: msa_merge_topk -> the global top_k, identical on all shards and
+ *      equal to what one bank holding every document would select;
+ *   4. each shard: msa_attend_partial over the selected documents it holds, the
+ *      sequence's owner shard with with_local = 1 -> (out_s, lse_s);
+ *   5. gather the partials at the owner: msa_merge_partials -> the step's output.
+ * The library moves no data between devices; the caller's collectives do. */
+
+/* Marks `bank` as the shard holding documents [doc_base, doc_base + n_docs) of a
+ * bank of n_docs_total documents whose longest document has max_doc_len_total
+ * tokens. Afterwards: msa_route returns global indices (doc_base + local index);
+ * attention calls read global indices, attend the ones in this shard and skip the
+ * other shards' (MSA_ERR_INVALID_ARG in the device error flag only outside
+ * [0, n_docs_total)); top_k may reach n_docs_total for attention (routing still
+ * needs top_k <= this shard's n_docs); the Global-RoPE offset is
+ * top_k * max_doc_len_total, the whole bank's. Attention on a shard runs the
+ * decode kernel (<= 16 rows per routing block and KV head) or, on fp32 banks, the
+ * fp32 kernel: many-row bf16 steps and the backward return MSA_ERR_UNSUPPORTED.
+ * MSA_ERR_INVALID_ARG for a NULL bank, doc_base < 0, a range past n_docs_total,
+ * or max_doc_len_total below this shard's longest document. Call it before the
+ * steps that use it (it is not ordered with work in flight). */
+msa_status msa_bank_set_shard(msa_bank* bank, int32_t doc_base, int32_t n_docs_total, int64_t max_doc_len_total);
+
+/* This shard's part of the routed attention for the selection topk_idx
+ * [B, nblk, Hkv, top_k] (global indices; the merged selection): for every query
+ * row, the softmax over the selected documents this bank holds -- and, when
+ * with_local = 1, the causal local context -- applied to their values (out
+ * [B, Hq, Tq, d] fp32), and that softmax's log-sum-exp (lse [B, Hq, Tq] fp32,
+ * natural log of sum_j exp(q_rot . k_j / sqrt(d))). A row with no key here gets
+ * out = 0 and lse = -inf. On a whole bank with with_local = 1 it equals
+ * msa_attend_lse. MSA_ERR_INVALID_ARG for a NULL pointer or with_local not 0/1;
+ * other errors as msa_attend. */
+msa_status msa_attend_partial(msa_bank* bank, const msa_query* q, int32_t top_k, const int32_t* topk_idx,
+                              int32_t with_local, float* out, float* lse, void* stream);
+
+/* Merges n_parts candidate lists into the global top_k: cand_scores / cand_idx
+ * [n_parts][rows][top_k] fp32 / int32 (the shards' msa_route outputs stacked part
+ * after part, as an all-gather leaves them), each list ordered (score desc, index
+ * asc) and no index in two lists -> topk_idx [rows][top_k] (and topk_scores, or
+ * NULL): the first top_k of the union in the same order. rows = B * nblk * Hkv.
+ * Device pointers, asynchronous on `stream`; no bank. MSA_ERR_INVALID_ARG for a
+ * NULL pointer or a size < 1; MSA_ERR_UNSUPPORTED for n_parts > 64, top_k > 64 or
+ * rows > 65535. The pages describe the gather, not this layout. */
+msa_status msa_merge_topk(int32_t n_parts, int32_t rows, int32_t top_k, const float* cand_scores,
+                          const int32_t* cand_idx, int32_t* topk_idx, float* topk_scores, void* stream);
+
+/* Merges n_parts partial attentions over disjoint key sets into one softmax over
+ * their union: part_out [n_parts][rows][head_dim] and part_lse [n_parts][rows]
+ * fp32 (msa_attend_partial outputs stacked part after part) -> out [rows][head_dim]
+ * = sum_s exp(part_lse[s] - L) part_out[s], L = log sum_s exp(part_lse[s]), and lse
+ * [rows] = L (or NULL). Parts with lse = -inf weigh nothing; a row empty in every
+ * part gets 0 and -inf. rows = B * Hq * Tq. Device pointers, asynchronous on
+ * `stream`; no bank. MSA_ERR_INVALID_ARG for a NULL pointer or a size < 1. */
+msa_status msa_merge_partials(int32_t n_parts, int64_t rows, int32_t head_dim, const float* part_out,
+                              const float* part_lse, float* out, float* lse, void* stream);
+
+/* One hop of Memory Interleave ("MSA (Memory Sparse Attention)", robocikowo.com,
+ * Komponenty: generation of document identifiers and context expansion alternate,
+ * so retrieval proceeds in several steps; "MSA架构…", §3.2: retrieval in rounds).
+ * There is no generating model in this library, so the next hop's routing query
+ * is a stated update in routing space (below). Per (sequence, routing block, KV
+ * head):
+ *   - the hop routes with q_r_in [B, Hkv, nblk, d_r] fp32 (NULL on the first hop:
+ *     the block means of q->qr, as msa_route forms them);
+ *   - it ranks only documents outside the context: context_idx
+ *     [B, nblk, Hkv, n_ctx] int32 (NULL when n_ctx = 0), the documents earlier
+ *     hops took;
+ *   - ctx_out [B, nblk, Hkv, n_ctx + top_k] receives the expanded context: the
+ *     n_ctx documents, then the hop's top_k new ones in (score desc, index asc)
+ *     order (topk_scores [B, nblk, Hkv, top_k] fp32 their scores, or NULL);
+ *   - q_r_out [B, Hkv, nblk, d_r] fp32 (or NULL) receives the next hop's query
+ *     q/|q| + (1/top_k) sum_j kbar_j/|kbar_j| over the hop's documents, kbar_j the
+ *     mean of document j's routing keys (its chunks' K_r weighted by their lengths).
+ * Attention over the expanded context is msa_attend with top_k = n_ctx + top_k and
+ * ctx_out as the selection (its Global-RoPE offset grows with the context). q->qr
+ * must be given on every hop (q, local_k, local_v are not read). Whole banks only
+ * (MSA_ERR_UNSUPPORTED on a shard). MSA_ERR_INVALID_ARG for a NULL ctx_out,
+ * n_ctx < 0, n_ctx + top_k > n_docs or an unaligned q_r_in; a context index
+ * outside [0, n_docs) raises MSA_ERR_INVALID_ARG in the device error flag. */
+msa_status msa_interleave_route(msa_bank* bank, const msa_query* q, int32_t top_k, const float* q_r_in,
+                                const int32_t* context_idx, int32_t n_ctx, int32_t* ctx_out, float* topk_scores,
+                                float* q_r_out, void* stream);
+
 /* Device-resident cache of selected K/V slabs for a pinned-host bank: the hot tier
  * of a hot/cold split ("MSA (Memory Sparse Attention)", robocikowo.com, Komponenty:
  * K_r in GPU memory, K/V in CPU RAM; "MSA：大模型高效推理的新突破，仅需2张A800显卡驱动1亿Token",

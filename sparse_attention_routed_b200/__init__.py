@@ -90,6 +90,11 @@ def _load():
         "msa_set_router_precision": ([vp, ctypes.c_int], ctypes.c_int),
         "msa_check_wait_timeout": ([vp, vp], ctypes.c_int),
         "msa_selftest_exp2_poly": ([vp, vp, vp, i64, vp], ctypes.c_int),
+        "msa_bank_set_shard": ([vp, i32, i32, i64], ctypes.c_int),
+        "msa_attend_partial": ([vp, ctypes.POINTER(msa_query), i32, vp, i32, vp, vp, vp], ctypes.c_int),
+        "msa_merge_topk": ([i32, i32, i32, vp, vp, vp, vp, vp], ctypes.c_int),
+        "msa_merge_partials": ([i32, i64, i32, vp, vp, vp, vp, vp], ctypes.c_int),
+        "msa_interleave_route": ([vp, ctypes.POINTER(msa_query), i32, vp, vp, i32, vp, vp, vp, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -117,7 +122,8 @@ def __getattr__(name):
 # Every symbol include/msa.h and include/msa_selftest.h declare, in declaration order.
 EXPORTED = ["msa_bank_create", "msa_bank_destroy", "msa_build_bank", "msa_bank_info", "msa_reserve",
             "msa_route", "msa_attend", "msa_attend_lse", "msa_attend_backward", "msa_attend_backward_saved",
-            "msa_forward", "msa_route_noalloc", "msa_set_kv_cache",
+            "msa_forward", "msa_route_noalloc", "msa_bank_set_shard", "msa_attend_partial", "msa_merge_topk",
+            "msa_merge_partials", "msa_interleave_route", "msa_set_kv_cache",
             "msa_kv_cache_stats", "msa_set_host_fetch", "msa_get_host_fetch", "msa_set_router_precision", "msa_check_wait_timeout", "msa_get_device_error",
             "msa_status_string", "msa_selftest_exp2_poly"]
 
@@ -295,6 +301,51 @@ def msa_check_wait_timeout(bank, stream=0) -> None:
 
 def msa_get_device_error(bank, stream=0) -> int:
     return lib().msa_get_device_error(bank, stream or None)
+
+
+def msa_bank_set_shard(bank, doc_base: int, n_docs_total: int, max_doc_len_total: int, check=True) -> int:
+    """Marks the bank as documents [doc_base, doc_base + n_docs) of an n_docs_total-document bank."""
+    st = lib().msa_bank_set_shard(bank, int(doc_base), int(n_docs_total), int(max_doc_len_total))
+    if check:
+        _check(st, "msa_bank_set_shard")
+    return st
+
+
+def msa_attend_partial(bank, query: msa_query, top_k: int, topk_idx: int, with_local: int, out: int, lse: int,
+                       stream=0, check=True) -> int:
+    st = lib().msa_attend_partial(bank, ctypes.byref(query), top_k, topk_idx or None, int(with_local), out or None,
+                                  lse or None, stream or None)
+    if check:
+        _check(st, "msa_attend_partial")
+    return st
+
+
+def msa_merge_topk(n_parts: int, rows: int, top_k: int, cand_scores: int, cand_idx: int, topk_idx: int,
+                   topk_scores: int, stream=0, check=True) -> int:
+    st = lib().msa_merge_topk(int(n_parts), int(rows), int(top_k), cand_scores or None, cand_idx or None,
+                              topk_idx or None, topk_scores or None, stream or None)
+    if check:
+        _check(st, "msa_merge_topk")
+    return st
+
+
+def msa_merge_partials(n_parts: int, rows: int, head_dim: int, part_out: int, part_lse: int, out: int, lse: int,
+                       stream=0, check=True) -> int:
+    st = lib().msa_merge_partials(int(n_parts), int(rows), int(head_dim), part_out or None, part_lse or None,
+                                  out or None, lse or None, stream or None)
+    if check:
+        _check(st, "msa_merge_partials")
+    return st
+
+
+def msa_interleave_route(bank, query: msa_query, top_k: int, q_r_in: int, context_idx: int, n_ctx: int,
+                         ctx_out: int, topk_scores: int, q_r_out: int, stream=0, check=True) -> int:
+    """One Memory Interleave hop: route over the documents outside the context, expand it, next query."""
+    st = lib().msa_interleave_route(bank, ctypes.byref(query), int(top_k), q_r_in or None, context_idx or None,
+                                    int(n_ctx), ctx_out or None, topk_scores or None, q_r_out or None, stream or None)
+    if check:
+        _check(st, "msa_interleave_route")
+    return st
 
 
 def msa_selftest_exp2_poly(x: int, y_poly: int, y_lib: int, n: int, stream=0) -> None:

@@ -134,13 +134,14 @@ __global__ void __launch_bounds__(S::THREADS, S::MINB)
   const int k = a.top_k;
 
   if (tid < k) {
-    const int j = a.sel[(int64_t)p * k + tid];
+    const int j = a.sel[(int64_t)p * k + tid];  // a global index on a shard bank
+    const int jl = j - a.doc_lo;
     int len = 0;
     long long base = 0;
-    if (j >= 0 && j < a.n_docs) {
-      len = a.doc_len[j];
-      base = a.sel_base ? (long long)a.sel_base[(int64_t)p * k + tid] : (long long)h * a.kv_rows + a.doc_row[j];
-    } else {
+    if (jl >= 0 && jl < a.n_docs) {
+      len = a.doc_len[jl];
+      base = a.sel_base ? (long long)a.sel_base[(int64_t)p * k + tid] : (long long)h * a.kv_rows + a.doc_row[jl];
+    } else if (j < 0 || j >= a.n_docs_index) {
       atomicCAS(a.err, 0, kErrInvalidArg);
     }
     doc_len_s[tid] = len;
@@ -161,7 +162,7 @@ __global__ void __launch_bounds__(S::THREADS, S::MINB)
       acc += (doc_len_s[d] + TILE - 1) / TILE;
     }
     tile_start[k] = acc;
-    tile_start[k + 1] = acc + (i_max + 1 + TILE - 1) / TILE;
+    tile_start[k + 1] = acc + (a.with_local ? (i_max + 1 + TILE - 1) / TILE : 0);
   }
   __syncthreads();
   // split boundaries in cost units: bank tiles cost 1, local tiles LOCAL_W

@@ -49,13 +49,14 @@ __global__ void __launch_bounds__(kWarps * 32) attend_f32_kernel(const AttendF32
   const int k = a.top_k;
 
   if (tid < k) {
-    const int j = a.sel[(int64_t)p * k + tid];
+    const int j = a.sel[(int64_t)p * k + tid];  // a global index on a shard bank
+    const int jl = j - a.doc_lo;
     int len = 0;
     long long base = 0;
-    if (j >= 0 && j < a.n_docs) {
-      len = a.doc_len[j];
-      base = (long long)h * a.kv_rows + a.doc_row[j];
-    } else {
+    if (jl >= 0 && jl < a.n_docs) {
+      len = a.doc_len[jl];
+      base = (long long)h * a.kv_rows + a.doc_row[jl];
+    } else if (j < 0 || j >= a.n_docs_index) {
       atomicCAS(a.err, 0, kErrInvalidArg);
     }
     len_s[tid] = len;
@@ -155,7 +156,7 @@ __global__ void __launch_bounds__(kWarps * 32) attend_f32_kernel(const AttendF32
   }
   // the local context up to this CTA's last row, Global RoPE at k_off + u
   const int64_t lrow0 = ((int64_t)b * a.n_kv_heads + h) * a.local_len;
-  for (int t0 = 0; t0 <= i_last; t0 += kTile) {
+  for (int t0 = 0; a.with_local && t0 <= i_last; t0 += kTile) {
     const int nk = min(kTile, i_last + 1 - t0);
     __syncthreads();
     for (int idx = tid; idx < kTile * (D / 2); idx += blockDim.x) {

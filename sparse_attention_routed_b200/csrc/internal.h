@@ -81,9 +81,12 @@ cudaError_t launch_route_tc(const RouteArgs& a, const RouteMaps& m, int sms, cud
 // Top-k per row of doc_scores, ordered (score desc, index asc).
 struct TopkArgs {
   const float* scores;  // [rows][n]
-  int32_t* idx;         // [rows][k]
+  int32_t* idx;         // [rows][out_ld] (out_ld 0: k): idx_base + the document's index in the score
+                        // row, written to columns [out_col, out_col + k)
   float* top_scores;    // [rows][k] or nullptr
   int32_t rows, n, k;
+  int32_t idx_base;     // global index of the row's first document (a shard of a larger bank), else 0
+  int32_t out_ld, out_col;
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 
@@ -107,6 +110,12 @@ struct AttendArgs {
   int32_t batch, n_q_heads, n_kv_heads, q_tokens, local_len, route_block, top_k, n_docs;
   int32_t n_splits;
   float scale_log2;         // log2(e) / sqrt(d)
+  // Memory Parallel (a bank that is one contiguous shard of a larger one): sel holds
+  // global document indices; those in [doc_lo, doc_lo + n_docs) are this bank's
+  // documents j - doc_lo, other indices in [0, n_docs_index) are skipped (another
+  // shard's), anything else raises the error flag. with_local = 0 leaves the local
+  // context out (another shard attends it). A whole bank: 0, n_docs, 1.
+  int32_t doc_lo, n_docs_index, with_local;
 };
 struct AttendMaps {
   CUtensorMap bank_k, bank_v, loc_k, loc_v;
@@ -211,9 +220,42 @@ struct AttendF32Args {
   int64_t kv_rows;
   int32_t batch, n_q_heads, n_kv_heads, q_tokens, local_len, route_block, top_k, n_docs;
   float scale_log2;         // log2(e) / sqrt(d)
+  int32_t doc_lo, n_docs_index, with_local;  // as AttendArgs
 };
 int attend_f32_rows();
 cudaError_t launch_attend_f32(const AttendF32Args& a, int head_dim, cudaStream_t s);
+
+// Memory Parallel merges. Candidates: n_parts lists of k (score, global index) per row,
+// each ordered (score desc, index asc) and with indices disjoint between parts ->
+// the first k of their union in the same order. Partials: softmax outputs and
+// log-sum-exps over disjoint key sets -> the softmax over their union.
+cudaError_t launch_merge_topk(int n_parts, int rows, int k, const float* cand_scores, const int32_t* cand_idx,
+                              int32_t* idx, float* scores, cudaStream_t s);
+cudaError_t launch_merge_partials(int n_parts, int64_t rows, int head_dim, const float* part_out,
+                                  const float* part_lse, float* out, float* lse, cudaStream_t s);
+
+// Memory Interleave. Context: the documents already in the context (ctx [rows_h][n_ctx],
+// global indices) are copied to columns [0, n_ctx) of ctx_out [rows_h][ld_out] and their
+// scores ([rows_h][n_docs], this bank's documents) set to -inf.
+cudaError_t launch_interleave_context(const int32_t* ctx, int n_ctx, int64_t rows_h, int n_docs, int doc_lo,
+                                      int n_docs_index, float* scores, int32_t* ctx_out, int ld_out, int* err,
+                                      cudaStream_t s);
+// Next routing query of a hop: q_r_out[b, h, blk] = q/|q| + (1/k) sum_j kbar_j/|kbar_j|
+// over the hop's k documents (columns [sel_col, sel_col + k) of sel [rows][Hkv][sel_ld]),
+// kbar_j = sum over document j's chunks of len_c * K_r[h, c].
+struct InterleaveUpdateArgs {
+  const float* q_r;         // [rows][Hkv][d_r] the hop's routing queries
+  const float* q_r_inv;     // [rows][Hkv]
+  const int32_t* sel;
+  int32_t sel_ld, sel_col, k;
+  const float* k_r;         // [Hkv][nch][d_r]
+  const int32_t* chunk_off; // [n_docs + 1]
+  const int32_t* chunk_len; // [nch]
+  int64_t nch;
+  int32_t rows, n_kv_heads, nblk, n_docs, doc_lo;
+  float* q_r_out;           // [B][Hkv][nblk][d_r]
+};
+cudaError_t launch_interleave_update(const InterleaveUpdateArgs& a, int route_dim, cudaStream_t s);
 
 // Pinned-host tier: one run of host-contiguous K/V rows and the staging rows it goes
 // to; jobs ascend in piece0, the index of their first piece (host_gather_piece_rows

@@ -130,6 +130,10 @@ struct msa_bank {
   // configuration
   int n_docs = 0, hkv = 0, d = 0, dr = 0, kv_loc = 0;
   bool f32 = false;  // MSA_DTYPE_F32: fp32 tensors and fp32 arithmetic (attend_f32_kernel)
+  // Memory Parallel: this bank holds documents [doc_lo, doc_lo + n_docs) of a bank of
+  // n_docs_total documents whose longest is koff_len tokens (a whole bank: 0, n_docs, max_len)
+  int doc_lo = 0, n_docs_total = 0;
+  int64_t koff_len = 0;
   double base = 10000.0;
   const void* k = nullptr;
   const void* v = nullptr;
@@ -259,7 +263,9 @@ msa_status check_query(const msa_bank* bank, const msa_query* q, int top_k, Step
     return MSA_ERR_INVALID_ARG;
   if (q->n_q_heads % bank->hkv) return MSA_ERR_INVALID_ARG;
   if (q->q_tokens > q->local_len || q->q_tokens % q->route_block) return MSA_ERR_INVALID_ARG;
-  if (top_k < 1 || top_k > bank->n_docs) return MSA_ERR_INVALID_ARG;
+  // routing ranks the bank's own documents; attention takes the selection of the whole
+  // (possibly sharded) bank
+  if (top_k < 1 || top_k > (need_attn ? bank->n_docs_total : bank->n_docs)) return MSA_ERR_INVALID_ARG;
   if (top_k > kMaxTopK) return MSA_ERR_UNSUPPORTED;
   if (!q->qr || !aligned16(q->qr)) return MSA_ERR_INVALID_ARG;
   s->B = q->batch;
@@ -387,18 +393,13 @@ msa_status ensure_gtab(msa_bank* bank, int64_t koff, int lc, cudaStream_t s) {
   return MSA_OK;
 }
 
-// The routing step. q_r / q_r_inv ([rows][Hkv][d_r], [rows][Hkv]) and score_scratch
-// ([rows][Hkv][n_docs], used when doc_scores is NULL) are the caller's scratch.
-msa_status route_into(msa_bank* bank, const msa_query* q, const StepShape& s, float* q_r, float* q_r_inv,
-                      float* score_scratch, float* doc_scores, int32_t* idx, float* top_scores, cudaStream_t st) {
+// Cosine of every routing row against every chunk and the per-document max into
+// `scores` [rows][Hkv][n_docs]: from q_r / q_r_inv ([rows][Hkv][d_r], [rows][Hkv]),
+// or, when `fuse`, with q_r formed inside the router from q->qr.
+msa_status run_router(msa_bank* bank, const msa_query* q, const StepShape& s, const float* q_r,
+                      const float* q_r_inv, float* scores, bool fuse, cudaStream_t st) {
   RouteArgs ra{};
-  const bool tc = route_tc_supported(bank->dr, s.B * s.nblk);
-  const bool fuse = !tc && !bank->f32 && s.Bq <= kRouteFuseMaxBlock;  // the router forms q_r itself
-  if (!fuse) {
-    QrArgs qa{bank->f32 ? nullptr : (const uint16_t*)q->qr, q_r, q_r_inv, s.B, bank->hkv, s.Tq, s.Bq, bank->dr,
-              bank->f32 ? (const float*)q->qr : nullptr};
-    MSA_CUDA(launch_qr_prep(qa, st));
-  } else {
+  if (fuse) {
     ra.qr = (const uint16_t*)q->qr;
     ra.q_tokens = s.Tq;
     ra.route_block = s.Bq;
@@ -406,7 +407,7 @@ msa_status route_into(msa_bank* bank, const msa_query* q, const StepShape& s, fl
   ra.chunk_off = bank->d_chunk_off;
   ra.q_r = q_r;
   ra.q_r_inv = q_r_inv;
-  ra.doc_scores = doc_scores ? doc_scores : score_scratch;
+  ra.doc_scores = scores;
   ra.nch = bank->nch;
   ra.rows = s.B * s.nblk;
   ra.n_kv_heads = bank->hkv;
@@ -414,12 +415,29 @@ msa_status route_into(msa_bank* bank, const msa_query* q, const StepShape& s, fl
   ra.route_dim = bank->dr;
   ra.err = bank->d_err;
   ra.kr_bf16 = bank->kr_bf16 ? 1 : 0;
-  if (tc) {
+  if (route_tc_supported(bank->dr, s.B * s.nblk)) {
     MSA_CUDA(launch_route_tc(ra, bank->route_maps, bank->sms, st));
   } else {
     MSA_CUDA(launch_route(ra, bank->route_maps, st));
   }
-  TopkArgs ta{ra.doc_scores, idx, top_scores, s.P, bank->n_docs, s.k};
+  return MSA_OK;
+}
+
+// The routing step. q_r / q_r_inv ([rows][Hkv][d_r], [rows][Hkv]) and score_scratch
+// ([rows][Hkv][n_docs], used when doc_scores is NULL) are the caller's scratch.
+msa_status route_into(msa_bank* bank, const msa_query* q, const StepShape& s, float* q_r, float* q_r_inv,
+                      float* score_scratch, float* doc_scores, int32_t* idx, float* top_scores, cudaStream_t st) {
+  const bool tc = route_tc_supported(bank->dr, s.B * s.nblk);
+  const bool fuse = !tc && !bank->f32 && s.Bq <= kRouteFuseMaxBlock;  // the router forms q_r itself
+  if (!fuse) {
+    QrArgs qa{bank->f32 ? nullptr : (const uint16_t*)q->qr, q_r, q_r_inv, s.B, bank->hkv, s.Tq, s.Bq, bank->dr,
+              bank->f32 ? (const float*)q->qr : nullptr};
+    MSA_CUDA(launch_qr_prep(qa, st));
+  }
+  float* scores = doc_scores ? doc_scores : score_scratch;
+  msa_status rc = run_router(bank, q, s, q_r, q_r_inv, scores, fuse, st);
+  if (rc != MSA_OK) return rc;
+  TopkArgs ta{scores, idx, top_scores, s.P, bank->n_docs, s.k, bank->doc_lo};
   MSA_CUDA(launch_topk(ta, st));
   return MSA_OK;
 }
@@ -549,8 +567,10 @@ msa_status stage_entries(msa_bank* bank, int k, size_t e0, size_t e1, std::unord
   std::vector<std::pair<int64_t, int64_t>> fresh;  // (host row of the slab's first token, doc * Hkv + head)
   for (size_t e = e0; e < e1; ++e) {
     const int h = (int)((e / k) % bank->hkv);
-    const int j = bank->h_idx[e];
-    if (j < 0 || j >= bank->n_docs) return MSA_ERR_INVALID_ARG;
+    const int jg = bank->h_idx[e];
+    const int j = jg - bank->doc_lo;  // a global index on a shard bank
+    if (jg < 0 || jg >= bank->n_docs_total) return MSA_ERR_INVALID_ARG;
+    if (j < 0 || j >= bank->n_docs) continue;  // another shard's document: nothing to stage
     const int64_t key = (int64_t)j * bank->hkv + h;
     if (slot.emplace(key, -1).second) fresh.emplace_back((int64_t)h * bank->kv_rows + bank->doc_rows[j], key);
   }
@@ -577,7 +597,8 @@ msa_status stage_entries(msa_bank* bank, int k, size_t e0, size_t e1, std::unord
   }
   for (size_t e = e0; e < e1; ++e) {
     const int h = (int)((e / k) % bank->hkv);
-    bank->h_base[e] = slot[(int64_t)bank->h_idx[e] * bank->hkv + h];
+    const int j = bank->h_idx[e] - bank->doc_lo;
+    bank->h_base[e] = (j >= 0 && j < bank->n_docs) ? slot[(int64_t)j * bank->hkv + h] : 0;
   }
   return MSA_OK;
 }
@@ -589,8 +610,13 @@ msa_status stage_entries_cached(msa_bank* bank, int k, size_t e0, size_t e1,
                                 std::unordered_map<int64_t, int64_t>& step, int& stream_rr) {
   for (size_t e = e0; e < e1; ++e) {
     const int h = (int)((e / k) % bank->hkv);
-    const int j = bank->h_idx[e];
-    if (j < 0 || j >= bank->n_docs) return MSA_ERR_INVALID_ARG;
+    const int jg = bank->h_idx[e];
+    const int j = jg - bank->doc_lo;  // a global index on a shard bank
+    if (jg < 0 || jg >= bank->n_docs_total) return MSA_ERR_INVALID_ARG;
+    if (j < 0 || j >= bank->n_docs) {  // another shard's document
+      bank->h_base[e] = 0;
+      continue;
+    }
     const int64_t key = (int64_t)j * bank->hkv + h;
     auto placed = step.find(key);
     if (placed != step.end()) {
@@ -667,9 +693,13 @@ msa_status host_fetch(msa_bank* bank, const StepShape& s, const int32_t* idx_dev
 
 // `staged`: for a pinned-host bank whose selection the caller has already staged,
 // the device table of staging rows (one per selection entry); NULL fetches here.
+bool is_shard(const msa_bank* bank) { return bank->doc_lo != 0 || bank->n_docs_total != bank->n_docs; }
+
 msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, int splits, const Workspace& w,
                        const int32_t* idx, float* out, cudaStream_t st, const int64_t* staged = nullptr,
-                       float* lse_out = nullptr) {
+                       float* lse_out = nullptr, int with_local = 1) {
+  // the prefill kernels take whole-bank selections with the local context only
+  if (s.rows > kMaxRows && !bank->f32 && (is_shard(bank) || !with_local)) return MSA_ERR_UNSUPPORTED;
   if (bank->f32) {
     AttendF32Args f{};
     f.q = (const float*)q->q;
@@ -694,6 +724,9 @@ msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, i
     f.top_k = s.k;
     f.n_docs = bank->n_docs;
     f.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)bank->d));
+    f.doc_lo = bank->doc_lo;
+    f.n_docs_index = bank->n_docs_total;
+    f.with_local = with_local;
     MSA_CUDA(launch_attend_f32(f, bank->d, st));
     return MSA_OK;
   }
@@ -753,6 +786,9 @@ msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, i
   a.n_splits = splits;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)bank->d));
   a.lse_out = lse_out;
+  a.doc_lo = bank->doc_lo;
+  a.n_docs_index = bank->n_docs_total;
+  a.with_local = with_local;
   if (tc) {
     MSA_CUDA(launch_attend_prefill_tc(a, maps, q_map, st));
   } else if (prefill) {
@@ -811,7 +847,7 @@ msa_status forward_host(msa_bank* bank, const msa_query* q, const StepShape& s, 
   Workspace w = layout(bank, sm, splits, nullptr);
   msa_status rc = ensure_workspace(bank, w.bytes, st);
   if (rc != MSA_OK) return rc;
-  if ((rc = ensure_gtab(bank, (int64_t)s.k * bank->max_len, s.Lc, st)) != MSA_OK) return rc;
+  if ((rc = ensure_gtab(bank, (int64_t)s.k * bank->koff_len, s.Lc, st)) != MSA_OK) return rc;
   w = layout(bank, sm, splits, bank->ws);
   const size_t n = (size_t)s.P * s.k;
   if ((rc = ensure_host_tier(bank, n)) != MSA_OK) return rc;
@@ -934,6 +970,8 @@ msa_status msa_bank_create(const msa_bank_config* cfg, msa_bank** out) {
   }
   b->ntok = b->doc_off[b->n_docs];
   b->nch = b->chunk_off[b->n_docs];
+  b->n_docs_total = b->n_docs;
+  b->koff_len = b->max_len;
   b->kv_rows = cfg->kv_rows > 0 ? cfg->kv_rows : b->ntok;
   b->doc_rows.resize(b->n_docs);
   for (int j = 0; j < b->n_docs; ++j) {
@@ -1087,7 +1125,7 @@ msa_status msa_reserve(msa_bank* bank, const msa_query* shape, int32_t top_k) {
   if (rc != MSA_OK) return rc;
   const int splits = choose_splits(bank, s);
   if ((rc = ensure_workspace(bank, layout(bank, s, splits, nullptr).bytes, nullptr)) != MSA_OK) return rc;
-  return ensure_gtab(bank, (int64_t)top_k * bank->max_len, s.Lc, nullptr);
+  return ensure_gtab(bank, (int64_t)top_k * bank->koff_len, s.Lc, nullptr);
 }
 
 msa_status msa_route(msa_bank* bank, const msa_query* q, int32_t top_k, float* doc_scores, int32_t* topk_idx,
@@ -1112,7 +1150,7 @@ msa_status msa_attend(msa_bank* bank, const msa_query* q, int32_t top_k, const i
   const int splits = choose_splits(bank, s);
   Workspace w = layout(bank, s, splits, nullptr);
   if ((rc = ensure_workspace(bank, w.bytes, (cudaStream_t)stream)) != MSA_OK) return rc;
-  if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->max_len, s.Lc, (cudaStream_t)stream)) != MSA_OK) return rc;
+  if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->koff_len, s.Lc, (cudaStream_t)stream)) != MSA_OK) return rc;
   w = layout(bank, s, splits, bank->ws);
   return attend_impl(bank, q, s, splits, w, topk_idx, out, (cudaStream_t)stream);
 }
@@ -1126,7 +1164,7 @@ msa_status msa_attend_lse(msa_bank* bank, const msa_query* q, int32_t top_k, con
   const int splits = choose_splits(bank, s);
   Workspace w = layout(bank, s, splits, nullptr);
   if ((rc = ensure_workspace(bank, w.bytes, (cudaStream_t)stream)) != MSA_OK) return rc;
-  if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->max_len, s.Lc, (cudaStream_t)stream)) != MSA_OK) return rc;
+  if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->koff_len, s.Lc, (cudaStream_t)stream)) != MSA_OK) return rc;
   w = layout(bank, s, splits, bank->ws);
   return attend_impl(bank, q, s, splits, w, topk_idx, out, (cudaStream_t)stream, nullptr, lse);
 }
@@ -1136,11 +1174,11 @@ msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_
   StepShape s;
   msa_status rc = check_query(bank, q, top_k, &s, true);
   if (rc != MSA_OK) return rc;
-  if (!topk_idx || !out) return MSA_ERR_INVALID_ARG;
+  if (!topk_idx || !out || top_k > bank->n_docs) return MSA_ERR_INVALID_ARG;
   const int splits = choose_splits(bank, s);
   Workspace w = layout(bank, s, splits, nullptr);
   if ((rc = ensure_workspace(bank, w.bytes, (cudaStream_t)stream)) != MSA_OK) return rc;
-  if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->max_len, s.Lc, (cudaStream_t)stream)) != MSA_OK) return rc;
+  if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->koff_len, s.Lc, (cudaStream_t)stream)) != MSA_OK) return rc;
   w = layout(bank, s, splits, bank->ws);
   cudaStream_t st = (cudaStream_t)stream;
   if (bank->kv_loc == MSA_KV_PINNED_HOST) return forward_host(bank, q, s, topk_idx, out, st);
@@ -1160,7 +1198,7 @@ msa_status backward_impl(msa_bank* bank, const msa_query* q, int32_t top_k, cons
   for (const void* p : {(const void*)d_out, (const void*)dq, (const void*)dlocal_k, (const void*)dlocal_v,
                         (const void*)dbank_k, (const void*)dbank_v})
     if (!aligned16(p)) return MSA_ERR_INVALID_ARG;
-  if (bank->kv_loc != MSA_KV_DEVICE || bank->f32) return MSA_ERR_UNSUPPORTED;
+  if (bank->kv_loc != MSA_KV_DEVICE || bank->f32 || is_shard(bank)) return MSA_ERR_UNSUPPORTED;
   cudaStream_t st = (cudaStream_t)stream;
   // workspace after the split counters: RoPE'd queries and local keys, row statistics
   const size_t qrot = align_up((size_t)s.B * s.Hq * s.Tq * bank->d * 2);
@@ -1189,7 +1227,7 @@ msa_status backward_impl(msa_bank* bank, const msa_query* q, int32_t top_k, cons
   const size_t base_ws = kCounterBytes + qrot + lrot + 2 * stats;
   if ((rc = ensure_workspace(bank, base_ws + dob + i_cnt + i_nit + i_items + i_prob + otmp + ltmp, st)) != MSA_OK)
     return rc;
-  if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->max_len, s.Lc, st)) != MSA_OK) return rc;
+  if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->koff_len, s.Lc, st)) != MSA_OK) return rc;
   uint8_t* ws = bank->ws + kCounterBytes;
   uint16_t* q_rot = reinterpret_cast<uint16_t*>(ws);
   uint16_t* l_rot = reinterpret_cast<uint16_t*>(ws + qrot);
@@ -1382,6 +1420,83 @@ msa_status msa_set_router_precision(msa_bank* bank, msa_kr_precision precision) 
 msa_status msa_check_wait_timeout(msa_bank* bank, void* stream) {
   if (!bank || !on_bank_device(bank)) return MSA_ERR_INVALID_ARG;
   MSA_CUDA(launch_wait_timeout(bank->d_err, (cudaStream_t)stream));
+  return MSA_OK;
+}
+
+msa_status msa_bank_set_shard(msa_bank* bank, int32_t doc_base, int32_t n_docs_total, int64_t max_doc_len_total) {
+  if (!bank || !on_bank_device(bank)) return MSA_ERR_INVALID_ARG;
+  if (doc_base < 0 || n_docs_total < 1 || (int64_t)doc_base + bank->n_docs > n_docs_total ||
+      max_doc_len_total < bank->max_len || max_doc_len_total >= (int64_t(1) << 30))
+    return MSA_ERR_INVALID_ARG;
+  bank->doc_lo = doc_base;
+  bank->n_docs_total = n_docs_total;
+  bank->koff_len = max_doc_len_total;
+  bank->gtab_koff = -1;  // the Global-RoPE offset follows the whole bank's longest document
+  return MSA_OK;
+}
+
+msa_status msa_attend_partial(msa_bank* bank, const msa_query* q, int32_t top_k, const int32_t* topk_idx,
+                              int32_t with_local, float* out, float* lse, void* stream) {
+  StepShape s;
+  msa_status rc = check_query(bank, q, top_k, &s, true);
+  if (rc != MSA_OK) return rc;
+  if (!topk_idx || !out || !lse || (with_local != 0 && with_local != 1)) return MSA_ERR_INVALID_ARG;
+  const int splits = choose_splits(bank, s);
+  Workspace w = layout(bank, s, splits, nullptr);
+  if ((rc = ensure_workspace(bank, w.bytes, (cudaStream_t)stream)) != MSA_OK) return rc;
+  if ((rc = ensure_gtab(bank, (int64_t)top_k * bank->koff_len, s.Lc, (cudaStream_t)stream)) != MSA_OK) return rc;
+  w = layout(bank, s, splits, bank->ws);
+  return attend_impl(bank, q, s, splits, w, topk_idx, out, (cudaStream_t)stream, nullptr, lse, with_local);
+}
+
+msa_status msa_merge_topk(int32_t n_parts, int32_t rows, int32_t top_k, const float* cand_scores,
+                          const int32_t* cand_idx, int32_t* topk_idx, float* topk_scores, void* stream) {
+  if (!cand_scores || !cand_idx || !topk_idx || n_parts < 1 || rows < 1 || top_k < 1) return MSA_ERR_INVALID_ARG;
+  if (n_parts > 64 || top_k > kMaxTopK || rows > 65535) return MSA_ERR_UNSUPPORTED;
+  return from_cuda(launch_merge_topk(n_parts, rows, top_k, cand_scores, cand_idx, topk_idx, topk_scores,
+                                     (cudaStream_t)stream));
+}
+
+msa_status msa_merge_partials(int32_t n_parts, int64_t rows, int32_t head_dim, const float* part_out,
+                              const float* part_lse, float* out, float* lse, void* stream) {
+  if (!part_out || !part_lse || !out || n_parts < 1 || rows < 1 || head_dim < 1) return MSA_ERR_INVALID_ARG;
+  if ((rows + 7) / 8 > 0x7fffffff) return MSA_ERR_UNSUPPORTED;
+  return from_cuda(launch_merge_partials(n_parts, rows, head_dim, part_out, part_lse, out, lse,
+                                         (cudaStream_t)stream));
+}
+
+msa_status msa_interleave_route(msa_bank* bank, const msa_query* q, int32_t top_k, const float* q_r_in,
+                                const int32_t* context_idx, int32_t n_ctx, int32_t* ctx_out, float* topk_scores,
+                                float* q_r_out, void* stream) {
+  StepShape s;
+  msa_status rc = check_query(bank, q, top_k, &s, false);
+  if (rc != MSA_OK) return rc;
+  if (is_shard(bank)) return MSA_ERR_UNSUPPORTED;
+  if (!ctx_out || n_ctx < 0 || (n_ctx > 0 && !context_idx) || (int64_t)n_ctx + top_k > bank->n_docs)
+    return MSA_ERR_INVALID_ARG;
+  if (q_r_in && !aligned16(q_r_in)) return MSA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  Workspace w = layout(bank, s, 1, nullptr);
+  if ((rc = ensure_workspace(bank, w.bytes, st)) != MSA_OK) return rc;
+  w = layout(bank, s, 1, bank->ws);
+  // the hop's routing query: the given one ([B, Hkv, nblk, d_r]: one "token" per block),
+  // or the block means of the routing queries on the first hop
+  QrArgs qa = q_r_in ? QrArgs{nullptr, w.q_r, w.q_r_inv, s.B, bank->hkv, s.nblk, 1, bank->dr, q_r_in}
+                     : QrArgs{bank->f32 ? nullptr : (const uint16_t*)q->qr, w.q_r, w.q_r_inv, s.B, bank->hkv,
+                              s.Tq, s.Bq, bank->dr, bank->f32 ? (const float*)q->qr : nullptr};
+  MSA_CUDA(launch_qr_prep(qa, st));
+  if ((rc = run_router(bank, q, s, w.q_r, w.q_r_inv, w.scores, false, st)) != MSA_OK) return rc;
+  const int ld = n_ctx + top_k;
+  MSA_CUDA(launch_interleave_context(context_idx, n_ctx, s.P, bank->n_docs, bank->doc_lo, bank->n_docs_total, w.scores,
+                                     ctx_out, ld, bank->d_err, st));
+  TopkArgs ta{w.scores, ctx_out, topk_scores, s.P, bank->n_docs, top_k, bank->doc_lo, ld, n_ctx};
+  MSA_CUDA(launch_topk(ta, st));
+  if (q_r_out) {
+    InterleaveUpdateArgs u{w.q_r, w.q_r_inv, ctx_out, ld, n_ctx, top_k, bank->d_kr, bank->d_chunk_off,
+                           bank->d_chunk_len, bank->nch, s.B * s.nblk, bank->hkv, s.nblk, bank->n_docs,
+                           bank->doc_lo, q_r_out};
+    MSA_CUDA(launch_interleave_update(u, bank->dr, st));
+  }
   return MSA_OK;
 }
 

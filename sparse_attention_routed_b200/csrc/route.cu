@@ -56,15 +56,17 @@ __global__ void qr_prep_kernel(QrArgs a) {
 // LO = false (the bf16 K_r variant) only Khat_hi is streamed, half the bytes,
 // and the score is Khat_hi . Qhat (the query keeps its hi + lo split).
 // Khat tiles of RITEM chunks arrive by 2-D TMA (128-byte swizzle) into a ring
-// whose slots each consumer warp owns; CTA (x, h) owns documents
-// x, x + gridDim.x, ... of KV head h, its j-th document going to warp
-// j % RWARPS, which keeps a running max per row over the document's chunks.
+// whose slots each consumer warp owns. The grid is one wave of resident CTAs;
+// CTA (x, h) owns the documents of KV head h whose first chunk lies in the x-th
+// of gridDim.x equal chunk ranges (a contiguous run of documents, found by binary
+// search in chunk_off), so every CTA streams the same number of K_r bytes to
+// within one document whatever the document lengths. Its j-th document goes to
+// warp j % RWARPS, which keeps a running max per row over the document's chunks.
 constexpr int RWARPS = 4;
 constexpr int RBUFS = 2;
 constexpr int RSLOTS = RWARPS * RBUFS;
 constexpr int RITEM = 16;            // chunks per tile (one m16 tile)
 constexpr int RNT_MAX = 2;           // n-tiles of 8 query rows per pass
-constexpr int RDOCS = 512;           // documents per CTA whose chunk ranges are staged in shared memory
 
 template <int DR, int NT>
 struct RouteShape {
@@ -74,9 +76,20 @@ struct RouteShape {
   static constexpr int SLOT_BYTES = 2 * MAT_BYTES;
   static constexpr int NR = NT * 8;
   static constexpr size_t bytes() {
-    return 1024 + (size_t)RSLOTS * SLOT_BYTES + 2 * RSLOTS * 8 + 2 * (size_t)NR * DR * 2 + 2 * RDOCS * 4;
+    return 1024 + (size_t)RSLOTS * SLOT_BYTES + 2 * RSLOTS * 8 + 2 * (size_t)NR * DR * 2;
   }
 };
+
+// First document whose first chunk is >= c (chunk_off is strictly increasing, n + 1 entries).
+__device__ __forceinline__ int first_doc_at(const int32_t* chunk_off, int n_docs, int64_t c) {
+  int lo = 0, hi = n_docs;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (chunk_off[mid] < c) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
 
 template <int DR, int NT, bool LO>
 __global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
@@ -94,8 +107,6 @@ __global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
   static_assert(SH::NR * DR * 4 <= RSLOTS * SH::SLOT_BYTES, "q_r scratch must fit in the ring");
   uint16_t* qhi = reinterpret_cast<uint16_t*>(empty + RSLOTS);  // [NR][DR] bf16
   uint16_t* qlo = qhi + NR * DR;                                // [NR][DR] bf16
-  int* c_beg = reinterpret_cast<int*>(qlo + NR * DR);           // [RDOCS] chunk range of the
-  int* c_end = c_beg + RDOCS;                                   // CTA's j-th document
   const int h = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nrows = min(NR, a.rows - row0);
@@ -107,12 +118,10 @@ __global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
     }
     fence_barrier_init();
   }
-  const int n_mine = (a.n_docs - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;  // <= RDOCS (host check)
-  for (int j = tid; j < n_mine; j += THREADS) {
-    const int doc = blockIdx.x + j * gridDim.x;
-    c_beg[j] = a.chunk_off[doc];
-    c_end[j] = a.chunk_off[doc + 1];
-  }
+  // this CTA's documents: those starting in chunks [x * nch / X, (x + 1) * nch / X)
+  const int d0 = first_doc_at(a.chunk_off, a.n_docs, (a.nch * blockIdx.x) / gridDim.x);
+  const int d1 = first_doc_at(a.chunk_off, a.n_docs, (a.nch * (blockIdx.x + 1)) / gridDim.x);
+  const int n_mine = d1 - d0;
   // ---- query rows of this pass: q_r (block mean) in fp32
   if (a.qr != nullptr) {
     const int nblk = a.q_tokens / a.route_block;
@@ -166,8 +175,8 @@ __global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
         for (int w = 0; w < RWARPS; ++w) {
           const int j = j0 + w;
           if (!ok || j >= n_mine) break;
-          const int c1 = c_end[j];
-          for (int cs = c_beg[j]; cs < c1; cs += RITEM) {
+          const int c1 = a.chunk_off[d0 + j + 1];
+          for (int cs = a.chunk_off[d0 + j]; cs < c1; cs += RITEM) {
             const int slot = w + RWARPS * (qw[w] % RBUFS), use = qw[w] / RBUFS;
             if (use > 0 && !mbar_wait_bounded(&empty[slot], (use - 1) & 1, a.err)) {
               ok = false;
@@ -211,13 +220,13 @@ __global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
   const int arow = (lane & 7) + ((lane >> 3) & 1) * 8;  // ldmatrix row of this lane
   int qc = 0;
   for (int j = warp; j < n_mine; j += RWARPS) {
-    const int doc = blockIdx.x + j * gridDim.x;
-    const int c1 = c_end[j];
+    const int doc = d0 + j;
+    const int c1 = a.chunk_off[doc + 1];
     float best[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) best[nt][0] = best[nt][1] = -INFINITY;
     bool ok = true;
-    for (int cs = c_beg[j]; cs < c1; cs += RITEM) {
+    for (int cs = a.chunk_off[doc]; cs < c1; cs += RITEM) {
       const int n = min(RITEM, c1 - cs);
       const int slot = warp + RWARPS * (qc % RBUFS), use = qc / RBUFS;
       ++qc;
@@ -277,12 +286,11 @@ cudaError_t launch_route_t(const RouteArgs& a, const RouteMaps& m, int row0, int
   const size_t smem = RouteShape<DR, NT>::bytes();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  int per_sm = (int)((227 * 1024) / (smem + 1024));
+  int per_sm = (int)((228 * 1024) / (smem + 1024));  // 228 KiB per SM, 1 KiB reserved per CTA
   per_sm = per_sm < 1 ? 1 : (per_sm > 3 ? 3 : per_sm);
-  // one wave of resident CTAs, unless a CTA would own more than RDOCS documents
+  // one wave of resident CTAs over the chunk ranges
   int gx = (sms * per_sm) / a.n_kv_heads;
   gx = gx < 1 ? 1 : (gx > a.n_docs ? a.n_docs : gx);
-  if ((a.n_docs + gx - 1) / gx > RDOCS) gx = (a.n_docs + RDOCS - 1) / RDOCS;
   if (gx > 65535) return cudaErrorInvalidValue;
   kern<<<dim3(gx, a.n_kv_heads), (RWARPS + 1) * 32, smem, s>>>(m.k_hat_hi, m.k_hat_lo, a, row0);
   return cudaGetLastError();
@@ -405,7 +413,7 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(TopkArgs a) {
       const uint32_t kj = sel_key[j];
       rank += (kj > kk) || (kj == kk && sel_idx[j] < ii);
     }
-    a.idx[(int64_t)row * a.k + rank] = ii;
+    a.idx[(int64_t)row * (a.out_ld ? a.out_ld : a.k) + a.out_col + rank] = a.idx_base + ii;
     if (a.top_scores) a.top_scores[(int64_t)row * a.k + rank] = sc[ii];
   }
 }

@@ -9,9 +9,10 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (MSA_DTYPE_BF16, MSA_DTYPE_F32, MSA_KV_DEVICE, make_query, msa_attend, msa_bank_create, msa_bank_destroy, msa_bank_info,
-               msa_build_bank, msa_forward, msa_get_device_error, msa_kv_cache_stats, msa_reserve, msa_route,
-               msa_set_kv_cache, ptr, msa_set_router_precision, msa_set_host_fetch, msa_get_host_fetch)
+from . import (MSA_DTYPE_BF16, MSA_DTYPE_F32, MSA_KV_DEVICE, make_query, msa_attend, msa_bank_create,
+               msa_bank_destroy, msa_bank_info, msa_bank_set_shard, msa_build_bank, msa_forward, msa_get_device_error,
+               msa_get_host_fetch, msa_kv_cache_stats, msa_reserve, msa_route, msa_set_host_fetch, msa_set_kv_cache,
+               msa_set_router_precision, ptr)
 
 
 class _DeviceArray:
@@ -108,6 +109,10 @@ class Bank:
                               dtype=torch.float32, device="cuda")
         msa_forward(self.handle, query, top_k, ptr(idx, torch.int32), ptr(out), _stream(stream))
         return idx, out
+
+    def set_shard(self, doc_base: int, n_docs_total: int, max_doc_len_total: int):
+        """This bank holds documents [doc_base, doc_base + n_docs) of a larger bank (Memory Parallel)."""
+        msa_bank_set_shard(self.handle, doc_base, n_docs_total, max_doc_len_total)
 
     def set_kv_cache(self, nbytes: int):
         """Device-resident slab cache of a pinned-host bank (0 turns it off)."""
