@@ -327,9 +327,8 @@ msa_status msa_route_noalloc(msa_bank* bank, const msa_query* q, int32_t top_k, 
  * other shards' (MSA_ERR_INVALID_ARG in the device error flag only outside
  * [0, n_docs_total)); top_k may reach n_docs_total for attention (routing still
  * needs top_k <= this shard's n_docs); the Global-RoPE offset is
- * top_k * max_doc_len_total, the whole bank's. Attention on a shard runs the
- * decode kernel (<= 16 rows per routing block and KV head) or, on fp32 banks, the
- * fp32 kernel: many-row bf16 steps and the backward return MSA_ERR_UNSUPPORTED.
+ * top_k * max_doc_len_total, the whole bank's. Every attention kernel takes
+ * shard selections; the backward returns MSA_ERR_UNSUPPORTED on a shard.
  * MSA_ERR_INVALID_ARG for a NULL bank, doc_base < 0, a range past n_docs_total,
  * or max_doc_len_total below this shard's longest document. Call it before the
  * steps that use it (it is not ordered with work in flight). */

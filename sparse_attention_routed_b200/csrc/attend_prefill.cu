@@ -96,13 +96,14 @@ __global__ void __launch_bounds__((PW + 1) * 32, 1)
   const int k = a.top_k;
 
   if (tid < k) {
-    const int j = a.sel[(int64_t)p * k + tid];
+    const int j = a.sel[(int64_t)p * k + tid];  // a global index on a shard bank
+    const int jl = j - a.doc_lo;
     int len = 0;
     long long base = 0;
-    if (j >= 0 && j < a.n_docs) {
-      len = a.doc_len[j];
-      base = a.sel_base ? (long long)a.sel_base[(int64_t)p * k + tid] : (long long)h * a.kv_rows + a.doc_row[j];
-    } else {
+    if (jl >= 0 && jl < a.n_docs) {
+      len = a.doc_len[jl];
+      base = a.sel_base ? (long long)a.sel_base[(int64_t)p * k + tid] : (long long)h * a.kv_rows + a.doc_row[jl];
+    } else if (j < 0 || j >= a.n_docs_index) {
       atomicCAS(a.err, 0, kErrInvalidArg);
     }
     doc_len_s[tid] = len;
@@ -123,7 +124,7 @@ __global__ void __launch_bounds__((PW + 1) * 32, 1)
       acc += (doc_len_s[d] + PT - 1) / PT;
     }
     tile_start[k] = acc;
-    tile_start[k + 1] = acc + (i_max + 1 + PT - 1) / PT;
+    tile_start[k + 1] = acc + (a.with_local ? (i_max + 1 + PT - 1) / PT : 0);
   }
   __syncthreads();
   const int T = tile_start[k + 1];

@@ -129,17 +129,43 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int k = a.top_k;
 
   if (tid < k) {
-    const int j = a.sel[(int64_t)p * k + tid];
+    const int j = a.sel[(int64_t)p * k + tid];  // a global index on a shard bank
+    const int jl = j - a.doc_lo;
     int len = 0;
     long long base = 0;
-    if (j >= 0 && j < a.n_docs) {
-      len = a.doc_len[j];
-      base = a.sel_base ? (long long)a.sel_base[(int64_t)p * k + tid] : (long long)h * a.kv_rows + a.doc_row[j];
-    } else {
+    if (jl >= 0 && jl < a.n_docs) {
+      len = a.doc_len[jl];
+      base = a.sel_base ? (long long)a.sel_base[(int64_t)p * k + tid] : (long long)h * a.kv_rows + a.doc_row[jl];
+    } else if (j < 0 || j >= a.n_docs_index) {
       atomicCAS(a.err, 0, kErrInvalidArg);
     }
     doc_len_s[tid] = len;
     doc_base_s[tid] = base;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int d = 0; d < k; ++d) {
+      tile_start[d] = acc;
+      acc += (doc_len_s[d] + TN - 1) / TN;
+    }
+    tile_start[k] = acc;
+    tile_start[k + 1] = acc + (a.with_local ? (i_max + 1 + TN - 1) / TN : 0);
+  }
+  __syncthreads();
+  const int T = tile_start[k + 1];
+  if (T == 0) {
+    // no key of this CTA's rows lives here (a shard without the local context and
+    // without any of the problem's selected documents): softmax over nothing
+    for (int idx = tid; idx < TM * TD; idx += THREADS) {
+      const int R = row0 + idx / TD;
+      const int hq = h * G + R / Bq;
+      const int t = blk * Bq + R % Bq;
+      const int64_t orow = ((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t;
+      a.out[orow * TD + idx % TD] = 0.f;
+      if (a.lse_out && idx % TD == 0) a.lse_out[orow] = -INFINITY;
+    }
+    return;
   }
   if (tid == 0) {
     // p_full collects one arrival per warp of a warpgroup; the rest one arrival each
@@ -151,17 +177,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (tid == 0) {
-    int acc = 0;
-    for (int d = 0; d < k; ++d) {
-      tile_start[d] = acc;
-      acc += (doc_len_s[d] + TN - 1) / TN;
-    }
-    tile_start[k] = acc;
-    tile_start[k + 1] = acc + (i_max + 1 + TN - 1) / TN;
-  }
-  __syncthreads();
-  const int T = tile_start[k + 1];
   const uint32_t tmem = *tmem_base_s;
   const uint32_t sbase = smem_addr(sm);
 

@@ -698,8 +698,6 @@ bool is_shard(const msa_bank* bank) { return bank->doc_lo != 0 || bank->n_docs_t
 msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, int splits, const Workspace& w,
                        const int32_t* idx, float* out, cudaStream_t st, const int64_t* staged = nullptr,
                        float* lse_out = nullptr, int with_local = 1) {
-  // the prefill kernels take whole-bank selections with the local context only
-  if (s.rows > kMaxRows && !bank->f32 && (is_shard(bank) || !with_local)) return MSA_ERR_UNSUPPORTED;
   if (bank->f32) {
     AttendF32Args f{};
     f.q = (const float*)q->q;
@@ -1269,6 +1267,8 @@ msa_status backward_impl(msa_bank* bank, const msa_query* q, int32_t top_k, cons
   a.route_block = s.Bq;
   a.top_k = s.k;
   a.n_docs = bank->n_docs;
+  a.n_docs_index = bank->n_docs;  // a whole bank (shards are refused above)
+  a.with_local = 1;
   a.n_splits = 1;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)bank->d));
   g.dout = d_out;

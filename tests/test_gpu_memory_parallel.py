@@ -10,7 +10,8 @@ C ABI, against the single bank and the oracle.
   the keys it holds); the owner's includes the local context.
 * The merge entry points alone against the oracle's merges: candidates with exact
   ties across shards, partials with empty (-inf) parts.
-* fp32 shards (1e-4) and pinned-host shards (bit for bit equal to device shards).
+* fp32 shards (1e-4), pinned-host shards (bit for bit equal to device shards), and
+  many-row steps on both prefill kernels, including CTAs that hold no key at all.
 """
 import math
 
@@ -30,6 +31,11 @@ CASES = {
     "blocks": (Workload("mp_blocks", 42, 2, 4, 2, 128, 24, 0, 160, 8, 4, 4, ragged=(100, 700)), 2),
     "d64_many_shards": (Workload("mp_d64", 43, 2, 8, 2, 64, 40, 0, 96, 2, 2, 5, ragged=(1, 400)), 5),
     "f32": (Workload("mp_f32", 44, 2, 8, 2, 128, 20, 0, 128, 1, 1, 4, ragged=(1, 500), dtype="f32"), 4),
+    # 4 heads x 64-token blocks = 256 rows per problem: the tcgen05 prefill kernel; with 3 shards
+    # and top_k 2 some problems hold none of a shard's documents (CTAs with no key at all)
+    "prefill_tc": (Workload("mp_prefill_tc", 47, 1, 8, 2, 128, 12, 0, 256, 128, 64, 2, ragged=(60, 300)), 3),
+    # 3 heads x 48-token blocks = 144 rows: the mma.sync prefill kernel, d = 64
+    "prefill_mma": (Workload("mp_prefill_mma", 48, 1, 6, 2, 64, 10, 0, 160, 96, 48, 3, ragged=(30, 400)), 2),
 }
 
 
@@ -201,8 +207,7 @@ def test_shard_limits():
     import sparse_attention_routed_b200 as msa
     from sparse_attention_routed_b200.runner import Bank
     from synth.device import bank_tensors, query_tensors
-    # a many-row (prefill) bf16 step on a shard bank is not supported; nor is the backward
-    w = Workload("mp_prefill", 46, 1, 8, 2, 128, 12, 0, 256, 128, 64, 3, ragged=(60, 300))
+    w = Workload("mp_limits", 46, 1, 8, 2, 128, 12, 0, 256, 128, 64, 3, ragged=(60, 300))
     K, V, R = bank_tensors(w)
     Q, Qr, LK, LV = query_tensors(w)
     bank = Bank(K, V, w.doc_lens(), w.rope_base)
@@ -217,10 +222,22 @@ def test_shard_limits():
     torch.cuda.synchronize()
     ix = idx.cpu().numpy()
     assert ix.min() >= 8 and ix.max() < 20
+    # the backward works on whole banks only
     out = torch.empty((1, 8, 128, 128), dtype=torch.float32, device="cuda")
+    g = [torch.zeros_like(out), torch.zeros_like(LK, dtype=torch.float32), torch.zeros_like(LV, dtype=torch.float32),
+         torch.zeros_like(K, dtype=torch.float32), torch.zeros_like(V, dtype=torch.float32)]
+    assert msa.msa_attend_backward(bank.handle, qry, w.top_k, idx.data_ptr(), out.data_ptr(),
+                                   *[t.data_ptr() for t in g], check=False) == msa.MSA_ERR_UNSUPPORTED
+    # an index outside the whole bank raises the device flag; another shard's is skipped silently
+    sel = torch.full_like(idx, 3)
     lse = torch.empty((1, 8, 128), dtype=torch.float32, device="cuda")
-    assert msa.msa_attend_partial(bank.handle, qry, w.top_k, idx.data_ptr(), 0, out.data_ptr(), lse.data_ptr(),
-                                  check=False) == msa.MSA_ERR_UNSUPPORTED
+    assert msa.msa_attend_partial(bank.handle, qry, w.top_k, sel.data_ptr(), 0, out.data_ptr(), lse.data_ptr(),
+                                  check=False) == msa.MSA_OK
     torch.cuda.synchronize()
     assert bank.device_error() == 0
+    assert torch.all(out == 0) and torch.all(torch.isinf(lse))
+    sel.fill_(25)
+    assert msa.msa_attend_partial(bank.handle, qry, w.top_k, sel.data_ptr(), 0, out.data_ptr(), lse.data_ptr(),
+                                  check=False) == msa.MSA_OK
+    assert bank.device_error() == msa.MSA_ERR_INVALID_ARG
     bank.close()
