@@ -24,6 +24,19 @@ extern "C" {
  * if the launch fails. */
 msa_status msa_selftest_exp2_poly(const float* x, float* y_poly, float* y_lib, int64_t n, void* stream);
 
+/* The document selection on its own: for each of `rows` rows of n fp32 scores
+ * (device, [rows][n], row-major), the k largest, ranked by score (descending) and,
+ * between equal scores, by index (ascending); scores compare through the IEEE
+ * total order of their bits (-0 below +0). idx[r][i] = the index in row r of
+ * rank i; top_scores[r][i] its score (or NULL). idx, top_scores: device,
+ * caller-owned [rows][k]. path 0 runs the kernel msa_route uses for this shape,
+ * 1 the block-per-row radix select (any n, k <= 64), 2 the warp-per-row select
+ * (n <= 2048, k <= 32). Asynchronous on `stream`. MSA_ERR_INVALID_ARG for a NULL
+ * scores or idx, rows < 1, n < 1, k outside [1, min(n, 64)], or a path that does
+ * not take the shape; MSA_ERR_CUDA if the launch fails. */
+msa_status msa_selftest_topk(const float* scores, int32_t rows, int32_t n, int32_t k, int32_t* idx,
+                             float* top_scores, int32_t path, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

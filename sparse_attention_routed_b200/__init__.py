@@ -90,6 +90,7 @@ def _load():
         "msa_set_router_precision": ([vp, ctypes.c_int], ctypes.c_int),
         "msa_check_wait_timeout": ([vp, vp], ctypes.c_int),
         "msa_selftest_exp2_poly": ([vp, vp, vp, i64, vp], ctypes.c_int),
+        "msa_selftest_topk": ([vp, i32, i32, i32, vp, vp, i32, vp], ctypes.c_int),
         "msa_bank_set_shard": ([vp, i32, i32, i64], ctypes.c_int),
         "msa_attend_partial": ([vp, ctypes.POINTER(msa_query), i32, vp, i32, vp, vp, vp], ctypes.c_int),
         "msa_merge_topk": ([i32, i32, i32, vp, vp, vp, vp, vp], ctypes.c_int),
@@ -125,7 +126,7 @@ EXPORTED = ["msa_bank_create", "msa_bank_destroy", "msa_build_bank", "msa_bank_i
             "msa_forward", "msa_route_noalloc", "msa_bank_set_shard", "msa_attend_partial", "msa_merge_topk",
             "msa_merge_partials", "msa_interleave_route", "msa_set_kv_cache",
             "msa_kv_cache_stats", "msa_set_host_fetch", "msa_get_host_fetch", "msa_set_router_precision", "msa_check_wait_timeout", "msa_get_device_error",
-            "msa_status_string", "msa_selftest_exp2_poly"]
+            "msa_status_string", "msa_selftest_exp2_poly", "msa_selftest_topk"]
 
 
 def msa_status_string(status: int) -> str:
@@ -352,3 +353,13 @@ def msa_selftest_exp2_poly(x: int, y_poly: int, y_lib: int, n: int, stream=0) ->
     """Self-test hook: the prefill kernel's polynomial 2^x and CUDA's exp2f over x [n] (device fp32)."""
     _check(lib().msa_selftest_exp2_poly(x or None, y_poly or None, y_lib or None, int(n), stream or None),
            "msa_selftest_exp2_poly")
+
+
+def msa_selftest_topk(scores: int, rows: int, n: int, k: int, idx: int, top_scores: int = 0, path: int = 0,
+                      stream=0, check=True) -> int:
+    """Self-test hook: top-k of [rows][n] device fp32 scores by the chosen kernel (0 auto, 1 block, 2 warp)."""
+    st = lib().msa_selftest_topk(scores or None, int(rows), int(n), int(k), idx or None, top_scores or None,
+                                 int(path), stream or None)
+    if check:
+        _check(st, "msa_selftest_topk")
+    return st

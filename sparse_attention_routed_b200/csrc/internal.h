@@ -63,6 +63,7 @@ struct RouteArgs {
   int32_t q_tokens, route_block;
   int* err;                // device error flag for expired waits, or nullptr
   int32_t kr_bf16;         // 1: read only the bf16 high part of the normalised K_r (half the bytes)
+  int32_t max_ctas_per_sm; // 0: as many as shared memory allows (3); fewer leaves room for a dependent kernel
 };
 // Largest routing block for which the router computes q_r itself.
 constexpr int kRouteFuseMaxBlock = 4;
@@ -87,8 +88,12 @@ struct TopkArgs {
   int32_t rows, n, k;
   int32_t idx_base;     // global index of the row's first document (a shard of a larger bank), else 0
   int32_t out_ld, out_col;
+  int32_t pdl;          // launch as a programmatic dependent of the previous kernel on the stream
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
+// path 0: the library's choice; 1: one 512-thread block per row (radix select, any
+// n, k <= 64); 2: one warp per row (n <= 2048, k <= 32). Same order, same output.
+cudaError_t launch_topk_path(const TopkArgs& a, int path, cudaStream_t s);
 
 // Split-KV routed attention for problems with at most 16 query rows.
 struct AttendArgs {
@@ -116,6 +121,14 @@ struct AttendArgs {
   // shard's), anything else raises the error flag. with_local = 0 leaves the local
   // context out (another shard attends it). A whole bank: 0, n_docs, 1.
   int32_t doc_lo, n_docs_index, with_local;
+  // Decode kernel: 0 cuts each problem's whole tile list (documents, then the local
+  // context) into n_splits ranges of equal cost. n > 0 gives the local context splits
+  // of its own: splits [0, n) cut the local tiles, splits [n, n_splits) the document
+  // tiles, and the CTAs of every problem's local splits come first in launch order.
+  // Those CTAs never read the selection, so with a programmatic dependent launch they
+  // run while the selection is still being made; the document CTAs wait for it.
+  int32_t n_local_splits;
+  int32_t pdl;              // launch as a programmatic dependent of the previous kernel on the stream
 };
 struct AttendMaps {
   CUtensorMap bank_k, bank_v, loc_k, loc_v;

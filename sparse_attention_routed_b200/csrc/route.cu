@@ -80,15 +80,25 @@ struct RouteShape {
   }
 };
 
-// First document whose first chunk is >= c (chunk_off is strictly increasing, n + 1 entries).
-__device__ __forceinline__ int first_doc_at(const int32_t* chunk_off, int n_docs, int64_t c) {
+// First document whose first chunk is >= c (chunk_off is strictly increasing, n + 1
+// entries, chunk_off[n] = nch >= c): a 32-ary search by one warp. Each round probes 32
+// evenly spaced entries of [lo, hi], the range the answer lies in, and keeps the span
+// between the last probe below c and the first at or above it, so 1024 documents take
+// two rounds of loads and 32K three.
+__device__ __forceinline__ int first_doc_at_warp(const int32_t* chunk_off, int n_docs, int64_t c, int lane) {
   int lo = 0, hi = n_docs;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (chunk_off[mid] < c) lo = mid + 1;
-    else hi = mid;
+  while (hi - lo > 31) {
+    const int stride = (hi - lo + 31) / 32;
+    const int q = min(lo + (lane + 1) * stride, hi);
+    const uint32_t ge = __ballot_sync(0xffffffffu, chunk_off[q] >= c);  // lane 31 probes hi: never 0
+    const int f = __ffs(ge) - 1;
+    const int new_hi = min(lo + (f + 1) * stride, hi);
+    lo = f == 0 ? lo : lo + f * stride + 1;
+    hi = new_hi;
   }
-  return lo;
+  const int q = lo + lane;
+  const uint32_t ge = __ballot_sync(0xffffffffu, q <= hi && chunk_off[q] >= c);
+  return lo + __ffs(ge) - 1;
 }
 
 template <int DR, int NT, bool LO>
@@ -97,19 +107,16 @@ __global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
                  const RouteArgs a, int row0) {
   using SH = RouteShape<DR, NT>;
   constexpr int NR = SH::NR;
-  constexpr int THREADS = (RWARPS + 1) * 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(ring + RSLOTS * SH::SLOT_BYTES);
   uint64_t* empty = full + RSLOTS;
-  // fp32 q_r rows live in the ring until the split below (before any TMA is issued)
-  float* qs = reinterpret_cast<float*>(ring);                   // [NR][DR] fp32
-  static_assert(SH::NR * DR * 4 <= RSLOTS * SH::SLOT_BYTES, "q_r scratch must fit in the ring");
   uint16_t* qhi = reinterpret_cast<uint16_t*>(empty + RSLOTS);  // [NR][DR] bf16
   uint16_t* qlo = qhi + NR * DR;                                // [NR][DR] bf16
   const int h = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nrows = min(NR, a.rows - row0);
+  __shared__ int doc_range[2];
 
   if (tid == 0) {
     for (int s = 0; s < RSLOTS; ++s) {
@@ -119,48 +126,13 @@ __global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
     fence_barrier_init();
   }
   // this CTA's documents: those starting in chunks [x * nch / X, (x + 1) * nch / X)
-  const int d0 = first_doc_at(a.chunk_off, a.n_docs, (a.nch * blockIdx.x) / gridDim.x);
-  const int d1 = first_doc_at(a.chunk_off, a.n_docs, (a.nch * (blockIdx.x + 1)) / gridDim.x);
-  const int n_mine = d1 - d0;
-  // ---- query rows of this pass: q_r (block mean) in fp32
-  if (a.qr != nullptr) {
-    const int nblk = a.q_tokens / a.route_block;
-    const float inv_b = 1.0f / (float)a.route_block;
-    for (int i = tid; i < NR * DR; i += THREADS) {
-      const int r = i / DR, dd = i % DR;
-      float v = 0.f;
-      if (r < nrows) {
-        const int row = row0 + r, bb = row / nblk, blk = row % nblk;
-        const uint16_t* src =
-            a.qr + (((int64_t)bb * a.n_kv_heads + h) * a.q_tokens + (int64_t)blk * a.route_block) * DR + dd;
-        for (int t = 0; t < a.route_block; ++t) v += __uint_as_float((uint32_t)src[(int64_t)t * DR] << 16);
-        v *= inv_b;
-      }
-      qs[i] = v;
-    }
-  } else {
-    for (int i = tid; i < NR * DR; i += THREADS) {
-      const int r = i / DR;
-      qs[i] = (r < nrows) ? a.q_r[((int64_t)(row0 + r) * a.n_kv_heads + h) * DR + (i % DR)] : 0.f;
-    }
+  if (warp < 2) {
+    const int d = first_doc_at_warp(a.chunk_off, a.n_docs, (a.nch * (blockIdx.x + warp)) / gridDim.x, lane);
+    if (lane == 0) doc_range[warp] = d;
   }
   __syncthreads();
-  // ---- normalise and split into bf16 hi + lo
-  for (int r = warp; r < NR; r += THREADS / 32) {
-    float ss = 0.f;
-    for (int i = lane; i < DR; i += 32) ss += qs[r * DR + i] * qs[r * DR + i];
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-30f);
-    for (int i = lane; i < DR; i += 32) {
-      const float x = qs[r * DR + i] * inv;
-      const __nv_bfloat16 hb = __float2bfloat16_rn(x);
-      const __nv_bfloat16 lb = __float2bfloat16_rn(x - __bfloat162float(hb));
-      qhi[r * DR + i] = *reinterpret_cast<const uint16_t*>(&hb);
-      qlo[r * DR + i] = *reinterpret_cast<const uint16_t*>(&lb);
-    }
-  }
-  __syncthreads();
+  const int d0 = doc_range[0];
+  const int n_mine = doc_range[1] - d0;
 
   if (warp == RWARPS) {
     // ------------------------------------------------------------ producer
@@ -204,6 +176,45 @@ __global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
   }
 
   // ------------------------------------------------------------ consumers
+  // q_r rows of this pass (the block mean of the routing queries, or given), normalised
+  // and split into bf16 hi + lo, while the producer's first copies are in flight.
+  for (int r = warp; r < NR; r += RWARPS) {
+    float v[DR / 32];
+#pragma unroll
+    for (int t = 0; t < DR / 32; ++t) v[t] = 0.f;
+    if (r < nrows) {
+      const int row = row0 + r;
+      if (a.qr != nullptr) {
+        const int nblk = a.q_tokens / a.route_block;
+        const int bb = row / nblk, blk = row % nblk;
+        const uint16_t* src = a.qr + (((int64_t)bb * a.n_kv_heads + h) * a.q_tokens + (int64_t)blk * a.route_block) * DR;
+        for (int t = 0; t < a.route_block; ++t)
+#pragma unroll
+          for (int u = 0; u < DR / 32; ++u) v[u] += __uint_as_float((uint32_t)src[(int64_t)t * DR + u * 32 + lane] << 16);
+        const float inv_b = 1.0f / (float)a.route_block;
+#pragma unroll
+        for (int u = 0; u < DR / 32; ++u) v[u] *= inv_b;
+      } else {
+#pragma unroll
+        for (int u = 0; u < DR / 32; ++u) v[u] = a.q_r[((int64_t)row * a.n_kv_heads + h) * DR + u * 32 + lane];
+      }
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < DR / 32; ++u) ss += v[u] * v[u];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-30f);
+#pragma unroll
+    for (int u = 0; u < DR / 32; ++u) {
+      const float x = v[u] * inv;
+      const __nv_bfloat16 hb = __float2bfloat16_rn(x);
+      const __nv_bfloat16 lb = __float2bfloat16_rn(x - __bfloat162float(hb));
+      qhi[r * DR + u * 32 + lane] = *reinterpret_cast<const uint16_t*>(&hb);
+      qlo[r * DR + u * 32 + lane] = *reinterpret_cast<const uint16_t*>(&lb);
+    }
+  }
+  named_barrier_sync(1, RWARPS * 32);
   const int g = lane >> 2, c = lane & 3;
   // B fragments (k = dims, n = rows): row 8*nt + g, dims 16ks + 2c (+1), +8.
   uint32_t bh[DR / 16][NT][2], bl[DR / 16][NT][2];
@@ -418,6 +429,133 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(TopkArgs a) {
   }
 }
 
+// ---------------------------------------------------------------- top-k, one warp per row
+// For rows of at most 32 * VPL scores and k <= 32: lane l holds scores i * 32 + l.
+// Every score becomes a distinct 64-bit key, its order key above the complement of
+// its index, so the larger key is the higher score and, between equal scores, the
+// lower index: the same order as the block kernel above. The k-th largest of the
+// 32 lane maxima, T0, bounds the k-th largest key from below (the k lanes with the
+// largest maxima each hold a key >= T0), so the k winners are among the keys >= T0.
+// When at most 64 keys pass, one warp-wide bitonic network over 64 elements sorts
+// them; otherwise the warp takes the maximum k times.
+constexpr int TOPKW_WARPS = 4;
+constexpr int TOPKW_CAP = 64;
+constexpr int TOPKW_MAX_N = 32 * 64;
+constexpr int TOPKW_MAX_K = 32;
+
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+__device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int src) {
+  const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)v, src);
+  const uint32_t hi = __shfl_sync(0xffffffffu, (uint32_t)(v >> 32), src);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+__device__ __forceinline__ uint64_t keep(uint64_t x, uint64_t p, bool keep_max) {
+  return keep_max ? (x > p ? x : p) : (x < p ? x : p);
+}
+
+// Bitonic sort of the 64 elements e = lane + 32 j (j = 0: r0, j = 1: r1), largest
+// first. An element of a block that sorts downward ((e & size) == 0) keeps the
+// larger of the pair when it is the pair's lower element.
+__device__ __forceinline__ void warp_sort64_desc(uint64_t& r0, uint64_t& r1, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 64; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride == 32) {  // size 64: one downward block; element lane is the lower one
+        const uint64_t hi = r0 > r1 ? r0 : r1, lo = r0 > r1 ? r1 : r0;
+        r0 = hi;
+        r1 = lo;
+      } else {
+        const uint64_t p0 = shfl_xor_u64(r0, stride), p1 = shfl_xor_u64(r1, stride);
+        const bool lower = (lane & stride) == 0;
+        r0 = keep(r0, p0, ((lane & size) == 0) == lower);
+        r1 = keep(r1, p1, (((lane + 32) & size) == 0) == lower);
+      }
+    }
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(TOPKW_WARPS * 32) topk_warp_kernel(TopkArgs a) {
+  __shared__ uint64_t cand[TOPKW_WARPS][TOPKW_CAP];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int row = blockIdx.x * TOPKW_WARPS + w;
+  if (row >= a.rows) return;  // a whole warp; no block-wide barrier follows
+  const float* sc = a.scores + (int64_t)row * a.n;
+  uint64_t key[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = i * 32 + lane;
+    key[i] = e < a.n ? ((uint64_t)float_order_key(sc[e]) << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)e) : 0ull;
+  }
+  uint64_t m = 0;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) m = key[i] > m ? key[i] : m;
+  // T0: the k-th largest lane maximum (bitonic sort of the 32 maxima across lanes).
+  uint64_t s = m;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1)
+      s = keep(s, shfl_xor_u64(s, stride), ((lane & size) == 0) == ((lane & stride) == 0));
+  const uint64_t t0 = shfl_u64(s, a.k - 1);
+  int c = 0;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) c += key[i] >= t0;
+  const int total = __reduce_add_sync(0xffffffffu, (unsigned)c);
+  uint64_t mine = 0;
+  if (total <= TOPKW_CAP) {
+    int off = c;  // inclusive scan of the counts, then exclusive
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, off, d);
+      if (lane >= d) off += v;
+    }
+    off -= c;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i)
+      if (key[i] >= t0) cand[w][off++] = key[i];
+    __syncwarp();
+    uint64_t r0 = lane < total ? cand[w][lane] : 0ull;
+    uint64_t r1 = lane + 32 < total ? cand[w][lane + 32] : 0ull;
+    warp_sort64_desc(r0, r1, lane);
+    mine = r0;  // element `lane` of the sorted candidates
+  } else {
+    uint64_t prev = 0;
+    for (int r = 0; r < a.k; ++r) {
+      uint64_t lm = 0;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if ((r == 0 || key[i] < prev) && key[i] > lm) lm = key[i];
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) {
+        const uint64_t o = shfl_xor_u64(lm, d);
+        lm = o > lm ? o : lm;
+      }
+      if (lane == r) mine = lm;
+      prev = lm;
+    }
+  }
+  if (lane < a.k) {
+    const int ii = (int)(0xFFFFFFFFu - (uint32_t)mine);
+    a.idx[(int64_t)row * (a.out_ld ? a.out_ld : a.k) + a.out_col + lane] = a.idx_base + ii;
+    // the score's bits, back from its order key (the key is a bijection of the bits)
+    const uint32_t ok = (uint32_t)(mine >> 32);
+    if (a.top_scores) a.top_scores[(int64_t)row * a.k + lane] = __uint_as_float(ok & 0x80000000u ? ok & 0x7FFFFFFFu : ~ok);
+  }
+}
+
+template <int VPL>
+cudaError_t launch_topk_warp_t(const TopkArgs& a, cudaStream_t s) {
+  topk_warp_kernel<VPL><<<(a.rows + TOPKW_WARPS - 1) / TOPKW_WARPS, TOPKW_WARPS * 32, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_qr_prep(const QrArgs& a, cudaStream_t s) {
@@ -434,9 +572,22 @@ cudaError_t launch_route(const RouteArgs& a, const RouteMaps& m, cudaStream_t s)
 
 int route_tile_rows() { return RITEM; }
 
-cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
-  topk_kernel<<<a.rows, TOPK_THREADS, 0, s>>>(a);
-  return cudaGetLastError();
+bool topk_warp_supported(const TopkArgs& a) { return a.k <= TOPKW_MAX_K && a.n <= TOPKW_MAX_N; }
+
+cudaError_t launch_topk_path(const TopkArgs& a, int path, cudaStream_t s) {
+  if (a.rows < 1 || a.n < 1 || a.k < 1 || a.k > a.n || a.k > TOPK_MAX) return cudaErrorInvalidValue;
+  if (path == 0) path = topk_warp_supported(a) ? 2 : 1;
+  if (path == 1) {
+    topk_kernel<<<a.rows, TOPK_THREADS, 0, s>>>(a);
+    return cudaGetLastError();
+  }
+  if (path != 2 || !topk_warp_supported(a)) return cudaErrorInvalidValue;
+  if (a.n <= 32 * 8) return launch_topk_warp_t<8>(a, s);
+  if (a.n <= 32 * 16) return launch_topk_warp_t<16>(a, s);
+  if (a.n <= 32 * 32) return launch_topk_warp_t<32>(a, s);
+  return launch_topk_warp_t<64>(a, s);
 }
+
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) { return launch_topk_path(a, 0, s); }
 
 }  // namespace msa

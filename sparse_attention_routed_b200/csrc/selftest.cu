@@ -62,3 +62,21 @@ extern "C" msa_status msa_selftest_exp2_poly(const float* x, float* y_poly, floa
   msa::exp2_poly_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_lib, n);
   return cudaGetLastError() == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------
+// Self-test of the document selection: either top-k kernel on caller scores.
+extern "C" msa_status msa_selftest_topk(const float* scores, int32_t rows, int32_t n, int32_t k, int32_t* idx,
+                                        float* top_scores, int32_t path, void* stream) {
+  if (!scores || !idx || rows < 1 || n < 1 || k < 1 || k > n || k > 64 || path < 0 || path > 2)
+    return MSA_ERR_INVALID_ARG;
+  msa::TopkArgs a{};
+  a.scores = scores;
+  a.idx = idx;
+  a.top_scores = top_scores;
+  a.rows = rows;
+  a.n = n;
+  a.k = k;
+  const cudaError_t e = msa::launch_topk_path(a, path, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorInvalidValue) return MSA_ERR_INVALID_ARG;
+  return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+}
