@@ -404,13 +404,15 @@ def job_throughput(world: int, units_per_step: float, steps: int, total_ms: floa
 
 def measure_device(args, wname: str, n: int, warmup: int, world: int, rank: int, local: int,
                    with_e2e: bool = True):
-    """Times n steps (route + attend through the C ABI) of a device-resident workload
-    after `warmup` untimed ones; returns the JSON line on rank 0 (None elsewhere)."""
+    """Times n steps (msa_forward: route + attend through the C ABI) of a device-resident
+    workload after `warmup` untimed ones, then n more as msa_route + msa_attend with an
+    event between them for the two phases' times; returns the JSON line on rank 0
+    (None elsewhere)."""
     import torch
     import torch.distributed as dist
 
     import synth
-    from sparse_attention_routed_b200 import MSA_KR_BF16, msa_attend, msa_route, ptr
+    from sparse_attention_routed_b200 import MSA_KR_BF16, msa_attend, msa_forward, msa_route, ptr
     from sparse_attention_routed_b200.runner import Bank
     from synth.device import bank_tensors, query_tensors
 
@@ -445,11 +447,12 @@ def measure_device(args, wname: str, n: int, warmup: int, world: int, rank: int,
     sh = stream.cuda_stream
 
     def step():
-        msa_route(bank.handle, qry, k, 0, idx.data_ptr(), 0, sh)
-        msa_attend(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
+        msa_forward(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
 
     for _ in range(max(3, warmup)):
         step()
+        msa_route(bank.handle, qry, k, 0, idx.data_ptr(), 0, sh)
+        msa_attend(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
     torch.cuda.synchronize()
     assert bank.device_error() == 0
 
@@ -481,12 +484,15 @@ def measure_device(args, wname: str, n: int, warmup: int, world: int, rank: int,
     clocks.mark(True)
     t_begin.record(stream)
     for i in range(n):
+        step()
+    t_end.record(stream)
+    # the two phases on their own (not the headline): the router + top-k, then the attention
+    for i in range(n):
         ev[i][0].record(stream)
         msa_route(bank.handle, qry, k, 0, idx.data_ptr(), 0, sh)
         ev[i][1].record(stream)
         msa_attend(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
         ev[i][2].record(stream)
-    t_end.record(stream)
     torch.cuda.synchronize()
     clocks.mark(False)
     if world > 1:
@@ -540,8 +546,7 @@ def measure_device(args, wname: str, n: int, warmup: int, world: int, rank: int,
                 stream.wait_event(ev_in[si])
                 if i >= 2:
                     stream.wait_event(ev_out[si])               # step i-2's result has left this set
-                msa_route(bank.handle, qy, k, 0, ix_d.data_ptr(), 0, sh)
-                msa_attend(bank.handle, qy, k, ix_d.data_ptr(), o_d.data_ptr(), sh)
+                msa_forward(bank.handle, qy, k, ix_d.data_ptr(), o_d.data_ptr(), sh)
                 ev_comp[si].record(stream)
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(ev_comp[si])

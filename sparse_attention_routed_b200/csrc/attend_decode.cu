@@ -11,6 +11,10 @@
 //    of TILE keys of each selected document followed by the local tiles up to
 //    the last query's position. The list is cut into n_splits equal ranges,
 //    one CTA each (split-KV), so ragged documents balance by construction.
+//    With n_local_splits > 0 the local tiles get splits of their own, whose
+//    CTAs never read the selection: launched as a programmatic dependent of the
+//    top-k, every CTA sets up while routing finishes, the local ones go on with
+//    their tiles, and only the document CTAs wait for the selection.
 //  * One producer lane streams K and V tiles with 2-D TMA loads (128-byte
 //    swizzle, evict-first L2 policy) into a ring of WARPS x BUFS slots; consumer
 //    warp w owns slots w, w + WARPS, ... and takes relative tiles w, w + WARPS, ...
@@ -23,6 +27,7 @@
 //    to finish (a wrapping atomic counter) merges all splits into the output.
 #include "common.cuh"
 #include "internal.h"
+#include "pdl.cuh"
 
 namespace msa {
 namespace {
@@ -122,9 +127,13 @@ __global__ void __launch_bounds__(S::THREADS, S::MINB)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int p = blockIdx.y, split = blockIdx.x;
   const int G = a.n_q_heads / a.n_kv_heads;
   const int nblk = a.q_tokens / a.route_block;
+  // CTA -> (problem, split), problem after problem, so that the local tiles (Global RoPE
+  // in shared memory) spread evenly over the waves.
+  const int nls = a.n_local_splits;
+  const int p = blockIdx.x / a.n_splits, split = blockIdx.x % a.n_splits;
+  const bool local_cta = split < nls;
   const int h = p % a.n_kv_heads;
   const int blk = (p / a.n_kv_heads) % nblk;
   const int b = p / (a.n_kv_heads * nblk);
@@ -133,7 +142,15 @@ __global__ void __launch_bounds__(S::THREADS, S::MINB)
   const int i_max = i_first + a.route_block - 1;
   const int k = a.top_k;
 
-  if (tid < k) {
+  if (tid == 0) {
+    for (int s = 0; s < S::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    fence_barrier_init();
+  }
+  if (!local_cta) pdl_wait();  // the selection comes from the top-k
+  if (tid < k && !local_cta) {
     const int j = a.sel[(int64_t)p * k + tid];  // a global index on a shard bank
     const int jl = j - a.doc_lo;
     int len = 0;
@@ -147,33 +164,36 @@ __global__ void __launch_bounds__(S::THREADS, S::MINB)
     doc_len_s[tid] = len;
     doc_base_s[tid] = base;
   }
-  if (tid == 0) {
-    for (int s = 0; s < S::STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    fence_barrier_init();
-  }
   __syncthreads();
+  const int local_tiles = a.with_local ? (i_max + 1 + TILE - 1) / TILE : 0;
   if (tid == 0) {
+    // A local CTA sees a list of local tiles only; a document CTA with splits of
+    // its own for the local context sees the document tiles only.
     int acc = 0;
     for (int d = 0; d < k; ++d) {
       tile_start[d] = acc;
-      acc += (doc_len_s[d] + TILE - 1) / TILE;
+      acc += local_cta ? 0 : (doc_len_s[d] + TILE - 1) / TILE;
     }
     tile_start[k] = acc;
-    tile_start[k + 1] = acc + (a.with_local ? (i_max + 1 + TILE - 1) / TILE : 0);
+    tile_start[k + 1] = acc + (local_cta || nls == 0 ? local_tiles : 0);
   }
   __syncthreads();
-  // split boundaries in cost units: bank tiles cost 1, local tiles LOCAL_W
   const int Tb = tile_start[k], T = tile_start[k + 1];
-  constexpr int LW = MSA_DECODE_LOCAL_W;
-  const long long cost = (long long)Tb + (long long)LW * (T - Tb);
-  auto tile_at = [&](long long cpos) -> int {
-    return cpos <= Tb ? (int)cpos : Tb + (int)((cpos - Tb + LW - 1) / LW);
-  };
-  const int t0 = tile_at((cost * split) / a.n_splits);
-  const int t1 = tile_at((cost * (split + 1)) / a.n_splits);
+  int t0, t1;
+  if (nls > 0) {
+    const int s0 = local_cta ? split : split - nls, ns = local_cta ? nls : a.n_splits - nls;
+    t0 = (int)(((long long)T * s0) / ns);
+    t1 = (int)(((long long)T * (s0 + 1)) / ns);
+  } else {
+    // split boundaries in cost units: bank tiles cost 1, local tiles LOCAL_W
+    constexpr int LW = MSA_DECODE_LOCAL_W;
+    const long long cost = (long long)Tb + (long long)LW * (T - Tb);
+    auto tile_at = [&](long long cpos) -> int {
+      return cpos <= Tb ? (int)cpos : Tb + (int)((cpos - Tb + LW - 1) / LW);
+    };
+    t0 = tile_at((cost * split) / a.n_splits);
+    t1 = tile_at((cost * (split + 1)) / a.n_splits);
+  }
   const int ntiles = t1 - t0;
 
   if (warp == WARPS) {
@@ -503,16 +523,21 @@ __global__ void __launch_bounds__(S::THREADS, S::MINB)
   if (!*flag_s) return;
   __threadfence();
   const int nS = a.n_splits;
-  const float* pm = a.part_ml + (int64_t)p * nS * rows * 2;
+  // Every split's (m, l) of every row into shared memory at once (the ring is free by
+  // now): one round of loads instead of two dependent chains of nS per row.
+  const float2* pm = reinterpret_cast<const float2*>(a.part_ml) + (int64_t)p * nS * rows;
+  float2* ml_s = reinterpret_cast<float2*>(ring);  // [nS][rows]
+  for (int i = tid; i < nS * rows; i += CT) ml_s[i] = __ldcg(pm + i);
+  named_barrier_sync(1, CT);
   for (int i = tid; i < rows; i += CT) {
     float M = -INFINITY;
-    for (int sp = 0; sp < nS; ++sp) M = fmaxf(M, __ldcg(pm + (sp * rows + i) * 2));
+    for (int sp = 0; sp < nS; ++sp) M = fmaxf(M, ml_s[sp * rows + i].x);
     float L = 0.f;
     for (int sp = 0; sp < nS; ++sp) {
-      const float m = __ldcg(pm + (sp * rows + i) * 2);
+      const float m = ml_s[sp * rows + i].x;
       const float f = (m == -INFINITY) ? 0.f : exp2f(m - M);
       wgt_s[sp * kRowsMax + i] = f;
-      L += f * __ldcg(pm + (sp * rows + i) * 2 + 1);
+      L += f * ml_s[sp * rows + i].y;
     }
     const float inv = (L > 0.f) ? 1.0f / L : 0.f;
     for (int sp = 0; sp < nS; ++sp) wgt_s[sp * kRowsMax + i] *= inv;
@@ -521,15 +546,52 @@ __global__ void __launch_bounds__(S::THREADS, S::MINB)
           L > 0.f ? (M + log2f(L)) * 0.693147180559945309f : -INFINITY;
   }
   named_barrier_sync(1, CT);
-  const float* po = a.part_o + (int64_t)p * nS * rows * D;
-  for (int idx = tid; idx < rows * D; idx += CT) {
-    const int r = idx / D, dim = idx % D;
-    float o = 0.f;
-#pragma unroll 8
-    for (int sp = 0; sp < nS; ++sp) o += wgt_s[sp * kRowsMax + r] * __ldcg(po + ((int64_t)sp * rows + r) * D + dim);
-    const int t = blk * a.route_block + r / G;
-    const int hq = h * G + r % G;
-    a.out[(((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t) * D + dim] = o;
+  // Outputs in items of 4 dims: a thread owns up to 4 items and keeps 4 splits x 4 items
+  // of loads in flight; each output still sums the splits in order, split 0 first.
+  constexpr int D4 = D / 4;
+  const int n4 = rows * D4;
+  const float4* po = reinterpret_cast<const float4*>(a.part_o) + (int64_t)p * nS * n4;
+  for (int base = 0; base < n4; base += 4 * CT) {
+    float4 o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp0 = 0; sp0 < nS; sp0 += 4) {
+      float4 x[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int item = base + j * CT + tid;
+          x[u][j] = (sp0 + u < nS && item < n4) ? __ldcg(po + (int64_t)(sp0 + u) * n4 + item)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (sp0 + u >= nS) break;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int item = base + j * CT + tid;
+          const float w = wgt_s[(sp0 + u) * kRowsMax + (item < n4 ? item / D4 : 0)];
+          o[j].x += w * x[u][j].x;
+          o[j].y += w * x[u][j].y;
+          o[j].z += w * x[u][j].z;
+          o[j].w += w * x[u][j].w;
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int item = base + j * CT + tid;
+      if (item >= n4) continue;
+      const int r = item / D4, dim = (item % D4) * 4;
+      const int t = blk * a.route_block + r / G;
+      const int hq = h * G + r % G;
+      float* dst = a.out + (((int64_t)b * a.n_q_heads + hq) * a.q_tokens + t) * D + dim;
+      dst[0] = o[j].x;
+      dst[1] = o[j].y;
+      dst[2] = o[j].z;
+      dst[3] = o[j].w;
+    }
   }
 }
 
@@ -540,9 +602,10 @@ cudaError_t launch_decode_t(const AttendArgs& a, const AttendMaps& m, cudaStream
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int nblk = a.q_tokens / a.route_block;
-  dim3 grid(a.n_splits, a.batch * nblk * a.n_kv_heads);
-  kern<<<grid, S::THREADS, smem, s>>>(m.bank_k, m.bank_v, m.loc_k, m.loc_v, a);
-  return cudaGetLastError();
+  const long long ctas = (long long)a.n_splits * a.batch * nblk * a.n_kv_heads;
+  if (ctas > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  return launch_maybe_pdl(kern, dim3((unsigned)ctas), dim3(S::THREADS), smem, s, a.pdl != 0, m.bank_k, m.bank_v,
+                          m.loc_k, m.loc_v, a);
 }
 
 }  // namespace
@@ -560,6 +623,8 @@ int attend_ctas_per_sm(int head_dim) {
 cudaError_t launch_attend_decode(const AttendArgs& a, const AttendMaps& m, int head_dim, cudaStream_t s) {
   const int rows = (a.n_q_heads / a.n_kv_heads) * a.route_block;
   if (a.n_splits < 1 || a.n_splits > kMaxSplits || rows > kRowsMax) return cudaErrorInvalidValue;
+  if (a.n_local_splits < 0 || a.n_local_splits >= a.n_splits || (a.n_local_splits > 0 && !a.with_local))
+    return cudaErrorInvalidValue;
   if (head_dim == 128) {
     if (rows <= 8) return launch_decode_t<Decode<128>, 1>(a, m, s);
     return launch_decode_t<Decode<128>, 2>(a, m, s);

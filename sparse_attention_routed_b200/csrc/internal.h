@@ -63,7 +63,6 @@ struct RouteArgs {
   int32_t q_tokens, route_block;
   int* err;                // device error flag for expired waits, or nullptr
   int32_t kr_bf16;         // 1: read only the bf16 high part of the normalised K_r (half the bytes)
-  int32_t max_ctas_per_sm; // 0: as many as shared memory allows (3); fewer leaves room for a dependent kernel
 };
 // Largest routing block for which the router computes q_r itself.
 constexpr int kRouteFuseMaxBlock = 4;
@@ -91,8 +90,9 @@ struct TopkArgs {
   int32_t pdl;          // launch as a programmatic dependent of the previous kernel on the stream
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
-// path 0: the library's choice; 1: one 512-thread block per row (radix select, any
-// n, k <= 64); 2: one warp per row (n <= 2048, k <= 32). Same order, same output.
+// path 0: the library's choice (the warp kernel for n <= 2048 and k <= 20); 1: one
+// 512-thread block per row (radix select, any n, k <= 64); 2: one warp per row
+// (n <= 2048, k <= 32). Same order, same output.
 cudaError_t launch_topk_path(const TopkArgs& a, int path, cudaStream_t s);
 
 // Split-KV routed attention for problems with at most 16 query rows.
@@ -124,9 +124,9 @@ struct AttendArgs {
   // Decode kernel: 0 cuts each problem's whole tile list (documents, then the local
   // context) into n_splits ranges of equal cost. n > 0 gives the local context splits
   // of its own: splits [0, n) cut the local tiles, splits [n, n_splits) the document
-  // tiles, and the CTAs of every problem's local splits come first in launch order.
-  // Those CTAs never read the selection, so with a programmatic dependent launch they
-  // run while the selection is still being made; the document CTAs wait for it.
+  // tiles. Those CTAs never read the selection, so with a programmatic dependent
+  // launch (pdl) they run while the selection is still being made; the document CTAs
+  // wait for it.
   int32_t n_local_splits;
   int32_t pdl;              // launch as a programmatic dependent of the previous kernel on the stream
 };

@@ -425,10 +425,15 @@ msa_status run_router(msa_bank* bank, const msa_query* q, const StepShape& s, co
 
 // The routing step. q_r / q_r_inv ([rows][Hkv][d_r], [rows][Hkv]) and score_scratch
 // ([rows][Hkv][n_docs], used when doc_scores is NULL) are the caller's scratch.
+// `overlap` (the decode router, with the decode attention queued right behind it on
+// `st`): the top-k is a programmatic dependent of the router, so that it and then the
+// attention (a programmatic dependent of the top-k) set up while the router finishes.
 msa_status route_into(msa_bank* bank, const msa_query* q, const StepShape& s, float* q_r, float* q_r_inv,
-                      float* score_scratch, float* doc_scores, int32_t* idx, float* top_scores, cudaStream_t st) {
+                      float* score_scratch, float* doc_scores, int32_t* idx, float* top_scores, cudaStream_t st,
+                      bool overlap = false) {
   const bool tc = route_tc_supported(bank->dr, s.B * s.nblk);
   const bool fuse = !tc && !bank->f32 && s.Bq <= kRouteFuseMaxBlock;  // the router forms q_r itself
+  overlap = overlap && fuse;
   if (!fuse) {
     QrArgs qa{bank->f32 ? nullptr : (const uint16_t*)q->qr, q_r, q_r_inv, s.B, bank->hkv, s.Tq, s.Bq, bank->dr,
               bank->f32 ? (const float*)q->qr : nullptr};
@@ -438,13 +443,14 @@ msa_status route_into(msa_bank* bank, const msa_query* q, const StepShape& s, fl
   msa_status rc = run_router(bank, q, s, q_r, q_r_inv, scores, fuse, st);
   if (rc != MSA_OK) return rc;
   TopkArgs ta{scores, idx, top_scores, s.P, bank->n_docs, s.k, bank->doc_lo};
+  ta.pdl = overlap ? 1 : 0;
   MSA_CUDA(launch_topk(ta, st));
   return MSA_OK;
 }
 
 msa_status route_impl(msa_bank* bank, const msa_query* q, const StepShape& s, const Workspace& w,
-                      float* doc_scores, int32_t* idx, float* top_scores, cudaStream_t st) {
-  return route_into(bank, q, s, w.q_r, w.q_r_inv, w.scores, doc_scores, idx, top_scores, st);
+                      float* doc_scores, int32_t* idx, float* top_scores, cudaStream_t st, bool overlap = false) {
+  return route_into(bank, q, s, w.q_r, w.q_r_inv, w.scores, doc_scores, idx, top_scores, st, overlap);
 }
 
 // Pinned-host tier ("MSA (Memory Sparse Attention)", robocikowo.com, Komponenty:
@@ -697,7 +703,7 @@ bool is_shard(const msa_bank* bank) { return bank->doc_lo != 0 || bank->n_docs_t
 
 msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, int splits, const Workspace& w,
                        const int32_t* idx, float* out, cudaStream_t st, const int64_t* staged = nullptr,
-                       float* lse_out = nullptr, int with_local = 1) {
+                       float* lse_out = nullptr, int with_local = 1, bool overlap = false) {
   if (bank->f32) {
     AttendF32Args f{};
     f.q = (const float*)q->q;
@@ -787,6 +793,16 @@ msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, i
   a.doc_lo = bank->doc_lo;
   a.n_docs_index = bank->n_docs_total;
   a.with_local = with_local;
+  if (!prefill && with_local && splits >= 2) {
+    // the local context's own splits, in proportion to its cost (a local tile costs
+    // about two bank tiles: Global RoPE in shared memory), at least one on each side
+    const int tile = attend_tile_rows();
+    const double doc_tiles = (double)s.k * std::ceil((double)bank->ntok / bank->n_docs / tile);
+    const double loc_cost = 2.0 * (double)((s.Lc + tile - 1) / tile);
+    const int nls = (int)std::lround(splits * loc_cost / (loc_cost + doc_tiles));
+    a.n_local_splits = std::max(1, std::min(splits - 1, nls));
+    a.pdl = overlap ? 1 : 0;
+  }
   if (tc) {
     MSA_CUDA(launch_attend_prefill_tc(a, maps, q_map, st));
   } else if (prefill) {
@@ -1180,8 +1196,11 @@ msa_status msa_forward(msa_bank* bank, const msa_query* q, int32_t top_k, int32_
   w = layout(bank, s, splits, bank->ws);
   cudaStream_t st = (cudaStream_t)stream;
   if (bank->kv_loc == MSA_KV_PINNED_HOST) return forward_host(bank, q, s, topk_idx, out, st);
-  if ((rc = route_impl(bank, q, s, w, nullptr, topk_idx, nullptr, st)) != MSA_OK) return rc;
-  return attend_impl(bank, q, s, splits, w, topk_idx, out, st);
+  // decode: the attention's local-context CTAs run beside the routing (programmatic
+  // dependent launches); the steps and their results are those of msa_route + msa_attend
+  const bool overlap = s.rows <= kMaxRows && !bank->f32;
+  if ((rc = route_impl(bank, q, s, w, nullptr, topk_idx, nullptr, st, overlap)) != MSA_OK) return rc;
+  return attend_impl(bank, q, s, splits, w, topk_idx, out, st, nullptr, nullptr, 1, overlap);
 }
 
 namespace {

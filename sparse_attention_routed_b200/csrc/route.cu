@@ -7,6 +7,7 @@
 //   Top-k: robocikowo.com, Hiperparametry (Top-k documents).
 #include "common.cuh"
 #include "internal.h"
+#include "pdl.cuh"
 
 namespace msa {
 namespace {
@@ -117,6 +118,9 @@ __global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nrows = min(NR, a.rows - row0);
   __shared__ int doc_range[2];
+  // A programmatic dependent (the top-k) may launch and set up at once; it waits for
+  // this grid to finish before it reads the scores.
+  pdl_launch_dependents();
 
   if (tid == 0) {
     for (int s = 0; s < RSLOTS; ++s) {
@@ -337,6 +341,8 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(TopkArgs a) {
   const int row = blockIdx.x;
   const float* sc = a.scores + (int64_t)row * a.n;
   const int tid = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();  // the scores come from the router
 
   uint32_t prefix = 0, mask = 0, remaining = (uint32_t)a.k;
   for (int shift = 24; shift >= 0; shift -= 8) {
@@ -442,6 +448,9 @@ constexpr int TOPKW_WARPS = 4;
 constexpr int TOPKW_CAP = 64;
 constexpr int TOPKW_MAX_N = 32 * 64;
 constexpr int TOPKW_MAX_K = 32;
+// Taken by default up to k = 20: for independent scores about 30 keys then pass T0, while
+// at k = 32 (T0 the smallest lane maximum) it is over 100 and the slow path runs.
+constexpr int TOPKW_AUTO_MAX_K = 20;
 
 __device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
   const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
@@ -485,7 +494,9 @@ __global__ void __launch_bounds__(TOPKW_WARPS * 32) topk_warp_kernel(TopkArgs a)
   __shared__ uint64_t cand[TOPKW_WARPS][TOPKW_CAP];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int row = blockIdx.x * TOPKW_WARPS + w;
+  pdl_launch_dependents();
   if (row >= a.rows) return;  // a whole warp; no block-wide barrier follows
+  pdl_wait();  // the scores come from the router
   const float* sc = a.scores + (int64_t)row * a.n;
   uint64_t key[VPL];
 #pragma unroll
@@ -552,8 +563,8 @@ __global__ void __launch_bounds__(TOPKW_WARPS * 32) topk_warp_kernel(TopkArgs a)
 
 template <int VPL>
 cudaError_t launch_topk_warp_t(const TopkArgs& a, cudaStream_t s) {
-  topk_warp_kernel<VPL><<<(a.rows + TOPKW_WARPS - 1) / TOPKW_WARPS, TOPKW_WARPS * 32, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_maybe_pdl(topk_warp_kernel<VPL>, dim3((a.rows + TOPKW_WARPS - 1) / TOPKW_WARPS),
+                          dim3(TOPKW_WARPS * 32), 0, s, a.pdl != 0, a);
 }
 
 }  // namespace
@@ -576,11 +587,8 @@ bool topk_warp_supported(const TopkArgs& a) { return a.k <= TOPKW_MAX_K && a.n <
 
 cudaError_t launch_topk_path(const TopkArgs& a, int path, cudaStream_t s) {
   if (a.rows < 1 || a.n < 1 || a.k < 1 || a.k > a.n || a.k > TOPK_MAX) return cudaErrorInvalidValue;
-  if (path == 0) path = topk_warp_supported(a) ? 2 : 1;
-  if (path == 1) {
-    topk_kernel<<<a.rows, TOPK_THREADS, 0, s>>>(a);
-    return cudaGetLastError();
-  }
+  if (path == 0) path = topk_warp_supported(a) && a.k <= TOPKW_AUTO_MAX_K ? 2 : 1;
+  if (path == 1) return launch_maybe_pdl(topk_kernel, dim3(a.rows), dim3(TOPK_THREADS), 0, s, a.pdl != 0, a);
   if (path != 2 || !topk_warp_supported(a)) return cudaErrorInvalidValue;
   if (a.n <= 32 * 8) return launch_topk_warp_t<8>(a, s);
   if (a.n <= 32 * 16) return launch_topk_warp_t<16>(a, s);
