@@ -353,7 +353,7 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- ours
 KERNEL_SOURCES = {
-    "attend_decode": ["attend_decode.cu", "common.cuh"],
+    "attend_decode": ["attend_decode.cu", "common.cuh", "pdl.cuh"],
     "attend_prefill_tc": ["attend_prefill_tc.cu", "common.cuh"],
 }
 
