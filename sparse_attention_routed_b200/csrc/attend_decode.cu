@@ -301,27 +301,43 @@ __global__ void __launch_bounds__(S::THREADS, S::MINB)
       for (int e = 0; e < 4; ++e) acc[md][nt][e] = 0.f;
   }
 
+  // Global RoPE of a local tile: lane l rotates the 8 pairs of 16-byte chunk l % PC
+  // (PC = D / 16 chunks per half row) of keys l / PC + STEP * i, STEP = 32 / PC.
+  constexpr int kPairChunks = D / 16;
+  constexpr int kStep = 32 / kPairChunks;
+  const int rch = lane % kPairChunks, rr0 = lane / kPairChunks;
   int hint = 0;
   for (int n = warp; n < ntiles; n += WARPS) {
     int stage, use;
     slot_of<S>(n, stage, use);
-    if (!mbar_wait_bounded(&full[stage], use & 1, a.err)) break;
     const TileRef tr = locate(tile_start, k, t0 + n, hint);
     hint = tr.di;
-    uint8_t* kt = ring + stage * S::STAGE_BYTES;
-    uint8_t* vt = kt + S::TILE_BYTES;
     const bool local = tr.di >= k;
     const int key0 = tr.tt * TILE;
+    // the lane's first key's (cos, sin) from the table (fetched into L1 before the wait);
+    // the later keys' by rotating STEP positions at a time (gstep)
+    const float4* cs_src = reinterpret_cast<const float4*>(a.gtab + (int64_t)(key0 + rr0) * (D / 2) + rch * 8);
+    if (local && key0 + rr0 < a.local_len) asm volatile("prefetch.global.L1 [%0];" ::"l"(cs_src));
+    if (!mbar_wait_bounded(&full[stage], use & 1, a.err)) break;
+    uint8_t* kt = ring + stage * S::STAGE_BYTES;
+    uint8_t* vt = kt + S::TILE_BYTES;
     const int nvalid = local ? 0 : min(TILE, doc_len_s[tr.di] - key0);
 
     if (local) {
       // Global RoPE of the local keys, in shared memory: pair (i, i + D/2)
       // lives in the same swizzled slot of chunk i/8 and chunk (i + D/2)/8.
-      constexpr int kPairChunks = D / 16;  // 16-byte chunks per half row
-      for (int unit = lane; unit < TILE * kPairChunks; unit += 32) {
-        const int r = unit / kPairChunks, ch = unit % kPairChunks;
+      float4 st[4], cs[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) st[j] = __ldg(reinterpret_cast<const float4*>(a.gstep + rch * 8) + j);
+      if (key0 + rr0 < a.local_len) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cs[j] = __ldg(cs_src + j);
+      }
+#pragma unroll 1
+      for (int it = 0; it < TILE / kStep; ++it) {
+        const int r = rr0 + kStep * it, ch = rch;
         const int u = key0 + r;
-        if (u >= a.local_len) continue;
+        if (u >= a.local_len) break;
         uint8_t* px;
         uint8_t* py;
         if constexpr (D == 128) {
@@ -333,14 +349,15 @@ __global__ void __launch_bounds__(S::THREADS, S::MINB)
         }
         uint4 xv = *reinterpret_cast<uint4*>(px), yv = *reinterpret_cast<uint4*>(py);
         uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w}, ys[4] = {yv.x, yv.y, yv.z, yv.w};
-        const float4* cs = reinterpret_cast<const float4*>(a.gtab + (int64_t)u * (D / 2) + ch * 8);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float4 t4 = __ldg(cs + j);
+          const float4 t4 = cs[j];
           const float x0 = bf16_lo(xs[j]), x1 = bf16_hi(xs[j]);
           const float y0 = bf16_lo(ys[j]), y1 = bf16_hi(ys[j]);
           xs[j] = pack_bf16(x0 * t4.x - y0 * t4.y, x1 * t4.z - y1 * t4.w);
           ys[j] = pack_bf16(y0 * t4.x + x0 * t4.y, y1 * t4.z + x1 * t4.w);
+          cs[j] = make_float4(t4.x * st[j].x - t4.y * st[j].y, t4.y * st[j].x + t4.x * st[j].y,
+                              t4.z * st[j].z - t4.w * st[j].w, t4.w * st[j].z + t4.z * st[j].w);
         }
         *reinterpret_cast<uint4*>(px) = make_uint4(xs[0], xs[1], xs[2], xs[3]);
         *reinterpret_cast<uint4*>(py) = make_uint4(ys[0], ys[1], ys[2], ys[3]);

@@ -104,6 +104,7 @@ struct AttendArgs {
                             // K/V tensor maps (host tier: the device staging pool)
   const int32_t* doc_len;   // [n_docs]
   const float2* gtab;       // [Lc][d/2] Global RoPE (cos, sin) at k_off + u
+  const float2* gstep;      // [d/2] (cos, sin) of the rotation by 512 / d positions
   float* part_o;            // [P][S][rows][d]   rows = G * route_block
   float* part_ml;           // [P][S][rows][2]   (running max in log2 units, sum)
   float* out;               // [B, Hq, Tq, d] fp32

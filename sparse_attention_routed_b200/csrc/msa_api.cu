@@ -376,6 +376,10 @@ msa_status ensure_gtab(msa_bank* bank, int64_t koff, int lc, cudaStream_t s) {
   if (bank->gtab_koff == koff && bank->gtab_lc >= lc) return MSA_OK;
   if (capturing(s)) return MSA_ERR_INVALID_ARG;
   std::vector<float2> t = rope_table(koff, lc, bank->d, bank->base);
+  // one more row: the rotation by 512 / d positions, the distance between the keys of a
+  // local tile that one lane of the decode kernel rotates (it steps the angles by it)
+  const std::vector<float2> step = rope_table(512 / bank->d, 1, bank->d, bank->base);
+  t.insert(t.end(), step.begin(), step.end());
   const size_t bytes = t.size() * sizeof(float2);
   if (bytes > bank->gtab_cap) {
     MSA_CUDA(cudaDeviceSynchronize());
@@ -773,6 +777,7 @@ msa_status attend_impl(msa_bank* bank, const msa_query* q, const StepShape& s, i
   a.sel_base = sel_base;
   a.doc_len = bank->d_doc_len;
   a.gtab = bank->d_gtab;
+  a.gstep = bank->d_gtab + (size_t)bank->gtab_lc * (bank->d / 2);
   a.part_o = w.part_o;
   a.part_ml = w.part_ml;
   a.out = out;
