@@ -13,8 +13,8 @@
 //    one CTA each (split-KV), so ragged documents balance by construction.
 //    With n_local_splits > 0 the local tiles get splits of their own, whose
 //    CTAs never read the selection: launched as a programmatic dependent of the
-//    top-k, every CTA sets up while routing finishes, the local ones go on with
-//    their tiles, and only the document CTAs wait for the selection.
+//    top-k, with those CTAs first, they stream the local context beside the
+//    router, and only the document CTAs wait for the selection.
 //  * One producer lane streams K and V tiles with 2-D TMA loads (128-byte
 //    swizzle, evict-first L2 policy) into a ring of WARPS x BUFS slots; consumer
 //    warp w owns slots w, w + WARPS, ... and takes relative tiles w, w + WARPS, ...
@@ -129,10 +129,25 @@ __global__ void __launch_bounds__(S::THREADS, S::MINB)
   const int warp = tid >> 5, lane = tid & 31;
   const int G = a.n_q_heads / a.n_kv_heads;
   const int nblk = a.q_tokens / a.route_block;
-  // CTA -> (problem, split), problem after problem, so that the local tiles (Global RoPE
-  // in shared memory) spread evenly over the waves.
+  // CTA -> (problem, split). Launched the ordinary way: problem after problem, so that
+  // the local tiles (Global RoPE in shared memory) spread evenly over the waves. As a
+  // programmatic dependent: every problem's local splits first (split 0 of every
+  // problem, then split 1, ...), so that they run beside the routing, then the document
+  // splits problem after problem. The order moves no tile to another split.
   const int nls = a.n_local_splits;
-  const int p = blockIdx.x / a.n_splits, split = blockIdx.x % a.n_splits;
+  const int n_problems = a.batch * nblk * a.n_kv_heads;
+  int p, split;
+  if (!a.pdl || nls == 0) {
+    p = blockIdx.x / a.n_splits;
+    split = blockIdx.x % a.n_splits;
+  } else if ((int)blockIdx.x < n_problems * nls) {
+    split = blockIdx.x / n_problems;
+    p = blockIdx.x % n_problems;
+  } else {
+    const int l = blockIdx.x - n_problems * nls, nds = a.n_splits - nls;
+    p = l / nds;
+    split = nls + l % nds;
+  }
   const bool local_cta = split < nls;
   const int h = p % a.n_kv_heads;
   const int blk = (p / a.n_kv_heads) % nblk;

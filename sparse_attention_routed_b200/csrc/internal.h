@@ -63,6 +63,7 @@ struct RouteArgs {
   int32_t q_tokens, route_block;
   int* err;                // device error flag for expired waits, or nullptr
   int32_t kr_bf16;         // 1: read only the bf16 high part of the normalised K_r (half the bytes)
+  int32_t max_ctas_per_sm; // 0: as many as shared memory allows (3); fewer leaves room beside the router
 };
 // Largest routing block for which the router computes q_r itself.
 constexpr int kRouteFuseMaxBlock = 4;
@@ -126,8 +127,8 @@ struct AttendArgs {
   // context) into n_splits ranges of equal cost. n > 0 gives the local context splits
   // of its own: splits [0, n) cut the local tiles, splits [n, n_splits) the document
   // tiles. Those CTAs never read the selection, so with a programmatic dependent
-  // launch (pdl) they run while the selection is still being made; the document CTAs
-  // wait for it.
+  // launch (pdl), which puts them first, they run while the selection is still being
+  // made; the document CTAs wait for it.
   int32_t n_local_splits;
   int32_t pdl;              // launch as a programmatic dependent of the previous kernel on the stream
 };

@@ -401,8 +401,9 @@ msa_status ensure_gtab(msa_bank* bank, int64_t koff, int lc, cudaStream_t s) {
 // `scores` [rows][Hkv][n_docs]: from q_r / q_r_inv ([rows][Hkv][d_r], [rows][Hkv]),
 // or, when `fuse`, with q_r formed inside the router from q->qr.
 msa_status run_router(msa_bank* bank, const msa_query* q, const StepShape& s, const float* q_r,
-                      const float* q_r_inv, float* scores, bool fuse, cudaStream_t st) {
+                      const float* q_r_inv, float* scores, bool fuse, cudaStream_t st, int max_ctas_per_sm = 0) {
   RouteArgs ra{};
+  ra.max_ctas_per_sm = max_ctas_per_sm;
   if (fuse) {
     ra.qr = (const uint16_t*)q->qr;
     ra.q_tokens = s.Tq;
@@ -430,8 +431,9 @@ msa_status run_router(msa_bank* bank, const msa_query* q, const StepShape& s, co
 // The routing step. q_r / q_r_inv ([rows][Hkv][d_r], [rows][Hkv]) and score_scratch
 // ([rows][Hkv][n_docs], used when doc_scores is NULL) are the caller's scratch.
 // `overlap` (the decode router, with the decode attention queued right behind it on
-// `st`): the top-k is a programmatic dependent of the router, so that it and then the
-// attention (a programmatic dependent of the top-k) set up while the router finishes.
+// `st`): the top-k is a programmatic dependent of the router, and the router keeps to 2
+// CTAs per SM, so that the attention (a programmatic dependent of the top-k) streams the
+// local context with one CTA per SM beside the router.
 msa_status route_into(msa_bank* bank, const msa_query* q, const StepShape& s, float* q_r, float* q_r_inv,
                       float* score_scratch, float* doc_scores, int32_t* idx, float* top_scores, cudaStream_t st,
                       bool overlap = false) {
@@ -444,7 +446,7 @@ msa_status route_into(msa_bank* bank, const msa_query* q, const StepShape& s, fl
     MSA_CUDA(launch_qr_prep(qa, st));
   }
   float* scores = doc_scores ? doc_scores : score_scratch;
-  msa_status rc = run_router(bank, q, s, q_r, q_r_inv, scores, fuse, st);
+  msa_status rc = run_router(bank, q, s, q_r, q_r_inv, scores, fuse, st, overlap ? 2 : 0);
   if (rc != MSA_OK) return rc;
   TopkArgs ta{scores, idx, top_scores, s.P, bank->n_docs, s.k, bank->doc_lo};
   ta.pdl = overlap ? 1 : 0;

@@ -118,7 +118,8 @@ __global__ void __launch_bounds__((RWARPS + 1) * 32, 3)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nrows = min(NR, a.rows - row0);
   __shared__ int doc_range[2];
-  // A programmatic dependent (the top-k) may launch and set up at once; it waits for
+  // A programmatic dependent (the top-k) may launch and set up at once (and the
+  // attention behind it run its local-context CTAs in the room left); it waits for
   // this grid to finish before it reads the scores.
   pdl_launch_dependents();
 
@@ -303,6 +304,7 @@ cudaError_t launch_route_t(const RouteArgs& a, const RouteMaps& m, int row0, int
   if (e != cudaSuccess) return e;
   int per_sm = (int)((228 * 1024) / (smem + 1024));  // 228 KiB per SM, 1 KiB reserved per CTA
   per_sm = per_sm < 1 ? 1 : (per_sm > 3 ? 3 : per_sm);
+  if (a.max_ctas_per_sm > 0 && per_sm > a.max_ctas_per_sm) per_sm = a.max_ctas_per_sm;
   // one wave of resident CTAs over the chunk ranges
   int gx = (sms * per_sm) / a.n_kv_heads;
   gx = gx < 1 ? 1 : (gx > a.n_docs ? a.n_docs : gx);
