@@ -479,28 +479,35 @@ def measure_device(args, wname: str, n: int, warmup: int, world: int, rank: int,
     torch.cuda.synchronize()
     clocks = ClockSampler(local)
     time.sleep(0.4)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(2 * n)]
     t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def phases(e):
+        # the two phases on their own (not the headline): the router + top-k, then the attention
+        for i in range(n):
+            e[i][0].record(stream)
+            msa_route(bank.handle, qry, k, 0, idx.data_ptr(), 0, sh)
+            e[i][1].record(stream)
+            msa_attend(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
+            e[i][2].record(stream)
+
     clocks.mark(True)
+    # n phase steps before and n after the timed steps, so that a clock that drifts under
+    # the power cap weighs on the phase times as on the timed steps
+    phases(ev[:n])
     t_begin.record(stream)
     for i in range(n):
         step()
     t_end.record(stream)
-    # the two phases on their own (not the headline): the router + top-k, then the attention
-    for i in range(n):
-        ev[i][0].record(stream)
-        msa_route(bank.handle, qry, k, 0, idx.data_ptr(), 0, sh)
-        ev[i][1].record(stream)
-        msa_attend(bank.handle, qry, k, idx.data_ptr(), out.data_ptr(), sh)
-        ev[i][2].record(stream)
+    phases(ev[n:])
     torch.cuda.synchronize()
     clocks.mark(False)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
     total_ms = t_begin.elapsed_time(t_end)
-    route_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / n
-    attend_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / n
+    route_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / len(ev)
+    attend_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / len(ev)
     assert bank.device_error() == 0
 
     e2e_ms, n_e2e, h2d, d2h = None, 0, 0, 0
