@@ -282,7 +282,7 @@ msa_status msa_attend_backward_saved(msa_bank* bank, const msa_query* q, int32_t
  * topk_idx [B, nblk, Hkv, top_k] receives the selection, out [B, Hq, Tq, d]
  * fp32 the attention. On a pinned-host bank the fetch overlaps the routing of
  * the next micro-batch of sequences. For decode-sized problems (at most 16 query
- * rows per problem) on a device bank, the top-k and the attention start as
+ * rows per problem) on a device bf16 bank, the top-k and the attention start as
  * programmatic dependents of the kernel before them, so the attention's CTAs
  * for the local context run while the selection is made; the outputs are
  * identical, bit for bit, to msa_route followed by msa_attend. Errors as
