@@ -552,7 +552,7 @@ def measure_device(args, wname: str, n: int, warmup: int, world: int, rank: int,
         out_h = [torch.empty(outbuf.shape, dtype=outbuf.dtype, pin_memory=True) for _ in range(2)]
         h2d = qin_h.numel() * 2 + kv_h.numel() * 2
         d2h = out_h[0].numel()
-        n_e2e = max(10, n // 2)
+        n_e2e = max(10, n)   # as many steps as the headline, so the pipeline's fill and drain weigh alike
         s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
         ev_in = [torch.cuda.Event() for _ in range(2)]
         ev_comp = [torch.cuda.Event() for _ in range(2)]
