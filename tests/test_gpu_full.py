@@ -1,6 +1,8 @@
 """Full-size parity on the benchmark workload (decode_4m: 4.19M-token bank,
-batch 8, 32/8 heads, top_k 16), in the launch configuration bench.py times
-(msa_route then msa_attend), on outputs the oracle computes one by one:
+batch 8, 32/8 heads, top_k 16), on outputs the oracle computes one by one, through
+msa_route then msa_attend; the launch configuration bench.py times (msa_forward:
+programmatic dependent launches, the local context's CTAs beside the router) must
+give the same selection and output bit for bit:
 
 * K_r of 256 random (head, chunk) pairs and the RoPE'd keys of 256 random tokens;
 * every document score and the top-16 of all 8 sequences for one KV head
@@ -34,10 +36,12 @@ def run():
     bank.reserve(qry, w.top_k)
     idx, tsc, scores = bank.route(qry, w.top_k)
     out = bank.attend(qry, w.top_k, idx)
+    idx_f, out_f = bank.forward(qry, w.top_k)
     torch.cuda.synchronize()
     assert bank.device_error() == 0
     res = dict(w=w, bank=bank, K=K, idx=idx.cpu().numpy(), tsc=tsc.cpu().numpy(),
-               scores=scores.cpu().numpy(), out=out.cpu().numpy(), kr=bank.k_r())
+               scores=scores.cpu().numpy(), out=out.cpu().numpy(), kr=bank.k_r(),
+               idx_f=idx_f.cpu().numpy(), out_f=out_f.cpu().numpy())
     yield res
     bank.close()
 
@@ -100,3 +104,9 @@ def test_all_attention_rows(run):
                 gots.append(run["out"][b, hq, 0])
     assert len(gots) == w.batch * w.n_q_heads
     P.check_out(np.stack(gots), np.stack(refs))
+
+
+def test_forward_equals_route_then_attend(run):
+    """msa_forward, as bench.py times it, gives the bits of msa_route + msa_attend."""
+    np.testing.assert_array_equal(run["idx_f"], run["idx"])
+    np.testing.assert_array_equal(run["out_f"], run["out"])
