@@ -7,7 +7,7 @@ give the same selection and output bit for bit:
 * K_r of 256 random (head, chunk) pairs and the RoPE'd keys of 256 random tokens;
 * every document score and the top-16 of all 8 sequences for one KV head
   (the oracle pools that head's whole bank: 16384 chunks);
-* the attention output of 8 random (sequence, query head) rows over the GPU's
+* the attention output of all 256 (sequence, query head) rows over the GPU's
   selection (checked above to be a correct top-k).
 """
 import numpy as np
