@@ -38,6 +38,9 @@ SMALL = {
     "prefill_bq128": Workload("prefill_bq128", 23, 1, 2, 2, 128, 10, 0, 256, 256, 128, 3, ragged=(60, 700)),
     # the largest top_k (64) over 80 short documents, decode kernel with G = 2
     "topk64": Workload("topk64", 24, 2, 4, 2, 128, 80, 0, 130, 1, 1, 64, ragged=(1, 200)),
+    # a long local context next to two short documents: most decode splits are the local
+    # context's own (and a single document split per problem)
+    "local_heavy": Workload("local_heavy", 26, 2, 8, 2, 128, 6, 100, 6000, 1, 1, 2),
 }
 
 
